@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Throughput of exact batched Lloyd k-means on B200 (iterations per second).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl fkm|reference]
+
+A step is one full Lloyd run of the workload (its configured iterations of
+assign + sort-inverse update through fkm_lloyd), inputs resident in HBM.  The
+metric is Lloyd iterations/sec on the B x N x K x D problem; the JSON line
+also carries the assign kernel's TFLOP/s and the update stages' GB/s, both
+from CUDA events recorded on the launching stream inside the timed region.
+
+Default workload: B=32, N=65536, D=128, K=1024, bf16 Dirichlet(0.5)-weighted
+Gaussian mixture, 10 iterations, tol=0 (512 MiB of points: larger than L2, so
+no flush is needed between steps).  Under torchrun (N > 1) every rank runs its
+own independent batch of problems (different seeds): weak scaling, no
+collective on the data path.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this build)
+on a bounded sample of the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import datagen  # noqa: E402
+
+METRIC = "Lloyd iterations/sec (assign+update) per BxNxKxD"
+UNIT = "iters/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "assign_traffic.json")
+ASSIGN_SRC = os.path.join(ROOT, "exact_means_clustering_b200", "csrc", "assign_tc.cu")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+def workload_config(w: datagen.Workload) -> dict:
+    return {"workload": w.name, "B": w.B, "N": w.N, "D": w.D, "K": w.K, "dtype": w.dtype,
+            "iters_per_step": w.iters, "tol": w.tol,
+            "data": ("seeded Gaussian mixture" if w.n_comp else "seeded standard normal"),
+            "l2": f"inputs larger than L2 ({w.x_bytes / 2**20:.0f} MiB of points), no flush"}
+
+
+def assign_flops(w):
+    return 2.0 * w.B * w.N * w.K * w.D
+
+
+def update_bytes(w):
+    # points read once, ids read, new centroids written + previous read, counts written
+    return (w.B * w.N * w.D * w.elem_bytes + 4.0 * w.B * w.N + 8.0 * w.B * w.K * w.D
+            + 4.0 * w.B * w.K)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def source_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def assign_traffic(config_name):
+    """DRAM bytes per assign launch from a committed ncu summary, when it was
+    taken on the current kernel source for this workload; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except OSError:
+        return None
+    if t.get("kernel_source_sha") != source_sha(ASSIGN_SRC):
+        return None
+    return t.get("per_launch_bytes", {}).get(config_name)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def window(self, t0, t1):
+        """Keep only samples read between host times t0 and t1 (the timed region)."""
+        self.t0, self.t1 = t0, t1
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", 1e30)
+        for ts, ln in self.lines:
+            if not (t0 <= ts <= t1 + 0.15):
+                continue
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 5:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+                bits = int(parts[4], 16)
+            except ValueError:
+                continue
+            for b, name in REASON_BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def oracle_sample(w, iters, rows=None):
+    """The fp64 oracle on batch 0 of the workload (its first `rows` points when
+    given) for `iters` Lloyd iterations.  Returns (seconds, scale, description):
+    the whole problem's iteration costs `scale` times the sample's."""
+    import oracle
+    n = w.N if rows is None else max(min(int(rows), w.N), w.K)
+    ws = w.scaled(B=1, N=n)
+    x = datagen.points(ws)
+    c0 = datagen.init_centroids(x, datagen.init_indices(ws), ws.dtype)
+    mir = w.dtype if w.dtype != "f32" else None
+    t0 = time.perf_counter()
+    oracle.lloyd(x, c0, iters, 0.0, dtype=w.dtype, mirror=mir)
+    dt = time.perf_counter() - t0
+    scale = w.B * (w.N / n)
+    part = "" if n == w.N else f"first {n} points of "
+    desc = (f"{part}batch 0 of {w.B} (N={w.N}, K={w.K}, D={w.D}, {w.dtype}), {iters} Lloyd "
+            f"iteration(s) of the fp64 oracle; rate scaled by 1/{scale:.4g} to the whole "
+            f"problem (cost is linear in B*N at fixed K)")
+    return dt, scale, desc
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    cores = cpu_cores()
+    # size each step's sample so that the whole run takes about two minutes
+    probe_rows = max(w.K, w.N // 64)
+    t_probe, _, _ = oracle_sample(w, 1, probe_rows)
+    per_step_budget = 120.0 / max(args.steps + args.warmup, 1)
+    rows = int(probe_rows * per_step_budget / max(t_probe, 1e-6))
+    for _ in range(args.warmup):
+        oracle_sample(w, 1, rows)
+    total, scale_sum, desc = 0.0, 0.0, ""
+    for _ in range(args.steps):
+        dt, scale, desc = oracle_sample(w, 1, rows)
+        total += dt * scale       # seconds one full-problem iteration would take
+        scale_sum += 1
+    value = args.steps / total
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(datagen.CONFIGS))
+    ap.add_argument("--impl", default="fkm", choices=["fkm", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-iters", type=int, default=10)
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = datagen.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    if w.host_resident:
+        print(json.dumps({"error": "use --config 1..4; the host-resident workload is timed by "
+                                   "bench_host (fkm_lloyd_host)"}))
+        return 2
+
+    import torch
+    import exact_means_clustering_b200 as fkm
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    # per rank: its own batch of problems (weak scaling)
+    wr = w.scaled(seed=w.seed + 1000 * rank)
+    x = datagen.points(wr)
+    c0 = datagen.init_centroids(x, datagen.init_indices(wr), wr.dtype)
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wr.dtype]
+    xh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if wr.dtype == "bf16"
+          else torch.from_numpy(x)).pin_memory()
+    ch = torch.from_numpy(c0).pin_memory()
+    dev = torch.device("cuda", local)
+    xt = xh.to(dev)
+    c0t = ch.to(dev)
+    B, N, D, K = wr.B, wr.N, wr.D, wr.K
+    ids = torch.empty(B, N, dtype=torch.int32, device=dev)
+    centers = torch.empty(B, K, D, dtype=torch.float32, device=dev)
+    counts = torch.empty(B, K, dtype=torch.int32, device=dev)
+    inertia = torch.empty(B, dtype=torch.float64, device=dev)
+    ws = fkm.workspace(fkm.fkm_workspace_size(B, N, K, D, tdt), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return fkm.fkm_lloyd(xt, c0t, wr.iters, wr.tol, ids, centers, counts, inertia, ws=ws,
+                             stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    fkm.fkm_profile(True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    fkm.fkm_profile_read(reset=True)
+    launches0 = fkm.fkm_kernel_launches()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    iters_done = 0
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)  # let the sampler start
+        barrier()
+        torch.cuda.synchronize(dev)
+        h0 = time.time()
+        e0.record(stream)
+        for _ in range(args.steps):
+            iters_done += step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        clk.window(h0, time.time())
+        barrier()
+    launches = fkm.fkm_kernel_launches() - launches0
+    prof = fkm.fkm_profile_read(reset=True)
+    fkm.fkm_profile(False)
+    elapsed_ms = e0.elapsed_time(e1)
+    t_max = elapsed_ms
+    total_iters = iters_done
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = t.item()
+        n = torch.tensor([iters_done], device=dev, dtype=torch.float64)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+        total_iters = int(n.item())
+    value = total_iters / (t_max / 1e3)
+
+    # --- per-stage rates from the events recorded inside the timed region
+    it = max(prof["iterations"], 1)
+    t_assign = prof["assign"] / it / 1e3
+    t_update = (prof["argsort"] + prof["segsum"] + prof["finalize"]) / it / 1e3
+    peaks, peak_src = load_peaks()
+    tflops = assign_flops(wr) / t_assign / 1e12 if t_assign > 0 else None
+    upd_gbs = update_bytes(wr) / t_update / 1e9 if t_update > 0 else None
+    peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if wr.dtype == "f32":
+        # split-bf16: the algorithmic FLOPs run as three bf16 products on the tensor cores
+        bound_note = "fp32 points as split bf16 (3 tensor-core products per algorithmic one)"
+    else:
+        bound_note = "bf16/fp16 operands, fp32 accumulate"
+    traffic = assign_traffic(wr.name)
+    roofline = {"bound": "tensor", "kernel": "assign_tc_kernel", "achieved": tflops,
+                "peak": peak_t, "unit": "TFLOP/s",
+                "frac": (tflops / peak_t) if tflops else None, "traffic": traffic,
+                "peak_source": f"{peak_src} (bf16 sustained, MEASURED_PEAKS.json)",
+                "note": bound_note,
+                "flops_per_launch": assign_flops(wr),
+                "launch_ms": t_assign * 1e3}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wr.dtype, "data": "synthetic", "config": workload_config(wr),
+            "roofline": roofline,
+            "stages_ms_per_iter": {k: prof[k] / it for k in fkm.STAGES},
+            "assign_tflops": tflops,
+            "update_gbs": upd_gbs,
+            "update_frac_of_hbm": (upd_gbs / peaks["hbm_gbs"]) if upd_gbs else None,
+            "gpu_launches": int(launches),
+            "clocks": clk.summary()}
+
+    # --- end to end through the C ABI with host buffers
+    if not args.no_e2e:
+        ids_h = torch.empty(B, N, dtype=torch.int32).pin_memory()
+        cen_h = torch.empty(B, K, D, dtype=torch.float32).pin_memory()
+        cnt_h = torch.empty(B, K, dtype=torch.int32).pin_memory()
+        ine_h = torch.empty(B, dtype=torch.float64).pin_memory()
+        x_e = torch.empty_like(xt)
+        c_e = torch.empty_like(c0t)
+
+        def e2e_step():
+            x_e.copy_(xh, non_blocking=True)
+            c_e.copy_(ch, non_blocking=True)
+            n_it = fkm.fkm_lloyd(x_e, c_e, wr.iters, wr.tol, ids, centers, counts, inertia,
+                                 ws=ws, stream=stream)
+            ids_h.copy_(ids, non_blocking=True)
+            cen_h.copy_(centers, non_blocking=True)
+            cnt_h.copy_(counts, non_blocking=True)
+            ine_h.copy_(inertia, non_blocking=True)
+            return n_it
+
+        for _ in range(max(args.warmup, 1)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0.record(stream)
+        n_e = 0
+        for _ in range(args.steps):
+            n_e += e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        t_e = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([t_e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            t_e = t.item()
+            n = torch.tensor([n_e], device=dev, dtype=torch.float64)
+            dist.all_reduce(n, op=dist.ReduceOp.SUM)
+            n_e = int(n.item())
+        line["e2e"] = {"value": n_e / (t_e / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": int(xh.numel() * xh.element_size()
+                                                 + ch.numel() * ch.element_size()),
+                       "d2h_bytes_per_step": int(ids_h.numel() * 4 + cen_h.numel() * 4
+                                                 + cnt_h.numel() * 4 + ine_h.numel() * 8)}
+
+    # --- the oracle on this host's cores (rank 0, one GPU only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, scale, desc = oracle_sample(wr, args.oracle_iters)
+        line["cpu_baseline"] = {"value": args.oracle_iters / (dt * scale), "unit": UNIT,
+                                "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

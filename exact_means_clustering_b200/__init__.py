@@ -1,0 +1,270 @@
+"""exact_means_clustering_b200 -- exact batched Lloyd k-means on NVIDIA B200.
+
+A thin ctypes binding over ``libfkm.so`` (C ABI in ``include/fkm.h``).  Every
+step of an iteration runs in the library's sm_100a kernels; this module only
+marshals torch tensors (device memory, streams) into pointers and sizes.  If
+the shared library is missing or a call fails, it raises: there is no
+fallback implementation.
+
+Functions named ``fkm_*`` mirror the C entry points one to one.  The
+convenience wrapper ``batch_kmeans_Euclid`` follows the call shape the
+Flash-KMeans README shows ("Usage": ``cluster_ids, centers, _ =
+batch_kmeans_Euclid(x, n_clusters, max_iters, tol)``); its third value is the
+number of iterations run.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfkm.so")
+
+FKM_OK = 0
+STATUS_NAMES = {0: "FKM_OK", 1: "FKM_ERR_INVALID_ARG", 2: "FKM_ERR_UNSUPPORTED",
+                3: "FKM_ERR_CUDA", 4: "FKM_ERR_WORKSPACE_TOO_SMALL", 5: "FKM_ERR_TIMEOUT",
+                6: "FKM_ERR_INTERNAL", 7: "FKM_ERR_BAD_ID"}
+DTYPES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+# every entry point of include/fkm.h: name -> (argtypes, restype)
+_P, _I, _L, _Z, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_SIG = {
+    "fkm_workspace_size": ([_I, _I, _I, _I, _I, ctypes.POINTER(_Z)], _I),
+    "fkm_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_lloyd": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _P, _P, ctypes.POINTER(_I), _P, _Z,
+                   _P], _I),
+    "fkm_host_workspace_size": ([_I, _I, _I, _I, _I, _L, ctypes.POINTER(_Z)], _I),
+    "fkm_lloyd_host": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _L, _P, _P, _P, _P,
+                        ctypes.POINTER(_I), _P, _Z, _P], _I),
+    "fkm_argsort_workspace_size": ([_L, _I, ctypes.POINTER(_Z)], _I),
+    "fkm_argsort": ([_P, _L, _I, _P, _P, _P, _Z, _P], _I),
+    "fkm_baseline_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_baseline_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_sync_status": ([_P, _Z, _P], _I),
+    "fkm_profile": ([_I], _I),
+    "fkm_profile_read": ([_P, ctypes.POINTER(ctypes.c_longlong), _I], _I),
+    "fkm_kernel_launches": ([], ctypes.c_longlong),
+    "fkm_status_string": ([_I], ctypes.c_char_p),
+    "fkm_last_error": ([], ctypes.c_char_p),
+    "fkm_version": ([], ctypes.c_char_p),
+}
+
+_lib = None
+
+
+class FkmError(RuntimeError):
+    def __init__(self, fn, code, detail):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)}: {detail}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfkm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m exact_means_clustering_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIG.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(fn, code):
+    if code != FKM_OK:
+        raise FkmError(fn, code, lib().fkm_last_error().decode(errors="replace"))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dt(x):
+    if isinstance(x, int):
+        return x
+    try:
+        return DTYPES[x if isinstance(x, torch.dtype) else x.dtype]
+    except KeyError as e:
+        raise TypeError(f"unsupported point dtype {x}") from e
+
+
+# ---------------------------------------------------------------- C mirrors
+def fkm_workspace_size(B, N, K, D, dtype) -> int:
+    out = ctypes.c_size_t(0)
+    _check("fkm_workspace_size", lib().fkm_workspace_size(B, N, K, D, _dt(dtype), ctypes.byref(out)))
+    return out.value
+
+
+def fkm_host_workspace_size(B, N, K, D, dtype, chunk_rows) -> int:
+    out = ctypes.c_size_t(0)
+    _check("fkm_host_workspace_size",
+           lib().fkm_host_workspace_size(B, N, K, D, _dt(dtype), chunk_rows, ctypes.byref(out)))
+    return out.value
+
+
+def fkm_argsort_workspace_size(n, n_keys) -> int:
+    out = ctypes.c_size_t(0)
+    _check("fkm_argsort_workspace_size",
+           lib().fkm_argsort_workspace_size(n, n_keys, ctypes.byref(out)))
+    return out.value
+
+
+def workspace(nbytes, device=None) -> torch.Tensor:
+    """A zero-filled device workspace (the library expects zeros on first use)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def fkm_assign(x, centers, ids, inertia=None, ws=None, stream=None):
+    B, N, D = x.shape
+    K = centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    _check("fkm_assign", lib().fkm_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers), _ptr(ids),
+                                          _ptr(inertia), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fkm_update(x, ids, prev_centers, centers, counts, shift=None, inertia=None, ws=None,
+               stream=None):
+    B, N, D = x.shape
+    K = prev_centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    _check("fkm_update", lib().fkm_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids),
+                                          _ptr(prev_centers), _ptr(centers), _ptr(counts),
+                                          _ptr(shift), _ptr(inertia), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
+
+
+def fkm_lloyd(x, init_centers, max_iters, tol, ids, centers, counts, inertia=None, ws=None,
+              stream=None) -> int:
+    B, N, D = x.shape
+    K = init_centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    n_iter = ctypes.c_int(0)
+    _check("fkm_lloyd", lib().fkm_lloyd(B, N, K, D, _dt(x), _ptr(x), _ptr(init_centers), max_iters,
+                                        float(tol), _ptr(ids), _ptr(centers), _ptr(counts),
+                                        _ptr(inertia), ctypes.byref(n_iter), _ptr(ws), ws.numel(),
+                                        _stream(stream)))
+    return n_iter.value
+
+
+def fkm_lloyd_host(x_host, init_centers, max_iters, tol, chunk_rows, ids, centers, counts,
+                   inertia=None, ws=None, stream=None, dtype=None, shape=None) -> int:
+    """x_host: a pinned CPU tensor [B, N, D] (or a raw address with dtype and shape)."""
+    if isinstance(x_host, int):
+        B, N, D = shape
+        dt = _dt(dtype)
+    else:
+        B, N, D = x_host.shape
+        dt = _dt(x_host)
+    K = init_centers.shape[1]
+    if ws is None:
+        ws = workspace(fkm_host_workspace_size(B, N, K, D, dt, chunk_rows), init_centers.device)
+    n_iter = ctypes.c_int(0)
+    _check("fkm_lloyd_host",
+           lib().fkm_lloyd_host(B, N, K, D, dt, _ptr(x_host), _ptr(init_centers), max_iters,
+                                float(tol), int(chunk_rows), _ptr(ids), _ptr(centers),
+                                _ptr(counts), _ptr(inertia), ctypes.byref(n_iter), _ptr(ws),
+                                ws.numel(), _stream(stream)))
+    return n_iter.value
+
+
+def fkm_argsort(keys, n_keys, idx, sorted_keys=None, ws=None, stream=None):
+    n = keys.numel()
+    ws = ws if ws is not None else workspace(fkm_argsort_workspace_size(n, n_keys), keys.device)
+    _check("fkm_argsort", lib().fkm_argsort(_ptr(keys), n, n_keys, _ptr(idx), _ptr(sorted_keys),
+                                            _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fkm_baseline_assign(x, centers, dist, ids, ws=None, stream=None):
+    B, N, D = x.shape
+    K = centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    _check("fkm_baseline_assign",
+           lib().fkm_baseline_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers), _ptr(dist),
+                                     _ptr(ids), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fkm_baseline_update(x, ids, prev_centers, centers, counts, ws=None, stream=None):
+    B, N, D = x.shape
+    K = prev_centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    _check("fkm_baseline_update",
+           lib().fkm_baseline_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids), _ptr(prev_centers),
+                                     _ptr(centers), _ptr(counts), _ptr(ws), ws.numel(),
+                                     _stream(stream)))
+
+
+def fkm_sync_status(ws, stream=None):
+    _check("fkm_sync_status", lib().fkm_sync_status(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fkm_profile(enable: bool) -> None:
+    _check("fkm_profile", lib().fkm_profile(1 if enable else 0))
+
+
+STAGES = ("assign", "argsort", "segsum", "finalize", "iteration")
+
+
+def fkm_profile_read(reset: bool = False) -> dict:
+    """Accumulated stage milliseconds of profiled fkm_lloyd calls, and iterations."""
+    ms = (ctypes.c_double * 5)()
+    it = ctypes.c_longlong(0)
+    _check("fkm_profile_read", lib().fkm_profile_read(ms, ctypes.byref(it), 1 if reset else 0))
+    out = {s: ms[i] for i, s in enumerate(STAGES)}
+    out["iterations"] = it.value
+    return out
+
+
+def fkm_kernel_launches() -> int:
+    return int(lib().fkm_kernel_launches())
+
+
+def fkm_version() -> str:
+    return lib().fkm_version().decode()
+
+
+# ---------------------------------------------------------------- wrapper
+def batch_kmeans_Euclid(x: torch.Tensor, n_clusters: int, max_iters: int = 100, tol: float = 0.0,
+                        init_centroids: torch.Tensor | None = None, seed: int = 0):
+    """Exact batched Lloyd k-means.  x: [B, N, D] (or [N, D]) CUDA tensor in
+    float32 / float16 / bfloat16.  Returns (cluster_ids int32 [B, N], centers
+    float32 [B, K, D], n_iter).  Default initial centroids: per batch, the
+    points at the first K positions of a seeded random permutation."""
+    squeeze = x.dim() == 2
+    if squeeze:
+        x = x.unsqueeze(0)
+    x = x.contiguous()
+    B, N, D = x.shape
+    K = int(n_clusters)
+    dev = x.device
+    if init_centroids is None:
+        g = torch.Generator(device="cpu").manual_seed(seed)
+        idx = torch.stack([torch.randperm(N, generator=g)[:K] for _ in range(B)]).to(dev)
+        init = torch.gather(x, 1, idx.unsqueeze(-1).expand(B, K, D)).float().contiguous()
+    else:
+        init = init_centroids.reshape(B, K, D).to(device=dev, dtype=torch.float32).contiguous()
+    ids = torch.empty(B, N, dtype=torch.int32, device=dev)
+    centers = torch.empty(B, K, D, dtype=torch.float32, device=dev)
+    counts = torch.empty(B, K, dtype=torch.int32, device=dev)
+    n_iter = fkm_lloyd(x, init, max_iters, tol, ids, centers, counts)
+    if squeeze:
+        return ids[0], centers[0], n_iter
+    return ids, centers, n_iter

@@ -1,0 +1,161 @@
+// Internal definitions shared by the library's translation units.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fkm.h"
+
+namespace fkm {
+
+// Bits of the device status word (workspace slot 0): kernels OR these in.
+enum : int {
+  ST_TIMEOUT = 1,     // a bounded wait on an mbarrier ran out
+  ST_BAD_ID = 2,      // fkm_update got an id outside [0, K)
+  ST_INTERNAL = 4,    // an internal consistency check failed
+};
+
+// Assign tiling: 128 points (TMEM lanes) x 256 centroids (TMEM columns) per
+// accumulator; K-chunks of 64 16-bit values (one 128-byte swizzled row).
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int KC = 64;
+constexpr int A_CHUNK_BYTES = BM * KC * 2;   // 16 KB
+constexpr int B_CHUNK_BYTES = BN * KC * 2;   // 32 KB
+constexpr int ASSIGN_THREADS = 192;          // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int TMEM_COLS = 512;               // two 256-column fp32 accumulators
+
+// Update tiling: sorted positions are cut into ranges of SEG_RANGE rows, one
+// warp per range.  A segment (run of equal keys) contained in one range is
+// finished by that warp; one that spans ranges is summed with fp64 atomics.
+constexpr int SEG_RANGE = 512;
+
+// Radix argsort: 8-bit digits, 256 threads x 16 keys per tile.
+constexpr int RADIX_BITS = 8;
+constexpr int RADIX_BINS = 1 << RADIX_BITS;
+constexpr int SORT_THREADS = 256;
+constexpr int SORT_ITEMS = 16;
+constexpr int SORT_TILE = SORT_THREADS * SORT_ITEMS;
+
+__host__ __device__ inline int elem_bytes(int dtype) { return dtype == FKM_F32 ? 4 : 2; }
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// thread-local error text (fkm_last_error)
+void set_error(const char* fmt, ...);
+fkm_status cuda_fail(cudaError_t e, const char* what);
+
+#define FKM_CUDA_TRY(call)                                  \
+  do {                                                      \
+    cudaError_t e_ = (call);                                \
+    if (e_ != cudaSuccess) return ::fkm::cuda_fail(e_, #call); \
+  } while (0)
+
+#define FKM_TRY(call)                   \
+  do {                                  \
+    fkm_status s_ = (call);             \
+    if (s_ != FKM_OK) return s_;        \
+  } while (0)
+
+// ---------------------------------------------------------------- workspace
+// Every buffer the library needs beyond the caller's inputs and outputs lives
+// in one caller-provided workspace, carved up by this layout.  Sizes depend on
+// B, N, K, D and dtype, never on N*K.
+struct Layout {
+  int B, N, K, D, dtype;
+  int Kp;          // K rounded up to BN
+  int Dp;          // D rounded up to 8 (the halves of a split row)
+  int Dq;          // columns of the quantised centroid / split-point rows
+  bool split;      // fp32 input: operands split into bf16 hi + lo
+  int m_tiles;     // ceil(N / BM)
+  int64_t n_sort;  // B * N keys
+  int n_sort_tiles;
+  int key_bits;
+  size_t status, cq, cn, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
+      segstart, segend, sums64, shiftk, cbuf, scal, total;
+};
+
+fkm_status make_layout(int B, int N, int K, int D, int dtype, Layout* L);
+
+template <typename T>
+inline T* ws_ptr(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ---------------------------------------------------------------- launchers
+struct AssignArgs {
+  int B, N, K, Kp, D, dtype;
+  bool split;
+  const void* xq;      // bf16/f16 points, or the split [hi|lo] rows for fp32
+  int x_row_elems;     // elements per row of xq (D, or 2D when split)
+  const void* cq;      // quantised centroids [B, Kp, Dq]
+  const float* cn;     // ||q(c)||^2 [B, Kp], +inf on padding rows
+  const float* xn;     // ||x||^2 [B, N] (comparison mode only)
+  int32_t* ids;        // [B, N]
+  int* status;
+  float* dist = nullptr;  // comparison mode: write the [B, N, K] distances here
+};
+fkm_status launch_assign(const AssignArgs& a, cudaStream_t st);
+bool assign_smem_plan(int D, bool split, int* nA, int* nS, size_t* smem);
+fkm_status assign_prepare();
+
+// q(c) rows [B][Kp][Dq] and ||q(c)||^2; split rows (fp32) are [hi | lo]
+// halves of round_up(D, 8) elements each.
+fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
+                                 void* cq, float* cn, cudaStream_t st);
+fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,
+                              cudaStream_t st);
+
+struct SortArgs {
+  const int32_t* ids;  // first-pass keys come from ids: key = (row / N) * K + id
+  int N, K;
+  int64_t n;           // number of keys
+  int key_bits;
+  int32_t *keys0, *vals0, *keys1, *vals1;
+  uint32_t* hist;      // [RADIX_BINS * tiles]
+  uint32_t* hist_part; // scan scratch
+  int* status;
+  int32_t* keys_out;   // set by the launcher: where the sorted keys / values ended up
+  int32_t* vals_out;
+};
+fkm_status launch_argsort_ids(SortArgs& a, cudaStream_t st);
+size_t argsort_scratch_words(int64_t n);
+
+fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
+                             int32_t* segend, cudaStream_t st);
+// Objective of the assignment being summed: chat is the centroid the assign
+// step measured against (q(c) in the points' 16-bit type [B][Kp][D], or the
+// fp32 centroids [B][K][D] for fp32 points), chat_bstride its batch stride
+// in elements; obj[b] (zeroed by the caller) receives sum ||x - chat||^2.
+struct ObjArgs {
+  const void* chat = nullptr;
+  int64_t chat_bstride = 0;
+  int K = 1;
+  double* obj = nullptr;
+};
+fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
+                         const int32_t* svals, int64_t n, int BK, const int32_t* segstart,
+                         const int32_t* segend, double* sums64, float* centers,
+                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st);
+// Direct objective of a given assignment: obj[b] += sum_i ||x_i - chat_{ids_i}||^2.
+fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const int32_t* ids,
+                            const ObjArgs& oa, cudaStream_t st);
+fkm_status launch_finalize(int B, int K, int D, int Kp, int dtype, const int32_t* segstart,
+                           const int32_t* segend, const int32_t* counts_in, double* sums64,
+                           const float* prev, float* centers, int32_t* counts, double* shiftk,
+                           void* cq, float* cn, cudaStream_t st);
+fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
+                               double* max_shift, cudaStream_t st);
+
+fkm_status launch_baseline_argmin(const float* dist, int64_t rows, int K, int32_t* ids,
+                                  cudaStream_t st);
+fkm_status launch_baseline_update(const void* x, int dtype, const int32_t* ids, int B, int N,
+                                  int K, int D, float* sums, int32_t* cnt, const float* prev,
+                                  float* centers, int32_t* counts, int* status, cudaStream_t st);
+
+int num_sms();
+
+// Counts kernel launches made by this library (fkm_kernel_launches).
+void note_launch(int n = 1);
+
+}  // namespace fkm

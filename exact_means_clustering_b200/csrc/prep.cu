@@ -1,0 +1,143 @@
+// Operand preparation for the assign kernel.
+//
+//  prep_centroids: q(c) = the fp32 centroid rounded (RNE) to the points'
+//    16-bit type, laid out [B, Kp, D] for TMA, and ||q(c)||^2 (summed in fp64,
+//    rounded once) -- the precomputed norm of the score ||c||^2 - 2 x.c
+//    ("Flash-KMeans：快速且内存高效精确K-Means聚类" summary, section 方法步骤详情
+//    step (1), which precomputes the norms).  Padding rows k >= K get q = 0
+//    and norm +inf so they never win the argmin.  For fp32 points each
+//    centroid is split into bf16 hi and lo = bf16(c - hi), rows [hi | lo], and
+//    the norm is that of the fp32 centroid.
+//  points_prep: for fp32 points, the bf16 [hi | lo] split rows the tensor
+//    cores consume (each half padded to a multiple of 8 elements); optionally
+//    ||x||^2 per point (fp64 sum rounded to fp32), which only the
+//    distance-materialising comparison path needs.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fkm_internal.cuh"
+
+namespace fkm {
+namespace {
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// one warp per padded centroid row
+__global__ void prep_centroids_kernel(const float* __restrict__ c, int B, int K, int Kp, int D,
+                                      int dtype, void* __restrict__ cq, float* __restrict__ cn) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (int64_t)B * Kp) return;
+  const int b = (int)(row / Kp), k = (int)(row % Kp);
+  const bool real = k < K;
+  const float* src = c + ((int64_t)b * K + k) * D;
+  double acc = 0.0;
+  if (dtype == FKM_F32) {
+    const int Dp = (D + 7) & ~7;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(cq) + row * (int64_t)(2 * Dp);
+    for (int d = lane; d < D; d += 32) {
+      float v = real ? src[d] : 0.0f;
+      __nv_bfloat16 h = __float2bfloat16_rn(v);
+      __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+      out[d] = h;
+      out[Dp + d] = l;
+      acc += (double)v * (double)v;
+    }
+  } else if (dtype == FKM_BF16) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(cq) + row * (int64_t)D;
+    for (int d = lane; d < D; d += 32) {
+      __nv_bfloat16 q = __float2bfloat16_rn(real ? src[d] : 0.0f);
+      out[d] = q;
+      double f = (double)__bfloat162float(q);
+      acc += f * f;
+    }
+  } else {
+    __half* out = static_cast<__half*>(cq) + row * (int64_t)D;
+    for (int d = lane; d < D; d += 32) {
+      __half q = __float2half_rn(real ? src[d] : 0.0f);
+      out[d] = q;
+      double f = (double)__half2float(q);
+      acc += f * f;
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) cn[row] = real ? (float)acc : INFINITY;
+}
+
+// one warp per point row
+__global__ void points_prep_kernel(const void* __restrict__ x, int64_t rows, int D, int dtype,
+                                   __nv_bfloat16* __restrict__ xs, float* __restrict__ xn) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  double acc = 0.0;
+  if (dtype == FKM_F32) {
+    const int Dp = (D + 7) & ~7;
+    const float* src = static_cast<const float*>(x) + row * D;
+    __nv_bfloat16* out = xs + row * (int64_t)(2 * Dp);
+    for (int d = lane; d < D; d += 32) {
+      float v = src[d];
+      __nv_bfloat16 h = __float2bfloat16_rn(v);
+      __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+      if (xs) {
+        out[d] = h;
+        out[Dp + d] = l;
+      }
+      acc += (double)v * (double)v;
+    }
+  } else {
+    // 16-bit points: 8-byte loads, four values per lane per step
+    const uint2* src = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + row * D);
+    const int nv = D / 4;
+    for (int v = lane; v < nv; v += 32) {
+      uint2 w = src[v];
+      uint32_t wd[2] = {w.x, w.y};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float a, bb;
+        if (dtype == FKM_BF16) {
+          a = __uint_as_float(wd[h] << 16);
+          bb = __uint_as_float(wd[h] & 0xFFFF0000u);
+        } else {
+          __half2 hv = *reinterpret_cast<__half2*>(&wd[h]);
+          float2 f = __half22float2(hv);
+          a = f.x;
+          bb = f.y;
+        }
+        acc += (double)a * a + (double)bb * bb;
+      }
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0 && xn) xn[row] = (float)acc;
+}
+
+}  // namespace
+
+fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
+                                 void* cq, float* cn, cudaStream_t st) {
+  const int64_t rows = (int64_t)B * Kp;
+  const int wpb = 8;
+  prep_centroids_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(centers, B, K, Kp, D,
+                                                                           dtype, cq, cn);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,
+                              cudaStream_t st) {
+  if (rows == 0) return FKM_OK;
+  const int wpb = 8;
+  points_prep_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(
+      x, rows, D, dtype, static_cast<__nv_bfloat16*>(xs), xn);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+}  // namespace fkm

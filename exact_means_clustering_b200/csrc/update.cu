@@ -1,0 +1,499 @@
+// Sort-Inverse Update, after the argsort ("Flash-KMeans：快速且内存高效精确K-Means
+// 聚类" summary, section 方法步骤详情 step (2); "Flash-KMeans: Fast and
+// Memory-Efficient Exact K-Means" summary, section "Method"):
+//
+//   seg_bounds  runs of equal keys in the sorted order: start/end per key, so
+//               counts = end - start are exact integers.
+//   segsum      the sorted order is cut into ranges of SEG_RANGE rows, one warp
+//               per range.  The warp walks its rows in order, gathering each
+//               row of the UNPERMUTED x by the sorted index with 16-byte loads
+//               (several rows per warp step when a row is narrower than 512 B)
+//               and adding it into fp64 registers.  When the key changes the
+//               partial sum is reduced across the warp with shuffles and
+//               flushed once: a run that lies inside this range is final, so
+//               the warp writes its centroid s/n directly; a run that crosses a
+//               range boundary is added to fp64 sums with one atomic per
+//               element (at most two such flushes per range), i.e. the pages'
+//               one atomic_add per segment boundary, O(K + N/B_N) of them.
+//               The same pass forms the objective of the assignment,
+//               sum ||x - c_hat||^2 with the direct difference (c_hat = the
+//               centroid the assign step measured against), so the reported
+//               inertia does not suffer the cancellation of the expanded form.
+//   finalize    per cluster: counts, c = s/n for crossing runs, the previous
+//               centroid for empty clusters (a reading: the pages give only
+//               c = s/n), the shift ||c_new - c_old||^2, and the next
+//               iteration's tensor-core operands q(c), ||q(c)||^2.
+//   batch_reduce  per batch, in fixed order: shift = sum_k shift_k.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fkm_internal.cuh"
+
+namespace fkm {
+namespace {
+
+__global__ void seg_bounds_kernel(const int32_t* __restrict__ skeys, int64_t n, int BK,
+                                  int32_t* __restrict__ segstart, int32_t* __restrict__ segend) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int32_t k = skeys[i];
+  if (k < 0 || k >= BK) return;  // sentinel of a rejected id
+  if (i == 0 || skeys[i - 1] != k) segstart[k] = (int32_t)i;
+  if (i == n - 1 || skeys[i + 1] != k) segend[k] = (int32_t)(i + 1);
+}
+
+struct SegParams {
+  const void* x;
+  const int32_t* skeys;
+  const int32_t* svals;
+  int64_t n;
+  int D;
+  int BK;
+  int64_t row_bytes;
+  int V;                 // 16-byte vectors per row
+  const int32_t* segstart;
+  const int32_t* segend;
+  double* sums64;
+  float* centers;
+  bool accumulate_all;   // out-of-core chunks: every run goes to sums64
+  ObjArgs oa;
+};
+
+// 16-byte vectors of the storage type, widened to float.
+template <int DT> struct Vec;
+template <> struct Vec<FKM_BF16> {
+  static constexpr int E = 8;
+  __device__ static void widen(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+template <> struct Vec<FKM_F16> {
+  static constexpr int E = 8;
+  __device__ static void widen(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+};
+template <> struct Vec<FKM_F32> {
+  static constexpr int E = 4;
+  __device__ static void widen(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+};
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Flush of one run: acc summed over the row groups (xor shuffles), then
+// written by group 0 either as the final centroid (run inside this range) or
+// added to the fp64 accumulators (run crossing a range boundary).
+template <int E, int LPR>
+__device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, int sub,
+                                          bool lane_has_vec, double (&acc)[E]) {
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  if (g == 0 && lane_has_vec) {
+    const int32_t s = p.segstart[key], t = p.segend[key];
+    const bool interior = !p.accumulate_all && (s / SEG_RANGE) == ((t - 1) / SEG_RANGE);
+    const int64_t col0 = (int64_t)sub * E;
+    if (interior) {
+      const double nk = (double)(t - s);
+      float* c = p.centers + (int64_t)key * p.D + col0;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (col0 + e < p.D) c[e] = (float)(acc[e] / nk);
+    } else {
+      double* sd = p.sums64 + (int64_t)key * p.D + col0;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (col0 + e < p.D) atomicAdd(sd + e, acc[e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.0;
+}
+
+// One warp per SEG_RANGE sorted rows; RPS rows per warp step, LPR = 32/RPS
+// lanes per row, lane `sub` of a row holds vector `sub` (when sub < V).
+template <int DT, int RPS>
+__global__ void __launch_bounds__(256) segsum_kernel(SegParams p) {
+  constexpr int E = Vec<DT>::E;
+  constexpr int LPR = 32 / RPS;
+  constexpr int U = RPS >= 8 ? 1 : (RPS >= 4 ? 2 : 4);  // warp steps loaded ahead
+  const int lane = threadIdx.x & 31;
+  const int g = lane / LPR, sub = lane % LPR;
+  const int64_t nranges = ceil_div(p.n, SEG_RANGE);
+  const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const bool lane_has_vec = sub < p.V;
+  const bool want_obj = p.oa.obj != nullptr;
+  const int64_t elem_bytes_ = p.row_bytes / p.D;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < nranges;
+       r += warps_total) {
+    const int64_t j0 = r * SEG_RANGE;
+    const int64_t j1 = (j0 + SEG_RANGE < p.n) ? j0 + SEG_RANGE : p.n;
+    double acc[E];
+    float chat[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      acc[e] = 0.0;
+      chat[e] = 0.0f;
+    }
+    double obj = 0.0;
+    int cur = -1, cur_b = -1;
+
+    for (int64_t jb = j0; jb < j1; jb += (int64_t)RPS * U) {
+      int32_t key[U];
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t jr = jb + (int64_t)u * RPS + g;
+        key[u] = -1;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (jr < j1) {
+          key[u] = p.skeys[jr];
+          if (key[u] >= p.BK) key[u] = -1;   // rejected id: skip the row
+          if (key[u] >= 0 && lane_has_vec) {
+            const int64_t rowi = p.svals[jr];
+            v[u] = ldg_nc_v4(static_cast<const char*>(p.x) + rowi * p.row_bytes + (int64_t)sub * 16);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+#pragma unroll
+        for (int gg = 0; gg < RPS; ++gg) {
+          const int kg = __shfl_sync(0xffffffffu, key[u], gg * LPR);
+          if (kg < 0) continue;
+          if (kg != cur) {
+            if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc);
+            cur = kg;
+            if (want_obj) {
+              const int b = kg / p.oa.K, k = kg % p.oa.K;
+              if (b != cur_b) {
+                if (cur_b >= 0) {
+                  const double t = warp_sum(obj);
+                  if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
+                }
+                obj = 0.0;
+                cur_b = b;
+              }
+              if (lane_has_vec) {
+                const char* row = static_cast<const char*>(p.oa.chat) +
+                                  ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.D) * elem_bytes_;
+                Vec<DT>::widen(ldg_nc_v4(row + (int64_t)sub * 16), chat);
+              }
+            }
+          }
+          if (g == gg && lane_has_vec) {
+            float f[E];
+            Vec<DT>::widen(v[u], f);
+            float d2 = 0.0f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              acc[e] += (double)f[e];
+              const float df = f[e] - chat[e];
+              d2 = fmaf(df, df, d2);
+            }
+            if (want_obj) obj += (double)d2;
+          }
+        }
+      }
+    }
+    if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc);
+    if (want_obj && cur_b >= 0) {
+      const double t = warp_sum(obj);
+      if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
+    }
+  }
+}
+
+// Direct objective of a given assignment, one warp per point row; grid.y = batch.
+template <int DT>
+__global__ void __launch_bounds__(256) objective_kernel(const void* __restrict__ x,
+                                                        const int32_t* __restrict__ ids, int N,
+                                                        int D, int V, int64_t row_bytes,
+                                                        ObjArgs oa, int rows_per_block) {
+  constexpr int E = Vec<DT>::E;
+  __shared__ double red[8];
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r0 = (int64_t)blockIdx.x * rows_per_block;
+  double acc = 0.0;
+  for (int64_t i = r0 + warp; i < r0 + rows_per_block && i < N; i += 8) {
+    const int id = ids[(int64_t)b * N + i];
+    if (id < 0 || id >= oa.K || lane >= V) continue;
+    float f[E], c[E];
+    Vec<DT>::widen(ldg_nc_v4(static_cast<const char*>(x) + ((int64_t)b * N + i) * row_bytes +
+                             lane * 16),
+                   f);
+    const char* crow = static_cast<const char*>(oa.chat) +
+                       ((int64_t)b * oa.chat_bstride + (int64_t)id * D) * (row_bytes / D);
+    Vec<DT>::widen(ldg_nc_v4(crow + lane * 16), c);
+    float d2 = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float df = f[e] - c[e];
+      d2 = fmaf(df, df, d2);
+    }
+    acc += (double)d2;
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) red[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < 8; ++w) t += red[w];
+    atomicAdd(oa.obj + b, t);
+  }
+}
+
+struct FinParams {
+  int B, K, D, Kp, dtype;
+  const int32_t* segstart;
+  const int32_t* segend;
+  double* sums64;
+  const float* prev;
+  float* centers;
+  int32_t* counts;
+  double* shiftk;
+  void* cq;
+  float* cn;
+  const int32_t* counts_in;  // out-of-core: accumulated counts (segstart/end unused)
+};
+
+// one warp per cluster
+__global__ void finalize_kernel(FinParams p) {
+  const int64_t key = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (key >= (int64_t)p.B * p.K) return;
+  int32_t nk;
+  bool interior = false;
+  if (p.counts_in) {
+    nk = p.counts_in[key];
+  } else {
+    const int32_t s = p.segstart[key], t = p.segend[key];
+    nk = t - s;
+    interior = nk > 0 && (s / SEG_RANGE) == ((t - 1) / SEG_RANGE);
+  }
+  if (lane == 0 && p.counts) p.counts[key] = nk;
+  const int b = (int)(key / p.K), k = (int)(key % p.K);
+  const int64_t qrow = (int64_t)b * p.Kp + k;
+  double sh = 0.0, nrm = 0.0;
+  for (int d = lane; d < p.D; d += 32) {
+    const int64_t e = key * p.D + d;
+    const float prev = p.prev[e];
+    float v;
+    if (nk == 0) {
+      v = prev;
+    } else if (interior) {
+      v = p.centers[e];
+    } else {
+      v = (float)(p.sums64[e] / (double)nk);
+      p.sums64[e] = 0.0;   // leave the accumulator clean for the next update
+    }
+    p.centers[e] = v;
+    const double df = (double)v - (double)prev;
+    sh += df * df;
+    if (p.cq) {
+      if (p.dtype == FKM_F32) {
+        const int Dp = (p.D + 7) & ~7;
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.cq) + qrow * (2 * Dp);
+        __nv_bfloat16 h = __float2bfloat16_rn(v);
+        o[d] = h;
+        o[Dp + d] = __float2bfloat16_rn(v - __bfloat162float(h));
+        nrm += (double)v * v;
+      } else if (p.dtype == FKM_BF16) {
+        __nv_bfloat16 q = __float2bfloat16_rn(v);
+        static_cast<__nv_bfloat16*>(p.cq)[qrow * p.D + d] = q;
+        const double f = __bfloat162float(q);
+        nrm += f * f;
+      } else {
+        __half q = __float2half_rn(v);
+        static_cast<__half*>(p.cq)[qrow * p.D + d] = q;
+        const double f = __half2float(q);
+        nrm += f * f;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sh += __shfl_xor_sync(0xffffffffu, sh, o);
+    nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
+  }
+  if (lane == 0) {
+    p.shiftk[key] = sh;
+    if (p.cq) p.cn[qrow] = (float)nrm;
+  }
+}
+
+// one block per batch; fixed-order tree sum
+__global__ void __launch_bounds__(256) batch_reduce_kernel(int K, const double* __restrict__ shiftk,
+                                                           double* shift_out, double* max_shift) {
+  __shared__ double s1[256];
+  const int b = blockIdx.x;
+  double a = 0.0;
+  for (int k = threadIdx.x; k < K; k += 256) a += shiftk[(int64_t)b * K + k];
+  s1[threadIdx.x] = a;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) s1[threadIdx.x] += s1[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    if (shift_out) shift_out[b] = s1[0];
+    if (max_shift)  // shift >= 0: the bit pattern orders like the value
+      atomicMax(reinterpret_cast<unsigned long long*>(max_shift),
+                (unsigned long long)__double_as_longlong(s1[0]));
+  }
+}
+
+template <int DT, int RPS>
+fkm_status run_segsum(const SegParams& sp, cudaStream_t st) {
+  const int64_t nranges = ceil_div(sp.n, SEG_RANGE);
+  const int wpb = 8;
+  int64_t blocks = ceil_div(nranges, wpb);
+  if (blocks < 1) blocks = 1;
+  segsum_kernel<DT, RPS><<<(unsigned)blocks, wpb * 32, 0, st>>>(sp);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+template <int DT>
+fkm_status run_segsum_dt(const SegParams& sp, cudaStream_t st) {
+  int lpr = 1;
+  while (lpr < sp.V) lpr <<= 1;
+  switch (32 / lpr) {
+    case 1: return run_segsum<DT, 1>(sp, st);
+    case 2: return run_segsum<DT, 2>(sp, st);
+    case 4: return run_segsum<DT, 4>(sp, st);
+    case 8: return run_segsum<DT, 8>(sp, st);
+    case 16: return run_segsum<DT, 16>(sp, st);
+    default: return run_segsum<DT, 32>(sp, st);
+  }
+}
+
+}  // namespace
+
+fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
+                             int32_t* segend, cudaStream_t st) {
+  FKM_CUDA_TRY(cudaMemsetAsync(segstart, 0, sizeof(int32_t) * (size_t)BK, st));
+  FKM_CUDA_TRY(cudaMemsetAsync(segend, 0, sizeof(int32_t) * (size_t)BK, st));
+  if (n > 0) {
+    seg_bounds_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(skeys, n, BK, segstart, segend);
+    note_launch();
+    FKM_CUDA_TRY(cudaGetLastError());
+  }
+  return FKM_OK;
+}
+
+fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
+                         const int32_t* svals, int64_t n, int BK, const int32_t* segstart,
+                         const int32_t* segend, double* sums64, float* centers,
+                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st) {
+  if (n == 0) return FKM_OK;
+  SegParams sp;
+  sp.x = x;
+  sp.skeys = skeys;
+  sp.svals = svals;
+  sp.n = n;
+  sp.D = D;
+  sp.BK = BK;
+  sp.row_bytes = (int64_t)D * elem_bytes(dtype);
+  sp.V = (int)(sp.row_bytes / 16);
+  sp.segstart = segstart;
+  sp.segend = segend;
+  sp.sums64 = sums64;
+  sp.centers = centers;
+  sp.accumulate_all = accumulate_all;
+  sp.oa = oa;
+  if (sp.V > 32) {
+    set_error("rows of %lld bytes exceed the update kernel's 512-byte limit",
+              (long long)sp.row_bytes);
+    return FKM_ERR_UNSUPPORTED;
+  }
+  if (dtype == FKM_BF16) return run_segsum_dt<FKM_BF16>(sp, st);
+  if (dtype == FKM_F16) return run_segsum_dt<FKM_F16>(sp, st);
+  return run_segsum_dt<FKM_F32>(sp, st);
+}
+
+fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const int32_t* ids,
+                            const ObjArgs& oa, cudaStream_t st) {
+  const int64_t row_bytes = (int64_t)D * elem_bytes(dtype);
+  const int V = (int)(row_bytes / 16);
+  const int rpb = 64;
+  dim3 grid((unsigned)ceil_div(N, rpb), (unsigned)B);
+  if (dtype == FKM_BF16)
+    objective_kernel<FKM_BF16><<<grid, 256, 0, st>>>(x, ids, N, D, V, row_bytes, oa, rpb);
+  else if (dtype == FKM_F16)
+    objective_kernel<FKM_F16><<<grid, 256, 0, st>>>(x, ids, N, D, V, row_bytes, oa, rpb);
+  else
+    objective_kernel<FKM_F32><<<grid, 256, 0, st>>>(x, ids, N, D, V, row_bytes, oa, rpb);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+fkm_status launch_finalize(int B, int K, int D, int Kp, int dtype, const int32_t* segstart,
+                           const int32_t* segend, const int32_t* counts_in, double* sums64,
+                           const float* prev, float* centers, int32_t* counts, double* shiftk,
+                           void* cq, float* cn, cudaStream_t st) {
+  FinParams fp;
+  fp.B = B;
+  fp.K = K;
+  fp.D = D;
+  fp.Kp = Kp;
+  fp.dtype = dtype;
+  fp.segstart = segstart;
+  fp.segend = segend;
+  fp.sums64 = sums64;
+  fp.prev = prev;
+  fp.centers = centers;
+  fp.counts = counts;
+  fp.shiftk = shiftk;
+  fp.cq = cq;
+  fp.cn = cn;
+  fp.counts_in = counts_in;
+  const int64_t keys = (int64_t)B * K;
+  const int wpb = 8;
+  finalize_kernel<<<(unsigned)ceil_div(keys, wpb), wpb * 32, 0, st>>>(fp);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
+                               double* max_shift, cudaStream_t st) {
+  batch_reduce_kernel<<<B, 256, 0, st>>>(K, shiftk, shift_out, max_shift);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+}  // namespace fkm

@@ -1,0 +1,200 @@
+/*
+ * fkm.h -- C ABI of libfkm: exact batched Lloyd k-means on NVIDIA B200 (sm_100a).
+ *
+ * The problem is the one the Flash-KMeans pages state with
+ * batch_kmeans_Euclid(x, n_clusters, max_iters, tol) -> (cluster_ids, centers, _)
+ * ("Flash-KMeans" GitHub README, section "Usage"): B independent problems, each
+ * N points of dimension D clustered into K centroids by Lloyd iterations
+ * (assign every point to its nearest centroid, then move every centroid to the
+ * mean of its points), minimising sum_i ||x_i - c_{a_i}||^2 ("Flash-KMeans：快速且
+ * 内存高效精确K-Means聚类" summary, section 前置知识 / K-Means聚类算法).
+ *
+ * Conventions shared by every entry point
+ *   Layout     x is [B, N, D] row-major and contiguous, in `dtype`.
+ *              Centroids are float32 [B, K, D]; ids int32 [B, N] (values in
+ *              [0, K)); counts int32 [B, K]; per-batch scalars are [B].
+ *   Pointers   "device" = memory the current CUDA device can address (cudaMalloc
+ *              or torch CUDA tensors); "host" = CPU memory.  Every pointer must
+ *              be 16-byte aligned.  The caller owns every buffer; the library
+ *              allocates no device memory of its own: scratch comes from the
+ *              caller's workspace (see fkm_workspace_size), whose size never
+ *              depends on N*K (the B x N x K distance matrix is never formed).
+ *   Streams    `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *              stream).  Work is stream-ordered; functions marked "async" return
+ *              before the GPU finishes.
+ *   Limits     B, N, K, D >= 1; D * sizeof(dtype) a multiple of 16 bytes
+ *              (D % 8 == 0 for bf16/fp16, D % 4 == 0 for fp32);
+ *              D <= 256 (fp32: D <= 128); B*N < 2^31; B*K < 2^31.
+ *   Errors     Arguments are validated before anything is launched; a violation
+ *              returns FKM_ERR_INVALID_ARG or FKM_ERR_UNSUPPORTED and launches
+ *              nothing.  There is no fallback path of any kind.  CUDA failures
+ *              return FKM_ERR_CUDA.  Kernels report what they detect (a bounded
+ *              wait that ran out, an out-of-range id) in a status word inside
+ *              the workspace, read by fkm_sync_status (and by fkm_lloyd itself).
+ *              fkm_last_error() gives a thread-local description of the last
+ *              failure.
+ */
+#ifndef FKM_H_
+#define FKM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FKM_API __attribute__((visibility("default")))
+#else
+#define FKM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FKM_OK = 0,
+  FKM_ERR_INVALID_ARG = 1,
+  FKM_ERR_UNSUPPORTED = 2,
+  FKM_ERR_CUDA = 3,
+  FKM_ERR_WORKSPACE_TOO_SMALL = 4,
+  FKM_ERR_TIMEOUT = 5,
+  FKM_ERR_INTERNAL = 6,
+  FKM_ERR_BAD_ID = 7
+} fkm_status;
+
+/* storage type of the points */
+typedef enum { FKM_F32 = 0, FKM_F16 = 1, FKM_BF16 = 2 } fkm_dtype;
+
+/* Bytes of device workspace fkm_assign / fkm_update / fkm_lloyd need for this
+ * shape (one size serves all three).  Host-only: makes no CUDA call.
+ * Returns FKM_ERR_INVALID_ARG / FKM_ERR_UNSUPPORTED for shapes the library
+ * rejects.  `bytes` (host) receives the size. */
+FKM_API fkm_status fkm_workspace_size(int B, int N, int K, int D, int dtype, size_t* bytes);
+
+/* Assign step (predict): ids[b,i] = argmin_k ||x[b,i] - q(c[b,k])||^2, ties to
+ * the lowest k, with q() the rounding of the fp32 centroid to `dtype` (the
+ * tensor-core operand type; for fp32 points the product is carried in split
+ * bf16 hi+lo form, relative error about 2^-17).  Computed as the online argmin
+ * of ||q(c)||^2 - 2 x.q(c) over centroid tiles on tcgen05 tensor cores, without
+ * ever writing a distance matrix ("Flash-KMeans: Fast and Memory-Efficient
+ * Exact K-Means" summary, section "Method", FlashAssign; "Flash-KMeans：快速且内存
+ * 高效精确K-Means聚类" summary, section 方法步骤详情 step (1)).
+ *   x        device [B,N,D] dtype        centers  device [B,K,D] float32
+ *   ids      device [B,N] int32 (out)
+ *   inertia  device [B] float64 (out) = sum_i ||x_i - q(c[b, ids_i])||^2 (direct
+ *            difference, fp32 terms summed in fp64), or NULL
+ *   ws       device workspace of ws_bytes >= fkm_workspace_size(...)
+ * Async. */
+FKM_API fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, const float* centers,
+                      int32_t* ids, double* inertia, void* ws, size_t ws_bytes, void* stream);
+
+/* Update step (sort-inverse update): stable radix argsort of the 1-D ids, one
+ * pass over contiguous runs of equal ids gathering rows of the UNPERMUTED x by
+ * the sorted index, fp64 sums per run, one flush per run per 512-row range of
+ * the sorted order ("Flash-KMeans: Fast and Memory-Efficient Exact K-Means"
+ * summary, section "Method", Sort-Inverse Update; "Flash-KMeans：快速且内存高效
+ * 精确K-Means聚类" summary, section 方法步骤详情 step (2)).
+ *   counts[b,k]   = number of i with ids[b,i] == k (exact)
+ *   centers[b,k]  = mean of those x_i (fp64 sum, rounded to fp32), or
+ *                   prev_centers[b,k] unchanged when counts[b,k] == 0
+ *   shift[b]      = sum_k ||centers[b,k] - prev_centers[b,k]||^2 (float64), or NULL
+ *   inertia[b]    = sum_i ||x_i - q(prev_centers[b, ids_i])||^2 (float64), the
+ *                   objective of the given assignment against the centroids an
+ *                   assign step would have used (q() as in fkm_assign), or NULL
+ *   x device [B,N,D] dtype; ids device [B,N] int32; prev_centers device [B,K,D];
+ *   centers device [B,K,D] (out, must not alias prev_centers); counts device
+ *   [B,K] int32 (out).  An id outside [0,K) sets FKM_ERR_BAD_ID in the status
+ *   word (rows with such ids are ignored).  Async. */
+FKM_API fkm_status fkm_update(int B, int N, int K, int D, int dtype, const void* x,
+                              const int32_t* ids, const float* prev_centers, float* centers,
+                              int32_t* counts, double* shift, double* inertia, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* Full Lloyd run (batch_kmeans_Euclid).  Starting from init_centers, for
+ * t < max_iters: assign, then update; stop after an update when
+ * max_b shift[b] < tol (strict, so tol = 0 runs max_iters iterations).
+ *   ids      device [B,N] (out): the last assignment
+ *   centers  device [B,K,D] (out): the centroids after the last update
+ *   counts   device [B,K] (out): sizes of the last assignment's clusters
+ *   inertia  device [B] float64 (out): objective of the last assignment against
+ *            the centroids it was made with (direct difference), or NULL
+ *   n_iter   host int (out): iterations run
+ * init_centers may alias centers.  With tol == 0 the iterations are replayed
+ * from one captured CUDA graph; with tol > 0 one 8-byte device-to-host read
+ * per iteration decides whether to stop.  Synchronous: returns after the
+ * stream has finished, with the status word checked. */
+FKM_API fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
+                     const float* init_centers, int max_iters, float tol, int32_t* ids,
+                     float* centers, int32_t* counts, double* inertia, int* n_iter, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* Device workspace for fkm_lloyd_host with chunks of `chunk_rows` points. */
+FKM_API fkm_status fkm_host_workspace_size(int B, int N, int K, int D, int dtype, int64_t chunk_rows,
+                                   size_t* bytes);
+
+/* Out-of-core Lloyd run: x stays in HOST memory (pinned, page-locked, e.g.
+ * cudaHostAlloc) and is streamed to the device in chunks of chunk_rows points
+ * through two device buffers: a copy stream fills one buffer (cudaMemcpyAsync)
+ * while the compute stream runs assign + chunk-local update on the other
+ * ("Flash-KMeans" GitHub README, section "Large tensor Benchmark"; "Flash-KMeans：
+ * 快速且内存高效精确K-Means聚类" summary, section 方法步骤详情 step (3)).
+ * Results are the same as fkm_lloyd's.  Outputs (ids, centers, counts,
+ * inertia) are device pointers as in fkm_lloyd; x_host is a host pointer.
+ * Synchronous. */
+FKM_API fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_host,
+                          const float* init_centers, int max_iters, float tol,
+                          int64_t chunk_rows, int32_t* ids, float* centers, int32_t* counts,
+                          double* inertia, int* n_iter, void* ws, size_t ws_bytes, void* stream);
+
+/* Stable argsort of n int32 keys in [0, n_keys) on the device (the sort inside
+ * fkm_update, exposed for tests): idx[r] = index of the r-th smallest key,
+ * equal keys in index order ("Flash-KMeans：快速且内存高效精确K-Means聚类" summary,
+ * section 前置知识 / argsort与分段规约, example [3,1,2,1,3,2] -> [1,3,2,5,0,4]).
+ * keys, idx: device int32 [n]; workspace from fkm_argsort_workspace_size.
+ * A key outside [0, n_keys) sets FKM_ERR_BAD_ID in the status word.  Async. */
+FKM_API fkm_status fkm_argsort_workspace_size(int64_t n, int n_keys, size_t* bytes);
+FKM_API fkm_status fkm_argsort(const int32_t* keys, int64_t n, int n_keys, int32_t* idx,
+                       int32_t* sorted_keys, void* ws, size_t ws_bytes, void* stream);
+
+/* Comparison point, NOT the method: the "standard" iteration the pages
+ * measure against.  Assign materialises the full fp32 distance matrix
+ * dist[b,i,k] = ||x||^2 + ||c||^2 - 2 x.c in `dist` (device, B*N*K floats,
+ * caller-allocated) and then argmins it; update scatters every point into
+ * its centroid with one atomicAdd per element ("Flash-KMeans: Fast and
+ * Memory-Efficient Exact K-Means" summary, section "Key claims" and "Method").
+ * Same outputs and workspace as fkm_assign / fkm_update.  Async. */
+FKM_API fkm_status fkm_baseline_assign(int B, int N, int K, int D, int dtype, const void* x,
+                               const float* centers, float* dist, int32_t* ids, void* ws,
+                               size_t ws_bytes, void* stream);
+FKM_API fkm_status fkm_baseline_update(int B, int N, int K, int D, int dtype, const void* x,
+                               const int32_t* ids, const float* prev_centers, float* centers,
+                               int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/* Stage timing of fkm_lloyd (tracing).  While enabled, fkm_lloyd records CUDA
+ * events on its stream (inside its captured graph too) around each stage of
+ * every iteration; fkm_profile_read returns the accumulated milliseconds per
+ * stage -- [0] assign, [1] argsort, [2] segment bounds + segment sums (+
+ * objective), [3] finalize + per-batch reduce, [4] whole iterations -- and
+ * the number of iterations timed, and optionally resets them.  Host pointers.
+ * Thread-safe; profiling serialises fkm_lloyd calls. */
+FKM_API fkm_status fkm_profile(int enable);
+FKM_API fkm_status fkm_profile_read(double* stage_ms /*[5]*/, long long* iterations, int reset);
+
+/* Number of kernels this library has launched in this process (graph replays
+ * count the kernels the graph holds). */
+FKM_API long long fkm_kernel_launches(void);
+
+/* Waits for `stream`, then reads and clears the workspace's status word:
+ * FKM_OK, FKM_ERR_TIMEOUT, FKM_ERR_BAD_ID or FKM_ERR_INTERNAL. */
+FKM_API fkm_status fkm_sync_status(void* ws, size_t ws_bytes, void* stream);
+
+FKM_API const char* fkm_status_string(fkm_status s);
+/* Thread-local text about the last failure in this thread ("" if none). */
+FKM_API const char* fkm_last_error(void);
+/* Library version string. */
+FKM_API const char* fkm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FKM_H_ */

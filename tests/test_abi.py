@@ -1,0 +1,103 @@
+"""The C ABI library: it builds, loads without a GPU, exports every entry point
+include/fkm.h declares, and its host-only paths (sizes, validation, status
+strings) behave as documented.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fkm.h")
+
+
+@pytest.fixture(scope="module")
+def fkm():
+    from exact_means_clustering_b200 import build
+    build.build()
+    import exact_means_clustering_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FKM_API\s+[\w\s\*]+?\b(fkm_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fkm_assign", "fkm_update", "fkm_lloyd", "fkm_lloyd_host",
+                     "fkm_workspace_size", "fkm_argsort", "fkm_sync_status", "fkm_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(fkm):
+    lib = ctypes.CDLL(fkm.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+    # and the binding wraps each of them under the same name
+    for n in declared_functions():
+        assert n in fkm._SIG
+
+
+def test_library_hides_internal_symbols(fkm):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", fkm.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {s for s in exported if s.startswith("fkm")}
+    assert ours == set(declared_functions())
+
+
+def test_workspace_size_is_independent_of_n_times_k(fkm):
+    a = fkm.fkm_workspace_size(1, 65536, 256, 128, 2)
+    b = fkm.fkm_workspace_size(1, 65536, 8192, 128, 2)
+    # growing K 32x grows only K-sized buffers, far below an N*K distance matrix
+    assert b - a < 65536 * (8192 - 256) * 4 / 100
+    c2 = fkm.fkm_workspace_size(32, 65536, 1024, 128, 2)
+    assert c2 < 32 * 65536 * 1024 * 4 / 50
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((0, 10, 4, 64, 2), 1),        # B < 1
+    ((1, 10, 0, 64, 2), 1),        # K < 1
+    ((1, 10, 4, 64, 9), 1),        # bad dtype
+    ((1, 10, 4, 12, 2), 2),        # 24-byte rows: not a multiple of 16
+    ((1, 10, 4, 6, 0), 2),         # 24-byte fp32 rows
+    ((1, 10, 4, 264, 2), 2),       # D too large for 16-bit points
+    ((1, 10, 4, 132, 0), 2),       # D too large for fp32 points
+    ((2, 1 << 30, 4, 64, 2), 2),   # B*N >= 2^31
+])
+def test_invalid_shapes_are_rejected(fkm, shape, code):
+    with pytest.raises(fkm.FkmError) as e:
+        fkm.fkm_workspace_size(*shape)
+    assert e.value.code == code
+    assert fkm.lib().fkm_last_error().decode()
+
+
+def test_null_pointers_rejected_before_any_launch(fkm):
+    L = fkm.lib()
+    ws = ctypes.create_string_buffer(1 << 20)
+    addr = (ctypes.addressof(ws) + 15) & ~15
+    rc = L.fkm_assign(1, 16, 4, 64, 2, None, addr, addr, None, addr, 1 << 19, None)
+    assert rc == 1
+    rc = L.fkm_update(1, 16, 4, 64, 2, addr, addr, addr, addr, addr, None, None, None, 0, None)
+    assert rc == 1
+    # workspace too small is its own status
+    rc = L.fkm_assign(1, 16, 4, 64, 2, addr, addr, addr, None, addr, 64, None)
+    assert rc == 4
+
+
+def test_status_strings_and_version(fkm):
+    L = fkm.lib()
+    assert L.fkm_status_string(0) == b"ok"
+    assert b"workspace" in L.fkm_status_string(4)
+    assert L.fkm_version().startswith(b"fkm")
+
+
+def test_argsort_workspace_size(fkm):
+    a = fkm.fkm_argsort_workspace_size(6, 4)
+    b = fkm.fkm_argsort_workspace_size(1 << 20, 4)
+    assert 0 < a < b
+    with pytest.raises(fkm.FkmError):
+        fkm.fkm_argsort_workspace_size(-1, 4)
