@@ -43,6 +43,7 @@ _SIG = {
     "fkm_argsort": ([_P, _L, _I, _P, _P, _P, _Z, _P], _I),
     "fkm_baseline_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_baseline_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_assign_noalloc": ([_I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
     "fkm_sync_status": ([_P, _Z, _P], _I),
     "fkm_profile": ([_I], _I),
     "fkm_profile_read": ([_P, ctypes.POINTER(ctypes.c_longlong), _I], _I),
@@ -210,6 +211,17 @@ def fkm_baseline_update(x, ids, prev_centers, centers, counts, ws=None, stream=N
            lib().fkm_baseline_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids), _ptr(prev_centers),
                                      _ptr(centers), _ptr(counts), _ptr(ws), ws.numel(),
                                      _stream(stream)))
+
+
+def fkm_assign_noalloc(x, centers, ids, stream=None):
+    """fkm_assign without a workspace, for callers that cannot allocate device
+    memory: its scratch is a static 16 MiB device array inside the library
+    (bf16/fp16 points only; calls that overlap on the GPU race)."""
+    B, N, D = x.shape
+    K = centers.shape[1]
+    _check("fkm_assign_noalloc", lib().fkm_assign_noalloc(B, N, K, D, _dt(x), _ptr(x),
+                                                          _ptr(centers), _ptr(ids),
+                                                          _stream(stream)))
 
 
 def fkm_sync_status(ws, stream=None):

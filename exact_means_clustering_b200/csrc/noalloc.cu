@@ -1,0 +1,111 @@
+// fkm_assign_noalloc: the assign step for callers that cannot allocate.
+//
+// Some callers are not allowed to allocate device memory at the point where
+// they need an assignment: code running inside a CUDA stream capture owned by
+// a framework that forbids allocations while capturing, real-time or embedded
+// services that reserve all memory up front in fixed pools, plugins handed
+// only their inputs and outputs by a host application.  They cannot call
+// cudaMalloc for the workspace that fkm_assign expects.
+//
+// This entry point keeps its scratch (the centroids rounded to the points'
+// 16-bit type, their squared norms, and a status word) in one file-scope
+// device array of FKM_NOALLOC_SCRATCH_BYTES.  Every GPU that loads the library
+// holds that array until the process exits.  The host-side name of the array
+// is only a stand-in: its device address is fetched with cudaGetSymbolAddress,
+// once per device, with that device current, on the first call made on it.
+#include <cstring>
+#include <mutex>
+
+#include "fkm_internal.cuh"
+
+namespace fkm {
+namespace {
+
+constexpr size_t kScratchBytes = FKM_NOALLOC_SCRATCH_BYTES;
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch array for the current device.
+fkm_status scratch_for_current_device(void** out) {
+  int dev = 0;
+  FKM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) {
+    set_error("device index %d out of range", dev);
+    return FKM_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      set_error("cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+      return FKM_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FKM_OK;
+}
+
+}  // namespace
+}  // namespace fkm
+
+using namespace fkm;
+
+extern "C" fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, const void* x,
+                                         const float* centers, int32_t* ids, void* stream) {
+  if (dtype != FKM_BF16 && dtype != FKM_F16) {
+    set_error("fkm_assign_noalloc takes bf16 or fp16 points only (fp32 points need scratch "
+              "proportional to N)");
+    return FKM_ERR_UNSUPPORTED;
+  }
+  size_t probe = 0;
+  FKM_TRY(fkm_workspace_size(B, N, K, D, dtype, &probe));  // shape validation
+  const uintptr_t need_align = 15;
+  if (!x || !centers || !ids || (reinterpret_cast<uintptr_t>(x) & need_align) ||
+      (reinterpret_cast<uintptr_t>(centers) & need_align) ||
+      (reinterpret_cast<uintptr_t>(ids) & need_align)) {
+    set_error("x, centers and ids must be non-null and 16-byte aligned");
+    return FKM_ERR_INVALID_ARG;
+  }
+  const int Kp = (int)round_up(K, BN);
+  const size_t status_bytes = 256;
+  const size_t cq_bytes = (size_t)round_up((int64_t)B * Kp * D * 2, 256);
+  const size_t cn_bytes = (size_t)round_up((int64_t)B * Kp * 4, 256);
+  if (status_bytes + cq_bytes + cn_bytes > kScratchBytes) {
+    set_error("B*Kp*(2*D + 4) = %zu bytes exceeds the %zu-byte static scratch of "
+              "fkm_assign_noalloc (Kp = K rounded up to 256)",
+              cq_bytes + cn_bytes, kScratchBytes - status_bytes);
+    return FKM_ERR_UNSUPPORTED;
+  }
+  void* base = nullptr;
+  FKM_TRY(scratch_for_current_device(&base));
+  char* p = static_cast<char*>(base);
+  int* status = reinterpret_cast<int*>(p);
+  void* cq = p + status_bytes;
+  float* cn = reinterpret_cast<float*>(p + status_bytes + cq_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the status word is the only scratch that must start at zero; the rest is
+  // fully rewritten by the centroid preparation below
+  FKM_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  FKM_TRY(launch_prep_centroids(centers, B, K, Kp, D, dtype, cq, cn, st));
+  AssignArgs a;
+  a.B = B;
+  a.N = N;
+  a.K = K;
+  a.Kp = Kp;
+  a.D = D;
+  a.dtype = dtype;
+  a.split = false;
+  a.xq = x;
+  a.x_row_elems = D;
+  a.cq = cq;
+  a.cn = cn;
+  a.xn = nullptr;
+  a.ids = ids;
+  a.status = status;
+  return launch_assign(a, st);
+}

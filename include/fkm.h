@@ -183,6 +183,34 @@ FKM_API fkm_status fkm_profile_read(double* stage_ms /*[5]*/, long long* iterati
  * count the kernels the graph holds). */
 FKM_API long long fkm_kernel_launches(void);
 
+/* Size of the static device scratch that fkm_assign_noalloc uses (16 MiB). */
+#define FKM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* fkm_assign for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is an interface for code that must not call cudaMalloc at
+ * the point it needs an assignment -- inside a stream capture owned by a
+ * framework that forbids allocating while capturing, in services that reserve
+ * all device memory up front, or in plugins that are handed only their inputs
+ * and outputs.  Same result as fkm_assign with inertia = NULL, but the
+ * scratch (the rounded centroids, their norms and a status word) lives in a
+ * file-scope device array of FKM_NOALLOC_SCRATCH_BYTES that every GPU loading
+ * the library keeps until the process exits; no workspace is passed and
+ * nothing is allocated.
+ *   x        device [B,N,D] bf16 or fp16 (fp32 points are rejected: their
+ *            split operands need scratch proportional to N)
+ *   centers  device [B,K,D] float32;  ids device [B,N] int32 (out)
+ * Limit: 256 + B*Kp*(2*D + 4) bytes (rounded to 256-byte blocks) must fit in
+ * FKM_NOALLOC_SCRATCH_BYTES, Kp = K rounded up to 256; larger shapes return
+ * FKM_ERR_UNSUPPORTED.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) and raises the kernel's shared-memory
+ * limit; make that first call before any stream capture.  All calls share
+ * the one array, which keeps the last call's contents: calls that can overlap
+ * on the GPU (other streams, other threads) race with each other, so
+ * serialise them.  Device-side status (a bounded wait that ran out) is not
+ * reported by this call.  Async. */
+FKM_API fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, const void* x,
+                                      const float* centers, int32_t* ids, void* stream);
+
 /* Waits for `stream`, then reads and clears the workspace's status word:
  * FKM_OK, FKM_ERR_TIMEOUT, FKM_ERR_BAD_ID or FKM_ERR_INTERNAL. */
 FKM_API fkm_status fkm_sync_status(void* ws, size_t ws_bytes, void* stream);
