@@ -9,16 +9,18 @@
 // The score is ||c||^2 - 2 x.c (the same page, section 核心方法: ||x||^2 is
 // constant per point and does not change the argmin).
 //
-// B200 design (one persistent CTA per SM, 192 threads):
+// B200 design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: the point tile [128 x D] once per work item into
 //               one of nA buffers, centroid tiles [256 x 64] through an
 //               nS-stage ring (128-byte swizzle, no multicast).
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators)
 //               and issues tcgen05.mma (M=128, N=256, K=16) from one thread.
-//   warps 2-5   epilogue: thread t owns TMEM lane t = point t of the tile; it
-//               reads its 256 accumulator columns (tcgen05.ld), forms
-//               score = ||q(c)||^2 - 2 acc with packed fp32x2 FMAs and keeps
-//               the running minimum; ties go to the lowest centroid index.
+//   warps 2-9   epilogue, two warpgroups: TMEM lane t = point t of the tile;
+//               warpgroup h reads columns [128h, 128h + 128) of every
+//               accumulator (tcgen05.ld), forms score = ||q(c)||^2 - 2 acc with
+//               packed fp32x2 FMAs and keeps its running minimum with 3-input
+//               min trees; the two halves are merged per work item.  Ties go
+//               to the lowest centroid index.
 // Accumulator double buffering lets the MMAs of tile t+1 run while the
 // epilogue reduces tile t; A double buffering overlaps the next work item's
 // point load with the current one's MMAs.
@@ -37,6 +39,7 @@
 #include <cuda_fp16.h>
 
 #include <cfloat>
+#include <cstddef>
 #include <cstdio>
 
 #include "fkm_internal.cuh"
@@ -69,11 +72,19 @@ struct __align__(8) SmemCtl {
   uint64_t b_full[8], b_empty[8];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t cn_full[2];
+  uint64_t merge_full, merge_empty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  float cn_s[2][BN];
+  __align__(16) float cn_s[2][BN];   // read with 16-byte loads
+  float2 merge[BM];   // (best score, index as float bits) of warpgroup 1
 };
+static_assert(offsetof(SmemCtl, cn_s) % 16 == 0, "cn_s must be 16-byte aligned");
+
+// Per epilogue thread, the scores of the chunk that last improved its
+// running minimum (32 floats), with the 16-byte units rotated by lane so the
+// predicated stores of a warp hit distinct banks.
+constexpr int kSaveBytes = 256 * 32 * 4;
 
 __device__ __forceinline__ float2 u2f2(uint32_t a, uint32_t b) {
   return make_float2(__uint_as_float(a), __uint_as_float(b));
@@ -99,29 +110,47 @@ __device__ __forceinline__ float min32(const float (&s)[32]) {
   return fminf(ptx::fmin3(n0, n1, n2), n3);
 }
 
-// Scores of one 32-column chunk, s = cn - 2 acc, folded into (best, bidx).
-// A chunk replaces the running minimum only when strictly smaller, and inside
-// a chunk the lowest column holding the minimum wins: over ascending columns
-// this keeps the lowest centroid index among exact ties.
+// Scores of one 32-column chunk, s = cn - 2 acc, folded into (best, bcol).
+// A chunk replaces the running minimum only when strictly smaller; then its
+// scores are saved so the lowest column holding the minimum can be found once
+// per work item (find_first), which keeps the lowest centroid index among
+// exact ties without a per-chunk search.
 __device__ __forceinline__ void fold_chunk(const uint32_t (&r)[32], const float* cn, int col0,
-                                           float& best, int& bidx) {
+                                           float& best, int& bcol, float4* save, int rot) {
   float s[32];
   const float2 m2 = make_float2(-2.0f, -2.0f);
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    float2 c2 = *reinterpret_cast<const float2*>(cn + j);
-    float2 v = __ffma2_rn(u2f2(r[j], r[j + 1]), m2, c2);
-    s[j] = v.x;
-    s[j + 1] = v.y;
+  for (int j = 0; j < 32; j += 4) {
+    const float4 c4 = *reinterpret_cast<const float4*>(cn + j);
+    const float2 v0 = __ffma2_rn(u2f2(r[j], r[j + 1]), m2, make_float2(c4.x, c4.y));
+    const float2 v1 = __ffma2_rn(u2f2(r[j + 2], r[j + 3]), m2, make_float2(c4.z, c4.w));
+    s[j] = v0.x;
+    s[j + 1] = v0.y;
+    s[j + 2] = v1.x;
+    s[j + 3] = v1.y;
   }
-  float cm = min32(s);
+  const float cm = min32(s);
   if (cm < best) {
     best = cm;
-    int idx = 31;
+    bcol = col0;
 #pragma unroll
-    for (int j = 30; j >= 0; --j) idx = (s[j] == cm) ? j : idx;
-    bidx = col0 + idx;
+    for (int k = 0; k < 8; ++k)
+      save[k ^ rot] = make_float4(s[4 * k], s[4 * k + 1], s[4 * k + 2], s[4 * k + 3]);
   }
+}
+
+// Lowest position j in the saved chunk whose score equals best.
+__device__ __forceinline__ int find_first(const float4* save, int rot, float best) {
+  uint32_t mask = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 v = save[k ^ rot];
+    mask |= (uint32_t)(v.x == best) << (4 * k);
+    mask |= (uint32_t)(v.y == best) << (4 * k + 1);
+    mask |= (uint32_t)(v.z == best) << (4 * k + 2);
+    mask |= (uint32_t)(v.w == best) << (4 * k + 3);
+  }
+  return mask ? __ffs(mask) - 1 : 0;
 }
 
 // kDist = true is the comparison ("standard") mode: the same tensor-core tiles,
@@ -141,6 +170,8 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   uint8_t* a_base = smem;
   uint8_t* b_base = a_base + (size_t)p.nA * p.a_bytes;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(b_base + (size_t)p.nS * p.s_bytes);
+  float4* save_base = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(ctl) +
+                                                ((sizeof(SmemCtl) + 127) & ~size_t(127)));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -157,9 +188,11 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&ctl->acc_full[i], 1);
-      ptx::mbar_init(&ctl->acc_empty[i], 4);
-      ptx::mbar_init(&ctl->cn_full[i], 128);
+      ptx::mbar_init(&ctl->acc_empty[i], 8);
+      ptx::mbar_init(&ctl->cn_full[i], 256);
     }
+    ptx::mbar_init(&ctl->merge_full, 128);
+    ptx::mbar_init(&ctl->merge_empty, 128);
     ptx::mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     ptx::fence_mbar_init();
@@ -200,16 +233,18 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
         }
         ++a_arms;
         for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
-          for (int dc = 0; dc < p.nD; ++dc) {
+          // one stage per 64-wide chunk; split operands put hi and lo in
+          // consecutive stages
+          for (int q = 0; q < p.nD * (kSplit ? 2 : 1); ++q) {
+            const int dc = kSplit ? (q >> 1) : q;
             const int sb = s_arms % p.nS;
             const uint32_t spar = ((s_arms / p.nS) & 1) ^ 1;
             if (!ptx::mbar_wait_bounded(&ctl->b_empty[sb], spar, abort_flag, p.status, ST_TIMEOUT,
                                         kWaitTimeoutNs)) { ok = false; break; }
             ptx::mbar_arrive_expect_tx(&ctl->b_full[sb], p.s_bytes);
             uint8_t* sbuf = b_base + (size_t)sb * p.s_bytes;
-            ptx::tma_load_3d(sbuf, &tm_c, &ctl->b_full[sb], dc * KC, kt * BN, b);
-            if (kSplit)
-              ptx::tma_load_3d(sbuf + B_CHUNK_BYTES, &tm_cl, &ctl->b_full[sb], dc * KC, kt * BN, b);
+            ptx::tma_load_3d(sbuf, (kSplit && (q & 1)) ? &tm_cl : &tm_c, &ctl->b_full[sb],
+                             dc * KC, kt * BN, b);
             ++s_arms;
           }
         }
@@ -244,28 +279,32 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
                                       p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-          for (int dc = 0; dc < p.nD; ++dc) {
+          for (int q = 0; q < p.nD * (kSplit ? 2 : 1); ++q) {
+            const int dc = kSplit ? (q >> 1) : q;
             const int sb = s_uses % p.nS;
             if (!ptx::mbar_wait_bounded(&ctl->b_full[sb], (s_uses / p.nS) & 1, abort_flag,
                                         p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t b_addr = ptx::smem_u32(b_base + (size_t)sb * p.s_bytes);
             const uint32_t xa = a_addr + dc * A_CHUNK_BYTES;
-#pragma unroll
-            for (int k = 0; k < KC / 16; ++k)
-              ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xa + 32 * k),
-                              ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc,
-                              (dc > 0 || k > 0) ? 1u : 0u);
-            if (kSplit) {
-              const uint32_t xl = a_addr + (p.nD + dc) * A_CHUNK_BYTES;
-              const uint32_t cl = b_addr + B_CHUNK_BYTES;
+            if (!(kSplit && (q & 1))) {
+              // xh . ch (or x . q(c)); the first product of the tile overwrites
 #pragma unroll
               for (int k = 0; k < KC / 16; ++k)
                 ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xa + 32 * k),
-                                ptx::umma_desc_sw128(cl + 32 * k), p.idesc, 1u);
+                                ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc,
+                                (q > 0 || k > 0) ? 1u : 0u);
+              if (kSplit) {   // xl . ch
+                const uint32_t xl = a_addr + (p.nD + dc) * A_CHUNK_BYTES;
+#pragma unroll
+                for (int k = 0; k < KC / 16; ++k)
+                  ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xl + 32 * k),
+                                  ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc, 1u);
+              }
+            } else {          // xh . cl
 #pragma unroll
               for (int k = 0; k < KC / 16; ++k)
-                ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xl + 32 * k),
+                ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xa + 32 * k),
                                 ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc, 1u);
             }
             issued = true;
@@ -288,33 +327,45 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;          // 0..127
+    const int et = threadIdx.x - 64;          // 0..255
+    const int ew = warp - 2;                  // epilogue warp 0..7
+    const int half = ew >> 2;                 // columns [128*half, 128*half + 128) of a tile
     const int quad = warp & 3;                // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;         // point within the tile
+    const int rot = lane & 7;
+    float4* save = save_base + (size_t)(ew * 32 + lane) * 8;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
-    uint32_t acc_uses = 0;
+    uint32_t acc_uses = 0, items = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < p.n_work && ok; w += gridDim.x) {
+    // ||q(c)||^2 of the next tile, loaded one tile ahead so the global load
+    // is off the critical path
+    float cn_pre = (blockIdx.x < (unsigned)p.n_work)
+                       ? p.cn[(size_t)(blockIdx.x / p.m_tiles) * p.Kp + et] : 0.0f;
+    for (int w = blockIdx.x; w < p.n_work && ok; w += gridDim.x, ++items) {
       const int b = w / p.m_tiles, mt = w % p.m_tiles;
       float best = INFINITY;
-      int bidx = 0;
+      int bcol = 0;
       for (int kt = 0; kt < p.k_tiles; ++kt) {
         const int acc = acc_uses & 1;
         const uint32_t par = (acc_uses >> 1) & 1;
+        const float cn_cur = cn_pre;
+        if (kt + 1 < p.k_tiles)
+          cn_pre = p.cn[(size_t)b * p.Kp + (size_t)(kt + 1) * BN + et];
+        else if (w + (int)gridDim.x < p.n_work)
+          cn_pre = p.cn[(size_t)((w + gridDim.x) / p.m_tiles) * p.Kp + et];
         // Stage ||q(c)||^2 of this centroid tile in shared memory.  Buffer acc
         // was last read two tiles ago, and every thread finished that tile
         // before it arrived for the previous one, so it is free to overwrite.
-        const float* cn_g = p.cn + (size_t)b * p.Kp + (size_t)kt * BN;
-        ctl->cn_s[acc][et] = cn_g[et];
-        ctl->cn_s[acc][et + 128] = cn_g[et + 128];
+        ctl->cn_s[acc][et] = cn_cur;
         ptx::mbar_arrive(&ctl->cn_full[acc]);
         if (!ptx::mbar_wait_bounded(&ctl->cn_full[acc], par, abort_flag, p.status, ST_TIMEOUT,
                                     kWaitTimeoutNs)) { ok = false; break; }
         if (!ptx::mbar_wait_bounded(&ctl->acc_full[acc], par, abort_flag, p.status, ST_TIMEOUT,
                                     kWaitTimeoutNs)) { ok = false; break; }
         ptx::tc_fence_after();
-        const uint32_t taddr = lane_addr + (uint32_t)(acc * BN);
-        const float* cn_s = ctl->cn_s[acc];
+        const uint32_t taddr = lane_addr + (uint32_t)(acc * BN + half * 128);
+        const float* cn_s = ctl->cn_s[acc] + half * 128;
+        const int colb = kt * BN + half * 128;
         uint32_t r0[32], r1[32];
         if (kDist) {
           const int gi = mt * BM + row;
@@ -322,15 +373,15 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
           float* drow = p.dist + ((size_t)b * p.N + (gi < p.N ? gi : 0)) * p.K;
           const bool vec4 = (p.K & 3) == 0;
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
+          for (int c = 0; c < 4; ++c) {
             ptx::tmem_ld32(taddr + c * 32, r0);
             ptx::tmem_wait_ld32(r0);
-            if (c == BN / 32 - 1) {
+            if (c == 3) {
               ptx::tc_fence_before();
               __syncwarp();
               if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
             }
-            const int col0 = kt * BN + c * 32;
+            const int col0 = colb + c * 32;
             if (gi < p.N && col0 < p.K) {
               float dv[32];
 #pragma unroll
@@ -353,28 +404,42 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
         }
         ptx::tmem_ld32(taddr, r0);
         ptx::tmem_wait_ld32(r0);
-#pragma unroll
-        for (int c = 0; c < BN / 32; c += 2) {
-          ptx::tmem_ld32(taddr + (c + 1) * 32, r1);
-          fold_chunk(r0, cn_s + c * 32, kt * BN + c * 32, best, bidx);
-          ptx::tmem_wait_ld32(r1);
-          if (c + 2 < BN / 32) {
-            ptx::tmem_ld32(taddr + (c + 2) * 32, r0);
-          } else {
-            // every column of this accumulator is in registers: hand it back
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
-          }
-          fold_chunk(r1, cn_s + (c + 1) * 32, kt * BN + (c + 1) * 32, best, bidx);
-          if (c + 2 < BN / 32) ptx::tmem_wait_ld32(r0);
-        }
+        ptx::tmem_ld32(taddr + 32, r1);
+        fold_chunk(r0, cn_s, colb, best, bcol, save, rot);
+        ptx::tmem_wait_ld32(r1);
+        ptx::tmem_ld32(taddr + 64, r0);
+        fold_chunk(r1, cn_s + 32, colb + 32, best, bcol, save, rot);
+        ptx::tmem_wait_ld32(r0);
+        ptx::tmem_ld32(taddr + 96, r1);
+        fold_chunk(r0, cn_s + 64, colb + 64, best, bcol, save, rot);
+        ptx::tmem_wait_ld32(r1);
+        // every column this warp reads from the accumulator is in registers
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
+        fold_chunk(r1, cn_s + 96, colb + 96, best, bcol, save, rot);
         ++acc_uses;
       }
       if (!ok) break;
       if (kDist) continue;
-      const int gi = mt * BM + row;
-      if (gi < p.N) p.ids[(size_t)b * p.N + gi] = bidx;
+      const int idx = bcol + find_first(save, rot, best);
+      // merge the two column halves of each row
+      const uint32_t mpar = items & 1;
+      if (half == 1) {
+        if (!ptx::mbar_wait_bounded(&ctl->merge_empty, mpar ^ 1, abort_flag, p.status,
+                                    ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+        ctl->merge[row] = make_float2(best, __int_as_float(idx));
+        ptx::mbar_arrive(&ctl->merge_full);
+      } else {
+        if (!ptx::mbar_wait_bounded(&ctl->merge_full, mpar, abort_flag, p.status, ST_TIMEOUT,
+                                    kWaitTimeoutNs)) { ok = false; break; }
+        const float2 o = ctl->merge[row];
+        ptx::mbar_arrive(&ctl->merge_empty);
+        const int oidx = __float_as_int(o.y);
+        const int fidx = (o.x < best || (o.x == best && oidx < idx)) ? oidx : idx;
+        const int gi = mt * BM + row;
+        if (gi < p.N) p.ids[(size_t)b * p.N + gi] = fidx;
+      }
     }
   }
 
@@ -440,8 +505,8 @@ constexpr int kSmemBudget = 232448 - 1024;  // opt-in maximum minus alignment sl
 bool assign_smem_plan(int D, bool split, int* nA_out, int* nS_out, size_t* smem_out) {
   const int nD = (int)ceil_div(D, KC);
   const long a_bytes = (long)(split ? 2 : 1) * nD * A_CHUNK_BYTES;
-  const long s_bytes = (long)(split ? 2 : 1) * B_CHUNK_BYTES;
-  const long ctl = (long)sizeof(SmemCtl);
+  const long s_bytes = B_CHUNK_BYTES;
+  const long ctl = (long)((sizeof(SmemCtl) + 127) & ~size_t(127)) + kSaveBytes;
   int nA = 2;
   long nS = (kSmemBudget - ctl - 2 * a_bytes) / s_bytes;
   if (nS < 2) {
@@ -512,7 +577,7 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
   p.nA = nA;
   p.nS = nS;
   p.a_bytes = (uint32_t)((a.split ? 2 : 1) * nD * A_CHUNK_BYTES);
-  p.s_bytes = (uint32_t)((a.split ? 2 : 1) * B_CHUNK_BYTES);
+  p.s_bytes = (uint32_t)B_CHUNK_BYTES;
   p.idesc = ptx::umma_idesc_f16(bf16, BM, BN);
   p.cn = a.cn;
   p.xn = a.xn;

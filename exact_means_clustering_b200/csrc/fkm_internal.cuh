@@ -22,13 +22,13 @@ constexpr int BN = 256;
 constexpr int KC = 64;
 constexpr int A_CHUNK_BYTES = BM * KC * 2;   // 16 KB
 constexpr int B_CHUNK_BYTES = BN * KC * 2;   // 32 KB
-constexpr int ASSIGN_THREADS = 192;          // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int ASSIGN_THREADS = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int TMEM_COLS = 512;               // two 256-column fp32 accumulators
 
 // Update tiling: sorted positions are cut into ranges of SEG_RANGE rows, one
 // warp per range.  A segment (run of equal keys) contained in one range is
 // finished by that warp; one that spans ranges is summed with fp64 atomics.
-constexpr int SEG_RANGE = 512;
+constexpr int SEG_RANGE = 256;
 
 // Radix argsort: 8-bit digits, 256 threads x 16 keys per tile.
 constexpr int RADIX_BITS = 8;

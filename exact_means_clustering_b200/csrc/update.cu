@@ -108,12 +108,18 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
-// Flush of one run: acc summed over the row groups (xor shuffles), then
-// written by group 0 either as the final centroid (run inside this range) or
-// added to the fp64 accumulators (run crossing a range boundary).
+// Flush of one run: the fp32 partial is folded into fp64, the partials are
+// summed over the row groups (xor shuffles), and group 0 writes either the
+// final centroid (run inside this range) or adds to the fp64 accumulators
+// (run crossing a range boundary).
 template <int E, int LPR>
 __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, int sub,
-                                          bool lane_has_vec, double (&acc)[E]) {
+                                          bool lane_has_vec, double (&acc)[E], float (&acc32)[E]) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    acc[e] += (double)acc32[e];
+    acc32[e] = 0.0f;
+  }
 #pragma unroll
   for (int o = LPR; o < 32; o <<= 1)
 #pragma unroll
@@ -139,97 +145,147 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
   for (int e = 0; e < E; ++e) acc[e] = 0.0;
 }
 
-// One warp per SEG_RANGE sorted rows; RPS rows per warp step, LPR = 32/RPS
-// lanes per row, lane `sub` of a row holds vector `sub` (when sub < V).
+constexpr int SEG_WARPS = 8;   // warps (ranges) per block
+constexpr int SEG_STAGES = 8;  // row-gather steps in flight per warp
+
+__device__ __forceinline__ void cp_async_16(void* smem, const void* gmem, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_stages() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(SEG_STAGES - 1) : "memory");
+}
+
+// One warp per SEG_RANGE sorted rows.  The range's (key, row) pairs are
+// staged in shared memory first; then every lane gathers its 16-byte piece of
+// the rows RPS at a time (LPR = 32 / RPS lanes per row, lane `sub` holding
+// vector `sub` of its row) with cp.async into a per-warp ring of SEG_STAGES
+// steps, so SEG_STAGES * RPS rows are in flight while the warp adds the
+// oldest step.  Rows are added in fp32 and folded into fp64 at every run
+// flush and every 16 steps.
 template <int DT, int RPS>
-__global__ void __launch_bounds__(256) segsum_kernel(SegParams p) {
+__global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) {
   constexpr int E = Vec<DT>::E;
   constexpr int LPR = 32 / RPS;
-  constexpr int U = RPS >= 8 ? 1 : (RPS >= 4 ? 2 : 4);  // warp steps loaded ahead
-  const int lane = threadIdx.x & 31;
+  __shared__ int2 kv_s[SEG_WARPS][SEG_RANGE];
+  __shared__ uint4 ring_s[SEG_WARPS][SEG_STAGES][32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int g = lane / LPR, sub = lane % LPR;
-  const int64_t nranges = ceil_div(p.n, SEG_RANGE);
-  const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   const bool lane_has_vec = sub < p.V;
   const bool want_obj = p.oa.obj != nullptr;
   const int64_t elem_bytes_ = p.row_bytes / p.D;
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < nranges;
-       r += warps_total) {
-    const int64_t j0 = r * SEG_RANGE;
-    const int64_t j1 = (j0 + SEG_RANGE < p.n) ? j0 + SEG_RANGE : p.n;
-    double acc[E];
-    float chat[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      acc[e] = 0.0;
-      chat[e] = 0.0f;
+  const int64_t r = (int64_t)blockIdx.x * SEG_WARPS + wid;
+  const int64_t nranges = ceil_div(p.n, SEG_RANGE);
+  if (r >= nranges) return;
+  const int64_t j0 = r * SEG_RANGE;
+  const int nrows = (int)((j0 + SEG_RANGE < p.n) ? SEG_RANGE : p.n - j0);
+  int2* kv = kv_s[wid];
+  uint4 (*ring)[32] = ring_s[wid];
+  for (int i = lane; i < SEG_RANGE; i += 32) {
+    int2 e = make_int2(-1, 0);
+    if (i < nrows) {
+      e.x = p.skeys[j0 + i];
+      e.y = p.svals[j0 + i];
+      if (e.x >= p.BK) e.x = -1;   // rejected id: skip the row
     }
-    double obj = 0.0;
-    int cur = -1, cur_b = -1;
+    kv[i] = e;
+  }
+  __syncwarp();
 
-    for (int64_t jb = j0; jb < j1; jb += (int64_t)RPS * U) {
-      int32_t key[U];
-      uint4 v[U];
+  const char* xb = static_cast<const char*>(p.x) + (int64_t)sub * 16;
+  const int nsteps = (nrows + RPS - 1) / RPS;
+  auto issue = [&](int s) {   // gather step s into ring slot s % SEG_STAGES
+    const int i = s * RPS + g;
+    bool valid = false;
+    const char* src = xb;
+    if (s < nsteps && i < nrows) {
+      const int2 e = kv[i];
+      valid = e.x >= 0 && lane_has_vec;
+      if (valid) src = xb + (int64_t)e.y * p.row_bytes;
+    }
+    cp_async_16(&ring[s % SEG_STAGES][lane], src, valid);
+    cp_async_commit();
+  };
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t jr = jb + (int64_t)u * RPS + g;
-        key[u] = -1;
-        v[u] = make_uint4(0, 0, 0, 0);
-        if (jr < j1) {
-          key[u] = p.skeys[jr];
-          if (key[u] >= p.BK) key[u] = -1;   // rejected id: skip the row
-          if (key[u] >= 0 && lane_has_vec) {
-            const int64_t rowi = p.svals[jr];
-            v[u] = ldg_nc_v4(static_cast<const char*>(p.x) + rowi * p.row_bytes + (int64_t)sub * 16);
+  for (int s = 0; s < SEG_STAGES - 1; ++s) issue(s);
+
+  double acc[E];
+  float acc32[E], chat[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    acc[e] = 0.0;
+    acc32[e] = 0.0f;
+    chat[e] = 0.0f;
+  }
+  double obj = 0.0;
+  float obj32 = 0.0f;
+  int cur = -1, cur_b = -1;
+
+#pragma unroll 1
+  for (int s = 0; s < nsteps; ++s) {
+    issue(s + SEG_STAGES - 1);
+    cp_async_wait_stages();   // step s has landed
+    __syncwarp();
+#pragma unroll
+    for (int gg = 0; gg < RPS; ++gg) {
+      const int kg = kv[s * RPS + gg].x;   // same address in every lane: broadcast
+      if (kg < 0) continue;
+      if (kg != cur) {
+        if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc, acc32);
+        cur = kg;
+        if (want_obj) {
+          obj += (double)obj32;
+          obj32 = 0.0f;
+          const int b = kg / p.oa.K, k = kg % p.oa.K;
+          if (b != cur_b) {
+            if (cur_b >= 0) {
+              const double t = warp_sum(obj);
+              if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
+            }
+            obj = 0.0;
+            cur_b = b;
+          }
+          if (lane_has_vec) {
+            const char* row = static_cast<const char*>(p.oa.chat) +
+                              ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.D) * elem_bytes_;
+            Vec<DT>::widen(ldg_nc_v4(row + (int64_t)sub * 16), chat);
           }
         }
       }
+      if (g == gg && lane_has_vec) {
+        float f[E];
+        Vec<DT>::widen(ring[s % SEG_STAGES][lane], f);
+        float d2 = 0.0f;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-#pragma unroll
-        for (int gg = 0; gg < RPS; ++gg) {
-          const int kg = __shfl_sync(0xffffffffu, key[u], gg * LPR);
-          if (kg < 0) continue;
-          if (kg != cur) {
-            if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc);
-            cur = kg;
-            if (want_obj) {
-              const int b = kg / p.oa.K, k = kg % p.oa.K;
-              if (b != cur_b) {
-                if (cur_b >= 0) {
-                  const double t = warp_sum(obj);
-                  if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
-                }
-                obj = 0.0;
-                cur_b = b;
-              }
-              if (lane_has_vec) {
-                const char* row = static_cast<const char*>(p.oa.chat) +
-                                  ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.D) * elem_bytes_;
-                Vec<DT>::widen(ldg_nc_v4(row + (int64_t)sub * 16), chat);
-              }
-            }
-          }
-          if (g == gg && lane_has_vec) {
-            float f[E];
-            Vec<DT>::widen(v[u], f);
-            float d2 = 0.0f;
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-              acc[e] += (double)f[e];
-              const float df = f[e] - chat[e];
-              d2 = fmaf(df, df, d2);
-            }
-            if (want_obj) obj += (double)d2;
-          }
+        for (int e = 0; e < E; ++e) {
+          acc32[e] += f[e];
+          const float df = f[e] - chat[e];
+          d2 = fmaf(df, df, d2);
         }
+        obj32 += d2;
       }
     }
-    if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc);
-    if (want_obj && cur_b >= 0) {
-      const double t = warp_sum(obj);
-      if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
+    if ((s & 15) == 15) {   // bound the fp32 partials to 16 rows per lane
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        acc[e] += (double)acc32[e];
+        acc32[e] = 0.0f;
+      }
+      obj += (double)obj32;
+      obj32 = 0.0f;
     }
+    __syncwarp();   // every lane is done with slot s before it is refilled
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc, acc32);
+  if (want_obj && cur_b >= 0) {
+    const double t = warp_sum(obj + (double)obj32);
+    if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
   }
 }
 
@@ -376,10 +432,8 @@ __global__ void __launch_bounds__(256) batch_reduce_kernel(int K, const double* 
 template <int DT, int RPS>
 fkm_status run_segsum(const SegParams& sp, cudaStream_t st) {
   const int64_t nranges = ceil_div(sp.n, SEG_RANGE);
-  const int wpb = 8;
-  int64_t blocks = ceil_div(nranges, wpb);
-  if (blocks < 1) blocks = 1;
-  segsum_kernel<DT, RPS><<<(unsigned)blocks, wpb * 32, 0, st>>>(sp);
+  const int64_t blocks = ceil_div(nranges, SEG_WARPS);
+  segsum_kernel<DT, RPS><<<(unsigned)blocks, SEG_WARPS * 32, 0, st>>>(sp);
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;

@@ -215,7 +215,7 @@ def test_lloyd_steps_match_single_calls():
     assert torch.equal(ids2, ids)
     assert torch.equal(counts2, n)
     assert torch.allclose(centers2, c, rtol=1e-6, atol=1e-6)
-    assert torch.allclose(inertia2, inertia, rtol=1e-9)
+    assert torch.allclose(inertia2, inertia, rtol=1e-6)
     # and the update's own objective equals the assign's for the same ids
     obj = torch.empty(w.B, dtype=torch.float64, device="cuda")
     c_prev = torch.from_numpy(c0).cuda()
@@ -223,7 +223,7 @@ def test_lloyd_steps_match_single_calls():
     inertia_a = torch.empty_like(obj)
     fkm.fkm_assign(xt, c_prev, ids_a, inertia_a)
     fkm.fkm_update(xt, ids_a, c_prev, torch.empty_like(c_prev), torch.empty_like(n), None, obj)
-    assert torch.allclose(obj, inertia_a, rtol=1e-9)
+    assert torch.allclose(obj, inertia_a, rtol=1e-6)
 
 
 def test_lloyd_tol_stops_and_repeats():
