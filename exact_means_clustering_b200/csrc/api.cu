@@ -143,6 +143,7 @@ fkm_status make_layout(int B, int N, int K, int D, int dtype, Layout* L) {
   };
   const size_t BN_ = (size_t)B * N, BK = (size_t)B * K;
   l.status = take(256);
+  l.mvec = take((size_t)B * D * 4);
   l.cq = take((size_t)B * l.Kp * l.Dq * 2);
   l.cn = take((size_t)B * l.Kp * 4);
   l.xs = take(l.split ? BN_ * l.Dq * 2 : 0);
@@ -228,6 +229,7 @@ static ObjArgs obj_args(const Ws& w, const float* prev, double* obj) {
   } else {
     o.chat = w.at<void>(L.cq);
     o.chat_bstride = (int64_t)L.Kp * L.D;
+    o.m = w.at<float>(L.mvec);
   }
   return o;
 }
@@ -261,10 +263,12 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK, segstart, segend,
                         w.at<double>(L.sums64), next, false, obj_args(w, prev, obj), st));
   if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[3], st, cudaEventRecordExternal));
-  FKM_TRY(launch_finalize(L.B, L.K, L.D, L.Kp, L.dtype, segstart, segend, nullptr,
-                          w.at<double>(L.sums64), prev, next, counts, w.at<double>(L.shiftk),
-                          requant ? w.at<void>(L.cq) : nullptr,
-                          requant ? w.at<float>(L.cn) : nullptr, st));
+  FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64), prev,
+                          next, counts, w.at<double>(L.shiftk), st));
+  // the next assign's operands: offsets of the new centroids from their mean
+  if (requant)
+    FKM_TRY(launch_prep_centroids(next, L.B, L.K, L.Kp, L.D, L.dtype, w.at<float>(L.mvec),
+                                  w.at<void>(L.cq), w.at<float>(L.cn), st));
   return FKM_OK;
 }
 
@@ -378,8 +382,8 @@ fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, cons
   if (inertia) FKM_TRY(check_ptr(inertia, "inertia"));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Ws w{ws, &L};
-  FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<void>(L.cq), w.at<float>(L.cn),
-                                st));
+  FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
+                                w.at<void>(L.cq), w.at<float>(L.cn), st));
   if (L.split)
     FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, w.at<void>(L.xs), nullptr, st));
   FKM_TRY(step_assign(w, x, ids, st));
@@ -411,8 +415,8 @@ fkm_status fkm_update(int B, int N, int K, int D, int dtype, const void* x, cons
   Ws w{ws, &L};
   FKM_CUDA_TRY(cudaMemsetAsync(w.at<double>(L.sums64), 0, (size_t)B * K * D * 8, st));
   if (inertia && !L.split)  // the objective measures against q(prev), the assign operand
-    FKM_TRY(launch_prep_centroids(prev_centers, B, K, L.Kp, D, dtype, w.at<void>(L.cq),
-                                  w.at<float>(L.cn), st));
+    FKM_TRY(launch_prep_centroids(prev_centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
+                                  w.at<void>(L.cq), w.at<float>(L.cn), st));
   FKM_TRY(step_update(w, x, ids, prev_centers, centers, counts, false, inertia, st));
   if (shift) FKM_TRY(launch_batch_reduce(B, K, w.at<double>(L.shiftk), shift, nullptr, st));
   return FKM_OK;
@@ -448,7 +452,8 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
   FKM_CUDA_TRY(cudaMemsetAsync(w.at<double>(L.sums64), 0, (size_t)B * K * D * 8, st));
   FKM_CUDA_TRY(cudaMemcpyAsync(cA, init_centers, cbytes, cudaMemcpyDeviceToDevice, st));
   if (L.split) FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, w.at<void>(L.xs), nullptr, st));
-  FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, w.at<void>(L.cq), w.at<float>(L.cn), st));
+  FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, w.at<float>(L.mvec), w.at<void>(L.cq),
+                                w.at<float>(L.cn), st));
 
   FKM_TRY(assign_prepare());
   const bool prof = g_prof.on.load();
@@ -608,10 +613,10 @@ fkm_status fkm_baseline_assign(int B, int N, int K, int D, int dtype, const void
   FKM_TRY(check_ptr(ids, "ids"));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Ws w{ws, &L};
-  FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<void>(L.cq), w.at<float>(L.cn),
-                                st));
+  FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
+                                w.at<void>(L.cq), w.at<float>(L.cn), st));
   FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, L.split ? w.at<void>(L.xs) : nullptr,
-                             w.at<float>(L.xn), st));
+                             w.at<float>(L.xn), st, w.at<float>(L.mvec), N));
   AssignArgs a;
   a.B = B;
   a.N = N;

@@ -154,8 +154,9 @@ __device__ __forceinline__ int find_first(const float4* save, int rot, float bes
 }
 
 // kDist = true is the comparison ("standard") mode: the same tensor-core tiles,
-// but the epilogue writes every distance ||x||^2 + ||c||^2 - 2 x.c to HBM
-// instead of reducing it, as the pages' baseline assignment does.
+// but the epilogue writes every distance ||x - c_hat||^2 = ||x - m||^2 +
+// norm_k - 2 x.q(c_k - m) to HBM instead of reducing it, as the pages'
+// baseline assignment does.
 template <bool kSplit, bool kDist>
 __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tm_x,   // points (hi part when split)
@@ -402,22 +403,21 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
           ++acc_uses;
           continue;
         }
+        // all 128 of this warp's columns in flight at once, one wait, then the
+        // accumulator goes straight back to the MMA warp
+        uint32_t r2[32], r3[32];
         ptx::tmem_ld32(taddr, r0);
-        ptx::tmem_wait_ld32(r0);
         ptx::tmem_ld32(taddr + 32, r1);
-        fold_chunk(r0, cn_s, colb, best, bcol, save, rot);
-        ptx::tmem_wait_ld32(r1);
-        ptx::tmem_ld32(taddr + 64, r0);
-        fold_chunk(r1, cn_s + 32, colb + 32, best, bcol, save, rot);
-        ptx::tmem_wait_ld32(r0);
-        ptx::tmem_ld32(taddr + 96, r1);
-        fold_chunk(r0, cn_s + 64, colb + 64, best, bcol, save, rot);
-        ptx::tmem_wait_ld32(r1);
-        // every column this warp reads from the accumulator is in registers
+        ptx::tmem_ld32(taddr + 64, r2);
+        ptx::tmem_ld32(taddr + 96, r3);
+        ptx::tmem_wait_ld128(r0, r1, r2, r3);
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
-        fold_chunk(r1, cn_s + 96, colb + 96, best, bcol, save, rot);
+        fold_chunk(r0, cn_s, colb, best, bcol, save, rot);
+        fold_chunk(r1, cn_s + 32, colb + 32, best, bcol, save, rot);
+        fold_chunk(r2, cn_s + 64, colb + 64, best, bcol, save, rot);
+        fold_chunk(r3, cn_s + 96, colb + 96, best, bcol, save, rot);
         ++acc_uses;
       }
       if (!ok) break;

@@ -71,7 +71,7 @@ struct Layout {
   int64_t n_sort;  // B * N keys
   int n_sort_tiles;
   int key_bits;
-  size_t status, cq, cn, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
+  size_t status, mvec, cq, cn, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
       segstart, segend, sums64, shiftk, cbuf, scal, total;
 };
 
@@ -90,7 +90,7 @@ struct AssignArgs {
   int x_row_elems;     // elements per row of xq (D, or 2D when split)
   const void* cq;      // quantised centroids [B, Kp, Dq]
   const float* cn;     // ||q(c)||^2 [B, Kp], +inf on padding rows
-  const float* xn;     // ||x||^2 [B, N] (comparison mode only)
+  const float* xn;     // ||x - m||^2 [B, N] (comparison mode only)
   int32_t* ids;        // [B, N]
   int* status;
   float* dist = nullptr;  // comparison mode: write the [B, N, K] distances here
@@ -99,12 +99,15 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st);
 bool assign_smem_plan(int D, bool split, int* nA, int* nS, size_t* smem);
 fkm_status assign_prepare();
 
-// q(c) rows [B][Kp][Dq] and ||q(c)||^2; split rows (fp32) are [hi | lo]
-// halves of round_up(D, 8) elements each.
+// Per batch mean centroid m [B][D]; q(c - m) rows [B][Kp][Dq] and the norm
+// term ||q(c-m)||^2 + 2 m.q(c-m); split rows (fp32) are [hi | lo] halves of
+// round_up(D, 8) elements each.
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
-                                 void* cq, float* cn, cudaStream_t st);
+                                 float* m, void* cq, float* cn, cudaStream_t st);
+// fp32 points: split rows into xs; xn (optional) = ||x - m[row / N]||^2
+// (||x||^2 when m is null).
 fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,
-                              cudaStream_t st);
+                              cudaStream_t st, const float* m = nullptr, int N = 1);
 
 struct SortArgs {
   const int32_t* ids;  // first-pass keys come from ids: key = (row / N) * K + id
@@ -123,13 +126,16 @@ size_t argsort_scratch_words(int64_t n);
 
 fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
                              int32_t* segend, cudaStream_t st);
-// Objective of the assignment being summed: chat is the centroid the assign
-// step measured against (q(c) in the points' 16-bit type [B][Kp][D], or the
-// fp32 centroids [B][K][D] for fp32 points), chat_bstride its batch stride
-// in elements; obj[b] (zeroed by the caller) receives sum ||x - chat||^2.
+// Objective of the assignment being summed against c_hat, the centroid the
+// assign step measured against: m + q(c - m) for 16-bit points (chat = the
+// q(c - m) rows [B][Kp][D], m = the per-batch mean centroid), the fp32
+// centroids themselves for fp32 points (chat = [B][K][D], m = nullptr);
+// chat_bstride is the batch stride of chat in elements; obj[b] (zeroed by the
+// caller) receives sum ||x - c_hat||^2.
 struct ObjArgs {
   const void* chat = nullptr;
   int64_t chat_bstride = 0;
+  const float* m = nullptr;   // 16-bit chat: c_hat = m[b] + chat (per batch [B][D])
   int K = 1;
   double* obj = nullptr;
 };
@@ -140,10 +146,9 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
 // Direct objective of a given assignment: obj[b] += sum_i ||x_i - chat_{ids_i}||^2.
 fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const int32_t* ids,
                             const ObjArgs& oa, cudaStream_t st);
-fkm_status launch_finalize(int B, int K, int D, int Kp, int dtype, const int32_t* segstart,
-                           const int32_t* segend, const int32_t* counts_in, double* sums64,
-                           const float* prev, float* centers, int32_t* counts, double* shiftk,
-                           void* cq, float* cn, cudaStream_t st);
+fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
+                           const int32_t* counts_in, double* sums64, const float* prev,
+                           float* centers, int32_t* counts, double* shiftk, cudaStream_t st);
 fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
                                double* max_shift, cudaStream_t st);
 

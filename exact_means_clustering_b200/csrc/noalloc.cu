@@ -7,8 +7,9 @@
 // only their inputs and outputs by a host application.  They cannot call
 // cudaMalloc for the workspace that fkm_assign expects.
 //
-// This entry point keeps its scratch (the centroids rounded to the points'
-// 16-bit type, their squared norms, and a status word) in one file-scope
+// This entry point keeps its scratch (the per-batch mean centroid, the
+// centroid offsets rounded to the points' 16-bit type, their norm terms, and
+// a status word) in one file-scope
 // device array of FKM_NOALLOC_SCRATCH_BYTES.  Every GPU that loads the library
 // holds that array until the process exits.  The host-side name of the array
 // is only a stand-in: its device address is fetched with cudaGetSymbolAddress,
@@ -73,25 +74,27 @@ extern "C" fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, 
   }
   const int Kp = (int)round_up(K, BN);
   const size_t status_bytes = 256;
+  const size_t m_bytes = (size_t)round_up((int64_t)B * D * 4, 256);
   const size_t cq_bytes = (size_t)round_up((int64_t)B * Kp * D * 2, 256);
   const size_t cn_bytes = (size_t)round_up((int64_t)B * Kp * 4, 256);
-  if (status_bytes + cq_bytes + cn_bytes > kScratchBytes) {
-    set_error("B*Kp*(2*D + 4) = %zu bytes exceeds the %zu-byte static scratch of "
+  if (status_bytes + m_bytes + cq_bytes + cn_bytes > kScratchBytes) {
+    set_error("B*(4*D + Kp*(2*D + 4)) = %zu bytes exceeds the %zu-byte static scratch of "
               "fkm_assign_noalloc (Kp = K rounded up to 256)",
-              cq_bytes + cn_bytes, kScratchBytes - status_bytes);
+              m_bytes + cq_bytes + cn_bytes, kScratchBytes - status_bytes);
     return FKM_ERR_UNSUPPORTED;
   }
   void* base = nullptr;
   FKM_TRY(scratch_for_current_device(&base));
   char* p = static_cast<char*>(base);
   int* status = reinterpret_cast<int*>(p);
-  void* cq = p + status_bytes;
-  float* cn = reinterpret_cast<float*>(p + status_bytes + cq_bytes);
+  float* m = reinterpret_cast<float*>(p + status_bytes);
+  void* cq = p + status_bytes + m_bytes;
+  float* cn = reinterpret_cast<float*>(p + status_bytes + m_bytes + cq_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the status word is the only scratch that must start at zero; the rest is
   // fully rewritten by the centroid preparation below
   FKM_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
-  FKM_TRY(launch_prep_centroids(centers, B, K, Kp, D, dtype, cq, cn, st));
+  FKM_TRY(launch_prep_centroids(centers, B, K, Kp, D, dtype, m, cq, cn, st));
   AssignArgs a;
   a.B = B;
   a.N = N;

@@ -37,7 +37,7 @@ struct HostLayout {
   int chunks_per_batch;
   int tiles_per_chunk;
   int key_bits;
-  size_t status, xbuf[2], cq, cn, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
+  size_t status, xbuf[2], mvec, cq, cn, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
       segstart, segend, sums64, counts_acc, shiftk, cbuf, total;
 };
 
@@ -86,6 +86,7 @@ fkm_status make_host_layout(int B, int N, int K, int D, int dtype, int64_t chunk
   l.status = take(256);
   l.xbuf[0] = take((size_t)R * D * s);
   l.xbuf[1] = take((size_t)R * D * s);
+  l.mvec = take((size_t)B * D * 4);
   l.cq = take((size_t)B * l.Kp * l.Dq * 2);
   l.cn = take((size_t)B * l.Kp * 4);
   l.xs = take(l.split ? (size_t)R * l.Dq * 2 : 0);
@@ -193,8 +194,9 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
   FKM_CUDA_TRY(cudaMemsetAsync(status, 0, 256, st));
   FKM_CUDA_TRY(cudaMemsetAsync(sums64, 0, (size_t)B * K * D * 8, st));
   FKM_CUDA_TRY(cudaMemcpyAsync(cA, init_centers, cbytes, cudaMemcpyDeviceToDevice, st));
-  FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, at(L.cq), static_cast<float*>(at(L.cn)),
-                                st));
+  float* mvec = static_cast<float*>(at(L.mvec));
+  FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, mvec, at(L.cq),
+                                static_cast<float*>(at(L.cn)), st));
   // the copy stream may only touch the workspace after the caller's earlier work
   FKM_CUDA_TRY(cudaEventRecord(ss.start, st));
   FKM_CUDA_TRY(cudaStreamWaitEvent(ss.copy, ss.start, 0));
@@ -265,6 +267,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
         } else {
           oa.chat = static_cast<const char*>(at(L.cq)) + (size_t)b * L.Kp * D * 2;
           oa.chat_bstride = 0;
+          oa.m = mvec + (size_t)b * D;
         }
         FKM_TRY(launch_segsum(xb, dtype, D, so.keys_out, so.vals_out, rows, K, segstart, segend,
                               sums64 + (size_t)b * K * D, nullptr, true, oa, st));
@@ -275,9 +278,10 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
         FKM_CUDA_TRY(cudaEventRecord(ss.freed[buf], st));
       }
     }
-    FKM_TRY(launch_finalize(B, K, D, L.Kp, dtype, nullptr, nullptr, counts_acc, sums64, cur, nxt,
-                            counts, static_cast<double*>(at(L.shiftk)), at(L.cq),
-                            static_cast<float*>(at(L.cn)), st));
+    FKM_TRY(launch_finalize(B, K, D, nullptr, nullptr, counts_acc, sums64, cur, nxt, counts,
+                            static_cast<double*>(at(L.shiftk)), st));
+    FKM_TRY(launch_prep_centroids(nxt, B, K, L.Kp, D, dtype, mvec, at(L.cq),
+                                  static_cast<float*>(at(L.cn)), st));
     if (tol > 0.0f) FKM_CUDA_TRY(cudaMemsetAsync(max_shift, 0, sizeof(double), st));
     FKM_TRY(launch_batch_reduce(B, K, static_cast<double*>(at(L.shiftk)), nullptr,
                                 tol > 0.0f ? max_shift : nullptr, st));

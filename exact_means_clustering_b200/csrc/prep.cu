@@ -1,16 +1,24 @@
 // Operand preparation for the assign kernel.
 //
-//  prep_centroids: q(c) = the fp32 centroid rounded (RNE) to the points'
-//    16-bit type, laid out [B, Kp, D] for TMA, and ||q(c)||^2 (summed in fp64,
-//    rounded once) -- the precomputed norm of the score ||c||^2 - 2 x.c
-//    ("Flash-KMeans：快速且内存高效精确K-Means聚类" summary, section 方法步骤详情
-//    step (1), which precomputes the norms).  Padding rows k >= K get q = 0
-//    and norm +inf so they never win the argmin.  For fp32 points each
-//    centroid is split into bf16 hi and lo = bf16(c - hi), rows [hi | lo], and
-//    the norm is that of the fp32 centroid.
+//  center: per batch the mean centroid m (fp64 sum over k in a fixed order --
+//    32 strided partial sums, then their sum -- divided by K, rounded to fp32).  The assignment works on offsets from m:
+//    k-means is translation invariant ("Flash-KMeans" README, section "Centre
+//    your data"), and with the offsets small the tensor-core products and
+//    their fp32 accumulation keep their precision even for data far from the
+//    origin.
+//  prep_centroids: delta = fp32(c - m); q(delta) = delta rounded (RNE) to the
+//    points' 16-bit type, laid out [B, Kp, D] for TMA; and the norm term
+//    ||q(delta)||^2 + 2 m.q(delta) (fp64, rounded once).  The score
+//    norm - 2 x.q(delta) equals ||x - c_hat||^2 - ||x - m||^2 + ||m||^2... up
+//    to terms constant per point, with c_hat = m + q(delta): the argmin of
+//    ||x - c_hat||^2 ("Flash-KMeans：快速且内存高效精确K-Means聚类" summary,
+//    section 方法步骤详情 step (1), which precomputes the norms).  Padding rows
+//    k >= K get q = 0 and norm +inf so they never win the argmin.  For fp32
+//    points delta is split into bf16 hi and lo = bf16(delta - hi), rows
+//    [hi | lo], and the norm term uses the fp32 delta.
 //  points_prep: for fp32 points, the bf16 [hi | lo] split rows the tensor
 //    cores consume (each half padded to a multiple of 8 elements); optionally
-//    ||x||^2 per point (fp64 sum rounded to fp32), which only the
+//    ||x - m||^2 per point (fp64 sum rounded to fp32), which only the
 //    distance-materialising comparison path needs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -26,55 +34,84 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
+// m[b][d] = fp32(S / K) with S summed in fp64 in a fixed order that does not
+// depend on the launch: 32 partial sums P_w = sum over k = w, w+32, w+64, ...
+// (each in ascending k), then S = P_0 + P_1 + ... + P_31 in that order.
+// Block (b, 32-dimension group) of 32 warps: warp w forms P_w for the 32
+// dimensions of its lanes (coalesced rows), warp 0 adds the partials.
+__global__ void __launch_bounds__(1024) center_kernel(const float* __restrict__ c, int B, int K,
+                                                      int D, float* __restrict__ m) {
+  __shared__ double part[32][33];
+  const int b = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int d = blockIdx.y * 32 + lane;
+  double s = 0.0;
+  if (d < D) {
+    const float* p = c + (int64_t)b * K * D + d;
+    for (int k = w; k < K; k += 32) s += (double)p[(int64_t)k * D];
+  }
+  part[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && d < D) {
+    double t = 0.0;
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) t += part[j][lane];
+    m[(int64_t)b * D + d] = (float)(t / (double)K);
+  }
+}
+
 // one warp per padded centroid row
-__global__ void prep_centroids_kernel(const float* __restrict__ c, int B, int K, int Kp, int D,
-                                      int dtype, void* __restrict__ cq, float* __restrict__ cn) {
+__global__ void prep_centroids_kernel(const float* __restrict__ c, const float* __restrict__ m,
+                                      int B, int K, int Kp, int D, int dtype,
+                                      void* __restrict__ cq, float* __restrict__ cn) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= (int64_t)B * Kp) return;
   const int b = (int)(row / Kp), k = (int)(row % Kp);
   const bool real = k < K;
   const float* src = c + ((int64_t)b * K + k) * D;
+  const float* mb = m + (int64_t)b * D;
   double acc = 0.0;
   if (dtype == FKM_F32) {
     const int Dp = (D + 7) & ~7;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(cq) + row * (int64_t)(2 * Dp);
     for (int d = lane; d < D; d += 32) {
-      float v = real ? src[d] : 0.0f;
+      const float v = real ? src[d] - mb[d] : 0.0f;
       __nv_bfloat16 h = __float2bfloat16_rn(v);
       __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
       out[d] = h;
       out[Dp + d] = l;
-      acc += (double)v * (double)v;
+      acc += (double)v * ((double)v + 2.0 * (double)mb[d]);
     }
   } else if (dtype == FKM_BF16) {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(cq) + row * (int64_t)D;
     for (int d = lane; d < D; d += 32) {
-      __nv_bfloat16 q = __float2bfloat16_rn(real ? src[d] : 0.0f);
+      __nv_bfloat16 q = __float2bfloat16_rn(real ? src[d] - mb[d] : 0.0f);
       out[d] = q;
-      double f = (double)__bfloat162float(q);
-      acc += f * f;
+      const double f = (double)__bfloat162float(q);
+      acc += f * (f + 2.0 * (double)mb[d]);
     }
   } else {
     __half* out = static_cast<__half*>(cq) + row * (int64_t)D;
     for (int d = lane; d < D; d += 32) {
-      __half q = __float2half_rn(real ? src[d] : 0.0f);
+      __half q = __float2half_rn(real ? src[d] - mb[d] : 0.0f);
       out[d] = q;
-      double f = (double)__half2float(q);
-      acc += f * f;
+      const double f = (double)__half2float(q);
+      acc += f * (f + 2.0 * (double)mb[d]);
     }
   }
   acc = warp_sum(acc);
   if (lane == 0) cn[row] = real ? (float)acc : INFINITY;
 }
 
-// one warp per point row
+// one warp per point row; xn[row] = ||x - m[batch]||^2 when m is given
 __global__ void points_prep_kernel(const void* __restrict__ x, int64_t rows, int D, int dtype,
-                                   __nv_bfloat16* __restrict__ xs, float* __restrict__ xn) {
+                                   __nv_bfloat16* __restrict__ xs, float* __restrict__ xn,
+                                   const float* __restrict__ m, int N) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   double acc = 0.0;
+  const float* mb = m ? m + (row / N) * D : nullptr;
   if (dtype == FKM_F32) {
     const int Dp = (D + 7) & ~7;
     const float* src = static_cast<const float*>(x) + row * D;
@@ -87,7 +124,8 @@ __global__ void points_prep_kernel(const void* __restrict__ x, int64_t rows, int
         out[d] = h;
         out[Dp + d] = l;
       }
-      acc += (double)v * (double)v;
+      const double dv = (double)v - (mb ? (double)mb[d] : 0.0);
+      acc += dv * dv;
     }
   } else {
     // 16-bit points: 8-byte loads, four values per lane per step
@@ -108,7 +146,9 @@ __global__ void points_prep_kernel(const void* __restrict__ x, int64_t rows, int
           a = f.x;
           bb = f.y;
         }
-        acc += (double)a * a + (double)bb * bb;
+        const double da = (double)a - (mb ? (double)mb[4 * v + 2 * h] : 0.0);
+        const double db = (double)bb - (mb ? (double)mb[4 * v + 2 * h + 1] : 0.0);
+        acc += da * da + db * db;
       }
     }
   }
@@ -119,22 +159,24 @@ __global__ void points_prep_kernel(const void* __restrict__ x, int64_t rows, int
 }  // namespace
 
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
-                                 void* cq, float* cn, cudaStream_t st) {
+                                 float* m, void* cq, float* cn, cudaStream_t st) {
+  center_kernel<<<dim3((unsigned)B, (unsigned)ceil_div(D, 32)), 1024, 0, st>>>(centers, B, K, D,
+                                                                              m);
   const int64_t rows = (int64_t)B * Kp;
   const int wpb = 8;
-  prep_centroids_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(centers, B, K, Kp, D,
-                                                                           dtype, cq, cn);
-  note_launch();
+  prep_centroids_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(centers, m, B, K, Kp,
+                                                                           D, dtype, cq, cn);
+  note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
 }
 
 fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,
-                              cudaStream_t st) {
+                              cudaStream_t st, const float* m, int N) {
   if (rows == 0) return FKM_OK;
   const int wpb = 8;
   points_prep_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(
-      x, rows, D, dtype, static_cast<__nv_bfloat16*>(xs), xn);
+      x, rows, D, dtype, static_cast<__nv_bfloat16*>(xs), xn, m, N > 0 ? N : 1);
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;

@@ -21,8 +21,7 @@
 //               inertia does not suffer the cancellation of the expanded form.
 //   finalize    per cluster: counts, c = s/n for crossing runs, the previous
 //               centroid for empty clusters (a reading: the pages give only
-//               c = s/n), the shift ||c_new - c_old||^2, and the next
-//               iteration's tensor-core operands q(c), ||q(c)||^2.
+//               c = s/n), and the shift ||c_new - c_old||^2.
 //   batch_reduce  per batch, in fixed order: shift = sum_k shift_k.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -254,6 +253,11 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
             const char* row = static_cast<const char*>(p.oa.chat) +
                               ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.D) * elem_bytes_;
             Vec<DT>::widen(ldg_nc_v4(row + (int64_t)sub * 16), chat);
+            if (p.oa.m) {
+              const float* mb = p.oa.m + (int64_t)b * p.D + (int64_t)sub * E;
+#pragma unroll
+              for (int e = 0; e < E; ++e) chat[e] += mb[e];
+            }
           }
         }
       }
@@ -311,6 +315,11 @@ __global__ void __launch_bounds__(256) objective_kernel(const void* __restrict__
     const char* crow = static_cast<const char*>(oa.chat) +
                        ((int64_t)b * oa.chat_bstride + (int64_t)id * D) * (row_bytes / D);
     Vec<DT>::widen(ldg_nc_v4(crow + lane * 16), c);
+    if (oa.m) {
+      const float* mb = oa.m + (int64_t)b * D + (int64_t)lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) c[e] += mb[e];
+    }
     float d2 = 0.0f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -330,7 +339,7 @@ __global__ void __launch_bounds__(256) objective_kernel(const void* __restrict__
 }
 
 struct FinParams {
-  int B, K, D, Kp, dtype;
+  int B, K, D;
   const int32_t* segstart;
   const int32_t* segend;
   double* sums64;
@@ -338,8 +347,6 @@ struct FinParams {
   float* centers;
   int32_t* counts;
   double* shiftk;
-  void* cq;
-  float* cn;
   const int32_t* counts_in;  // out-of-core: accumulated counts (segstart/end unused)
 };
 
@@ -358,9 +365,7 @@ __global__ void finalize_kernel(FinParams p) {
     interior = nk > 0 && (s / SEG_RANGE) == ((t - 1) / SEG_RANGE);
   }
   if (lane == 0 && p.counts) p.counts[key] = nk;
-  const int b = (int)(key / p.K), k = (int)(key % p.K);
-  const int64_t qrow = (int64_t)b * p.Kp + k;
-  double sh = 0.0, nrm = 0.0;
+  double sh = 0.0;
   for (int d = lane; d < p.D; d += 32) {
     const int64_t e = key * p.D + d;
     const float prev = p.prev[e];
@@ -376,36 +381,10 @@ __global__ void finalize_kernel(FinParams p) {
     p.centers[e] = v;
     const double df = (double)v - (double)prev;
     sh += df * df;
-    if (p.cq) {
-      if (p.dtype == FKM_F32) {
-        const int Dp = (p.D + 7) & ~7;
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.cq) + qrow * (2 * Dp);
-        __nv_bfloat16 h = __float2bfloat16_rn(v);
-        o[d] = h;
-        o[Dp + d] = __float2bfloat16_rn(v - __bfloat162float(h));
-        nrm += (double)v * v;
-      } else if (p.dtype == FKM_BF16) {
-        __nv_bfloat16 q = __float2bfloat16_rn(v);
-        static_cast<__nv_bfloat16*>(p.cq)[qrow * p.D + d] = q;
-        const double f = __bfloat162float(q);
-        nrm += f * f;
-      } else {
-        __half q = __float2half_rn(v);
-        static_cast<__half*>(p.cq)[qrow * p.D + d] = q;
-        const double f = __half2float(q);
-        nrm += f * f;
-      }
-    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    sh += __shfl_xor_sync(0xffffffffu, sh, o);
-    nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
-  }
-  if (lane == 0) {
-    p.shiftk[key] = sh;
-    if (p.cq) p.cn[qrow] = (float)nrm;
-  }
+  for (int o = 16; o > 0; o >>= 1) sh += __shfl_xor_sync(0xffffffffu, sh, o);
+  if (lane == 0) p.shiftk[key] = sh;
 }
 
 // one block per batch; fixed-order tree sum
@@ -514,16 +493,13 @@ fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const
   return FKM_OK;
 }
 
-fkm_status launch_finalize(int B, int K, int D, int Kp, int dtype, const int32_t* segstart,
-                           const int32_t* segend, const int32_t* counts_in, double* sums64,
-                           const float* prev, float* centers, int32_t* counts, double* shiftk,
-                           void* cq, float* cn, cudaStream_t st) {
+fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
+                           const int32_t* counts_in, double* sums64, const float* prev,
+                           float* centers, int32_t* counts, double* shiftk, cudaStream_t st) {
   FinParams fp;
   fp.B = B;
   fp.K = K;
   fp.D = D;
-  fp.Kp = Kp;
-  fp.dtype = dtype;
   fp.segstart = segstart;
   fp.segend = segend;
   fp.sums64 = sums64;
@@ -531,8 +507,6 @@ fkm_status launch_finalize(int B, int K, int D, int Kp, int dtype, const int32_t
   fp.centers = centers;
   fp.counts = counts;
   fp.shiftk = shiftk;
-  fp.cq = cq;
-  fp.cn = cn;
   fp.counts_in = counts_in;
   const int64_t keys = (int64_t)B * K;
   const int wpb = 8;

@@ -70,17 +70,22 @@ typedef enum { FKM_F32 = 0, FKM_F16 = 1, FKM_BF16 = 2 } fkm_dtype;
  * rejects.  `bytes` (host) receives the size. */
 FKM_API fkm_status fkm_workspace_size(int B, int N, int K, int D, int dtype, size_t* bytes);
 
-/* Assign step (predict): ids[b,i] = argmin_k ||x[b,i] - q(c[b,k])||^2, ties to
- * the lowest k, with q() the rounding of the fp32 centroid to `dtype` (the
- * tensor-core operand type; for fp32 points the product is carried in split
- * bf16 hi+lo form, relative error about 2^-17).  Computed as the online argmin
- * of ||q(c)||^2 - 2 x.q(c) over centroid tiles on tcgen05 tensor cores, without
- * ever writing a distance matrix ("Flash-KMeans: Fast and Memory-Efficient
- * Exact K-Means" summary, section "Method", FlashAssign; "Flash-KMeans：快速且内存
- * 高效精确K-Means聚类" summary, section 方法步骤详情 step (1)).
+/* Assign step (predict): ids[b,i] = argmin_k ||x[b,i] - c_hat[b,k]||^2, ties to
+ * the lowest k, where c_hat = m_b + q(c - m_b): m_b is the batch's mean
+ * centroid (fp64 sum over k in index order / K, rounded to fp32) and q() the
+ * RNE rounding of the fp32 offset c - m_b to `dtype` -- the tensor-core
+ * operand.  Centring keeps the products small, so data far from the origin
+ * keeps its precision; k-means is translation invariant ("Flash-KMeans"
+ * README, section "Centre your data").  For fp32 points the offset is carried
+ * in split bf16 hi+lo form (relative error about 2^-17) and c_hat ~= c.
+ * Computed as the online argmin of the score over centroid tiles on tcgen05
+ * tensor cores, without ever writing a distance matrix ("Flash-KMeans: Fast
+ * and Memory-Efficient Exact K-Means" summary, section "Method", FlashAssign;
+ * "Flash-KMeans：快速且内存高效精确K-Means聚类" summary, section 方法步骤详情
+ * step (1)).
  *   x        device [B,N,D] dtype        centers  device [B,K,D] float32
  *   ids      device [B,N] int32 (out)
- *   inertia  device [B] float64 (out) = sum_i ||x_i - q(c[b, ids_i])||^2 (direct
+ *   inertia  device [B] float64 (out) = sum_i ||x_i - c_hat[b, ids_i]||^2 (direct
  *            difference, fp32 terms summed in fp64), or NULL
  *   ws       device workspace of ws_bytes >= fkm_workspace_size(...)
  * Async. */
@@ -97,9 +102,10 @@ FKM_API fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void*
  *   centers[b,k]  = mean of those x_i (fp64 sum, rounded to fp32), or
  *                   prev_centers[b,k] unchanged when counts[b,k] == 0
  *   shift[b]      = sum_k ||centers[b,k] - prev_centers[b,k]||^2 (float64), or NULL
- *   inertia[b]    = sum_i ||x_i - q(prev_centers[b, ids_i])||^2 (float64), the
- *                   objective of the given assignment against the centroids an
- *                   assign step would have used (q() as in fkm_assign), or NULL
+ *   inertia[b]    = sum_i ||x_i - c_hat[b, ids_i]||^2 (float64), the objective of
+ *                   the given assignment against the centroids an assign step
+ *                   would have used (c_hat of prev_centers, as in fkm_assign),
+ *                   or NULL
  *   x device [B,N,D] dtype; ids device [B,N] int32; prev_centers device [B,K,D];
  *   centers device [B,K,D] (out, must not alias prev_centers); counts device
  *   [B,K] int32 (out).  An id outside [0,K) sets FKM_ERR_BAD_ID in the status
@@ -192,16 +198,17 @@ FKM_API long long fkm_kernel_launches(void);
  * framework that forbids allocating while capturing, in services that reserve
  * all device memory up front, or in plugins that are handed only their inputs
  * and outputs.  Same result as fkm_assign with inertia = NULL, but the
- * scratch (the rounded centroids, their norms and a status word) lives in a
+ * scratch (the mean centroids, the rounded centroid offsets, their norm terms
+ * and a status word) lives in a
  * file-scope device array of FKM_NOALLOC_SCRATCH_BYTES that every GPU loading
  * the library keeps until the process exits; no workspace is passed and
  * nothing is allocated.
  *   x        device [B,N,D] bf16 or fp16 (fp32 points are rejected: their
  *            split operands need scratch proportional to N)
  *   centers  device [B,K,D] float32;  ids device [B,N] int32 (out)
- * Limit: 256 + B*Kp*(2*D + 4) bytes (rounded to 256-byte blocks) must fit in
- * FKM_NOALLOC_SCRATCH_BYTES, Kp = K rounded up to 256; larger shapes return
- * FKM_ERR_UNSUPPORTED.  The first call on a device looks up the array's
+ * Limit: 256 + B*(4*D + Kp*(2*D + 4)) bytes (each part rounded to 256-byte
+ * blocks) must fit in FKM_NOALLOC_SCRATCH_BYTES, Kp = K rounded up to 256;
+ * larger shapes return FKM_ERR_UNSUPPORTED.  The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) and raises the kernel's shared-memory
  * limit; make that first call before any stream capture.  All calls share
  * the one array, which keeps the last call's contents: calls that can overlap

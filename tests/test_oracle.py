@@ -55,13 +55,20 @@ def test_argsort_rejects_out_of_range():
 # ------------------------------------------------------------------ assign
 def _grid_problem(rng, B, N, K, D, spacing=16, jitter=3):
     """Centroids on a coarse integer lattice, points = centroid + small integer offset.
-    With spacing > 2*jitter*sqrt(D)... the owner is the strict nearest by construction."""
+    Neighbouring lattice centroids are `spacing` apart, so a point at most
+    `jitter` from its own centroid in every coordinate is strictly nearest to
+    it.  The centroid set is symmetric (v and -v), so its mean is exactly zero
+    and the centred operand of mirror mode equals the centroid itself."""
     c = np.zeros((B, K, D))
     for b in range(B):
         pts = set()
-        while len(pts) < K:
-            pts.add(tuple(rng.integers(-4, 5, size=D) * spacing))
-        c[b] = np.array(sorted(pts), dtype=np.float64)[rng.permutation(K)]
+        while len(pts) < K // 2:
+            v = tuple(rng.integers(-4, 5, size=D) * spacing)
+            if any(v) and tuple(-t for t in v) not in pts:
+                pts.add(v)
+        half = np.array(sorted(pts), dtype=np.float64)
+        full = np.concatenate([half, -half] + ([np.zeros((1, D))] if K % 2 else []))
+        c[b] = full[rng.permutation(K)]
     owner = rng.integers(0, K, size=(B, N))
     off = rng.integers(-jitter, jitter + 1, size=(B, N, D))
     x = np.take_along_axis(c, owner[..., None], axis=1) + off
@@ -129,18 +136,68 @@ def test_assign_matches_numpy_table_tiny():
         assert np.allclose(J, tab.min(-1).sum(-1), rtol=1e-12)
 
 
-def test_mirror_mode_is_assign_against_rounded_centroids():
+def _centred_operand(c, mirror):
+    """The mirror-mode centroid written out independently with numpy / torch:
+    m = fp32(S / K) per batch, S the fp64 sum of the fp32 centroids taken as
+    32 strided partials (k = w, w+32, ... ascending) added in order w = 0..31;
+    c_hat = m + q(fp32(c32 - m))."""
+    c32 = np.asarray(c, np.float32)
+    B, K, D = c32.shape
+    s = np.zeros((B, D))
+    for w in range(32):
+        part = np.zeros((B, D))
+        for k in range(w, K, 32):
+            part = part + c32[:, k].astype(np.float64)
+        s = s + part
+    m = (s / K).astype(np.float32)
+    delta = c32 - m[:, None, :]                      # float32 arithmetic, RNE
+    if mirror == "bf16":
+        q = _bf16_value(delta)
+    else:
+        q = delta.astype(np.float16).astype(np.float64)
+    return m.astype(np.float64)[:, None, :] + q
+
+
+def test_mirror_mode_is_assign_against_centred_rounded_centroids():
     rng = np.random.default_rng(5)
-    x = rng.standard_normal((1, 500, 16)).astype(np.float16)
-    c = rng.standard_normal((1, 40, 16))
+    x = (rng.standard_normal((2, 500, 16)) + 20).astype(np.float16)
+    c = rng.standard_normal((2, 40, 16)) + 20
+    ref = _centred_operand(c, "f16")
+    assert np.array_equal(oracle.chat(c, "f16"), ref)
     ids_m, d1_m, _, _ = oracle.assign(x, c, dtype="f16", mirror="f16")
-    cq = c.astype(np.float32).astype(np.float16).astype(np.float64)
-    ids_p, d1_p, _, _ = oracle.assign(x, cq, dtype="f16", mirror=None)
+    ids_p, d1_p, _, _ = oracle.assign(x, ref, dtype="f16", mirror=None)
     assert np.array_equal(ids_m, ids_p) and np.array_equal(d1_m, d1_p)
-    xb = _bf16_bits(rng.standard_normal((1, 500, 16)))
-    ids_m, _, _, _ = oracle.assign(xb, c, dtype="bf16", mirror="bf16")
-    ids_p, _, _, _ = oracle.assign(xb, _bf16_value(c), dtype="bf16", mirror=None)
+    xb = _bf16_bits(rng.standard_normal((1, 500, 16)) * 3 - 40)
+    cb = rng.standard_normal((1, 40, 16)) * 3 - 40
+    refb = _centred_operand(cb, "bf16")
+    assert np.array_equal(oracle.chat(cb, "bf16"), refb)
+    ids_m, _, _, _ = oracle.assign(xb, cb, dtype="bf16", mirror="bf16")
+    ids_p, _, _, _ = oracle.assign(xb, refb, dtype="bf16", mirror=None)
     assert np.array_equal(ids_m, ids_p)
+
+
+def test_centred_operand_error_scales_with_spread_not_offset():
+    """RNE to bf16 moves each offset by at most half an ulp: |c_hat - c| is
+    bounded by 2^-8 |c - m| (plus the fp32 rounding of c and of c - m),
+    however far the centroids sit from the origin."""
+    rng = np.random.default_rng(21)
+    for offset in (0.0, 64.0, -5000.0):
+        c = rng.standard_normal((3, 30, 8)) + offset
+        c32 = c.astype(np.float32).astype(np.float64)
+        ch = oracle.chat(c, "bf16")
+        assert np.array_equal(ch, _centred_operand(c, "bf16"))
+        spread = np.abs(c32 - c32.mean(axis=1, keepdims=True))
+        assert np.all(np.abs(ch - c32) <= 2.0 ** -8 * spread + 2.0 ** -22 * np.abs(c32))
+
+
+def test_centred_operand_is_translation_invariant():
+    """Shifting every centroid by a small integer vector shifts c_hat by the
+    same vector exactly (values on a 1/64 grid keep every step exact)."""
+    rng = np.random.default_rng(22)
+    c = np.round(rng.standard_normal((2, 16, 8)) * 64) / 64
+    mu = rng.integers(-20, 20, size=(2, 1, 8)).astype(np.float64)
+    for mir in ("bf16", "f16"):
+        assert np.array_equal(oracle.chat(c + mu, mir), oracle.chat(c, mir) + mu)
 
 
 # ---------------------------------------------------------- storage rounding
