@@ -145,7 +145,7 @@ fkm_status make_layout(int B, int N, int K, int D, int dtype, Layout* L) {
   l.status = take(256);
   l.mvec = take((size_t)B * D * 4);
   l.cq = take((size_t)B * l.Kp * l.Dq * 2);
-  l.cn = take((size_t)B * l.Kp * 4);
+  l.caug = take((size_t)B * l.Kp * AUG_SLAB * 2);
   l.xs = take(l.split ? BN_ * l.Dq * 2 : 0);
   l.xn = take(BN_ * 4);
   l.keys0 = take(BN_ * 4);
@@ -208,7 +208,7 @@ static fkm_status step_assign(const Ws& w, const void* x, int32_t* ids, cudaStre
   a.xq = L.split ? w.at<void>(L.xs) : x;
   a.x_row_elems = L.split ? L.Dq : L.D;
   a.cq = w.at<void>(L.cq);
-  a.cn = w.at<float>(L.cn);
+  a.caug = w.at<void>(L.caug);
   a.xn = nullptr;
   a.ids = ids;
   a.status = w.status();
@@ -268,7 +268,7 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   // the next assign's operands: offsets of the new centroids from their mean
   if (requant)
     FKM_TRY(launch_prep_centroids(next, L.B, L.K, L.Kp, L.D, L.dtype, w.at<float>(L.mvec),
-                                  w.at<void>(L.cq), w.at<float>(L.cn), st));
+                                  w.at<void>(L.cq), w.at<void>(L.caug), st));
   return FKM_OK;
 }
 
@@ -383,7 +383,7 @@ fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Ws w{ws, &L};
   FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
-                                w.at<void>(L.cq), w.at<float>(L.cn), st));
+                                w.at<void>(L.cq), w.at<void>(L.caug), st));
   if (L.split)
     FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, w.at<void>(L.xs), nullptr, st));
   FKM_TRY(step_assign(w, x, ids, st));
@@ -416,7 +416,7 @@ fkm_status fkm_update(int B, int N, int K, int D, int dtype, const void* x, cons
   FKM_CUDA_TRY(cudaMemsetAsync(w.at<double>(L.sums64), 0, (size_t)B * K * D * 8, st));
   if (inertia && !L.split)  // the objective measures against q(prev), the assign operand
     FKM_TRY(launch_prep_centroids(prev_centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
-                                  w.at<void>(L.cq), w.at<float>(L.cn), st));
+                                  w.at<void>(L.cq), w.at<void>(L.caug), st));
   FKM_TRY(step_update(w, x, ids, prev_centers, centers, counts, false, inertia, st));
   if (shift) FKM_TRY(launch_batch_reduce(B, K, w.at<double>(L.shiftk), shift, nullptr, st));
   return FKM_OK;
@@ -453,7 +453,7 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
   FKM_CUDA_TRY(cudaMemcpyAsync(cA, init_centers, cbytes, cudaMemcpyDeviceToDevice, st));
   if (L.split) FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, w.at<void>(L.xs), nullptr, st));
   FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, w.at<float>(L.mvec), w.at<void>(L.cq),
-                                w.at<float>(L.cn), st));
+                                w.at<void>(L.caug), st));
 
   FKM_TRY(assign_prepare());
   const bool prof = g_prof.on.load();
@@ -614,7 +614,7 @@ fkm_status fkm_baseline_assign(int B, int N, int K, int D, int dtype, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Ws w{ws, &L};
   FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
-                                w.at<void>(L.cq), w.at<float>(L.cn), st));
+                                w.at<void>(L.cq), w.at<void>(L.caug), st));
   FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, L.split ? w.at<void>(L.xs) : nullptr,
                              w.at<float>(L.xn), st, w.at<float>(L.mvec), N));
   AssignArgs a;
@@ -628,7 +628,7 @@ fkm_status fkm_baseline_assign(int B, int N, int K, int D, int dtype, const void
   a.xq = L.split ? w.at<void>(L.xs) : x;
   a.x_row_elems = L.split ? L.Dq : D;
   a.cq = w.at<void>(L.cq);
-  a.cn = w.at<float>(L.cn);
+  a.caug = w.at<void>(L.caug);
   a.xn = w.at<float>(L.xn);
   a.ids = ids;
   a.status = w.status();

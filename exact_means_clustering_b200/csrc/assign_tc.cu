@@ -3,24 +3,38 @@
 // "Flash-KMeans: Fast and Memory-Efficient Exact K-Means" summary, section
 // "Method" (FlashAssign), and the "Flash-KMeans：快速且内存高效精确K-Means聚类"
 // summary, section 方法步骤详情 step (1): tile the points (B_N) and the
-// centroids (B_K); per point keep a running (min score, index) that starts at
-// +inf; per centroid tile compute the local B_N x B_K block on chip, take its
-// row minima and fold them into the running state; write the final index once.
-// The score is ||c||^2 - 2 x.c (the same page, section 核心方法: ||x||^2 is
-// constant per point and does not change the argmin).
+// centroids (B_K); per point keep a running (best score, index); per centroid
+// tile compute the local B_N x B_K block on chip, take its row extrema and fold
+// them into the running state; write the final index once.  The score is
+// ||c||^2 - 2 x.c (the same page, section 核心方法: ||x||^2 is constant per
+// point and does not change the argmin).
+//
+// Operands (see prep.cu): centroid offsets q(c - m) from the batch's mean
+// centroid m, and a 16-column "bias" slab per centroid holding -n/2 as three
+// 16-bit parts, n = ||q(c-m)||^2 + 2 m.q(c-m).  Each point tile is extended by
+// a constant slab [a0, a1, a2, 0...] (a = 1, 1, 1 for bf16; 2^15, 2^4, 2^-7
+// for fp16, whose parts are scaled to stay in range), so one extra K=16 MMA
+// adds the bias and the accumulator holds
+//     acc = x.q(c - m) - n/2 = -(score)/2 + (a per-point constant),
+// and the nearest centroid is the argmax of acc: the epilogue only compares.
 //
 // B200 design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: the point tile [128 x D] once per work item into
-//               one of nA buffers, centroid tiles [256 x 64] through an
-//               nS-stage ring (128-byte swizzle, no multicast).
+//               one of nA buffers; per centroid tile, 256 x 64 chunks through
+//               an nS-stage ring (128-byte swizzle, no multicast), the tile's
+//               bias slab (256 x 16, 32-byte swizzle) riding with its first
+//               chunk.
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators)
-//               and issues tcgen05.mma (M=128, N=256, K=16) from one thread.
+//               and issues tcgen05.mma (M=128, N=256, K=16) from one thread:
+//               the bias product, then the point . centroid products.
 //   warps 2-9   epilogue, two warpgroups: TMEM lane t = point t of the tile;
 //               warpgroup h reads columns [128h, 128h + 128) of every
-//               accumulator (tcgen05.ld), forms score = ||q(c)||^2 - 2 acc with
-//               packed fp32x2 FMAs and keeps its running minimum with 3-input
-//               min trees; the two halves are merged per work item.  Ties go
-//               to the lowest centroid index.
+//               accumulator (four tcgen05.ld in flight, one wait), hands the
+//               accumulator back, and keeps the running maximum with 3-input
+//               max trees; the chunk that improves it is saved to shared
+//               memory so the lowest column holding the maximum is found once
+//               per work item.  The two halves are merged per work item.
+//               Ties go to the lowest centroid index.
 // Accumulator double buffering lets the MMAs of tile t+1 run while the
 // epilogue reduces tile t; A double buffering overlaps the next work item's
 // point load with the current one's MMAs.
@@ -49,21 +63,24 @@ namespace fkm {
 namespace {
 
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;  // 4 s
+constexpr int AUG_COLS = 16;                             // the bias slab: one K=16 MMA
+constexpr int AUG_A_BYTES = BM * AUG_COLS * 2;           // 4 KB, constant per CTA
+constexpr int AUG_B_BYTES = BN * AUG_COLS * 2;           // 8 KB per centroid tile
+constexpr int STAGE_BYTES = B_CHUNK_BYTES + AUG_B_BYTES; // chunk + bias slot
 
 struct AssignKParams {
-  int B, N, Kp;
+  int B, N, Kp, K;
   int nD;          // 64-wide D chunks
   int m_tiles;     // point tiles per batch
   int k_tiles;     // centroid tiles per batch
   int n_work;      // B * m_tiles
   int nA, nS;      // point buffers, centroid stages
-  uint32_t a_bytes, s_bytes;
+  uint32_t a_bytes;
   uint32_t idesc;
-  const float* cn;
-  const float* xn;  // ||x||^2, comparison mode only
+  int f16;         // fp16 operands: scaled bias parts
+  const float* xn;  // ||x - m||^2, comparison mode only
   int32_t* ids;
   int* status;
-  int K;           // real centroids (materialised rows are K wide)
   float* dist;     // comparison mode only: the full [B, N, K] distance matrix
 };
 
@@ -71,66 +88,54 @@ struct __align__(8) SmemCtl {
   uint64_t a_full[2], a_empty[2];
   uint64_t b_full[8], b_empty[8];
   uint64_t acc_full[2], acc_empty[2];
-  uint64_t cn_full[2];
   uint64_t merge_full, merge_empty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  __align__(16) float cn_s[2][BN];   // read with 16-byte loads
-  float2 merge[BM];   // (best score, index as float bits) of warpgroup 1
+  float2 merge[BM];   // (best, index as float bits) of warpgroup 1
 };
-static_assert(offsetof(SmemCtl, cn_s) % 16 == 0, "cn_s must be 16-byte aligned");
 
-// Per epilogue thread, the scores of the chunk that last improved its
-// running minimum (32 floats), with the 16-byte units rotated by lane so the
+// Per epilogue thread, the 32 accumulator values of the chunk that last
+// improved its running maximum, with the 16-byte units rotated by lane so the
 // predicated stores of a warp hit distinct banks.
 constexpr int kSaveBytes = 256 * 32 * 4;
 
-__device__ __forceinline__ float2 u2f2(uint32_t a, uint32_t b) {
-  return make_float2(__uint_as_float(a), __uint_as_float(b));
+__device__ __forceinline__ float max32(const float (&s)[32]) {
+  float m0 = ptx::fmax3(s[0], s[1], s[2]);
+  float m1 = ptx::fmax3(s[3], s[4], s[5]);
+  float m2 = ptx::fmax3(s[6], s[7], s[8]);
+  float m3 = ptx::fmax3(s[9], s[10], s[11]);
+  float m4 = ptx::fmax3(s[12], s[13], s[14]);
+  float m5 = ptx::fmax3(s[15], s[16], s[17]);
+  float m6 = ptx::fmax3(s[18], s[19], s[20]);
+  float m7 = ptx::fmax3(s[21], s[22], s[23]);
+  float m8 = ptx::fmax3(s[24], s[25], s[26]);
+  float m9 = ptx::fmax3(s[27], s[28], s[29]);
+  float m10 = fmaxf(s[30], s[31]);
+  float n0 = ptx::fmax3(m0, m1, m2);
+  float n1 = ptx::fmax3(m3, m4, m5);
+  float n2 = ptx::fmax3(m6, m7, m8);
+  float n3 = fmaxf(m9, m10);
+  return fmaxf(ptx::fmax3(n0, n1, n2), n3);
 }
 
-// Minimum of 32 scores with 3-input min instructions.
-__device__ __forceinline__ float min32(const float (&s)[32]) {
-  float m0 = ptx::fmin3(s[0], s[1], s[2]);
-  float m1 = ptx::fmin3(s[3], s[4], s[5]);
-  float m2 = ptx::fmin3(s[6], s[7], s[8]);
-  float m3 = ptx::fmin3(s[9], s[10], s[11]);
-  float m4 = ptx::fmin3(s[12], s[13], s[14]);
-  float m5 = ptx::fmin3(s[15], s[16], s[17]);
-  float m6 = ptx::fmin3(s[18], s[19], s[20]);
-  float m7 = ptx::fmin3(s[21], s[22], s[23]);
-  float m8 = ptx::fmin3(s[24], s[25], s[26]);
-  float m9 = ptx::fmin3(s[27], s[28], s[29]);
-  float m10 = fminf(s[30], s[31]);
-  float n0 = ptx::fmin3(m0, m1, m2);
-  float n1 = ptx::fmin3(m3, m4, m5);
-  float n2 = ptx::fmin3(m6, m7, m8);
-  float n3 = fminf(m9, m10);
-  return fminf(ptx::fmin3(n0, n1, n2), n3);
-}
-
-// Scores of one 32-column chunk, s = cn - 2 acc, folded into (best, bcol).
-// A chunk replaces the running minimum only when strictly smaller; then its
-// scores are saved so the lowest column holding the minimum can be found once
-// per work item (find_first), which keeps the lowest centroid index among
-// exact ties without a per-chunk search.
-__device__ __forceinline__ void fold_chunk(const uint32_t (&r)[32], const float* cn, int col0,
-                                           float& best, int& bcol, float4* save, int rot) {
+// One 32-column chunk folded into (best, bcol).  A chunk replaces the running
+// maximum only when strictly larger; its values are then saved so the lowest
+// column holding the maximum is found once per work item (find_first): over
+// ascending columns this keeps the lowest centroid index among exact ties.
+// Columns at or past K (padding of the last tile) are excluded.
+__device__ __forceinline__ void fold_chunk(const uint32_t (&r)[32], int col0, int K, float& best,
+                                           int& bcol, float4* save, int rot) {
   float s[32];
-  const float2 m2 = make_float2(-2.0f, -2.0f);
 #pragma unroll
-  for (int j = 0; j < 32; j += 4) {
-    const float4 c4 = *reinterpret_cast<const float4*>(cn + j);
-    const float2 v0 = __ffma2_rn(u2f2(r[j], r[j + 1]), m2, make_float2(c4.x, c4.y));
-    const float2 v1 = __ffma2_rn(u2f2(r[j + 2], r[j + 3]), m2, make_float2(c4.z, c4.w));
-    s[j] = v0.x;
-    s[j + 1] = v0.y;
-    s[j + 2] = v1.x;
-    s[j + 3] = v1.y;
+  for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(r[j]);
+  if (col0 + 32 > K) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j >= K) s[j] = -INFINITY;
   }
-  const float cm = min32(s);
-  if (cm < best) {
+  const float cm = max32(s);
+  if (cm > best) {
     best = cm;
     bcol = col0;
 #pragma unroll
@@ -139,7 +144,7 @@ __device__ __forceinline__ void fold_chunk(const uint32_t (&r)[32], const float*
   }
 }
 
-// Lowest position j in the saved chunk whose score equals best.
+// Lowest position j in the saved chunk whose value equals best.
 __device__ __forceinline__ int find_first(const float4* save, int rot, float best) {
   uint32_t mask = 0;
 #pragma unroll
@@ -153,24 +158,49 @@ __device__ __forceinline__ int find_first(const float4* save, int rot, float bes
   return mask ? __ffs(mask) - 1 : 0;
 }
 
+// The constant bias slab of a point tile: row r = [a0, a1, a2, 0 ... 0] (16
+// values) in the 32-byte swizzle (rows of 32 bytes, 8-row groups of 256
+// bytes; the two 16-byte halves of rows 4-7 of a group trade places), the
+// layout a K-major tcgen05 operand with SWIZZLE_32B reads.
+__device__ __forceinline__ void write_aug_a(uint8_t* base, int f16) {
+  if (threadIdx.x >= 2 * BM) return;
+  const int r = threadIdx.x >> 1, h = threadIdx.x & 1;
+  const int phys = h ^ ((r & 7) >> 2);
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (h == 0) {
+    uint16_t a0, a1, a2;
+    if (f16) {
+      a0 = __half_as_ushort(__float2half_rn(32768.0f));
+      a1 = __half_as_ushort(__float2half_rn(16.0f));
+      a2 = __half_as_ushort(__float2half_rn(0.0078125f));
+    } else {
+      a0 = a1 = a2 = __bfloat16_as_ushort(__float2bfloat16_rn(1.0f));
+    }
+    v.x = (uint32_t)a0 | ((uint32_t)a1 << 16);
+    v.y = (uint32_t)a2;
+  }
+  *reinterpret_cast<uint4*>(base + (r >> 3) * 256 + (r & 7) * 32 + phys * 16) = v;
+}
+
 // kDist = true is the comparison ("standard") mode: the same tensor-core tiles,
-// but the epilogue writes every distance ||x - c_hat||^2 = ||x - m||^2 +
-// norm_k - 2 x.q(c_k - m) to HBM instead of reducing it, as the pages'
-// baseline assignment does.
+// but the epilogue writes every distance ||x - c_hat||^2 = ||x - m||^2 - 2 acc
+// to HBM instead of reducing it, as the pages' baseline assignment does.
 template <bool kSplit, bool kDist>
 __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
-    assign_tc_kernel(const __grid_constant__ CUtensorMap tm_x,   // points (hi part when split)
-                     const __grid_constant__ CUtensorMap tm_xl,  // lo part (split only)
-                     const __grid_constant__ CUtensorMap tm_c,   // centroids (hi part when split)
-                     const __grid_constant__ CUtensorMap tm_cl,  // lo part (split only)
+    assign_tc_kernel(const __grid_constant__ CUtensorMap tm_x,    // points (hi part when split)
+                     const __grid_constant__ CUtensorMap tm_xl,   // lo part (split only)
+                     const __grid_constant__ CUtensorMap tm_c,    // centroid offsets (hi when split)
+                     const __grid_constant__ CUtensorMap tm_cl,   // lo part (split only)
+                     const __grid_constant__ CUtensorMap tm_aug,  // bias slabs [B][Kp][16]
                      const AssignKParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* a_base = smem;
-  uint8_t* b_base = a_base + (size_t)p.nA * p.a_bytes;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(b_base + (size_t)p.nS * p.s_bytes);
+  uint8_t* aug_a = a_base + (size_t)p.nA * p.a_bytes;
+  uint8_t* b_base = aug_a + AUG_A_BYTES;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(b_base + (size_t)p.nS * STAGE_BYTES);
   float4* save_base = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(ctl) +
                                                 ((sizeof(SmemCtl) + 127) & ~size_t(127)));
 
@@ -178,6 +208,9 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &ctl->abort;
 
+  write_aug_a(aug_a, p.f16);
+  // the generic-proxy stores above are read by the tensor cores (async proxy)
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.nA; ++i) {
       ptx::mbar_init(&ctl->a_full[i], 1);
@@ -190,7 +223,6 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&ctl->acc_full[i], 1);
       ptx::mbar_init(&ctl->acc_empty[i], 8);
-      ptx::mbar_init(&ctl->cn_full[i], 256);
     }
     ptx::mbar_init(&ctl->merge_full, 128);
     ptx::mbar_init(&ctl->merge_empty, 128);
@@ -206,12 +238,14 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+  const int nQ = p.nD * (kSplit ? 2 : 1);   // stages per centroid tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       ptx::prefetch_tmap(&tm_x);
       ptx::prefetch_tmap(&tm_c);
+      ptx::prefetch_tmap(&tm_aug);
       if (kSplit) {
         ptx::prefetch_tmap(&tm_xl);
         ptx::prefetch_tmap(&tm_cl);
@@ -234,18 +268,21 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
         }
         ++a_arms;
         for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
-          // one stage per 64-wide chunk; split operands put hi and lo in
-          // consecutive stages
-          for (int q = 0; q < p.nD * (kSplit ? 2 : 1); ++q) {
+          // one stage per 64-wide chunk (split operands: hi and lo in
+          // consecutive stages); the tile's bias slab rides with its first chunk
+          for (int q = 0; q < nQ; ++q) {
             const int dc = kSplit ? (q >> 1) : q;
             const int sb = s_arms % p.nS;
             const uint32_t spar = ((s_arms / p.nS) & 1) ^ 1;
             if (!ptx::mbar_wait_bounded(&ctl->b_empty[sb], spar, abort_flag, p.status, ST_TIMEOUT,
                                         kWaitTimeoutNs)) { ok = false; break; }
-            ptx::mbar_arrive_expect_tx(&ctl->b_full[sb], p.s_bytes);
-            uint8_t* sbuf = b_base + (size_t)sb * p.s_bytes;
+            ptx::mbar_arrive_expect_tx(&ctl->b_full[sb],
+                                       B_CHUNK_BYTES + (q == 0 ? AUG_B_BYTES : 0));
+            uint8_t* sbuf = b_base + (size_t)sb * STAGE_BYTES;
             ptx::tma_load_3d(sbuf, (kSplit && (q & 1)) ? &tm_cl : &tm_c, &ctl->b_full[sb],
                              dc * KC, kt * BN, b);
+            if (q == 0)
+              ptx::tma_load_3d(sbuf + B_CHUNK_BYTES, &tm_aug, &ctl->b_full[sb], 0, kt * BN, b);
             ++s_arms;
           }
         }
@@ -265,6 +302,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      const uint32_t aug_a_addr = ptx::smem_u32(aug_a);
       uint32_t a_uses = 0, s_uses = 0, acc_uses = 0;
       bool ok = true;
       bool issued = false;
@@ -280,21 +318,23 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
                                       p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-          for (int q = 0; q < p.nD * (kSplit ? 2 : 1); ++q) {
+          for (int q = 0; q < nQ; ++q) {
             const int dc = kSplit ? (q >> 1) : q;
             const int sb = s_uses % p.nS;
             if (!ptx::mbar_wait_bounded(&ctl->b_full[sb], (s_uses / p.nS) & 1, abort_flag,
                                         p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
             ptx::tc_fence_after();
-            const uint32_t b_addr = ptx::smem_u32(b_base + (size_t)sb * p.s_bytes);
+            const uint32_t b_addr = ptx::smem_u32(b_base + (size_t)sb * STAGE_BYTES);
             const uint32_t xa = a_addr + dc * A_CHUNK_BYTES;
+            if (q == 0)   // the bias product starts the tile's accumulation
+              ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw32(aug_a_addr),
+                              ptx::umma_desc_sw32(b_addr + B_CHUNK_BYTES), p.idesc, 0u);
             if (!(kSplit && (q & 1))) {
-              // xh . ch (or x . q(c)); the first product of the tile overwrites
+              // xh . ch (or x . q(c - m))
 #pragma unroll
               for (int k = 0; k < KC / 16; ++k)
                 ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xa + 32 * k),
-                                ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc,
-                                (q > 0 || k > 0) ? 1u : 0u);
+                                ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc, 1u);
               if (kSplit) {   // xl . ch
                 const uint32_t xl = a_addr + (p.nD + dc) * A_CHUNK_BYTES;
 #pragma unroll
@@ -328,7 +368,6 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;          // 0..255
     const int ew = warp - 2;                  // epilogue warp 0..7
     const int half = ew >> 2;                 // columns [128*half, 128*half + 128) of a tile
     const int quad = warp & 3;                // TMEM lane quadrant this warp may access
@@ -338,74 +377,22 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
     uint32_t acc_uses = 0, items = 0;
     bool ok = true;
-    // ||q(c)||^2 of the next tile, loaded one tile ahead so the global load
-    // is off the critical path
-    float cn_pre = (blockIdx.x < (unsigned)p.n_work)
-                       ? p.cn[(size_t)(blockIdx.x / p.m_tiles) * p.Kp + et] : 0.0f;
     for (int w = blockIdx.x; w < p.n_work && ok; w += gridDim.x, ++items) {
       const int b = w / p.m_tiles, mt = w % p.m_tiles;
-      float best = INFINITY;
+      const int gi = mt * BM + row;
+      float best = -INFINITY;
       int bcol = 0;
       for (int kt = 0; kt < p.k_tiles; ++kt) {
         const int acc = acc_uses & 1;
         const uint32_t par = (acc_uses >> 1) & 1;
-        const float cn_cur = cn_pre;
-        if (kt + 1 < p.k_tiles)
-          cn_pre = p.cn[(size_t)b * p.Kp + (size_t)(kt + 1) * BN + et];
-        else if (w + (int)gridDim.x < p.n_work)
-          cn_pre = p.cn[(size_t)((w + gridDim.x) / p.m_tiles) * p.Kp + et];
-        // Stage ||q(c)||^2 of this centroid tile in shared memory.  Buffer acc
-        // was last read two tiles ago, and every thread finished that tile
-        // before it arrived for the previous one, so it is free to overwrite.
-        ctl->cn_s[acc][et] = cn_cur;
-        ptx::mbar_arrive(&ctl->cn_full[acc]);
-        if (!ptx::mbar_wait_bounded(&ctl->cn_full[acc], par, abort_flag, p.status, ST_TIMEOUT,
-                                    kWaitTimeoutNs)) { ok = false; break; }
         if (!ptx::mbar_wait_bounded(&ctl->acc_full[acc], par, abort_flag, p.status, ST_TIMEOUT,
                                     kWaitTimeoutNs)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t taddr = lane_addr + (uint32_t)(acc * BN + half * 128);
-        const float* cn_s = ctl->cn_s[acc] + half * 128;
         const int colb = kt * BN + half * 128;
-        uint32_t r0[32], r1[32];
-        if (kDist) {
-          const int gi = mt * BM + row;
-          const float xv = (gi < p.N) ? p.xn[(size_t)b * p.N + gi] : 0.0f;
-          float* drow = p.dist + ((size_t)b * p.N + (gi < p.N ? gi : 0)) * p.K;
-          const bool vec4 = (p.K & 3) == 0;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            ptx::tmem_ld32(taddr + c * 32, r0);
-            ptx::tmem_wait_ld32(r0);
-            if (c == 3) {
-              ptx::tc_fence_before();
-              __syncwarp();
-              if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
-            }
-            const int col0 = colb + c * 32;
-            if (gi < p.N && col0 < p.K) {
-              float dv[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                dv[j] = xv + fmaf(-2.0f, __uint_as_float(r0[j]), cn_s[c * 32 + j]);
-              if (vec4 && col0 + 32 <= p.K) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                  *reinterpret_cast<float4*>(drow + col0 + j) =
-                      make_float4(dv[j], dv[j + 1], dv[j + 2], dv[j + 3]);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (col0 + j < p.K) drow[col0 + j] = dv[j];
-              }
-            }
-          }
-          ++acc_uses;
-          continue;
-        }
         // all 128 of this warp's columns in flight at once, one wait, then the
         // accumulator goes straight back to the MMA warp
-        uint32_t r2[32], r3[32];
+        uint32_t r0[32], r1[32], r2[32], r3[32];
         ptx::tmem_ld32(taddr, r0);
         ptx::tmem_ld32(taddr + 32, r1);
         ptx::tmem_ld32(taddr + 64, r2);
@@ -414,15 +401,29 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ctl->acc_empty[acc]);
-        fold_chunk(r0, cn_s, colb, best, bcol, save, rot);
-        fold_chunk(r1, cn_s + 32, colb + 32, best, bcol, save, rot);
-        fold_chunk(r2, cn_s + 64, colb + 64, best, bcol, save, rot);
-        fold_chunk(r3, cn_s + 96, colb + 96, best, bcol, save, rot);
         ++acc_uses;
+        if (kDist) {
+          if (gi < p.N) {
+            const float xv = p.xn[(size_t)b * p.N + gi];
+            float* drow = p.dist + ((size_t)b * p.N + gi) * p.K;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (colb + j < p.K) drow[colb + j] = fmaf(-2.0f, __uint_as_float(r0[j]), xv);
+              if (colb + 32 + j < p.K) drow[colb + 32 + j] = fmaf(-2.0f, __uint_as_float(r1[j]), xv);
+              if (colb + 64 + j < p.K) drow[colb + 64 + j] = fmaf(-2.0f, __uint_as_float(r2[j]), xv);
+              if (colb + 96 + j < p.K) drow[colb + 96 + j] = fmaf(-2.0f, __uint_as_float(r3[j]), xv);
+            }
+          }
+          continue;
+        }
+        fold_chunk(r0, colb, p.K, best, bcol, save, rot);
+        fold_chunk(r1, colb + 32, p.K, best, bcol, save, rot);
+        fold_chunk(r2, colb + 64, p.K, best, bcol, save, rot);
+        fold_chunk(r3, colb + 96, p.K, best, bcol, save, rot);
       }
       if (!ok) break;
       if (kDist) continue;
-      const int idx = bcol + find_first(save, rot, best);
+      const int idx = best > -INFINITY ? bcol + find_first(save, rot, best) : 0;
       // merge the two column halves of each row
       const uint32_t mpar = items & 1;
       if (half == 1) {
@@ -436,8 +437,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
         const float2 o = ctl->merge[row];
         ptx::mbar_arrive(&ctl->merge_empty);
         const int oidx = __float_as_int(o.y);
-        const int fidx = (o.x < best || (o.x == best && oidx < idx)) ? oidx : idx;
-        const int gi = mt * BM + row;
+        const int fidx = (o.x > best || (o.x == best && oidx < idx)) ? oidx : idx;
         if (gi < p.N) p.ids[(size_t)b * p.N + gi] = fidx;
       }
     }
@@ -472,10 +472,11 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // 3-D map over [batches][rows][cols] 16-bit elements with a row pitch of
-// row_elems; the box is box_cols x box_rows x 1 with the 128-byte swizzle.
-// Elements outside [cols) x [rows) read as zero.
+// row_elems; the box is box_cols x box_rows x 1.  Elements outside
+// [cols) x [rows) read as zero.
 fkm_status make_map(CUtensorMap* m, const void* base, bool bf16, int cols, int rows, int batches,
-                    int row_elems, int box_cols, int box_rows) {
+                    int row_elems, int box_cols, int box_rows,
+                    CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) {
     set_error("cuTensorMapEncodeTiled is not available from the CUDA driver");
@@ -487,8 +488,7 @@ fkm_status make_map(CUtensorMap* m, const void* base, bool bf16, int cols, int r
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                    const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_error("cuTensorMapEncodeTiled failed (%d) for a %d x %d x %d map", (int)r, cols, rows,
               batches);
@@ -505,8 +505,8 @@ constexpr int kSmemBudget = 232448 - 1024;  // opt-in maximum minus alignment sl
 bool assign_smem_plan(int D, bool split, int* nA_out, int* nS_out, size_t* smem_out) {
   const int nD = (int)ceil_div(D, KC);
   const long a_bytes = (long)(split ? 2 : 1) * nD * A_CHUNK_BYTES;
-  const long s_bytes = B_CHUNK_BYTES;
-  const long ctl = (long)((sizeof(SmemCtl) + 127) & ~size_t(127)) + kSaveBytes;
+  const long s_bytes = STAGE_BYTES;
+  const long ctl = (long)((sizeof(SmemCtl) + 127) & ~size_t(127)) + kSaveBytes + AUG_A_BYTES;
   int nA = 2;
   long nS = (kSmemBudget - ctl - 2 * a_bytes) / s_bytes;
   if (nS < 2) {
@@ -550,13 +550,15 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
   }
   const int nD = (int)ceil_div(a.D, KC);
   const bool bf16 = a.split || a.dtype == FKM_BF16;
-  CUtensorMap tx, txl, tc, tcl;
+  CUtensorMap tx, txl, tc, tcl, taug;
   // split rows are [hi | lo] with each half padded to a multiple of 8
   // elements, so the lo half starts 16-byte aligned
   const int Dp = (int)round_up(a.D, 8);
   const int Dq = a.split ? 2 * Dp : a.D;
   FKM_TRY(make_map(&tx, a.xq, bf16, a.D, a.N, a.B, a.x_row_elems, KC, BM));
   FKM_TRY(make_map(&tc, a.cq, bf16, a.D, a.Kp, a.B, Dq, KC, BN));
+  FKM_TRY(make_map(&taug, a.caug, bf16, AUG_COLS, a.Kp, a.B, AUG_COLS, AUG_COLS, BN,
+                   CU_TENSOR_MAP_SWIZZLE_32B));
   if (a.split) {
     FKM_TRY(make_map(&txl, static_cast<const uint16_t*>(a.xq) + Dp, true, a.D, a.N, a.B,
                      a.x_row_elems, KC, BM));
@@ -570,6 +572,7 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
   p.B = a.B;
   p.N = a.N;
   p.Kp = a.Kp;
+  p.K = a.K;
   p.nD = nD;
   p.m_tiles = (int)ceil_div(a.N, BM);
   p.k_tiles = a.Kp / BN;
@@ -577,26 +580,24 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
   p.nA = nA;
   p.nS = nS;
   p.a_bytes = (uint32_t)((a.split ? 2 : 1) * nD * A_CHUNK_BYTES);
-  p.s_bytes = (uint32_t)B_CHUNK_BYTES;
   p.idesc = ptx::umma_idesc_f16(bf16, BM, BN);
-  p.cn = a.cn;
+  p.f16 = bf16 ? 0 : 1;
   p.xn = a.xn;
   p.ids = a.ids;
   p.status = a.status;
-  p.K = a.K;
   p.dist = a.dist;
   const int sms = num_sms();
   const int grid = p.n_work < sms ? p.n_work : sms;
   FKM_TRY(assign_prepare());
   if (a.dist) {
     if (a.split)
-      assign_tc_kernel<true, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, p);
+      assign_tc_kernel<true, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
     else
-      assign_tc_kernel<false, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, p);
+      assign_tc_kernel<false, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
   } else if (a.split) {
-    assign_tc_kernel<true, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, p);
+    assign_tc_kernel<true, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
   } else {
-    assign_tc_kernel<false, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, p);
+    assign_tc_kernel<false, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
   }
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());

@@ -71,7 +71,7 @@ struct Layout {
   int64_t n_sort;  // B * N keys
   int n_sort_tiles;
   int key_bits;
-  size_t status, mvec, cq, cn, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
+  size_t status, mvec, cq, caug, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
       segstart, segend, sums64, shiftk, cbuf, scal, total;
 };
 
@@ -88,8 +88,8 @@ struct AssignArgs {
   bool split;
   const void* xq;      // bf16/f16 points, or the split [hi|lo] rows for fp32
   int x_row_elems;     // elements per row of xq (D, or 2D when split)
-  const void* cq;      // quantised centroids [B, Kp, Dq]
-  const float* cn;     // ||q(c)||^2 [B, Kp], +inf on padding rows
+  const void* cq;      // centroid offsets q(c - m) [B, Kp, Dq]
+  const void* caug;    // bias slabs [B, Kp, 16]: -n/2 in three 16-bit parts
   const float* xn;     // ||x - m||^2 [B, N] (comparison mode only)
   int32_t* ids;        // [B, N]
   int* status;
@@ -99,11 +99,13 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st);
 bool assign_smem_plan(int D, bool split, int* nA, int* nS, size_t* smem);
 fkm_status assign_prepare();
 
-// Per batch mean centroid m [B][D]; q(c - m) rows [B][Kp][Dq] and the norm
-// term ||q(c-m)||^2 + 2 m.q(c-m); split rows (fp32) are [hi | lo] halves of
-// round_up(D, 8) elements each.
+// Per batch mean centroid m [B][D]; q(c - m) rows [B][Kp][Dq] (split rows
+// for fp32 are [hi | lo] halves of round_up(D, 8) elements each); and per
+// centroid the bias slab [B][Kp][16]: -n/2 as three 16-bit parts, n =
+// ||q(c-m)||^2 + 2 m.q(c-m) (zero on padding rows).
+constexpr int AUG_SLAB = 16;
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
-                                 float* m, void* cq, float* cn, cudaStream_t st);
+                                 float* m, void* cq, void* caug, cudaStream_t st);
 // fp32 points: split rows into xs; xn (optional) = ||x - m[row / N]||^2
 // (||x||^2 when m is null).
 fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,

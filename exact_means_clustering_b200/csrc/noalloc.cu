@@ -8,7 +8,7 @@
 // cudaMalloc for the workspace that fkm_assign expects.
 //
 // This entry point keeps its scratch (the per-batch mean centroid, the
-// centroid offsets rounded to the points' 16-bit type, their norm terms, and
+// centroid offsets rounded to the points' 16-bit type, their bias slabs, and
 // a status word) in one file-scope
 // device array of FKM_NOALLOC_SCRATCH_BYTES.  Every GPU that loads the library
 // holds that array until the process exits.  The host-side name of the array
@@ -76,11 +76,11 @@ extern "C" fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, 
   const size_t status_bytes = 256;
   const size_t m_bytes = (size_t)round_up((int64_t)B * D * 4, 256);
   const size_t cq_bytes = (size_t)round_up((int64_t)B * Kp * D * 2, 256);
-  const size_t cn_bytes = (size_t)round_up((int64_t)B * Kp * 4, 256);
-  if (status_bytes + m_bytes + cq_bytes + cn_bytes > kScratchBytes) {
-    set_error("B*(4*D + Kp*(2*D + 4)) = %zu bytes exceeds the %zu-byte static scratch of "
+  const size_t aug_bytes = (size_t)round_up((int64_t)B * Kp * AUG_SLAB * 2, 256);
+  if (status_bytes + m_bytes + cq_bytes + aug_bytes > kScratchBytes) {
+    set_error("B*(4*D + Kp*(2*D + 32)) = %zu bytes exceeds the %zu-byte static scratch of "
               "fkm_assign_noalloc (Kp = K rounded up to 256)",
-              m_bytes + cq_bytes + cn_bytes, kScratchBytes - status_bytes);
+              m_bytes + cq_bytes + aug_bytes, kScratchBytes - status_bytes);
     return FKM_ERR_UNSUPPORTED;
   }
   void* base = nullptr;
@@ -89,12 +89,12 @@ extern "C" fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, 
   int* status = reinterpret_cast<int*>(p);
   float* m = reinterpret_cast<float*>(p + status_bytes);
   void* cq = p + status_bytes + m_bytes;
-  float* cn = reinterpret_cast<float*>(p + status_bytes + m_bytes + cq_bytes);
+  void* caug = p + status_bytes + m_bytes + cq_bytes;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the status word is the only scratch that must start at zero; the rest is
   // fully rewritten by the centroid preparation below
   FKM_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
-  FKM_TRY(launch_prep_centroids(centers, B, K, Kp, D, dtype, m, cq, cn, st));
+  FKM_TRY(launch_prep_centroids(centers, B, K, Kp, D, dtype, m, cq, caug, st));
   AssignArgs a;
   a.B = B;
   a.N = N;
@@ -106,7 +106,7 @@ extern "C" fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, 
   a.xq = x;
   a.x_row_elems = D;
   a.cq = cq;
-  a.cn = cn;
+  a.caug = caug;
   a.xn = nullptr;
   a.ids = ids;
   a.status = status;

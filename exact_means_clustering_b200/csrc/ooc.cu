@@ -37,7 +37,7 @@ struct HostLayout {
   int chunks_per_batch;
   int tiles_per_chunk;
   int key_bits;
-  size_t status, xbuf[2], mvec, cq, cn, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
+  size_t status, xbuf[2], mvec, cq, caug, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
       segstart, segend, sums64, counts_acc, shiftk, cbuf, total;
 };
 
@@ -88,7 +88,7 @@ fkm_status make_host_layout(int B, int N, int K, int D, int dtype, int64_t chunk
   l.xbuf[1] = take((size_t)R * D * s);
   l.mvec = take((size_t)B * D * 4);
   l.cq = take((size_t)B * l.Kp * l.Dq * 2);
-  l.cn = take((size_t)B * l.Kp * 4);
+  l.caug = take((size_t)B * l.Kp * AUG_SLAB * 2);
   l.xs = take(l.split ? (size_t)R * l.Dq * 2 : 0);
   l.xn = take((size_t)R * 4);
   l.keys0 = take((size_t)R * 4);
@@ -196,7 +196,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
   FKM_CUDA_TRY(cudaMemcpyAsync(cA, init_centers, cbytes, cudaMemcpyDeviceToDevice, st));
   float* mvec = static_cast<float*>(at(L.mvec));
   FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, mvec, at(L.cq),
-                                static_cast<float*>(at(L.cn)), st));
+                                at(L.caug), st));
   // the copy stream may only touch the workspace after the caller's earlier work
   FKM_CUDA_TRY(cudaEventRecord(ss.start, st));
   FKM_CUDA_TRY(cudaStreamWaitEvent(ss.copy, ss.start, 0));
@@ -235,7 +235,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
         a.xq = L.split ? at(L.xs) : xb;
         a.x_row_elems = L.split ? L.Dq : D;
         a.cq = static_cast<const char*>(at(L.cq)) + (size_t)b * L.Kp * L.Dq * 2;
-        a.cn = static_cast<const float*>(at(L.cn)) + (size_t)b * L.Kp;
+        a.caug = static_cast<const char*>(at(L.caug)) + (size_t)b * L.Kp * AUG_SLAB * 2;
         a.xn = nullptr;
         a.ids = ids_c;
         a.status = status;
@@ -281,7 +281,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
     FKM_TRY(launch_finalize(B, K, D, nullptr, nullptr, counts_acc, sums64, cur, nxt, counts,
                             static_cast<double*>(at(L.shiftk)), st));
     FKM_TRY(launch_prep_centroids(nxt, B, K, L.Kp, D, dtype, mvec, at(L.cq),
-                                  static_cast<float*>(at(L.cn)), st));
+                                  at(L.caug), st));
     if (tol > 0.0f) FKM_CUDA_TRY(cudaMemsetAsync(max_shift, 0, sizeof(double), st));
     FKM_TRY(launch_batch_reduce(B, K, static_cast<double*>(at(L.shiftk)), nullptr,
                                 tol > 0.0f ? max_shift : nullptr, st));

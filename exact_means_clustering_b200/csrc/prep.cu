@@ -8,13 +8,14 @@
 //    origin.
 //  prep_centroids: delta = fp32(c - m); q(delta) = delta rounded (RNE) to the
 //    points' 16-bit type, laid out [B, Kp, D] for TMA; and the norm term
-//    ||q(delta)||^2 + 2 m.q(delta) (fp64, rounded once).  The score
-//    norm - 2 x.q(delta) equals ||x - c_hat||^2 - ||x - m||^2 + ||m||^2... up
-//    to terms constant per point, with c_hat = m + q(delta): the argmin of
-//    ||x - c_hat||^2 ("Flash-KMeans：快速且内存高效精确K-Means聚类" summary,
-//    section 方法步骤详情 step (1), which precomputes the norms).  Padding rows
-//    k >= K get q = 0 and norm +inf so they never win the argmin.  For fp32
-//    points delta is split into bf16 hi and lo = bf16(delta - hi), rows
+//    n = ||q(delta)||^2 + 2 m.q(delta) (fp64), stored as the bias slab
+//    [-n/2 in three 16-bit parts, 0 x 13] that one extra tensor-core product
+//    adds to x.q(delta).  Up to terms constant per point, n - 2 x.q(delta) is
+//    ||x - c_hat||^2 with c_hat = m + q(delta), so the argmax of
+//    x.q(delta) - n/2 is the nearest centroid ("Flash-KMeans：快速且内存高效精确
+//    K-Means聚类" summary, section 方法步骤详情 step (1), which precomputes the
+//    norms).  Padding rows k >= K are zero (their columns are masked).  For
+//    fp32 points delta is split into bf16 hi and lo = bf16(delta - hi), rows
 //    [hi | lo], and the norm term uses the fp32 delta.
 //  points_prep: for fp32 points, the bf16 [hi | lo] split rows the tensor
 //    cores consume (each half padded to a multiple of 8 elements); optionally
@@ -59,10 +60,40 @@ __global__ void __launch_bounds__(1024) center_kernel(const float* __restrict__ 
   }
 }
 
+// v split into three 16-bit parts whose weighted sum is v to about 24 bits:
+// bf16 parts are successive residuals (weights 1, 1, 1); fp16 parts are scaled
+// by 2^-15, 2^-4, 2^7 (weights 2^15, 2^4, 2^-7) so |v| up to 2^31 stays in
+// range.  Parts below the type's smallest normal are flushed to zero so no
+// operand is subnormal.
+__device__ __forceinline__ void bias_parts(double v, bool f16, uint16_t out[3]) {
+  if (!f16) {
+    double r = v;
+    for (int i = 0; i < 3; ++i) {
+      __nv_bfloat16 q = __double2bfloat16(r);
+      float qf = __bfloat162float(q);
+      if (fabsf(qf) < 1.17549435e-38f) { q = __float2bfloat16_rn(0.0f); qf = 0.0f; }
+      out[i] = __bfloat16_as_ushort(q);
+      r -= (double)qf;
+    }
+  } else {
+    const double scale[3] = {1.0 / 32768.0, 1.0 / 16.0, 128.0};   // 1 / weight
+    double r = v;
+    for (int i = 0; i < 3; ++i) {
+      double t = r * scale[i];
+      t = fmin(fmax(t, -65504.0), 65504.0);
+      __half q = __double2half(t);
+      float qf = __half2float(q);
+      if (fabsf(qf) < 6.1035156e-5f) { q = __float2half_rn(0.0f); qf = 0.0f; }
+      out[i] = __half_as_ushort(q);
+      r -= (double)qf / scale[i];
+    }
+  }
+}
+
 // one warp per padded centroid row
 __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* __restrict__ m,
                                       int B, int K, int Kp, int D, int dtype,
-                                      void* __restrict__ cq, float* __restrict__ cn) {
+                                      void* __restrict__ cq, uint16_t* __restrict__ caug) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= (int64_t)B * Kp) return;
@@ -100,7 +131,11 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
     }
   }
   acc = warp_sum(acc);
-  if (lane == 0) cn[row] = real ? (float)acc : INFINITY;
+  // the bias slab: [-n/2 in three parts, 0 x 13]; padding rows are all zero
+  // (the assign kernel masks their columns)
+  uint16_t parts[3] = {0, 0, 0};
+  if (real) bias_parts(-0.5 * acc, dtype == FKM_F16, parts);
+  if (lane < AUG_SLAB) caug[row * AUG_SLAB + lane] = lane < 3 ? parts[lane] : (uint16_t)0;
 }
 
 // one warp per point row; xn[row] = ||x - m[batch]||^2 when m is given
@@ -159,13 +194,13 @@ __global__ void points_prep_kernel(const void* __restrict__ x, int64_t rows, int
 }  // namespace
 
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
-                                 float* m, void* cq, float* cn, cudaStream_t st) {
+                                 float* m, void* cq, void* caug, cudaStream_t st) {
   center_kernel<<<dim3((unsigned)B, (unsigned)ceil_div(D, 32)), 1024, 0, st>>>(centers, B, K, D,
                                                                               m);
   const int64_t rows = (int64_t)B * Kp;
   const int wpb = 8;
-  prep_centroids_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(centers, m, B, K, Kp,
-                                                                           D, dtype, cq, cn);
+  prep_centroids_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(
+      centers, m, B, K, Kp, D, dtype, cq, static_cast<uint16_t*>(caug));
   note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;

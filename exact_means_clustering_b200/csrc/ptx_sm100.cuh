@@ -194,6 +194,13 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return d;
 }
 
+// 3-input maximum (sm_100a).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ------------------------------------------------- UMMA descriptors (sm_100)
 // Shared-memory matrix descriptor, K-major operand in the 128-byte swizzle
 // layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B: rows of 128 B, 8-row
@@ -208,6 +215,18 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   d |= (uint64_t)(1024u >> 4) << 32;   // stride byte offset: 8 rows x 128 B
   d |= (uint64_t)1 << 46;              // descriptor version
   d |= (uint64_t)2 << 61;              // SWIZZLE_128B
+  return d;
+}
+
+// The same for a K-major operand in the 32-byte swizzle (one 16-element K
+// slab of 16-bit values per row): rows of 32 B, 8-row groups 256 B apart.
+__device__ __forceinline__ uint64_t umma_desc_sw32(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(16u >> 4) << 16;     // leading byte offset: unused for swizzled K-major
+  d |= (uint64_t)(256u >> 4) << 32;    // stride byte offset: 8 rows x 32 B
+  d |= (uint64_t)1 << 46;              // descriptor version
+  d |= (uint64_t)6 << 61;              // SWIZZLE_32B
   return d;
 }
 
