@@ -214,12 +214,13 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
   for (int s = 0; s < SEG_STAGES - 1; ++s) issue(s);
 
   double acc[E];
-  float acc32[E], chat[E];
+  float acc32[E], chat[E], nchat[E];   // nchat = -chat for the packed fast path
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     acc[e] = 0.0;
     acc32[e] = 0.0f;
     chat[e] = 0.0f;
+    nchat[e] = 0.0f;
   }
   double obj = 0.0;
   float obj32 = 0.0f;
@@ -230,6 +231,27 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
     issue(s + SEG_STAGES - 1);
     cp_async_wait_stages();   // step s has landed
     __syncwarp();
+    // Fast path: the keys are sorted, so when the first and the last row of
+    // the step belong to the current run every row does, and all lanes add
+    // their own row at once (packed fp32x2 adds and FMAs).
+    const int kfirst = kv[s * RPS].x, klast = kv[s * RPS + RPS - 1].x;
+    if (kfirst == cur && klast == cur) {
+      if (lane_has_vec) {
+        float f[E];
+        Vec<DT>::widen(ring[s % SEG_STAGES][lane], f);
+        float2 d2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          const float2 fe = make_float2(f[e], f[e + 1]);
+          const float2 a = __fadd2_rn(make_float2(acc32[e], acc32[e + 1]), fe);
+          acc32[e] = a.x;
+          acc32[e + 1] = a.y;
+          const float2 df = __fadd2_rn(fe, make_float2(nchat[e], nchat[e + 1]));
+          d2 = __ffma2_rn(df, df, d2);
+        }
+        obj32 += d2.x + d2.y;
+      }
+    } else {
 #pragma unroll
     for (int gg = 0; gg < RPS; ++gg) {
       const int kg = kv[s * RPS + gg].x;   // same address in every lane: broadcast
@@ -258,6 +280,8 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
 #pragma unroll
               for (int e = 0; e < E; ++e) chat[e] += mb[e];
             }
+#pragma unroll
+            for (int e = 0; e < E; ++e) nchat[e] = -chat[e];
           }
         }
       }
@@ -273,6 +297,7 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
         }
         obj32 += d2;
       }
+    }
     }
     if ((s & 15) == 15) {   // bound the fp32 partials to 16 rows per lane
 #pragma unroll
