@@ -1,6 +1,7 @@
 // C ABI of libfkm: argument validation, workspace layout, stream-ordered
 // launch sequences, the Lloyd loop and status reporting.  Every step of an
 // iteration runs in this library's kernels; there is no fallback path.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -152,8 +153,16 @@ fkm_status make_layout(int B, int N, int K, int D, int dtype, Layout* L) {
   l.vals0 = take(BN_ * 4);
   l.keys1 = take(BN_ * 4);
   l.vals1 = take(BN_ * 4);
-  l.hist = take((size_t)l.n_sort_tiles * RADIX_BINS * 4);
-  l.hist_part = take(argsort_scratch_words(l.n_sort) * 4);
+  l.count_sort = K <= CS_MAX_K;
+  {
+    size_t hw = (size_t)l.n_sort_tiles * RADIX_BINS, pw = argsort_scratch_words(l.n_sort);
+    if (l.count_sort) {
+      hw = std::max(hw, (size_t)cs_hist_words(B, N, K));
+      pw = std::max(pw, cs_scan_scratch_words(B, N, K));
+    }
+    l.hist = take(hw * 4);
+    l.hist_part = take(pw * 4);
+  }
   l.segstart = take(BK * 4);
   l.segend = take(BK * 4);
   l.sums64 = take(BK * D * 8);
@@ -253,14 +262,18 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   s.hist = w.at<uint32_t>(L.hist);
   s.hist_part = w.at<uint32_t>(L.hist_part);
   s.status = w.status();
-  FKM_TRY(launch_argsort_ids(s, st));
-  if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[2], st, cudaEventRecordExternal));
   const int BK = L.B * L.K;
   int32_t* segstart = w.at<int32_t>(L.segstart);
   int32_t* segend = w.at<int32_t>(L.segend);
-  FKM_TRY(launch_seg_bounds(s.keys_out, L.n_sort, BK, segstart, segend, st));
+  if (L.count_sort) {
+    FKM_TRY(launch_count_sort_ids(s, L.B, segstart, segend, st));
+  } else {
+    FKM_TRY(launch_argsort_ids(s, st));
+    FKM_TRY(launch_seg_bounds(s.keys_out, L.n_sort, BK, segstart, segend, st));
+  }
+  if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[2], st, cudaEventRecordExternal));
   if (obj) FKM_CUDA_TRY(cudaMemsetAsync(obj, 0, sizeof(double) * L.B, st));
-  FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK, segstart, segend,
+  FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK,
                         w.at<double>(L.sums64), next, false, obj_args(w, prev, obj), st));
   if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[3], st, cudaEventRecordExternal));
   FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64), prev,
@@ -455,7 +468,10 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
   FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, w.at<float>(L.mvec), w.at<void>(L.cq),
                                 w.at<void>(L.caug), st));
 
+  // kernel attributes are set here, before any stream capture
   FKM_TRY(assign_prepare());
+  FKM_TRY(segsum_prepare());
+  FKM_TRY(count_sort_prepare());
   const bool prof = g_prof.on.load();
   std::unique_lock<std::mutex> prof_lock(g_prof.mu, std::defer_lock);
   if (prof) {
@@ -550,16 +566,33 @@ fkm_status fkm_profile_read(double* stage_ms, long long* iterations, int reset) 
 
 long long fkm_kernel_launches(void) { return g_launches.load(); }
 
+// Scratch of fkm_argsort: histogram, scan scratch and (counting sort only)
+// segment bounds, in 4-byte words.
+static void argsort_ws_words(int64_t n, int n_keys, size_t* hist_w, size_t* part_w,
+                             size_t* bounds_w) {
+  const int64_t m = n > 0 ? n : 1;
+  *hist_w = (size_t)ceil_div(m, SORT_TILE) * RADIX_BINS;
+  *part_w = argsort_scratch_words(m);
+  *bounds_w = 0;
+  if (n_keys <= CS_MAX_K) {   // the one-pass counting sort of the Lloyd loop
+    *hist_w = std::max(*hist_w, (size_t)cs_hist_words(1, (int)m, n_keys));
+    *part_w = std::max(*part_w, cs_scan_scratch_words(1, (int)m, n_keys));
+    *bounds_w = 2 * (size_t)n_keys;
+  }
+}
+
 fkm_status fkm_argsort_workspace_size(int64_t n, int n_keys, size_t* bytes) {
   if (!bytes || n < 0 || n >= (int64_t(1) << 31) || n_keys < 1 || n_keys >= (1 << 30)) {
     set_error("invalid argsort size");
     return FKM_ERR_INVALID_ARG;
   }
-  const int64_t tiles = ceil_div(n > 0 ? n : 1, SORT_TILE);
+  size_t hist_w, part_w, bounds_w;
+  argsort_ws_words(n, n_keys, &hist_w, &part_w, &bounds_w);
   size_t off = 256;  // status
   off += 4 * (((size_t)n * 4 + 255) & ~size_t(255));
-  off += ((size_t)tiles * RADIX_BINS * 4 + 255) & ~size_t(255);
-  off += (argsort_scratch_words(n > 0 ? n : 1) * 4 + 255) & ~size_t(255);
+  off += (hist_w * 4 + 255) & ~size_t(255);
+  off += (part_w * 4 + 255) & ~size_t(255);
+  off += (bounds_w * 4 + 255) & ~size_t(255);
   *bytes = off;
   return FKM_OK;
 }
@@ -578,7 +611,10 @@ fkm_status fkm_argsort(const int32_t* keys, int64_t n, int n_keys, int32_t* idx,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* p = static_cast<char*>(ws);
   const size_t vec = ((size_t)n * 4 + 255) & ~size_t(255);
-  const int64_t tiles = ceil_div(n, SORT_TILE);
+  size_t hist_w, part_w, bounds_w;
+  argsort_ws_words(n, n_keys, &hist_w, &part_w, &bounds_w);
+  const size_t hist_b = (hist_w * 4 + 255) & ~size_t(255);
+  const size_t part_b = (part_w * 4 + 255) & ~size_t(255);
   SortArgs s;
   s.ids = keys;
   s.N = (int)n;
@@ -591,9 +627,13 @@ fkm_status fkm_argsort(const int32_t* keys, int64_t n, int n_keys, int32_t* idx,
   s.keys1 = reinterpret_cast<int32_t*>(p + 256 + 2 * vec);
   s.vals1 = reinterpret_cast<int32_t*>(p + 256 + 3 * vec);
   s.hist = reinterpret_cast<uint32_t*>(p + 256 + 4 * vec);
-  s.hist_part = reinterpret_cast<uint32_t*>(p + 256 + 4 * vec +
-                                            (((size_t)tiles * RADIX_BINS * 4 + 255) & ~size_t(255)));
-  FKM_TRY(launch_argsort_ids(s, st));
+  s.hist_part = reinterpret_cast<uint32_t*>(p + 256 + 4 * vec + hist_b);
+  if (bounds_w) {
+    int32_t* bounds = reinterpret_cast<int32_t*>(p + 256 + 4 * vec + hist_b + part_b);
+    FKM_TRY(launch_count_sort_ids(s, 1, bounds, bounds + n_keys, st));
+  } else {
+    FKM_TRY(launch_argsort_ids(s, st));
+  }
   FKM_CUDA_TRY(cudaMemcpyAsync(idx, s.vals_out, (size_t)n * 4, cudaMemcpyDeviceToDevice, st));
   if (sorted_keys)
     FKM_CUDA_TRY(

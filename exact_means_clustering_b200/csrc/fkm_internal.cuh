@@ -71,6 +71,7 @@ struct Layout {
   int64_t n_sort;  // B * N keys
   int n_sort_tiles;
   int key_bits;
+  bool count_sort;  // one-pass counting sort (K <= CS_MAX_K) instead of LSD radix
   size_t status, mvec, cq, caug, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
       segstart, segend, sums64, shiftk, cbuf, scal, total;
 };
@@ -126,6 +127,18 @@ struct SortArgs {
 fkm_status launch_argsort_ids(SortArgs& a, cudaStream_t st);
 size_t argsort_scratch_words(int64_t n);
 
+// One-pass counting sort of the same keys for K <= CS_MAX_K: rows of a batch
+// are contiguous, so per-batch stable sorts by id concatenate into the stable
+// sort by key.  Also writes segstart / segend ([B*K], positions in the sorted
+// order; equal for an empty cluster).  hist needs cs_hist_words(B, N, K)
+// words, hist_part argsort_scratch_words-style scan scratch for that length.
+constexpr int CS_MAX_K = 2048;
+int64_t cs_hist_words(int B, int N, int K);
+size_t cs_scan_scratch_words(int B, int N, int K);
+fkm_status launch_count_sort_ids(SortArgs& a, int B, int32_t* segstart, int32_t* segend,
+                                 cudaStream_t st);
+fkm_status count_sort_prepare();
+
 fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
                              int32_t* segend, cudaStream_t st);
 // Objective of the assignment being summed against c_hat, the centroid the
@@ -142,9 +155,11 @@ struct ObjArgs {
   double* obj = nullptr;
 };
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
-                         const int32_t* svals, int64_t n, int BK, const int32_t* segstart,
-                         const int32_t* segend, double* sums64, float* centers,
+                         const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
                          bool accumulate_all, const ObjArgs& oa, cudaStream_t st);
+// Raises the segment-sum kernels' dynamic shared-memory limit once per device
+// (outside any stream capture).
+fkm_status segsum_prepare();
 // Direct objective of a given assignment: obj[b] += sum_i ||x_i - chat_{ids_i}||^2.
 fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const int32_t* ids,
                             const ObjArgs& oa, cudaStream_t st);

@@ -269,7 +269,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
           oa.chat_bstride = 0;
           oa.m = mvec + (size_t)b * D;
         }
-        FKM_TRY(launch_segsum(xb, dtype, D, so.keys_out, so.vals_out, rows, K, segstart, segend,
+        FKM_TRY(launch_segsum(xb, dtype, D, so.keys_out, so.vals_out, rows, K,
                               sums64 + (size_t)b * K * D, nullptr, true, oa, st));
         accumulate_counts_kernel<<<(unsigned)ceil_div(K, 256), 256, 0, st>>>(
             segstart, segend, K, counts_acc + (size_t)b * K);

@@ -17,6 +17,15 @@
 // The first pass forms the keys from the ids on the fly and validates them:
 // an id outside [0, K) sets ST_BAD_ID and gets the sentinel key B*K, which
 // sorts after every real key.
+//
+// For K <= CS_MAX_K the Lloyd loop uses a one-pass counting sort instead.
+// The rows of batch b are contiguous, so the stable sort by b*K + id is the
+// concatenation of per-batch stable sorts by id: tiles of SORT_TILE rows that
+// never straddle a batch count their ids into K bins (plus one bin for
+// rejected ids), one exclusive scan over the bins in (batch, id, tile) order
+// gives every (id, tile) its output base, and a scatter pass ranks the keys
+// stably inside their tile.  The scanned bins are also the segment bounds of
+// every cluster, so no separate bounds pass is needed.
 #include "fkm_internal.cuh"
 
 namespace fkm {
@@ -239,6 +248,124 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_downsweep(KeySrc s, int64_
   }
 }
 
+// ---- one-pass counting sort ----
+struct CsArgs {
+  const int32_t* ids;
+  int B, N, K;
+  int tpb;               // tiles per batch
+  uint32_t* hist;        // [(b*K + k) * tpb + t], then [B*K*tpb + tile] rejected ids
+  int* status;
+  int32_t* keys_out;
+  int32_t* vals_out;
+  int32_t* segstart;
+  int32_t* segend;
+};
+
+// Tile histogram: bins 0..K-1 are the ids, bin K the rejected ids.
+__global__ void __launch_bounds__(SORT_THREADS) cs_hist_kernel(CsArgs a) {
+  extern __shared__ uint32_t h[];   // K + 1
+  const int tg = blockIdx.x, b = tg / a.tpb, t = tg % a.tpb;
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i <= a.K; i += SORT_THREADS) h[i] = 0;
+  __syncthreads();
+  const int64_t row0 = (int64_t)b * a.N + (int64_t)t * SORT_TILE;
+  const int nrows = (a.N - t * SORT_TILE) < SORT_TILE ? (a.N - t * SORT_TILE) : SORT_TILE;
+  int id[SORT_ITEMS];
+#pragma unroll
+  for (int it = 0; it < SORT_ITEMS; ++it) {
+    const int i = it * SORT_THREADS + threadIdx.x;
+    id[it] = i < nrows ? a.ids[row0 + i] : -2;
+  }
+  bool bad = false;
+#pragma unroll
+  for (int it = 0; it < SORT_ITEMS; ++it) {
+    const int i = it * SORT_THREADS + threadIdx.x;
+    int bin = a.K + 1;   // past the tile: counted nowhere
+    if (i < nrows) {
+      if (id[it] < 0 || id[it] >= a.K) {
+        bin = a.K;
+        bad = true;
+      } else {
+        bin = id[it];
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    if (bin <= a.K && lane == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(a.status, ST_BAD_ID);
+  for (int k = threadIdx.x; k < a.K; k += SORT_THREADS)
+    a.hist[((int64_t)b * a.K + k) * a.tpb + t] = h[k];
+  if (threadIdx.x == 0) a.hist[(int64_t)a.B * a.K * a.tpb + tg] = h[a.K];
+}
+
+// Stable scatter of one tile: warp w ranks rows [512 w, 512 w + 512) of the
+// tile in order with per-warp bin counters (match_any), the counters are
+// turned into output positions (scanned base + earlier warps' counts), and
+// every row writes its key and index.  Tile 0 of each batch also writes that
+// batch's segment bounds.
+__global__ void __launch_bounds__(SORT_THREADS) cs_scatter_kernel(CsArgs a) {
+  constexpr int NW = SORT_THREADS / 32;
+  constexpr int PER_WARP = SORT_TILE / NW;
+  extern __shared__ uint32_t cnt[];   // NW * (K + 1)
+  const int KB = a.K + 1;
+  const int tg = blockIdx.x, b = tg / a.tpb, t = tg % a.tpb;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < NW * KB; i += SORT_THREADS) cnt[i] = 0;
+  const int64_t row0 = (int64_t)b * a.N + (int64_t)t * SORT_TILE;
+  const int nrows = (a.N - t * SORT_TILE) < SORT_TILE ? (a.N - t * SORT_TILE) : SORT_TILE;
+  int bin[SORT_ITEMS];
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    const int i = warp * PER_WARP + r * 32 + lane;
+    bin[r] = a.K + 1;
+    if (i < nrows) {
+      const int id = a.ids[row0 + i];
+      bin[r] = (id < 0 || id >= a.K) ? a.K : id;
+    }
+  }
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  uint32_t* wc = cnt + warp * KB;
+  uint32_t rank[SORT_ITEMS];
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    const unsigned peers = __match_any_sync(0xffffffffu, bin[r]);
+    uint32_t before = 0;
+    if (bin[r] <= a.K) before = wc[bin[r]];
+    rank[r] = before + __popc(peers & lt_mask);
+    __syncwarp();
+    if (bin[r] <= a.K && lane == __ffs(peers) - 1) wc[bin[r]] = before + __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < KB; k += SORT_THREADS) {
+    uint32_t base = k < a.K ? a.hist[((int64_t)b * a.K + k) * a.tpb + t]
+                            : a.hist[(int64_t)a.B * a.K * a.tpb + tg];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t c = cnt[w * KB + k];
+      cnt[w * KB + k] = base;
+      base += c;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    if (bin[r] <= a.K) {
+      const uint32_t pos = wc[bin[r]] + rank[r];
+      a.keys_out[pos] = bin[r] < a.K ? b * a.K + bin[r] : a.B * a.K;
+      a.vals_out[pos] = (int32_t)(row0 + warp * PER_WARP + r * 32 + lane);
+    }
+  }
+  if (t == 0) {
+    for (int k = threadIdx.x; k < a.K; k += SORT_THREADS) {
+      const int64_t key = (int64_t)b * a.K + k;
+      a.segstart[key] = (int32_t)a.hist[key * a.tpb];
+      a.segend[key] = (int32_t)a.hist[(key + 1) * a.tpb];
+    }
+  }
+}
+
 fkm_status device_scan(uint32_t* data, int64_t len, uint32_t* part, cudaStream_t st) {
   const int64_t nparts = ceil_div(len, kScanChunk);
   scan_reduce<<<(unsigned)nparts, kScanBlock, 0, st>>>(data, len, part);
@@ -256,6 +383,57 @@ static_assert(SORT_THREADS == RADIX_BINS, "downsweep maps one thread per digit")
 size_t argsort_scratch_words(int64_t n) {
   const int64_t tiles = ceil_div(n, SORT_TILE);
   return (size_t)ceil_div(tiles * RADIX_BINS, kScanChunk) + 1;
+}
+
+int64_t cs_hist_words(int B, int N, int K) {
+  const int64_t tpb = ceil_div(N, SORT_TILE);
+  return (int64_t)B * K * tpb + (int64_t)B * tpb;
+}
+
+size_t cs_scan_scratch_words(int B, int N, int K) {
+  return (size_t)ceil_div(cs_hist_words(B, N, K), kScanChunk) + 1;
+}
+
+fkm_status count_sort_prepare() {
+  static bool done[64] = {false};
+  int dev = 0;
+  FKM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && done[dev]) return FKM_OK;
+  const int b = (SORT_THREADS / 32) * (CS_MAX_K + 1) * 4;
+  FKM_CUDA_TRY(cudaFuncSetAttribute(cs_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
+  if (dev >= 0 && dev < 64) done[dev] = true;
+  return FKM_OK;
+}
+
+fkm_status launch_count_sort_ids(SortArgs& s, int B, int32_t* segstart, int32_t* segend,
+                                 cudaStream_t st) {
+  if (s.K > CS_MAX_K || s.n != (int64_t)B * s.N) {
+    set_error("count sort: K = %d exceeds %d or n != B*N", s.K, CS_MAX_K);
+    return FKM_ERR_INTERNAL;
+  }
+  FKM_TRY(count_sort_prepare());
+  CsArgs a;
+  a.ids = s.ids;
+  a.B = B;
+  a.N = s.N;
+  a.K = s.K;
+  a.tpb = (int)ceil_div(s.N, SORT_TILE);
+  a.hist = s.hist;
+  a.status = s.status;
+  a.keys_out = s.keys0;
+  a.vals_out = s.vals0;
+  a.segstart = segstart;
+  a.segend = segend;
+  s.keys_out = s.keys0;
+  s.vals_out = s.vals0;
+  if (s.n == 0) return FKM_OK;
+  const unsigned tiles = (unsigned)((int64_t)B * a.tpb);
+  cs_hist_kernel<<<tiles, SORT_THREADS, (a.K + 1) * 4, st>>>(a);
+  FKM_TRY(device_scan(a.hist, cs_hist_words(B, s.N, s.K), s.hist_part, st));
+  cs_scatter_kernel<<<tiles, SORT_THREADS, (SORT_THREADS / 32) * (a.K + 1) * 4, st>>>(a);
+  note_launch(2);
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
 }
 
 // Sorts a.n keys formed from a.ids; leaves sorted keys / values in

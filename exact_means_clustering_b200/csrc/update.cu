@@ -50,8 +50,6 @@ struct SegParams {
   int BK;
   int64_t row_bytes;
   int V;                 // 16-byte vectors per row
-  const int32_t* segstart;
-  const int32_t* segend;
   double* sums64;
   float* centers;
   bool accumulate_all;   // out-of-core chunks: every run goes to sums64
@@ -109,11 +107,12 @@ __device__ __forceinline__ double warp_sum(double v) {
 
 // Flush of one run: the fp32 partial is folded into fp64, the partials are
 // summed over the row groups (xor shuffles), and group 0 writes either the
-// final centroid (run inside this range) or adds to the fp64 accumulators
-// (run crossing a range boundary).
+// final centroid (run inside this range, nk rows) or adds to the fp64
+// accumulators (run crossing a range boundary).
 template <int E, int LPR>
 __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, int sub,
-                                          bool lane_has_vec, double (&acc)[E], float (&acc32)[E]) {
+                                          bool lane_has_vec, bool interior, int nk,
+                                          double (&acc)[E], float (&acc32)[E]) {
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     acc[e] += (double)acc32[e];
@@ -124,15 +123,13 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
   if (g == 0 && lane_has_vec) {
-    const int32_t s = p.segstart[key], t = p.segend[key];
-    const bool interior = !p.accumulate_all && (s / SEG_RANGE) == ((t - 1) / SEG_RANGE);
     const int64_t col0 = (int64_t)sub * E;
     if (interior) {
-      const double nk = (double)(t - s);
+      const double n = (double)nk;
       float* c = p.centers + (int64_t)key * p.D + col0;
 #pragma unroll
       for (int e = 0; e < E; ++e)
-        if (col0 + e < p.D) c[e] = (float)(acc[e] / nk);
+        if (col0 + e < p.D) c[e] = (float)(acc[e] / n);
     } else {
       double* sd = p.sums64 + (int64_t)key * p.D + col0;
 #pragma unroll
@@ -144,8 +141,23 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
   for (int e = 0; e < E; ++e) acc[e] = 0.0;
 }
 
-constexpr int SEG_WARPS = 8;   // warps (ranges) per block
-constexpr int SEG_STAGES = 8;  // row-gather steps in flight per warp
+#ifndef FKM_SEG_STAGES
+#define FKM_SEG_STAGES 8
+#endif
+#ifndef FKM_SEG_MIN_BLOCKS
+#define FKM_SEG_MIN_BLOCKS 3
+#endif
+constexpr int SEG_WARPS = 8;                // warps (ranges) per block
+constexpr int SEG_STAGES = FKM_SEG_STAGES;  // row-gather steps in flight per warp
+
+// Per-warp shared memory: the range's (key, row) pairs, the start position of
+// every run (plus an end sentinel), and the gather ring.
+struct SegWarpSmem {
+  int2 kv[SEG_RANGE];
+  uint4 ring[SEG_STAGES][32];
+  int16_t runs[SEG_RANGE + 1];
+};
+constexpr size_t SEG_SMEM_BYTES = sizeof(SegWarpSmem) * SEG_WARPS;
 
 __device__ __forceinline__ void cp_async_16(void* smem, const void* gmem, bool valid) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -161,19 +173,24 @@ __device__ __forceinline__ void cp_async_wait_stages() {
 }
 
 // One warp per SEG_RANGE sorted rows.  The range's (key, row) pairs are
-// staged in shared memory first; then every lane gathers its 16-byte piece of
-// the rows RPS at a time (LPR = 32 / RPS lanes per row, lane `sub` holding
-// vector `sub` of its row) with cp.async into a per-warp ring of SEG_STAGES
-// steps, so SEG_STAGES * RPS rows are in flight while the warp adds the
-// oldest step.  Rows are added in fp32 and folded into fp64 at every run
-// flush and every 16 steps.
+// staged in shared memory first, together with the start of every run of
+// equal keys and the keys just outside the range, so a run's length and
+// whether it crosses the range boundary are known without touching global
+// memory.  Then every lane gathers its 16-byte piece of the rows RPS at a
+// time (LPR = 32 / RPS lanes per row, lane `sub` holding vector `sub` of its
+// row) with cp.async into a per-warp ring of SEG_STAGES steps, so
+// SEG_STAGES * RPS rows are in flight while the warp adds the oldest step.
+// Rows are added in fp32 and folded into fp64 at every run flush and every 16
+// steps.  For the objective, the centroid row of the next run is loaded when
+// the current run starts, so it has arrived by the time it is needed.
 template <int DT, int RPS>
-__global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) {
+__global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
+    segsum_kernel(SegParams p) {
   constexpr int E = Vec<DT>::E;
   constexpr int LPR = 32 / RPS;
-  __shared__ int2 kv_s[SEG_WARPS][SEG_RANGE];
-  __shared__ uint4 ring_s[SEG_WARPS][SEG_STAGES][32];
+  extern __shared__ __align__(16) uint8_t seg_smem[];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  SegWarpSmem& ws = reinterpret_cast<SegWarpSmem*>(seg_smem)[wid];
   const int g = lane / LPR, sub = lane % LPR;
   const bool lane_has_vec = sub < p.V;
   const bool want_obj = p.oa.obj != nullptr;
@@ -183,17 +200,44 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
   if (r >= nranges) return;
   const int64_t j0 = r * SEG_RANGE;
   const int nrows = (int)((j0 + SEG_RANGE < p.n) ? SEG_RANGE : p.n - j0);
-  int2* kv = kv_s[wid];
-  uint4 (*ring)[32] = ring_s[wid];
-  for (int i = lane; i < SEG_RANGE; i += 32) {
-    int2 e = make_int2(-1, 0);
+
+  // ---- staging: all loads first, then the stores
+  int2 e_[SEG_RANGE / 32];
+#pragma unroll
+  for (int t = 0; t < SEG_RANGE / 32; ++t) {
+    const int i = t * 32 + lane;
+    e_[t] = make_int2(-1, 0);
     if (i < nrows) {
-      e.x = p.skeys[j0 + i];
-      e.y = p.svals[j0 + i];
-      if (e.x >= p.BK) e.x = -1;   // rejected id: skip the row
+      e_[t].x = p.skeys[j0 + i];
+      e_[t].y = p.svals[j0 + i];
     }
-    kv[i] = e;
   }
+  int kedge = -1;   // lane 0: the key before the range; lane 1: the key after it
+  if (lane == 0 && j0 > 0) kedge = p.skeys[j0 - 1];
+  if (lane == 1 && j0 + nrows < p.n) kedge = p.skeys[j0 + nrows];
+#pragma unroll
+  for (int t = 0; t < SEG_RANGE / 32; ++t) {
+    if (e_[t].x >= p.BK) e_[t].x = -1;   // rejected id: skip the row
+    ws.kv[t * 32 + lane] = e_[t];
+  }
+  const int key_before = __shfl_sync(0xffffffffu, kedge, 0);
+  const int key_after = __shfl_sync(0xffffffffu, kedge, 1);
+  __syncwarp();
+  // run starts (ids that are rejected sort after every valid key, so the
+  // valid rows are a prefix of the range)
+  int nruns = 0, nvalid = 0;
+#pragma unroll
+  for (int t = 0; t < SEG_RANGE / 32; ++t) {
+    const int i = t * 32 + lane;
+    const int k = ws.kv[i].x;
+    const int kp = i > 0 ? ws.kv[i - 1].x : -1;
+    const bool start = k >= 0 && (i == 0 || k != kp);
+    const unsigned bal = __ballot_sync(0xffffffffu, start);
+    if (start) ws.runs[nruns + __popc(bal & ((1u << lane) - 1u))] = (int16_t)i;
+    nruns += __popc(bal);
+    nvalid += __popc(__ballot_sync(0xffffffffu, k >= 0));
+  }
+  if (lane == 0) ws.runs[nruns] = (int16_t)nvalid;
   __syncwarp();
 
   const char* xb = static_cast<const char*>(p.x) + (int64_t)sub * 16;
@@ -203,28 +247,46 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
     bool valid = false;
     const char* src = xb;
     if (s < nsteps && i < nrows) {
-      const int2 e = kv[i];
+      const int2 e = ws.kv[i];
       valid = e.x >= 0 && lane_has_vec;
       if (valid) src = xb + (int64_t)e.y * p.row_bytes;
     }
-    cp_async_16(&ring[s % SEG_STAGES][lane], src, valid);
+    cp_async_16(&ws.ring[s % SEG_STAGES][lane], src, valid);
     cp_async_commit();
   };
 #pragma unroll
   for (int s = 0; s < SEG_STAGES - 1; ++s) issue(s);
 
+  // centroid rows for the objective: raw 16-byte piece of the next run's row
+  uint4 chat_next = make_uint4(0, 0, 0, 0);
+  auto prefetch_chat = [&](int run) {
+    if (!want_obj || run >= nruns || !lane_has_vec) return;
+    const int kg = ws.kv[ws.runs[run]].x;
+    const int b = kg / p.oa.K, k = kg % p.oa.K;
+    const char* row = static_cast<const char*>(p.oa.chat) +
+                      ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.D) * elem_bytes_;
+    chat_next = ldg_nc_v4(row + (int64_t)sub * 16);
+  };
+  prefetch_chat(0);
+
   double acc[E];
-  float acc32[E], chat[E], nchat[E];   // nchat = -chat for the packed fast path
+  float acc32[E], chat[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     acc[e] = 0.0;
     acc32[e] = 0.0f;
     chat[e] = 0.0f;
-    nchat[e] = 0.0f;
   }
   double obj = 0.0;
   float obj32 = 0.0f;
-  int cur = -1, cur_b = -1;
+  int cur = -1, cur_b = -1, run = -1, run_start = 0;
+  const float2 neg1 = make_float2(-1.0f, -1.0f);
+  auto flush = [&](int run_end) {
+    const bool crossing = (run_start == 0 && key_before == cur) ||
+                          (run_end == nrows && key_after == cur);
+    flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, !p.accumulate_all && !crossing,
+                      run_end - run_start, acc, acc32);
+  };
 
 #pragma unroll 1
   for (int s = 0; s < nsteps; ++s) {
@@ -234,11 +296,11 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
     // Fast path: the keys are sorted, so when the first and the last row of
     // the step belong to the current run every row does, and all lanes add
     // their own row at once (packed fp32x2 adds and FMAs).
-    const int kfirst = kv[s * RPS].x, klast = kv[s * RPS + RPS - 1].x;
+    const int kfirst = ws.kv[s * RPS].x, klast = ws.kv[s * RPS + RPS - 1].x;
     if (kfirst == cur && klast == cur) {
       if (lane_has_vec) {
         float f[E];
-        Vec<DT>::widen(ring[s % SEG_STAGES][lane], f);
+        Vec<DT>::widen(ws.ring[s % SEG_STAGES][lane], f);
         float2 d2 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int e = 0; e < E; e += 2) {
@@ -246,58 +308,58 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
           const float2 a = __fadd2_rn(make_float2(acc32[e], acc32[e + 1]), fe);
           acc32[e] = a.x;
           acc32[e + 1] = a.y;
-          const float2 df = __fadd2_rn(fe, make_float2(nchat[e], nchat[e + 1]));
+          const float2 df = __ffma2_rn(make_float2(chat[e], chat[e + 1]), neg1, fe);
           d2 = __ffma2_rn(df, df, d2);
         }
         obj32 += d2.x + d2.y;
       }
     } else {
 #pragma unroll
-    for (int gg = 0; gg < RPS; ++gg) {
-      const int kg = kv[s * RPS + gg].x;   // same address in every lane: broadcast
-      if (kg < 0) continue;
-      if (kg != cur) {
-        if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc, acc32);
-        cur = kg;
-        if (want_obj) {
-          obj += (double)obj32;
-          obj32 = 0.0f;
-          const int b = kg / p.oa.K, k = kg % p.oa.K;
-          if (b != cur_b) {
-            if (cur_b >= 0) {
-              const double t = warp_sum(obj);
-              if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
+      for (int gg = 0; gg < RPS; ++gg) {
+        const int i = s * RPS + gg;
+        const int kg = ws.kv[i].x;   // same address in every lane: broadcast
+        if (kg < 0) continue;
+        if (kg != cur) {
+          if (cur >= 0) flush(i);
+          cur = kg;
+          ++run;
+          run_start = i;
+          if (want_obj) {
+            obj += (double)obj32;
+            obj32 = 0.0f;
+            const int b = kg / p.oa.K;
+            if (b != cur_b) {
+              if (cur_b >= 0) {
+                const double t = warp_sum(obj);
+                if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
+              }
+              obj = 0.0;
+              cur_b = b;
             }
-            obj = 0.0;
-            cur_b = b;
-          }
-          if (lane_has_vec) {
-            const char* row = static_cast<const char*>(p.oa.chat) +
-                              ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.D) * elem_bytes_;
-            Vec<DT>::widen(ldg_nc_v4(row + (int64_t)sub * 16), chat);
-            if (p.oa.m) {
-              const float* mb = p.oa.m + (int64_t)b * p.D + (int64_t)sub * E;
+            if (lane_has_vec) {
+              Vec<DT>::widen(chat_next, chat);
+              if (p.oa.m) {   // the batch's mean centroid: a few KB, cache-resident
+                const float* mb = p.oa.m + (int64_t)b * p.D + (int64_t)sub * E;
 #pragma unroll
-              for (int e = 0; e < E; ++e) chat[e] += mb[e];
+                for (int e = 0; e < E; ++e) chat[e] += mb[e];
+              }
             }
-#pragma unroll
-            for (int e = 0; e < E; ++e) nchat[e] = -chat[e];
+            prefetch_chat(run + 1);
           }
         }
-      }
-      if (g == gg && lane_has_vec) {
-        float f[E];
-        Vec<DT>::widen(ring[s % SEG_STAGES][lane], f);
-        float d2 = 0.0f;
+        if (g == gg && lane_has_vec) {
+          float f[E];
+          Vec<DT>::widen(ws.ring[s % SEG_STAGES][lane], f);
+          float d2 = 0.0f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-          acc32[e] += f[e];
-          const float df = f[e] - chat[e];
-          d2 = fmaf(df, df, d2);
+          for (int e = 0; e < E; ++e) {
+            acc32[e] += f[e];
+            const float df = f[e] - chat[e];
+            d2 = fmaf(df, df, d2);
+          }
+          obj32 += d2;
         }
-        obj32 += d2;
       }
-    }
     }
     if ((s & 15) == 15) {   // bound the fp32 partials to 16 rows per lane
 #pragma unroll
@@ -311,7 +373,7 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, 3) segsum_kernel(SegParams p) 
     __syncwarp();   // every lane is done with slot s before it is refilled
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
-  if (cur >= 0) flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, acc, acc32);
+  if (cur >= 0) flush(nvalid);
   if (want_obj && cur_b >= 0) {
     const double t = warp_sum(obj + (double)obj32);
     if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
@@ -375,7 +437,9 @@ struct FinParams {
   const int32_t* counts_in;  // out-of-core: accumulated counts (segstart/end unused)
 };
 
-// one warp per cluster
+// One warp per cluster.  When D is a multiple of 4 each lane moves four
+// consecutive elements per step (16-byte loads and stores), so a cluster of
+// D <= 128 takes one step.
 __global__ void finalize_kernel(FinParams p) {
   const int64_t key = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -391,21 +455,45 @@ __global__ void finalize_kernel(FinParams p) {
   }
   if (lane == 0 && p.counts) p.counts[key] = nk;
   double sh = 0.0;
-  for (int d = lane; d < p.D; d += 32) {
-    const int64_t e = key * p.D + d;
-    const float prev = p.prev[e];
-    float v;
-    if (nk == 0) {
-      v = prev;
-    } else if (interior) {
-      v = p.centers[e];
-    } else {
-      v = (float)(p.sums64[e] / (double)nk);
-      p.sums64[e] = 0.0;   // leave the accumulator clean for the next update
+  if ((p.D & 3) == 0) {
+    for (int d = 4 * lane; d < p.D; d += 128) {
+      const int64_t e = key * p.D + d;
+      const float4 pv = *reinterpret_cast<const float4*>(p.prev + e);
+      float4 v;
+      if (nk == 0) {
+        v = pv;
+      } else if (interior) {
+        v = *reinterpret_cast<const float4*>(p.centers + e);
+      } else {
+        double2* s2 = reinterpret_cast<double2*>(p.sums64 + e);
+        const double2 a = s2[0], b = s2[1];
+        const double n = (double)nk;
+        v = make_float4((float)(a.x / n), (float)(a.y / n), (float)(b.x / n), (float)(b.y / n));
+        s2[0] = make_double2(0.0, 0.0);   // leave the accumulator clean for the next update
+        s2[1] = make_double2(0.0, 0.0);
+      }
+      *reinterpret_cast<float4*>(p.centers + e) = v;
+      const double d0 = (double)v.x - (double)pv.x, d1 = (double)v.y - (double)pv.y;
+      const double d2 = (double)v.z - (double)pv.z, d3 = (double)v.w - (double)pv.w;
+      sh += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
     }
-    p.centers[e] = v;
-    const double df = (double)v - (double)prev;
-    sh += df * df;
+  } else {
+    for (int d = lane; d < p.D; d += 32) {
+      const int64_t e = key * p.D + d;
+      const float prev = p.prev[e];
+      float v;
+      if (nk == 0) {
+        v = prev;
+      } else if (interior) {
+        v = p.centers[e];
+      } else {
+        v = (float)(p.sums64[e] / (double)nk);
+        p.sums64[e] = 0.0;
+      }
+      p.centers[e] = v;
+      const double df = (double)v - (double)prev;
+      sh += df * df;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sh += __shfl_xor_sync(0xffffffffu, sh, o);
@@ -437,9 +525,21 @@ template <int DT, int RPS>
 fkm_status run_segsum(const SegParams& sp, cudaStream_t st) {
   const int64_t nranges = ceil_div(sp.n, SEG_RANGE);
   const int64_t blocks = ceil_div(nranges, SEG_WARPS);
-  segsum_kernel<DT, RPS><<<(unsigned)blocks, SEG_WARPS * 32, 0, st>>>(sp);
+  segsum_kernel<DT, RPS><<<(unsigned)blocks, SEG_WARPS * 32, SEG_SMEM_BYTES, st>>>(sp);
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+template <int DT>
+fkm_status set_segsum_smem() {
+  const int b = (int)SEG_SMEM_BYTES;
+  FKM_CUDA_TRY(cudaFuncSetAttribute(segsum_kernel<DT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(segsum_kernel<DT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(segsum_kernel<DT, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(segsum_kernel<DT, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(segsum_kernel<DT, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(segsum_kernel<DT, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
   return FKM_OK;
 }
 
@@ -459,6 +559,18 @@ fkm_status run_segsum_dt(const SegParams& sp, cudaStream_t st) {
 
 }  // namespace
 
+fkm_status segsum_prepare() {
+  static bool done[64] = {false};
+  int dev = 0;
+  FKM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && done[dev]) return FKM_OK;
+  FKM_TRY(set_segsum_smem<FKM_BF16>());
+  FKM_TRY(set_segsum_smem<FKM_F16>());
+  FKM_TRY(set_segsum_smem<FKM_F32>());
+  if (dev >= 0 && dev < 64) done[dev] = true;
+  return FKM_OK;
+}
+
 fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
                              int32_t* segend, cudaStream_t st) {
   FKM_CUDA_TRY(cudaMemsetAsync(segstart, 0, sizeof(int32_t) * (size_t)BK, st));
@@ -472,10 +584,10 @@ fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* s
 }
 
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
-                         const int32_t* svals, int64_t n, int BK, const int32_t* segstart,
-                         const int32_t* segend, double* sums64, float* centers,
+                         const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
                          bool accumulate_all, const ObjArgs& oa, cudaStream_t st) {
   if (n == 0) return FKM_OK;
+  FKM_TRY(segsum_prepare());
   SegParams sp;
   sp.x = x;
   sp.skeys = skeys;
@@ -485,8 +597,6 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
   sp.BK = BK;
   sp.row_bytes = (int64_t)D * elem_bytes(dtype);
   sp.V = (int)(sp.row_bytes / 16);
-  sp.segstart = segstart;
-  sp.segend = segend;
   sp.sums64 = sums64;
   sp.centers = centers;
   sp.accumulate_all = accumulate_all;

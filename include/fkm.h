@@ -156,7 +156,10 @@ FKM_API fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const v
  * equal keys in index order ("Flash-KMeans：快速且内存高效精确K-Means聚类" summary,
  * section 前置知识 / argsort与分段规约, example [3,1,2,1,3,2] -> [1,3,2,5,0,4]).
  * keys, idx: device int32 [n]; workspace from fkm_argsort_workspace_size.
- * A key outside [0, n_keys) sets FKM_ERR_BAD_ID in the status word.  Async. */
+ * n_keys <= 2048 takes the one-pass counting sort that fkm_update and
+ * fkm_lloyd use for K <= 2048; larger key ranges take the LSD radix sort
+ * (8-bit digits) used for larger K.  A key outside [0, n_keys) sorts after
+ * every valid key and sets FKM_ERR_BAD_ID in the status word.  Async. */
 FKM_API fkm_status fkm_argsort_workspace_size(int64_t n, int n_keys, size_t* bytes);
 FKM_API fkm_status fkm_argsort(const int32_t* keys, int64_t n, int n_keys, int32_t* idx,
                        int32_t* sorted_keys, void* ws, size_t ws_bytes, void* stream);

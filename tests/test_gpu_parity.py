@@ -50,7 +50,9 @@ def test_argsort_pages_example(golden_dir):
     assert sk.tolist() == g["sorted_keys"]
 
 
+# n_keys <= 2048 takes the one-pass counting sort, larger the LSD radix sort
 @pytest.mark.parametrize("n,n_keys", [(1, 1), (4096, 7), (3 * 4096 + 77, 300),
+                                      (2 * 4096 + 5, 2048), (2 * 4096 + 5, 2049),
                                       (100003, 40000), (70001, 70000), (50000, 1)])
 def test_argsort_matches_oracle(n, n_keys):
     rng = np.random.default_rng(n + n_keys)
