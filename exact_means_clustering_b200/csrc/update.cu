@@ -60,6 +60,12 @@ struct SegParams {
 template <int DT> struct Vec;
 template <> struct Vec<FKM_BF16> {
   static constexpr int E = 8;
+  __device__ static void widen2(const uint4& v, float2* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  }
   __device__ static void widen(const uint4& v, float* f) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -71,6 +77,11 @@ template <> struct Vec<FKM_BF16> {
 };
 template <> struct Vec<FKM_F16> {
   static constexpr int E = 8;
+  __device__ static void widen2(const uint4& v, float2* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+  }
   __device__ static void widen(const uint4& v, float* f) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -83,6 +94,10 @@ template <> struct Vec<FKM_F16> {
 };
 template <> struct Vec<FKM_F32> {
   static constexpr int E = 4;
+  __device__ static void widen2(const uint4& v, float2* f) {
+    f[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+    f[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+  }
   __device__ static void widen(const uint4& v, float* f) {
     f[0] = __uint_as_float(v.x);
     f[1] = __uint_as_float(v.y);
@@ -105,19 +120,14 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
-// Flush of one run: the fp32 partial is folded into fp64, the partials are
-// summed over the row groups (xor shuffles), and group 0 writes either the
-// final centroid (run inside this range, nk rows) or adds to the fp64
-// accumulators (run crossing a range boundary).
+// Flush of one run (its fp32 partials already folded into acc): the
+// partials are summed over the row groups (xor shuffles), and group 0 writes
+// either the final centroid (run inside this range, nk rows) or adds to the
+// fp64 accumulators (run crossing a range boundary).
 template <int E, int LPR>
 __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, int sub,
                                           bool lane_has_vec, bool interior, int nk,
-                                          double (&acc)[E], float (&acc32)[E]) {
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    acc[e] += (double)acc32[e];
-    acc32[e] = 0.0f;
-  }
+                                          double (&acc)[E]) {
 #pragma unroll
   for (int o = LPR; o < 32; o <<= 1)
 #pragma unroll
@@ -142,19 +152,27 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
 }
 
 #ifndef FKM_SEG_STAGES
-#define FKM_SEG_STAGES 8
+#define FKM_SEG_STAGES 4
 #endif
 #ifndef FKM_SEG_MIN_BLOCKS
 #define FKM_SEG_MIN_BLOCKS 3
 #endif
+#ifndef FKM_SEG_PREFETCH
+#define FKM_SEG_PREFETCH 0
+#endif
 constexpr int SEG_WARPS = 8;                // warps (ranges) per block
 constexpr int SEG_STAGES = FKM_SEG_STAGES;  // row-gather steps in flight per warp
+static_assert((SEG_STAGES & (SEG_STAGES - 1)) == 0, "the ring index is a mask");
+// When non-zero, the rows of step s + SEG_PREFETCH are prefetched into L2
+// (one prefetch per 128-byte line) while step s is added.
+constexpr int SEG_PREFETCH = FKM_SEG_PREFETCH;
 
 // Per-warp shared memory: the range's (key, row) pairs, the start position of
 // every run (plus an end sentinel), and the gather ring.
 struct SegWarpSmem {
-  int2 kv[SEG_RANGE];
+  int2 kv[SEG_RANGE + 1];   // + a (-1, 0) sentinel read by gathers past the range
   uint4 ring[SEG_STAGES][32];
+  double2 acc[4][32];   // per lane fp64 sums of its vector: [element pair][lane]
   int16_t runs[SEG_RANGE + 1];
 };
 constexpr size_t SEG_SMEM_BYTES = sizeof(SegWarpSmem) * SEG_WARPS;
@@ -220,6 +238,7 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     if (e_[t].x >= p.BK) e_[t].x = -1;   // rejected id: skip the row
     ws.kv[t * 32 + lane] = e_[t];
   }
+  if (lane == 0) ws.kv[SEG_RANGE] = make_int2(-1, 0);
   const int key_before = __shfl_sync(0xffffffffu, kedge, 0);
   const int key_after = __shfl_sync(0xffffffffu, kedge, 1);
   __syncwarp();
@@ -242,18 +261,28 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
 
   const char* xb = static_cast<const char*>(p.x) + (int64_t)sub * 16;
   const int nsteps = (nrows + RPS - 1) / RPS;
-  auto issue = [&](int s) {   // gather step s into ring slot s % SEG_STAGES
-    const int i = s * RPS + g;
-    bool valid = false;
-    const char* src = xb;
-    if (s < nsteps && i < nrows) {
-      const int2 e = ws.kv[i];
-      valid = e.x >= 0 && lane_has_vec;
-      if (valid) src = xb + (int64_t)e.y * p.row_bytes;
-    }
-    cp_async_16(&ws.ring[s % SEG_STAGES][lane], src, valid);
+  // Gather step s into ring slot s % SEG_STAGES.  Rows past the range read
+  // the (-1, 0) entries (the staged tail and the sentinel), so the copy is a
+  // zero fill from a valid address; so is the copy of a lane past the row's
+  // last vector.  Each lane reads back only the piece it copied itself, so
+  // the ring needs no warp barrier.
+  const int novec = lane_has_vec ? 0 : (int)0x80000000;
+  const int rb = (int)p.row_bytes;
+  auto issue = [&](int s) {
+    const int i = min(s * RPS + g, SEG_RANGE);
+    const int2 e = ws.kv[i];
+    cp_async_16(&ws.ring[s & (SEG_STAGES - 1)][lane], xb + (int64_t)e.y * rb, (e.x | novec) >= 0);
     cp_async_commit();
   };
+  auto prefetch = [&](int s) {
+    const int i = min(s * RPS + g, SEG_RANGE);
+    if (SEG_PREFETCH > 0 && (sub & 7) == 0 && lane_has_vec) {
+      const int2 e = ws.kv[i];
+      if (e.x >= 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(xb + (int64_t)e.y * rb));
+    }
+  };
+#pragma unroll 1
+  for (int s = 0; s < SEG_PREFETCH; ++s) prefetch(s);
 #pragma unroll
   for (int s = 0; s < SEG_STAGES - 1; ++s) issue(s);
 
@@ -269,51 +298,101 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
   };
   prefetch_chat(0);
 
-  double acc[E];
-  float acc32[E], chat[E];
+  // Lanes without a vector of the row (sub >= V) gather zeros and keep a zero
+  // centroid piece, so they add nothing and need no test on the hot path.
+  // fp64 sums live in shared memory (registers hold the fp32 partials)
+  float2 acc2[E / 2], chat2[E / 2];
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    acc[e] = 0.0;
-    acc32[e] = 0.0f;
-    chat[e] = 0.0f;
+  for (int e = 0; e < E / 2; ++e) {
+    acc2[e] = make_float2(0.0f, 0.0f);
+    chat2[e] = make_float2(0.0f, 0.0f);
+    ws.acc[e][lane] = make_double2(0.0, 0.0);
   }
+  float2 obj2 = make_float2(0.0f, 0.0f);
   double obj = 0.0;
-  float obj32 = 0.0f;
-  int cur = -1, cur_b = -1, run = -1, run_start = 0;
+  int cur = -1, cur_b = -1, run = -1, run_start = 0, run_end = 0, since_fold = 0;
   const float2 neg1 = make_float2(-1.0f, -1.0f);
-  auto flush = [&](int run_end) {
+  auto fold_obj = [&]() {
+    obj += (double)obj2.x + (double)obj2.y;
+    obj2 = make_float2(0.0f, 0.0f);
+  };
+  // the fp32 partials hold at most 16 rows per lane before going to fp64
+  auto fold = [&]() {
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      double2 a = ws.acc[e][lane];
+      a.x += (double)acc2[e].x;
+      a.y += (double)acc2[e].y;
+      ws.acc[e][lane] = a;
+      acc2[e] = make_float2(0.0f, 0.0f);
+    }
+    fold_obj();
+    since_fold = 0;
+  };
+  // one row of the current run: this lane's vector of it
+  auto add_row = [&](const uint4& v) {
+    float2 f[E / 2];
+    Vec<DT>::widen2(v, f);
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      acc2[e] = __fadd2_rn(acc2[e], f[e]);
+      const float2 df = __ffma2_rn(chat2[e], neg1, f[e]);
+      obj2 = __ffma2_rn(df, df, obj2);
+    }
+  };
+  auto flush = [&](int end) {
+    fold();
     const bool crossing = (run_start == 0 && key_before == cur) ||
-                          (run_end == nrows && key_after == cur);
+                          (end == nrows && key_after == cur);
+    double acc[E];
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      const double2 a = ws.acc[e][lane];
+      acc[2 * e] = a.x;
+      acc[2 * e + 1] = a.y;
+      ws.acc[e][lane] = make_double2(0.0, 0.0);
+    }
     flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, !p.accumulate_all && !crossing,
-                      run_end - run_start, acc, acc32);
+                      end - run_start, acc);
+  };
+  auto start_run = [&](int kg, int i) {
+    cur = kg;
+    ++run;
+    run_start = i;
+    run_end = ws.runs[run + 1];
+    if (!want_obj) return;
+    fold_obj();
+    const int b = kg / p.oa.K;
+    if (b != cur_b) {
+      if (cur_b >= 0) {
+        const double t = warp_sum(obj);
+        if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
+      }
+      obj = 0.0;
+      cur_b = b;
+    }
+    if (lane_has_vec) {
+      float2 c2[E / 2];
+      Vec<DT>::widen2(chat_next, c2);
+      if (p.oa.m) {   // the batch's mean centroid: a few KB, cache-resident
+        const float2* mb = reinterpret_cast<const float2*>(p.oa.m + (int64_t)b * p.D) + sub * (E / 2);
+#pragma unroll
+        for (int e = 0; e < E / 2; ++e) c2[e] = __fadd2_rn(c2[e], mb[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < E / 2; ++e) chat2[e] = c2[e];
+    }
+    prefetch_chat(run + 1);
   };
 
+  int s = 0;
 #pragma unroll 1
-  for (int s = 0; s < nsteps; ++s) {
+  while (s < nsteps) {
+    // a general step: the rows may start new runs
     issue(s + SEG_STAGES - 1);
     cp_async_wait_stages();   // step s has landed
-    __syncwarp();
-    // Fast path: the keys are sorted, so when the first and the last row of
-    // the step belong to the current run every row does, and all lanes add
-    // their own row at once (packed fp32x2 adds and FMAs).
-    const int kfirst = ws.kv[s * RPS].x, klast = ws.kv[s * RPS + RPS - 1].x;
-    if (kfirst == cur && klast == cur) {
-      if (lane_has_vec) {
-        float f[E];
-        Vec<DT>::widen(ws.ring[s % SEG_STAGES][lane], f);
-        float2 d2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int e = 0; e < E; e += 2) {
-          const float2 fe = make_float2(f[e], f[e + 1]);
-          const float2 a = __fadd2_rn(make_float2(acc32[e], acc32[e + 1]), fe);
-          acc32[e] = a.x;
-          acc32[e + 1] = a.y;
-          const float2 df = __ffma2_rn(make_float2(chat[e], chat[e + 1]), neg1, fe);
-          d2 = __ffma2_rn(df, df, d2);
-        }
-        obj32 += d2.x + d2.y;
-      }
-    } else {
+    {
+      const uint4 v = ws.ring[s & (SEG_STAGES - 1)][lane];
 #pragma unroll
       for (int gg = 0; gg < RPS; ++gg) {
         const int i = s * RPS + gg;
@@ -321,61 +400,30 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
         if (kg < 0) continue;
         if (kg != cur) {
           if (cur >= 0) flush(i);
-          cur = kg;
-          ++run;
-          run_start = i;
-          if (want_obj) {
-            obj += (double)obj32;
-            obj32 = 0.0f;
-            const int b = kg / p.oa.K;
-            if (b != cur_b) {
-              if (cur_b >= 0) {
-                const double t = warp_sum(obj);
-                if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
-              }
-              obj = 0.0;
-              cur_b = b;
-            }
-            if (lane_has_vec) {
-              Vec<DT>::widen(chat_next, chat);
-              if (p.oa.m) {   // the batch's mean centroid: a few KB, cache-resident
-                const float* mb = p.oa.m + (int64_t)b * p.D + (int64_t)sub * E;
-#pragma unroll
-                for (int e = 0; e < E; ++e) chat[e] += mb[e];
-              }
-            }
-            prefetch_chat(run + 1);
-          }
+          start_run(kg, i);
         }
-        if (g == gg && lane_has_vec) {
-          float f[E];
-          Vec<DT>::widen(ws.ring[s % SEG_STAGES][lane], f);
-          float d2 = 0.0f;
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            acc32[e] += f[e];
-            const float df = f[e] - chat[e];
-            d2 = fmaf(df, df, d2);
-          }
-          obj32 += d2;
-        }
+        if (g == gg) add_row(v);
       }
     }
-    if ((s & 15) == 15) {   // bound the fp32 partials to 16 rows per lane
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        acc[e] += (double)acc32[e];
-        acc32[e] = 0.0f;
-      }
-      obj += (double)obj32;
-      obj32 = 0.0f;
+    if (++since_fold == 16) fold();
+    ++s;
+    // the steps that lie wholly inside the current run: keys sorted, so no
+    // per-row test is needed
+    const int s_end = cur >= 0 ? min(nsteps, run_end / RPS) : s;
+#pragma unroll 1
+    while (s < s_end) {
+      issue(s + SEG_STAGES - 1);
+      cp_async_wait_stages();
+      add_row(ws.ring[s & (SEG_STAGES - 1)][lane]);
+      if (++since_fold == 16) fold();
+      ++s;
     }
-    __syncwarp();   // every lane is done with slot s before it is refilled
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   if (cur >= 0) flush(nvalid);
   if (want_obj && cur_b >= 0) {
-    const double t = warp_sum(obj + (double)obj32);
+    fold_obj();
+    const double t = warp_sum(obj);
     if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
   }
 }
