@@ -181,6 +181,19 @@ def oracle_sample(w, iters, rows=None):
     return dt, scale, desc
 
 
+def cpu_baseline(w, max_iters, budget_s=15.0):
+    """The oracle's iteration rate on a bounded sample of the workload: a probe
+    on a few thousand points of batch 0 sizes the sample (points of batch 0,
+    and iterations up to max_iters) to about budget_s seconds of CPU work."""
+    probe_rows = max(w.K, min(w.N, 4096))
+    t_probe, _, _ = oracle_sample(w, 1, probe_rows)
+    per_row = max(t_probe, 1e-6) / probe_rows
+    rows = int(min(w.N, max(probe_rows, budget_s / per_row)))
+    iters = int(max(1, min(max_iters, budget_s / (per_row * rows))))
+    dt, scale, desc = oracle_sample(w, iters, rows)
+    return iters / (dt * scale), desc
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -212,6 +225,149 @@ def run_reference(args, w):
     return 0
 
 
+HOST_CHUNK_ROWS = 1 << 23   # rows per streamed chunk of the host-resident workload
+
+
+def measure_h2d_gbs(torch, dev, nbytes=1 << 30):
+    """Pinned host -> device copy bandwidth (best of 5, CUDA events)."""
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    best = float("inf")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(6):
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        best = min(best, e0.elapsed_time(e1))
+    return nbytes / (best / 1e3) / 1e9
+
+
+def run_host(args, w):
+    """The host-resident workload: points stay in pinned host memory and every
+    iteration streams them through the GPU in chunks (fkm_lloyd_host).  Its
+    bound is the host link, so the roofline is taken against the measured
+    pinned host-to-device bandwidth."""
+    import torch
+    import exact_means_clustering_b200 as fkm
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=dev)
+    wr = w.scaled(seed=w.seed + 1000 * rank)
+    B, N, D, K = wr.B, wr.N, wr.D, wr.K
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wr.dtype]
+    xh = torch.empty((B, N, D), dtype=tdt, pin_memory=True)
+    for b in range(B):
+        datagen.fill_points(wr, b, xh[b].data_ptr())
+    xv = xh.view(torch.int16).numpy().view(np.uint16) if wr.dtype == "bf16" else xh.numpy()
+    c0 = datagen.init_centroids(xv, datagen.init_indices(wr), wr.dtype)
+    ch = torch.from_numpy(c0).pin_memory()
+    c0t = ch.to(dev)
+    ids = torch.empty(B, N, dtype=torch.int32, device=dev)
+    centers = torch.empty(B, K, D, dtype=torch.float32, device=dev)
+    counts = torch.empty(B, K, dtype=torch.int32, device=dev)
+    inertia = torch.empty(B, dtype=torch.float64, device=dev)
+    ws = fkm.workspace(fkm.fkm_host_workspace_size(B, N, K, D, tdt, HOST_CHUNK_ROWS), dev)
+    stream = torch.cuda.current_stream(dev)
+    h2d = measure_h2d_gbs(torch, dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        h0 = time.time()
+        e0.record(stream)
+        n = 0
+        for _ in range(args.steps):
+            n += fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        h1 = time.time()
+        barrier()
+        t = e0.elapsed_time(e1)
+        if dist is not None:
+            tt = torch.tensor([t], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t = tt.item()
+            nn = torch.tensor([n], device=dev, dtype=torch.float64)
+            dist.all_reduce(nn, op=dist.ReduceOp.SUM)
+            n = int(nn.item())
+        return n, t, (h0, h1)
+
+    def step():
+        return fkm.fkm_lloyd_host(xh, c0t, wr.iters, wr.tol, HOST_CHUNK_ROWS, ids, centers,
+                                  counts, inertia, ws=ws, stream=stream)
+
+    launches0 = fkm.fkm_kernel_launches()
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        n_it, t_ms, (h0, h1) = timed(step)
+        clk.window(h0, h1)
+    launches = (fkm.fkm_kernel_launches() - launches0) / max(args.steps + args.warmup, 1) \
+        * args.steps
+    value = n_it / (t_ms / 1e3)
+    per_iter_s = (t_ms / 1e3) / max(n_it / world, 1)
+    x_bytes = wr.x_bytes
+    achieved = x_bytes / per_iter_s / 1e9
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wr.dtype, "data": "synthetic",
+            "config": dict(workload_config(wr), chunk_rows=HOST_CHUNK_ROWS,
+                           l2=f"points stream from pinned host memory "
+                              f"({x_bytes / 2**30:.0f} GiB per iteration), no flush"),
+            "roofline": {"bound": "h2d", "kernel": "whole iteration (host link)",
+                         "achieved": achieved, "peak": h2d, "unit": "GB/s",
+                         "frac": achieved / h2d, "traffic": None,
+                         "peak_source": "measured pinned host-to-device copy, 1 GiB, this run"},
+            "gpu_launches": int(launches),
+            "clocks": clk.summary()}
+    if not args.no_e2e:
+        ids_h = torch.empty(B, N, dtype=torch.int32).pin_memory()
+        cen_h = torch.empty(B, K, D, dtype=torch.float32).pin_memory()
+        ine_h = torch.empty(B, dtype=torch.float64).pin_memory()
+
+        def e2e_step():
+            c0t.copy_(ch, non_blocking=True)
+            n = step()
+            ids_h.copy_(ids, non_blocking=True)
+            cen_h.copy_(centers, non_blocking=True)
+            ine_h.copy_(inertia, non_blocking=True)
+            return n
+
+        n_e, t_e, _ = timed(e2e_step)
+        line["e2e"] = {"value": n_e / (t_e / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": int(wr.iters * x_bytes + ch.numel() * 4),
+                       "d2h_bytes_per_step": int(ids_h.numel() * 4 + cen_h.numel() * 4
+                                                 + ine_h.numel() * 8)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        value_c, desc = cpu_baseline(wr, 1)
+        line["cpu_baseline"] = {"value": value_c, "unit": UNIT, "cores": cpu_cores(),
+                                "kind": "oracle", "sample": desc}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -231,9 +387,7 @@ def main():
     if args.impl == "reference":
         return run_reference(args, w)
     if w.host_resident:
-        print(json.dumps({"error": "use --config 1..4; the host-resident workload is timed by "
-                                   "bench_host (fkm_lloyd_host)"}))
-        return 2
+        return run_host(args, w)
 
     import torch
     import exact_means_clustering_b200 as fkm
@@ -390,9 +544,9 @@ def main():
 
     # --- the oracle on this host's cores (rank 0, one GPU only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, scale, desc = oracle_sample(wr, args.oracle_iters)
-        line["cpu_baseline"] = {"value": args.oracle_iters / (dt * scale), "unit": UNIT,
-                                "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+        value_c, desc = cpu_baseline(wr, args.oracle_iters)
+        line["cpu_baseline"] = {"value": value_c, "unit": UNIT, "cores": cpu_cores(),
+                                "kind": "oracle", "sample": desc}
 
     if dist is not None:
         dist.barrier()

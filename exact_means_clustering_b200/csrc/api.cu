@@ -71,6 +71,18 @@ static fkm_status prof_reserve(int iters) {
 }
 
 
+// A stage boundary: inside a stream capture the record must become a graph
+// node (cudaEventRecordExternal); outside one a plain record is required.
+static fkm_status record_stage(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  FKM_CUDA_TRY(cudaStreamIsCapturing(st, &cs));
+  if (cs == cudaStreamCaptureStatusActive)
+    FKM_CUDA_TRY(cudaEventRecordWithFlags(e, st, cudaEventRecordExternal));
+  else
+    FKM_CUDA_TRY(cudaEventRecord(e, st));
+  return FKM_OK;
+}
+
 static void prof_collect(int iters) {
   for (int t = 0; t < iters; ++t) {
     cudaEvent_t* e = &g_prof.ev[(size_t)t * 5];
@@ -271,11 +283,11 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
     FKM_TRY(launch_argsort_ids(s, st));
     FKM_TRY(launch_seg_bounds(s.keys_out, L.n_sort, BK, segstart, segend, st));
   }
-  if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[2], st, cudaEventRecordExternal));
+  if (ev) FKM_TRY(record_stage(ev[2], st));
   if (obj) FKM_CUDA_TRY(cudaMemsetAsync(obj, 0, sizeof(double) * L.B, st));
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK,
                         w.at<double>(L.sums64), next, false, obj_args(w, prev, obj), st));
-  if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[3], st, cudaEventRecordExternal));
+  if (ev) FKM_TRY(record_stage(ev[3], st));
   FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64), prev,
                           next, counts, w.at<double>(L.shiftk), st));
   // the next assign's operands: offsets of the new centroids from their mean
@@ -341,14 +353,14 @@ static fkm_status lloyd_iterations(const Ws& w, const void* x, int iters, int32_
     float* cur = (t & 1) ? cB : cA;
     float* nxt = (t & 1) ? cA : cB;
     cudaEvent_t* ev = ev_base ? ev_base + (size_t)t * 5 : nullptr;
-    if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[0], st, cudaEventRecordExternal));
+    if (ev) FKM_TRY(record_stage(ev[0], st));
     FKM_TRY(step_assign(w, x, ids, st));
-    if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[1], st, cudaEventRecordExternal));
+    if (ev) FKM_TRY(record_stage(ev[1], st));
     FKM_TRY(step_update(w, x, ids, cur, nxt, counts, true, inertia, st, ev));
     if (track_max) FKM_CUDA_TRY(cudaMemsetAsync(w.max_shift(), 0, sizeof(double), st));
     FKM_TRY(launch_batch_reduce(L.B, L.K, w.at<double>(L.shiftk), shift_dev,
                                 track_max ? w.max_shift() : nullptr, st));
-    if (ev) FKM_CUDA_TRY(cudaEventRecordWithFlags(ev[4], st, cudaEventRecordExternal));
+    if (ev) FKM_TRY(record_stage(ev[4], st));
   }
   return FKM_OK;
 }

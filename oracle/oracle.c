@@ -49,6 +49,7 @@
  * segmented reduction), which works the example [3,1,2,1,3,2]].
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -226,15 +227,21 @@ int orc_update(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xd
       if (k < 0 || k >= K) { free(n); free(s); return -1; }
       n[b * K + k] += 1;
     }
-  /* sums: every element summed over its cluster's points in index order;
-   * the (b, d) pairs are independent, so they run in parallel. */
-#pragma omp parallel for collapse(2) schedule(static)
-  for (int64_t b = 0; b < B; ++b)
-    for (int64_t d = 0; d < D; ++d)
+  /* sums: every element summed over its cluster's points in index order.
+   * Clusters are independent: thread t of T owns the clusters with
+   * k % T == t and walks the points in index order adding only the rows of
+   * its own clusters, so every row of x is read once, by one thread. */
+#pragma omp parallel
+  {
+    const int64_t T = omp_get_num_threads(), t = omp_get_thread_num();
+    for (int64_t b = 0; b < B; ++b)
       for (int64_t i = 0; i < N; ++i) {
-        int64_t k = ids[b * N + i];
-        s[(b * K + k) * D + d] += orc_read(x, xdt, (b * N + i) * D + d);
+        const int64_t k = ids[b * N + i];
+        if (k % T != t) continue;
+        double* sk = s + (b * K + k) * D;
+        for (int64_t d = 0; d < D; ++d) sk[d] += orc_read(x, xdt, (b * N + i) * D + d);
       }
+  }
   for (int64_t b = 0; b < B; ++b) {
     double sh = 0.0;
     for (int64_t k = 0; k < K; ++k) {

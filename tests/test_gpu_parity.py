@@ -396,3 +396,22 @@ def test_baseline_matches_oracle(dtype, B, N, K, D):
     c_ref, n_ref, _ = oracle.update(x, g, c0.astype(np.float64), dtype=dtype)
     assert np.array_equal(cnt.cpu().numpy(), n_ref)
     assert np.allclose(cn.cpu().numpy(), c_ref, rtol=1e-4, atol=1e-4)
+
+
+def test_stage_profile_with_and_without_graph():
+    """Stage timing works for the graph-captured loop (tol = 0) and for the
+    stepped loop that reads the shift every iteration (tol > 0)."""
+    w = datagen.CONFIGS[3].scaled(B=2, N=3000, K=100, iters=3)
+    x, xt, c0 = problem(w)
+    ids, centers, counts = _empty(w.B, w.N, w.K, w.D)
+    fkm.fkm_profile(True)
+    try:
+        fkm.fkm_profile_read(reset=True)
+        for tol in (0.0, 1e-12):
+            n = fkm.fkm_lloyd(xt, torch.from_numpy(c0).cuda(), 3, tol, ids, centers, counts)
+            torch.cuda.synchronize()
+            p = fkm.fkm_profile_read(reset=True)
+            assert p["iterations"] == n
+            assert all(p[s] > 0 for s in fkm.STAGES), p
+    finally:
+        fkm.fkm_profile(False)
