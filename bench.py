@@ -160,6 +160,23 @@ def cpu_cores():
         return os.cpu_count()
 
 
+def rank_workload(w, rank):
+    """Rank r's own problems (weak scaling): the same recipe, seed + 1000 r."""
+    return w.scaled(seed=w.seed + 1000 * rank)
+
+
+def over_ranks(torch, dist, dev, t_ms, n_iters):
+    """(max over ranks of the timed milliseconds, sum over ranks of the
+    iterations done): the whole-job time is the slowest rank's."""
+    if dist is None:
+        return t_ms, n_iters
+    t = torch.tensor([t_ms], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    n = torch.tensor([n_iters], device=dev, dtype=torch.float64)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return t.item(), int(n.item())
+
+
 def oracle_sample(w, iters, rows=None):
     """The fp64 oracle on batch 0 of the workload (its first `rows` points when
     given) for `iters` Lloyd iterations.  Returns (seconds, scale, description):
@@ -179,6 +196,48 @@ def oracle_sample(w, iters, rows=None):
             f"iteration(s) of the fp64 oracle; rate scaled by 1/{scale:.4g} to the whole "
             f"problem (cost is linear in B*N at fixed K)")
     return dt, scale, desc
+
+
+def comparison(fkm, torch, w, xt, c0t, ws, stream, dev, reps=3):
+    """Milliseconds of one assign and one update by the pages' "standard"
+    path (B x N x K fp32 distance matrix written to HBM then read back for the
+    argmin; one fp32 atomicAdd per point per dimension) and by the fused path,
+    on the workload's initial centroids."""
+    B, N, K, D = w.B, w.N, w.K, w.D
+    dist_bytes = 4 * B * N * K
+    free, _ = torch.cuda.mem_get_info(dev)
+    ids = torch.empty(B, N, dtype=torch.int32, device=dev)
+    cen = torch.empty(B, K, D, dtype=torch.float32, device=dev)
+    cnt = torch.empty(B, K, dtype=torch.int32, device=dev)
+
+    def t(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    out = {"centroids": "the initial centroids", "reps": reps}
+    out["assign_fused_ms"] = t(lambda: fkm.fkm_assign(xt, c0t, ids, ws=ws, stream=stream))
+    out["update_sort_inverse_ms"] = t(lambda: fkm.fkm_update(xt, ids, c0t, cen, cnt, ws=ws,
+                                                             stream=stream))
+    out["update_scatter_ms"] = t(lambda: fkm.fkm_baseline_update(xt, ids, c0t, cen, cnt, ws=ws,
+                                                                 stream=stream))
+    out["update_scatter_gbs"] = update_bytes(w) / (out["update_scatter_ms"] / 1e3) / 1e9
+    if dist_bytes > 0.8 * free:
+        out["assign_materialise"] = (f"not run: the distance matrix needs "
+                                     f"{dist_bytes / 2**30:.0f} GiB")
+    else:
+        dist = torch.empty(B, N, K, dtype=torch.float32, device=dev)
+        out["assign_materialise_ms"] = t(lambda: fkm.fkm_baseline_assign(xt, c0t, dist, ids,
+                                                                         ws=ws, stream=stream))
+        out["distance_matrix_bytes"] = dist_bytes
+        del dist
+    return out
 
 
 def cpu_baseline(w, max_iters, budget_s=15.0):
@@ -262,7 +321,7 @@ def run_host(args, w):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=dev)
-    wr = w.scaled(seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     B, N, D, K = wr.B, wr.N, wr.D, wr.K
     tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wr.dtype]
     xh = torch.empty((B, N, D), dtype=tdt, pin_memory=True)
@@ -300,14 +359,7 @@ def run_host(args, w):
         torch.cuda.synchronize(dev)
         h1 = time.time()
         barrier()
-        t = e0.elapsed_time(e1)
-        if dist is not None:
-            tt = torch.tensor([t], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t = tt.item()
-            nn = torch.tensor([n], device=dev, dtype=torch.float64)
-            dist.all_reduce(nn, op=dist.ReduceOp.SUM)
-            n = int(nn.item())
+        t, n = over_ranks(torch, dist, dev, e0.elapsed_time(e1), n)
         return n, t, (h0, h1)
 
     def step():
@@ -377,6 +429,7 @@ def main():
     ap.add_argument("--impl", default="fkm", choices=["fkm", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparison", action="store_true")
     ap.add_argument("--oracle-iters", type=int, default=10)
     args = ap.parse_args()
 
@@ -401,7 +454,7 @@ def main():
                                 device_id=torch.device("cuda", local))
 
     # per rank: its own batch of problems (weak scaling)
-    wr = w.scaled(seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     x = datagen.points(wr)
     c0 = datagen.init_centroids(x, datagen.init_indices(wr), wr.dtype)
     tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wr.dtype]
@@ -451,16 +504,7 @@ def main():
     launches = fkm.fkm_kernel_launches() - launches0
     prof = fkm.fkm_profile_read(reset=True)
     fkm.fkm_profile(False)
-    elapsed_ms = e0.elapsed_time(e1)
-    t_max = elapsed_ms
-    total_iters = iters_done
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = t.item()
-        n = torch.tensor([iters_done], device=dev, dtype=torch.float64)
-        dist.all_reduce(n, op=dist.ReduceOp.SUM)
-        total_iters = int(n.item())
+    t_max, total_iters = over_ranks(torch, dist, dev, e0.elapsed_time(e1), iters_done)
     value = total_iters / (t_max / 1e3)
 
     # --- per-stage rates from the events recorded inside the timed region
@@ -497,45 +541,69 @@ def main():
             "gpu_launches": int(launches),
             "clocks": clk.summary()}
 
-    # --- end to end through the C ABI with host buffers
+    # --- the pages' comparison point (not the method): materialised distances
+    # + argmin read-back, and the scatter-atomic update, against the fused
+    # calls on the same inputs (outside the timed region)
+    if not args.no_comparison:
+        line["comparison"] = comparison(fkm, torch, wr, xt, c0t, ws, stream, dev)
+
+    # --- end to end through the C ABI with host buffers.  Every step copies its
+    # points and initial centroids from pinned host memory and reads its
+    # results back; the copy of step k+1 runs on a copy stream while step k
+    # computes (two device buffers), as a service running back-to-back
+    # problems would do.
     if not args.no_e2e:
         ids_h = torch.empty(B, N, dtype=torch.int32).pin_memory()
         cen_h = torch.empty(B, K, D, dtype=torch.float32).pin_memory()
         cnt_h = torch.empty(B, K, dtype=torch.int32).pin_memory()
         ine_h = torch.empty(B, dtype=torch.float64).pin_memory()
-        x_e = torch.empty_like(xt)
-        c_e = torch.empty_like(c0t)
+        x_e = [torch.empty_like(xt), torch.empty_like(xt)]
+        c_e = [torch.empty_like(c0t), torch.empty_like(c0t)]
+        copy_stream = torch.cuda.Stream(dev)
+        ready = [torch.cuda.Event(), torch.cuda.Event()]
+        done = [torch.cuda.Event(), torch.cuda.Event()]
+        for ev in done:
+            ev.record(stream)
 
-        def e2e_step():
-            x_e.copy_(xh, non_blocking=True)
-            c_e.copy_(ch, non_blocking=True)
-            n_it = fkm.fkm_lloyd(x_e, c_e, wr.iters, wr.tol, ids, centers, counts, inertia,
+        def issue_copy(k):
+            s = k % 2
+            copy_stream.wait_event(done[s])   # step k-2 is finished with buffer s
+            with torch.cuda.stream(copy_stream):
+                x_e[s].copy_(xh, non_blocking=True)
+                c_e[s].copy_(ch, non_blocking=True)
+                ready[s].record(copy_stream)
+
+        def e2e_step(k):
+            s = k % 2
+            stream.wait_event(ready[s])
+            n_it = fkm.fkm_lloyd(x_e[s], c_e[s], wr.iters, wr.tol, ids, centers, counts, inertia,
                                  ws=ws, stream=stream)
+            done[s].record(stream)
             ids_h.copy_(ids, non_blocking=True)
             cen_h.copy_(centers, non_blocking=True)
             cnt_h.copy_(counts, non_blocking=True)
             ine_h.copy_(inertia, non_blocking=True)
             return n_it
 
-        for _ in range(max(args.warmup, 1)):
-            e2e_step()
+        def e2e_run(steps):
+            issue_copy(0)
+            n = 0
+            for k in range(steps):
+                if k + 1 < steps:
+                    issue_copy(k + 1)
+                n += e2e_step(k)
+            return n
+
+        e2e_run(max(args.warmup, 1))
         torch.cuda.synchronize(dev)
         barrier()
         e0.record(stream)
-        n_e = 0
-        for _ in range(args.steps):
-            n_e += e2e_step()
+        copy_stream.wait_event(e0)
+        n_e = e2e_run(args.steps)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        t_e = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([t_e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_e = t.item()
-            n = torch.tensor([n_e], device=dev, dtype=torch.float64)
-            dist.all_reduce(n, op=dist.ReduceOp.SUM)
-            n_e = int(n.item())
+        t_e, n_e = over_ranks(torch, dist, dev, e0.elapsed_time(e1), n_e)
         line["e2e"] = {"value": n_e / (t_e / 1e3), "unit": UNIT,
                        "h2d_bytes_per_step": int(xh.numel() * xh.element_size()
                                                  + ch.numel() * ch.element_size()),

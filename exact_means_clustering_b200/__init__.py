@@ -32,6 +32,7 @@ DTYPES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 _P, _I, _L, _Z, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
 _SIG = {
     "fkm_workspace_size": ([_I, _I, _I, _I, _I, ctypes.POINTER(_Z)], _I),
+    "fkm_selftest_wait_timeout": ([ctypes.c_uint64, _P, _Z, _P], _I),
     "fkm_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_lloyd": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _P, _P, ctypes.POINTER(_I), _P, _Z,
@@ -222,6 +223,12 @@ def fkm_assign_noalloc(x, centers, ids, stream=None):
     _check("fkm_assign_noalloc", lib().fkm_assign_noalloc(B, N, K, D, _dt(x), _ptr(x),
                                                           _ptr(centers), _ptr(ids),
                                                           _stream(stream)))
+
+
+def fkm_selftest_wait_timeout(timeout_ns, ws, stream=None):
+    """Launch a kernel whose bounded wait runs out after timeout_ns (see fkm.h)."""
+    _check("fkm_selftest_wait_timeout",
+           lib().fkm_selftest_wait_timeout(int(timeout_ns), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def fkm_sync_status(ws, stream=None):

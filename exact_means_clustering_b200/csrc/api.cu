@@ -331,10 +331,19 @@ struct GraphKey {
   bool operator==(const GraphKey& o) const { return memcmp(this, &o, sizeof(GraphKey)) == 0; }
 };
 
+// A few recent loops stay instantiated (callers that alternate buffers, e.g.
+// double-buffered inputs, replay without re-capturing); least recently used
+// goes first.
+struct GraphEntry {
+  GraphKey key;
+  cudaGraphExec_t exec;
+  long long launches;   // kernels one replay launches
+  long long last_use;
+};
+constexpr size_t kGraphCacheSize = 8;
 static std::mutex g_graph_mu;
-static GraphKey g_graph_key;
-static cudaGraphExec_t g_graph_exec = nullptr;
-static long long g_graph_launches = 0;  // kernels one replay launches
+static std::vector<GraphEntry> g_graphs;
+static long long g_graph_clock = 0;
 
 }  // namespace fkm
 
@@ -503,11 +512,18 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
     key.counts = counts; key.inertia = inertia; key.ws = ws; key.st = st; key.dev = dev;
     key.prof_gen = prof ? g_prof.gen : -1;
     std::lock_guard<std::mutex> lock(g_graph_mu);
-    if (!(g_graph_exec && g_graph_key == key)) {
-      if (g_graph_exec) {
-        cudaGraphExecDestroy(g_graph_exec);
-        g_graph_exec = nullptr;
+    GraphEntry* hit = nullptr;
+    for (auto& ge : g_graphs)
+      if (ge.key == key) hit = &ge;
+    if (!hit) {
+      if (g_graphs.size() >= kGraphCacheSize) {
+        size_t lru = 0;
+        for (size_t i = 1; i < g_graphs.size(); ++i)
+          if (g_graphs[i].last_use < g_graphs[lru].last_use) lru = i;
+        cudaGraphExecDestroy(g_graphs[lru].exec);
+        g_graphs.erase(g_graphs.begin() + (long)lru);
       }
+      cudaGraphExec_t exec = nullptr;
       cudaStream_t cap;
       FKM_CUDA_TRY(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
       cudaGraph_t g = nullptr;
@@ -523,21 +539,22 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
         s = cuda_fail(e, "cudaStreamBeginCapture");
       }
       if (s == FKM_OK) {
-        e = cudaGraphInstantiate(&g_graph_exec, g, 0);
+        e = cudaGraphInstantiate(&exec, g, 0);
         if (e != cudaSuccess) {
-          g_graph_exec = nullptr;
+          exec = nullptr;
           s = cuda_fail(e, "cudaGraphInstantiate");
         }
       }
       if (g) cudaGraphDestroy(g);
       cudaStreamDestroy(cap);
       if (s != FKM_OK) return s;
-      g_graph_key = key;
-      g_graph_launches = g_launches.load() - l0;
+      g_graphs.push_back(GraphEntry{key, exec, g_launches.load() - l0, 0});
+      hit = &g_graphs.back();
     } else {
-      note_launch((int)g_graph_launches);  // the replay launches what the capture counted
+      note_launch((int)hit->launches);  // the replay launches what the capture counted
     }
-    FKM_CUDA_TRY(cudaGraphLaunch(g_graph_exec, st));
+    hit->last_use = ++g_graph_clock;
+    FKM_CUDA_TRY(cudaGraphLaunch(hit->exec, st));
     done = max_iters;
   } else {
     for (int t = 0; t < max_iters; ++t) {

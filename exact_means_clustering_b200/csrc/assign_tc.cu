@@ -158,6 +158,26 @@ __device__ __forceinline__ int find_first(const float4* save, int rot, float bes
   return mask ? __ffs(mask) - 1 : 0;
 }
 
+// Comparison mode: 32 distances ||x - c_hat||^2 = xv - 2 acc of one row,
+// written as 16-byte vectors when the row allows it (K a multiple of 4), so a
+// thread's 128 bytes go out whole.
+__device__ __forceinline__ void store_dist_chunk(const uint32_t (&r)[32], float* drow, int col0,
+                                                 int K, float xv) {
+  if (col0 + 32 <= K && (K & 3) == 0) {
+    float4* d4 = reinterpret_cast<float4*>(drow + col0);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      d4[k] = make_float4(fmaf(-2.0f, __uint_as_float(r[4 * k]), xv),
+                          fmaf(-2.0f, __uint_as_float(r[4 * k + 1]), xv),
+                          fmaf(-2.0f, __uint_as_float(r[4 * k + 2]), xv),
+                          fmaf(-2.0f, __uint_as_float(r[4 * k + 3]), xv));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < K) drow[col0 + j] = fmaf(-2.0f, __uint_as_float(r[j]), xv);
+  }
+}
+
 // The constant bias slab of a point tile: row r = [a0, a1, a2, 0 ... 0] (16
 // values) in the 32-byte swizzle (rows of 32 bytes, 8-row groups of 256
 // bytes; the two 16-byte halves of rows 4-7 of a group trade places), the
@@ -406,13 +426,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
           if (gi < p.N) {
             const float xv = p.xn[(size_t)b * p.N + gi];
             float* drow = p.dist + ((size_t)b * p.N + gi) * p.K;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (colb + j < p.K) drow[colb + j] = fmaf(-2.0f, __uint_as_float(r0[j]), xv);
-              if (colb + 32 + j < p.K) drow[colb + 32 + j] = fmaf(-2.0f, __uint_as_float(r1[j]), xv);
-              if (colb + 64 + j < p.K) drow[colb + 64 + j] = fmaf(-2.0f, __uint_as_float(r2[j]), xv);
-              if (colb + 96 + j < p.K) drow[colb + 96 + j] = fmaf(-2.0f, __uint_as_float(r3[j]), xv);
-            }
+            store_dist_chunk(r0, drow, colb, p.K, xv);
+            store_dist_chunk(r1, drow, colb + 32, p.K, xv);
+            store_dist_chunk(r2, drow, colb + 64, p.K, xv);
+            store_dist_chunk(r3, drow, colb + 96, p.K, xv);
           }
           continue;
         }

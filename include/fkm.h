@@ -225,6 +225,17 @@ FKM_API fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, con
  * FKM_OK, FKM_ERR_TIMEOUT, FKM_ERR_BAD_ID or FKM_ERR_INTERNAL. */
 FKM_API fkm_status fkm_sync_status(void* ws, size_t ws_bytes, void* stream);
 
+/* Self-test of failure detection (no counterpart in the pages): launches one
+ * kernel whose bounded mbarrier wait is made to run out -- it waits
+ * timeout_ns (1 us .. 1 s) for an arrival nobody makes, then sets the
+ * timeout bit in the workspace's status word and returns, as every bounded
+ * wait in the library does.  A following fkm_sync_status on the same
+ * workspace returns FKM_ERR_TIMEOUT, and the context stays usable.  ws:
+ * device, >= 256 bytes, 16-byte aligned (its first word is the status).
+ * Async. */
+FKM_API fkm_status fkm_selftest_wait_timeout(uint64_t timeout_ns, void* ws, size_t ws_bytes,
+                                             void* stream);
+
 FKM_API const char* fkm_status_string(fkm_status s);
 /* Thread-local text about the last failure in this thread ("" if none). */
 FKM_API const char* fkm_last_error(void);

@@ -415,3 +415,20 @@ def test_stage_profile_with_and_without_graph():
             assert all(p[s] > 0 for s in fkm.STAGES), p
     finally:
         fkm.fkm_profile(False)
+
+
+def test_bounded_wait_runs_out_without_a_fault():
+    """Failure detection: a wait nobody satisfies ends with FKM_ERR_TIMEOUT in
+    the status word after its limit, and the context stays usable."""
+    w = datagen.CONFIGS[2].scaled(B=1, N=2000, K=64, iters=1)
+    x, xt, c0 = problem(w)
+    ws = fkm.workspace(fkm.fkm_workspace_size(w.B, w.N, w.K, w.D, xt.dtype))
+    fkm.fkm_selftest_wait_timeout(2_000_000, ws)   # 2 ms
+    with pytest.raises(fkm.FkmError) as e:
+        fkm.fkm_sync_status(ws)
+    assert e.value.code == 5
+    fkm.fkm_sync_status(ws)                       # the status was cleared
+    ids = torch.empty(w.B, w.N, dtype=torch.int32, device="cuda")
+    fkm.fkm_assign(xt, torch.from_numpy(c0).cuda(), ids, ws=ws)
+    fkm.fkm_sync_status(ws)
+    check_assign(x, w.dtype, c0, ids.cpu().numpy())
