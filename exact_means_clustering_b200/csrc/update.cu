@@ -157,15 +157,10 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
 #ifndef FKM_SEG_MIN_BLOCKS
 #define FKM_SEG_MIN_BLOCKS 3
 #endif
-#ifndef FKM_SEG_PREFETCH
-#define FKM_SEG_PREFETCH 0
-#endif
 constexpr int SEG_WARPS = 8;                // warps (ranges) per block
 constexpr int SEG_STAGES = FKM_SEG_STAGES;  // row-gather steps in flight per warp
 static_assert((SEG_STAGES & (SEG_STAGES - 1)) == 0, "the ring index is a mask");
-// When non-zero, the rows of step s + SEG_PREFETCH are prefetched into L2
-// (one prefetch per 128-byte line) while step s is added.
-constexpr int SEG_PREFETCH = FKM_SEG_PREFETCH;
+
 
 // Per-warp shared memory: the range's (key, row) pairs, the start position of
 // every run (plus an end sentinel), and the gather ring.
@@ -274,15 +269,6 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     cp_async_16(&ws.ring[s & (SEG_STAGES - 1)][lane], xb + (int64_t)e.y * rb, (e.x | novec) >= 0);
     cp_async_commit();
   };
-  auto prefetch = [&](int s) {
-    const int i = min(s * RPS + g, SEG_RANGE);
-    if (SEG_PREFETCH > 0 && (sub & 7) == 0 && lane_has_vec) {
-      const int2 e = ws.kv[i];
-      if (e.x >= 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(xb + (int64_t)e.y * rb));
-    }
-  };
-#pragma unroll 1
-  for (int s = 0; s < SEG_PREFETCH; ++s) prefetch(s);
 #pragma unroll
   for (int s = 0; s < SEG_STAGES - 1; ++s) issue(s);
 
