@@ -377,6 +377,12 @@ def run_host(args, w):
     per_iter_s = (t_ms / 1e3) / max(n_it / world, 1)
     x_bytes = wr.x_bytes
     achieved = x_bytes / per_iter_s / 1e9
+    peaks, _ = load_peaks()
+    products = 3 if wr.dtype == "f32" else 1   # fp32 points: split-bf16, three products
+    tensor_s = products * assign_flops(wr) / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12)
+    tensor_note = (f"the other bound: {products} x 2*N*K*D tensor-core FLOP per iteration at the "
+                   f"measured sustained bf16 peak takes {tensor_s:.3f} s; the larger of the two "
+                   f"terms binds")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -387,7 +393,10 @@ def run_host(args, w):
             "roofline": {"bound": "h2d", "kernel": "whole iteration (host link)",
                          "achieved": achieved, "peak": h2d, "unit": "GB/s",
                          "frac": achieved / h2d, "traffic": None,
-                         "peak_source": "measured pinned host-to-device copy, 1 GiB, this run"},
+                         "peak_source": "measured pinned host-to-device copy, 1 GiB, this run",
+                         "terms_s_per_iter": {"h2d": x_bytes / (h2d * 1e9),
+                                              "tensor": tensor_s},
+                         "note": tensor_note},
             "gpu_launches": int(launches),
             "clocks": clk.summary()}
     if not args.no_e2e:

@@ -15,6 +15,7 @@
 // it overlaps the previous iteration's finalize (the README's prefetch of the
 // first block of the next iteration, "Multi-GPU Support").
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "fkm_internal.cuh"
@@ -121,6 +122,17 @@ struct StreamSet {
   }
 };
 
+// Host-side fault injection for the failure-detection tests (off unless the
+// environment asks for it): FKM_FAULT_INJECT=h2d@chunk:<n> makes the copy of
+// the n-th streamed chunk (counted over the whole call) fail as a CUDA error
+// would, before it is issued.  Nothing is done on the GPU to cause it.
+int64_t injected_h2d_fault_chunk() {
+  const char* v = std::getenv("FKM_FAULT_INJECT");
+  long long n = -1;
+  if (v && std::sscanf(v, "h2d@chunk:%lld", &n) == 1 && n >= 0) return (int64_t)n;
+  return -1;
+}
+
 }  // namespace
 }  // namespace fkm
 
@@ -203,6 +215,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
 
   int done = 0;
   int64_t chunk_no = 0;
+  const int64_t fault_chunk = injected_h2d_fault_chunk();
   for (int t = 0; t < max_iters; ++t) {
     float* cur = (t & 1) ? cB : cA;
     float* nxt = (t & 1) ? cA : cB;
@@ -215,6 +228,11 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
         const int rows = (int)((N - n0) < L.R ? (N - n0) : L.R);
         void* xb = at(L.xbuf[buf]);
         FKM_CUDA_TRY(cudaStreamWaitEvent(ss.copy, ss.freed[buf], 0));
+        if (chunk_no == fault_chunk) {
+          set_error("injected fault (FKM_FAULT_INJECT): host-to-device copy of chunk %lld",
+                    (long long)chunk_no);
+          return FKM_ERR_CUDA;
+        }
         FKM_CUDA_TRY(cudaMemcpyAsync(xb,
                                      static_cast<const char*>(x_host) +
                                          ((size_t)b * N + n0) * D * s,

@@ -145,7 +145,10 @@ FKM_API fkm_status fkm_host_workspace_size(int B, int N, int K, int D, int dtype
  * 快速且内存高效精确K-Means聚类" summary, section 方法步骤详情 step (3)).
  * Results are the same as fkm_lloyd's.  Outputs (ids, centers, counts,
  * inertia) are device pointers as in fkm_lloyd; x_host is a host pointer.
- * Synchronous. */
+ * Synchronous.  For failure-detection tests, the environment variable
+ * FKM_FAULT_INJECT=h2d@chunk:<n> makes the copy of the n-th streamed chunk
+ * fail (FKM_ERR_CUDA) on the host before it is issued; the call then returns
+ * with its copy stream and events released. */
 FKM_API fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_host,
                           const float* init_centers, int max_iters, float tol,
                           int64_t chunk_rows, int32_t* ids, float* centers, int32_t* counts,

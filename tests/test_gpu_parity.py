@@ -432,3 +432,26 @@ def test_bounded_wait_runs_out_without_a_fault():
     fkm.fkm_assign(xt, torch.from_numpy(c0).cuda(), ids, ws=ws)
     fkm.fkm_sync_status(ws)
     check_assign(x, w.dtype, c0, ids.cpu().numpy())
+
+
+def test_lloyd_host_injected_copy_failure(monkeypatch):
+    """Failure detection on the host: a streamed copy made to fail (no GPU
+    fault) is reported as FKM_ERR_CUDA, and the next call, without the
+    injection, runs cleanly and matches a run that never failed."""
+    w = datagen.Workload("ooc_fault", 1, 9000, 64, 40, "f32", 40, sigma=0.5, iters=3, seed=77)
+    x, xt, c0 = problem(w)
+    xh = xt.cpu().pin_memory()
+    c0t = torch.from_numpy(c0).cuda()
+    ids, centers, counts = _empty(w.B, w.N, w.K, w.D)
+    monkeypatch.setenv("FKM_FAULT_INJECT", "h2d@chunk:4")
+    with pytest.raises(fkm.FkmError) as e:
+        fkm.fkm_lloyd_host(xh, c0t, 3, 0.0, 2048, ids, centers, counts)
+    assert e.value.code == 3 and "injected" in str(e.value)
+    monkeypatch.delenv("FKM_FAULT_INJECT")
+    torch.cuda.synchronize()
+    n = fkm.fkm_lloyd_host(xh, c0t, 3, 0.0, 2048, ids, centers, counts)
+    i2, c2, n2 = _empty(w.B, w.N, w.K, w.D)
+    fkm.fkm_lloyd_host(xh, c0t, 3, 0.0, 2048, i2, c2, n2)
+    assert n == 3
+    assert torch.equal(ids, i2) and torch.equal(counts, n2)
+    assert torch.allclose(centers, c2, rtol=1e-6, atol=1e-7)
