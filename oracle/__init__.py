@@ -62,7 +62,9 @@ def _load():
         L.orc_lloyd.argtypes = [_I, _I, _I, _I, _P, ctypes.c_int, _P, ctypes.c_int,
                                 ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
         L.orc_argsort_stable.argtypes = [_P, _I, _I, _P]
-        for f in ("orc_assign", "orc_inertia", "orc_update", "orc_lloyd", "orc_argsort_stable"):
+        L.orc_centre.argtypes = [_I, _I, _I, _P, ctypes.c_int, _P, _P, _P]
+        for f in ("orc_assign", "orc_inertia", "orc_update", "orc_lloyd", "orc_argsort_stable",
+                  "orc_centre"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -200,3 +202,18 @@ def argsort_stable(keys, n_keys=None):
     if rc:
         raise RuntimeError("orc_argsort_stable failed")
     return idx
+
+
+def centre(x, dtype="f32", mu=None):
+    """Centred points and their mean (README "Centre your data"): returns
+    (xc in the storage form of dtype, mu float32 [B, D]).  mu: optional given
+    mean [B, D] (float32) to subtract instead of the computed one."""
+    x, code = _x3(x, dtype)
+    B, N, D = x.shape
+    xc = np.empty_like(x)
+    mu_out = np.empty((B, D), np.float32)
+    mu_in = None if mu is None else np.ascontiguousarray(mu, dtype=np.float32).reshape(B, D)
+    rc = _load().orc_centre(B, N, D, _ptr(x), code, _ptr(mu_in), _ptr(mu_out), _ptr(xc))
+    if rc:
+        raise RuntimeError("orc_centre failed")
+    return xc, mu_out

@@ -262,6 +262,59 @@ int orc_update(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xd
   return 0;
 }
 
+/* ---------- centring ----------
+ * k-means is translation invariant, so data with a large common offset can be
+ * clustered after subtracting its mean and the centroids shifted back
+ * ("Flash-KMeans" GitHub README, section "Centre your data").
+ *   mu[b,d] = fp32( (sum over i of x[b,i,d], fp64, index order) / N )
+ *   xc[b,i,d] = RNE_dtype( fp32(x[b,i,d]) - mu[b,d] ), the subtraction one IEEE
+ *               fp32 operation; xc is written in the storage form of the dtype
+ *               (fp32 values, fp16 values, bf16 bit patterns).
+ * mu_in, when non-null, replaces the computed mean (to check the subtraction
+ * for a given mean); mu_out (optional) receives the mean used. */
+static void orc_store(void* out, int dt, int64_t idx, float v) {
+  if (dt == ORC_F32) {
+    ((float*)out)[idx] = v;
+  } else if (dt == ORC_F16) {
+    _Float16 h = (_Float16)v;
+    memcpy((uint16_t*)out + idx, &h, 2);
+  } else {
+    const float r = (float)orc_round_bf16(v);
+    uint32_t u;
+    memcpy(&u, &r, 4);
+    ((uint16_t*)out)[idx] = (uint16_t)(u >> 16);
+  }
+}
+
+int orc_centre(int64_t B, int64_t N, int64_t D, const void* x, int xdt, const float* mu_in,
+               float* mu_out, void* xc_out) {
+  if (B < 1 || N < 1 || D < 1 || !x || !xc_out) return -1;
+  float* mu = (float*)malloc(sizeof(float) * (size_t)(B * D));
+  if (!mu) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t d = 0; d < D; ++d) {
+      if (mu_in) {
+        mu[b * D + d] = mu_in[b * D + d];
+        continue;
+      }
+      double s = 0.0;
+      for (int64_t i = 0; i < N; ++i) s += orc_read(x, xdt, (b * N + i) * D + d);
+      mu[b * D + d] = (float)(s / (double)N);
+    }
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t i = 0; i < N; ++i)
+      for (int64_t d = 0; d < D; ++d) {
+        const int64_t e = (b * N + i) * D + d;
+        const float v = (float)orc_read(x, xdt, e) - mu[b * D + d];
+        orc_store(xc_out, xdt, e, v);
+      }
+  if (mu_out) memcpy(mu_out, mu, sizeof(float) * (size_t)(B * D));
+  free(mu);
+  return 0;
+}
+
 /* ---------- Lloyd loop ---------- */
 /* centers starts as c0 and ends as the centroids after the last update.
  * J_hist / shift_hist (optional, [max_iters * B]) record every iteration. */

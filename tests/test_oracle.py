@@ -18,7 +18,9 @@ import os
 import numpy as np
 import pytest
 
+import datagen
 import oracle
+import torch
 
 
 def _bf16_bits(a):
@@ -400,3 +402,61 @@ def test_lloyd_tol_semantics():
     r = oracle.lloyd(x, c0, max_iters=30, tol=1e-3)
     sh = r["shift_hist"]
     assert sh[-1].max() < 1e-3 and np.all(sh[:-1].max(1) >= 1e-3)
+
+
+# ---------------------------------------------------------------- centring
+# README "Centre your data": k-means is translation invariant; centring
+# subtracts the per-batch mean of the points.
+
+def _store(x32, dtype):
+    if dtype == "bf16":
+        return (torch.from_numpy(x32).to(torch.bfloat16).view(torch.int16).numpy()
+                .view(np.uint16))
+    return x32.astype(np.float16 if dtype == "f16" else np.float32)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_centre_integer_grid_is_exact(dtype):
+    rng = np.random.default_rng(5)
+    B, N, D = 2, 64, 8
+    x = rng.integers(-20, 21, size=(B, N, D)).astype(np.float32)
+    x -= x.mean(axis=1, keepdims=True).round()       # column sums now small integers
+    x[:, -1, :] -= x.sum(axis=1)                      # ... and exactly zero: mean 0
+    x += np.arange(D, dtype=np.float32) * 4           # mean = 4 d, exact
+    xs = _store(x, dtype)
+    xc, mu = oracle.centre(xs, dtype)
+    assert np.array_equal(mu, np.broadcast_to(np.arange(D, dtype=np.float32) * 4, (B, D)))
+    assert np.array_equal(datagen.widen(xc, dtype), x - mu[:, None, :])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_centre_subtraction_matches_library_rounding(dtype):
+    rng = np.random.default_rng(6)
+    B, N, D = 2, 300, 16
+    x32 = (rng.standard_normal((B, N, D)) * 3 + 50).astype(np.float32)
+    xs = _store(x32, dtype)
+    mu = rng.standard_normal((B, D)).astype(np.float32) * 7
+    xc, mu_used = oracle.centre(xs, dtype, mu=mu)
+    assert np.array_equal(mu_used, mu)
+    ref = _store(datagen.widen(xs, dtype) - mu[:, None, :], dtype)   # fp32 subtract, library RNE
+    assert np.array_equal(xc.view(np.uint8), ref.view(np.uint8))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_centre_mean_matches_numpy(dtype):
+    rng = np.random.default_rng(7)
+    x32 = (rng.standard_normal((3, 1000, 24)) + 64).astype(np.float32)
+    xs = _store(x32, dtype)
+    _, mu = oracle.centre(xs, dtype)
+    ref = datagen.widen(xs, dtype).astype(np.float64).mean(axis=1).astype(np.float32)
+    assert np.all(np.abs(mu.view(np.int32).astype(np.int64) - ref.view(np.int32)) <= 1)
+
+
+def test_centre_is_translation_free():
+    """Centring x and x + t (t exact, every value exact) gives the same points."""
+    rng = np.random.default_rng(8)
+    x = rng.integers(-50, 50, size=(1, 128, 8)).astype(np.float32)
+    t = np.array([64, -32, 0, 8, 1, 2, 3, 4], np.float32)
+    a, _ = oracle.centre(x, "f32")
+    b, _ = oracle.centre(x + t, "f32")
+    assert np.array_equal(a, b)
