@@ -228,6 +228,14 @@ def comparison(fkm, torch, w, xt, c0t, ws, stream, dev, reps=3):
     out["update_scatter_ms"] = t(lambda: fkm.fkm_baseline_update(xt, ids, c0t, cen, cnt, ws=ws,
                                                                  stream=stream))
     out["update_scatter_gbs"] = update_bytes(w) / (out["update_scatter_ms"] / 1e3) / 1e9
+    # the optional centring pass (README "Centre your data"): the mean reads x,
+    # the subtraction reads and writes it
+    xc = torch.empty_like(xt)
+    mu = torch.empty(B, D, dtype=torch.float32, device=dev)
+    cws = fkm.workspace(fkm.fkm_centre_workspace_size_bytes(B, N, D), dev)
+    out["centre_ms"] = t(lambda: fkm.fkm_centre(xt, mu=mu, out=xc, ws=cws, stream=stream))
+    out["centre_gbs"] = 3 * w.x_bytes / (out["centre_ms"] / 1e3) / 1e9
+    del xc
     if dist_bytes > 0.8 * free:
         out["assign_materialise"] = (f"not run: the distance matrix needs "
                                      f"{dist_bytes / 2**30:.0f} GiB")

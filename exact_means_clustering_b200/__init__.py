@@ -33,6 +33,8 @@ _P, _I, _L, _Z, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_siz
 _SIG = {
     "fkm_workspace_size": ([_I, _I, _I, _I, _I, ctypes.POINTER(_Z)], _I),
     "fkm_selftest_wait_timeout": ([ctypes.c_uint64, _P, _Z, _P], _I),
+    "fkm_centre_workspace_size": ([_I, _I, _I, ctypes.POINTER(_Z)], _I),
+    "fkm_centre": ([_I, _I, _I, _I, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_lloyd": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _P, _P, ctypes.POINTER(_I), _P, _Z,
@@ -225,6 +227,25 @@ def fkm_assign_noalloc(x, centers, ids, stream=None):
                                                           _stream(stream)))
 
 
+def fkm_centre_workspace_size_bytes(B, N, D) -> int:
+    n = ctypes.c_size_t(0)
+    _check("fkm_centre_workspace_size", lib().fkm_centre_workspace_size(B, N, D, ctypes.byref(n)))
+    return n.value
+
+
+def fkm_centre(x, mu=None, out=None, ws=None, stream=None):
+    """Per-batch mean of x [B, N, D] and x minus it, rounded to x's dtype (see
+    fkm.h).  out may be x itself.  Returns (out, mu float32 [B, D])."""
+    B, N, D = x.shape
+    mu = mu if mu is not None else torch.empty(B, D, dtype=torch.float32, device=x.device)
+    out = out if out is not None else torch.empty_like(x)
+    if ws is None:
+        ws = workspace(fkm_centre_workspace_size_bytes(B, N, D), x.device)
+    _check("fkm_centre", lib().fkm_centre(B, N, D, _dt(x), _ptr(x), _ptr(mu), _ptr(out), _ptr(ws),
+                                          ws.numel(), _stream(stream)))
+    return out, mu
+
+
 def fkm_selftest_wait_timeout(timeout_ns, ws, stream=None):
     """Launch a kernel whose bounded wait runs out after timeout_ns (see fkm.h)."""
     _check("fkm_selftest_wait_timeout",
@@ -287,3 +308,119 @@ def batch_kmeans_Euclid(x: torch.Tensor, n_clusters: int, max_iters: int = 100, 
     if squeeze:
         return ids[0], centers[0], n_iter
     return ids, centers, n_iter
+
+
+# ---------------------------------------------------------------- class API
+class FlashKMeans:
+    """Exact Lloyd k-means with the class-style calls of the "Flash-KMeans"
+    GitHub README (section "Usage"): fit, predict, fit_predict, and train for
+    data held in host memory.
+
+    d, k       point dimension and number of clusters
+    niter      maximum Lloyd iterations; tol: stop once every batch's squared
+               centroid shift is below it (0 runs all niter iterations)
+    dtype      storage type the points are clustered in (bf16, fp16 or fp32;
+               None keeps the input's)
+    centre     subtract the per-batch mean of the points first and add it back
+               to the centroids (README, "Centre your data"); costs one extra
+               copy of x
+    chunk_rows rows per streamed chunk when the points are in host memory
+
+    Points are [N, D] or [B, N, D] (B independent problems).  After fit:
+    centroids [B, K, D] float32 (or [K, D]), labels_ int32 [B, N] (or [N]),
+    n_iter, inertia [B] (the objective of the last assignment).
+    """
+
+    def __init__(self, d, k, niter=100, tol=0.0, dtype=None, centre=False, seed=0,
+                 chunk_rows=1 << 23, device=None):
+        self.d, self.k, self.niter, self.tol = int(d), int(k), int(niter), float(tol)
+        self.dtype, self.centre, self.seed = dtype, bool(centre), int(seed)
+        self.chunk_rows = int(chunk_rows)
+        self.device = torch.device(device) if device is not None else torch.device("cuda")
+        self.centroids = None
+        self.labels_ = None
+        self.n_iter = 0
+        self.inertia = None
+        self._squeeze = False
+
+    def _shape(self, x):
+        if x.dim() == 2:
+            x = x.unsqueeze(0)
+        if x.dim() != 3 or x.shape[-1] != self.d:
+            raise ValueError(f"points must be [N, {self.d}] or [B, N, {self.d}], got {tuple(x.shape)}")
+        if self.dtype is not None and x.dtype != self.dtype:
+            x = x.to(self.dtype)
+        return x.contiguous()
+
+    def _init(self, x, init_centroids):
+        B, N, D = x.shape
+        if init_centroids is not None:
+            return init_centroids.reshape(B, self.k, D).to(self.device, torch.float32).contiguous()
+        g = torch.Generator(device="cpu").manual_seed(self.seed)
+        idx = torch.stack([torch.randperm(N, generator=g)[:self.k] for _ in range(B)])
+        rows = torch.gather(x, 1, idx.to(x.device).unsqueeze(-1).expand(B, self.k, D))
+        return rows.to(self.device, torch.float32).contiguous()
+
+    def fit(self, x, init_centroids=None):
+        self._squeeze = x.dim() == 2
+        x = self._shape(x)
+        if not x.is_cuda:
+            return self._fit_host(x, init_centroids)
+        B, N, D = x.shape
+        mu = None
+        if self.centre:
+            x, mu = fkm_centre(x)
+            if init_centroids is not None:
+                init_centroids = init_centroids.reshape(B, self.k, D).to(x.device) - mu[:, None, :]
+        init = self._init(x, init_centroids)
+        ids = torch.empty(B, N, dtype=torch.int32, device=x.device)
+        centers = torch.empty(B, self.k, D, dtype=torch.float32, device=x.device)
+        counts = torch.empty(B, self.k, dtype=torch.int32, device=x.device)
+        inertia = torch.empty(B, dtype=torch.float64, device=x.device)
+        self.n_iter = fkm_lloyd(x, init, self.niter, self.tol, ids, centers, counts, inertia)
+        if mu is not None:
+            centers += mu[:, None, :]
+        self._store(ids, centers, inertia)
+        return self
+
+    def _fit_host(self, x, init_centroids):
+        B, N, D = x.shape
+        if self.centre:
+            raise ValueError("centre=True needs the points on the GPU (one extra device copy)")
+        xh = x if x.is_pinned() else x.pin_memory()
+        init = self._init(xh, init_centroids)
+        ids = torch.empty(B, N, dtype=torch.int32, device=self.device)
+        centers = torch.empty(B, self.k, D, dtype=torch.float32, device=self.device)
+        counts = torch.empty(B, self.k, dtype=torch.int32, device=self.device)
+        inertia = torch.empty(B, dtype=torch.float64, device=self.device)
+        self.n_iter = fkm_lloyd_host(xh, init, self.niter, self.tol, self.chunk_rows, ids, centers,
+                                     counts, inertia)
+        self._store(ids, centers, inertia)
+        return self
+
+    def _store(self, ids, centers, inertia):
+        self.labels_ = ids[0] if self._squeeze else ids
+        self.centroids = centers[0] if self._squeeze else centers
+        self.inertia = inertia
+
+    def train(self, data, init_centroids=None):
+        """fit, under the README's name for training on large data (host
+        tensors are streamed to the GPU in chunks)."""
+        return self.fit(data, init_centroids)
+
+    def predict(self, x):
+        """Nearest-centroid ids of the points x (on the GPU) for the fitted centroids."""
+        if self.centroids is None:
+            raise RuntimeError("predict before fit")
+        squeeze = x.dim() == 2
+        x = self._shape(x).to(self.device)
+        B, N, D = x.shape
+        c = self.centroids.reshape(-1, self.k, D)
+        if c.shape[0] != B:
+            raise ValueError("predict needs as many batches as fit")
+        ids = torch.empty(B, N, dtype=torch.int32, device=x.device)
+        fkm_assign(x, c.contiguous(), ids)
+        return ids[0] if squeeze else ids
+
+    def fit_predict(self, x, init_centroids=None):
+        return self.fit(x, init_centroids).labels_

@@ -167,6 +167,20 @@ FKM_API fkm_status fkm_argsort_workspace_size(int64_t n, int n_keys, size_t* byt
 FKM_API fkm_status fkm_argsort(const int32_t* keys, int64_t n, int n_keys, int32_t* idx,
                        int32_t* sorted_keys, void* ws, size_t ws_bytes, void* stream);
 
+/* Centring ("Flash-KMeans" GitHub README, section "Centre your data"):
+ * k-means is translation invariant, so points with a large common offset can
+ * be clustered after subtracting their mean and the centroids shifted back
+ * by it; the tensor-core products then keep their precision.
+ *   mu[b, d]      = fp32((sum over i of x[b, i, d], in fp64) / N)
+ *   x_out[b,i,d]  = x[b,i,d] - mu[b,d], one fp32 subtraction rounded RNE
+ *                   to `dtype` (x_out may be x: centring in place)
+ * x, x_out: device [B, N, D] in dtype; mu: device float32 [B, D]; ws: device
+ * scratch of fkm_centre_workspace_size bytes.  Limits as for fkm_assign
+ * (D * element size a multiple of 16, B * N < 2^31).  Async. */
+FKM_API fkm_status fkm_centre_workspace_size(int B, int N, int D, size_t* bytes);
+FKM_API fkm_status fkm_centre(int B, int N, int D, int dtype, const void* x, float* mu,
+                              void* x_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Comparison point, NOT the method: the "standard" iteration the pages
  * measure against.  Assign materialises the full fp32 distance matrix
  * dist[b,i,k] = ||x||^2 + ||c||^2 - 2 x.c in `dist` (device, B*N*K floats,
