@@ -123,6 +123,10 @@ CONFIGS = {
                 1.1, 1.0, 0.3, 5, 0.0, 20260004),
     5: Workload("mixture_f32_host_B1_N268435456_D64_K16384", 1, 1 << 28, 64, 16384, "f32", 16384,
                 W_EQUAL, 0.0, 1.0, 0.5, 3, 0.0, 20260005, host_resident=True),
+    # large D (README "Large-D and dtype support" runs d = 2048): the assign
+    # kernel streams the point tile with the centroids
+    6: Workload("mixture_bf16_B1_N1048576_D2048_K1024", 1, 1 << 20, 2048, 1024, "bf16", 1024,
+                W_EQUAL, 0.0, 1.0, 0.5, 10, 0.0, 20260006),
 }
 
 

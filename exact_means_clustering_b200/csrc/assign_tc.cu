@@ -67,6 +67,11 @@ constexpr int AUG_COLS = 16;                             // the bias slab: one K
 constexpr int AUG_A_BYTES = BM * AUG_COLS * 2;           // 4 KB, constant per CTA
 constexpr int AUG_B_BYTES = BN * AUG_COLS * 2;           // 8 KB per centroid tile
 constexpr int STAGE_BYTES = B_CHUNK_BYTES + AUG_B_BYTES; // chunk + bias slot
+// Large D (the point tile does not fit shared memory): every stage also
+// carries the 128 x 64 point chunk its products need, so the point tile is
+// streamed once per centroid tile (from L2 after the first) while the TMEM
+// accumulator persists across the D chunks.
+constexpr int STAGE_BYTES_STREAM = B_CHUNK_BYTES + A_CHUNK_BYTES + AUG_B_BYTES;
 
 struct AssignKParams {
   int B, N, Kp, K;
@@ -205,7 +210,7 @@ __device__ __forceinline__ void write_aug_a(uint8_t* base, int f16) {
 // kDist = true is the comparison ("standard") mode: the same tensor-core tiles,
 // but the epilogue writes every distance ||x - c_hat||^2 = ||x - m||^2 - 2 acc
 // to HBM instead of reducing it, as the pages' baseline assignment does.
-template <bool kSplit, bool kDist>
+template <bool kSplit, bool kDist, bool kStreamA>
 __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tm_x,    // points (hi part when split)
                      const __grid_constant__ CUtensorMap tm_xl,   // lo part (split only)
@@ -217,10 +222,12 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  constexpr int kStageBytes = kStreamA ? STAGE_BYTES_STREAM : STAGE_BYTES;
+  constexpr int kAugOff = kStreamA ? B_CHUNK_BYTES + A_CHUNK_BYTES : B_CHUNK_BYTES;
   uint8_t* a_base = smem;
-  uint8_t* aug_a = a_base + (size_t)p.nA * p.a_bytes;
+  uint8_t* aug_a = a_base + (kStreamA ? 0 : (size_t)p.nA * p.a_bytes);
   uint8_t* b_base = aug_a + AUG_A_BYTES;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(b_base + (size_t)p.nS * STAGE_BYTES);
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(b_base + (size_t)p.nS * kStageBytes);
   float4* save_base = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(ctl) +
                                                 ((sizeof(SmemCtl) + 127) & ~size_t(127)));
 
@@ -274,19 +281,22 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
       bool ok = true;
       for (int w = blockIdx.x; w < p.n_work && ok; w += gridDim.x) {
         const int b = w / p.m_tiles, mt = w % p.m_tiles;
-        const int ab = a_arms % p.nA;
-        const uint32_t apar = ((a_arms / p.nA) & 1) ^ 1;
-        if (!ptx::mbar_wait_bounded(&ctl->a_empty[ab], apar, abort_flag, p.status, ST_TIMEOUT,
-                                    kWaitTimeoutNs)) { ok = false; break; }
-        ptx::mbar_arrive_expect_tx(&ctl->a_full[ab], p.a_bytes);
-        uint8_t* abuf = a_base + (size_t)ab * p.a_bytes;
-        for (int dc = 0; dc < p.nD; ++dc) {
-          ptx::tma_load_3d(abuf + dc * A_CHUNK_BYTES, &tm_x, &ctl->a_full[ab], dc * KC, mt * BM, b);
-          if (kSplit)
-            ptx::tma_load_3d(abuf + (p.nD + dc) * A_CHUNK_BYTES, &tm_xl, &ctl->a_full[ab], dc * KC,
-                             mt * BM, b);
+        if (!kStreamA) {
+          const int ab = a_arms % p.nA;
+          const uint32_t apar = ((a_arms / p.nA) & 1) ^ 1;
+          if (!ptx::mbar_wait_bounded(&ctl->a_empty[ab], apar, abort_flag, p.status, ST_TIMEOUT,
+                                      kWaitTimeoutNs)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&ctl->a_full[ab], p.a_bytes);
+          uint8_t* abuf = a_base + (size_t)ab * p.a_bytes;
+          for (int dc = 0; dc < p.nD; ++dc) {
+            ptx::tma_load_3d(abuf + dc * A_CHUNK_BYTES, &tm_x, &ctl->a_full[ab], dc * KC, mt * BM,
+                             b);
+            if (kSplit)
+              ptx::tma_load_3d(abuf + (p.nD + dc) * A_CHUNK_BYTES, &tm_xl, &ctl->a_full[ab],
+                               dc * KC, mt * BM, b);
+          }
+          ++a_arms;
         }
-        ++a_arms;
         for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
           // one stage per 64-wide chunk (split operands: hi and lo in
           // consecutive stages); the tile's bias slab rides with its first chunk
@@ -297,18 +307,21 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
             if (!ptx::mbar_wait_bounded(&ctl->b_empty[sb], spar, abort_flag, p.status, ST_TIMEOUT,
                                         kWaitTimeoutNs)) { ok = false; break; }
             ptx::mbar_arrive_expect_tx(&ctl->b_full[sb],
-                                       B_CHUNK_BYTES + (q == 0 ? AUG_B_BYTES : 0));
-            uint8_t* sbuf = b_base + (size_t)sb * STAGE_BYTES;
+                                       B_CHUNK_BYTES + (kStreamA ? A_CHUNK_BYTES : 0) +
+                                           (q == 0 ? AUG_B_BYTES : 0));
+            uint8_t* sbuf = b_base + (size_t)sb * kStageBytes;
             ptx::tma_load_3d(sbuf, (kSplit && (q & 1)) ? &tm_cl : &tm_c, &ctl->b_full[sb],
                              dc * KC, kt * BN, b);
+            if (kStreamA)   // the point chunk these products need
+              ptx::tma_load_3d(sbuf + B_CHUNK_BYTES, &tm_x, &ctl->b_full[sb], dc * KC, mt * BM, b);
             if (q == 0)
-              ptx::tma_load_3d(sbuf + B_CHUNK_BYTES, &tm_aug, &ctl->b_full[sb], 0, kt * BN, b);
+              ptx::tma_load_3d(sbuf + kAugOff, &tm_aug, &ctl->b_full[sb], 0, kt * BN, b);
             ++s_arms;
           }
         }
       }
       // Drain: every buffer's most recent load must have landed before exit.
-      for (uint32_t i = 0; i < (uint32_t)p.nA && i < a_arms; ++i) {
+      for (uint32_t i = 0; !kStreamA && i < (uint32_t)p.nA && i < a_arms; ++i) {
         uint32_t last = i + p.nA * ((a_arms - 1 - i) / p.nA);
         ptx::mbar_wait_bounded(&ctl->a_full[i], (last / p.nA) & 1, abort_flag, p.status,
                                ST_TIMEOUT, kWaitTimeoutNs);
@@ -327,10 +340,12 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
       bool ok = true;
       bool issued = false;
       for (int w = blockIdx.x; w < p.n_work && ok; w += gridDim.x) {
-        const int ab = a_uses % p.nA;
-        if (!ptx::mbar_wait_bounded(&ctl->a_full[ab], (a_uses / p.nA) & 1, abort_flag, p.status,
-                                    ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
-        ptx::tc_fence_after();
+        const int ab = kStreamA ? 0 : a_uses % p.nA;
+        if (!kStreamA) {
+          if (!ptx::mbar_wait_bounded(&ctl->a_full[ab], (a_uses / p.nA) & 1, abort_flag,
+                                      p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+          ptx::tc_fence_after();
+        }
         const uint32_t a_addr = ptx::smem_u32(a_base + (size_t)ab * p.a_bytes);
         for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
           const int acc = acc_uses & 1;
@@ -344,11 +359,11 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
             if (!ptx::mbar_wait_bounded(&ctl->b_full[sb], (s_uses / p.nS) & 1, abort_flag,
                                         p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
             ptx::tc_fence_after();
-            const uint32_t b_addr = ptx::smem_u32(b_base + (size_t)sb * STAGE_BYTES);
-            const uint32_t xa = a_addr + dc * A_CHUNK_BYTES;
+            const uint32_t b_addr = ptx::smem_u32(b_base + (size_t)sb * kStageBytes);
+            const uint32_t xa = kStreamA ? b_addr + B_CHUNK_BYTES : a_addr + dc * A_CHUNK_BYTES;
             if (q == 0)   // the bias product starts the tile's accumulation
               ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw32(aug_a_addr),
-                              ptx::umma_desc_sw32(b_addr + B_CHUNK_BYTES), p.idesc, 0u);
+                              ptx::umma_desc_sw32(b_addr + kAugOff), p.idesc, 0u);
             if (!(kSplit && (q & 1))) {
               // xh . ch (or x . q(c - m))
 #pragma unroll
@@ -377,8 +392,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
           ++acc_uses;
         }
         if (!ok) break;
-        ptx::mma_commit(&ctl->a_empty[ab]);
-        ++a_uses;
+        if (!kStreamA) {
+          ptx::mma_commit(&ctl->a_empty[ab]);
+          ++a_uses;
+        }
       }
       // Drain: all MMAs this thread issued must finish before TMEM is freed.
       if (issued) {
@@ -519,22 +536,34 @@ constexpr int kSmemBudget = 232448 - 1024;  // opt-in maximum minus alignment sl
 }  // namespace
 
 // Shared-memory plan of the assign kernel for D (also used by validation).
-bool assign_smem_plan(int D, bool split, int* nA_out, int* nS_out, size_t* smem_out) {
+// The point tile stays resident (double-buffered when it fits) up to D = 256;
+// beyond that, 16-bit points are streamed chunk by chunk with the centroids.
+bool assign_smem_plan(int D, bool split, int* nA_out, int* nS_out, size_t* smem_out,
+                      bool* stream_out) {
   const int nD = (int)ceil_div(D, KC);
   const long a_bytes = (long)(split ? 2 : 1) * nD * A_CHUNK_BYTES;
-  const long s_bytes = STAGE_BYTES;
   const long ctl = (long)((sizeof(SmemCtl) + 127) & ~size_t(127)) + kSaveBytes + AUG_A_BYTES;
-  int nA = 2;
-  long nS = (kSmemBudget - ctl - 2 * a_bytes) / s_bytes;
-  if (nS < 2) {
-    nA = 1;
-    nS = (kSmemBudget - ctl - a_bytes) / s_bytes;
+  int nA = 0;
+  long nS = 0, s_bytes = STAGE_BYTES;
+  bool stream = false;
+  if (D <= 256) {
+    nA = 2;
+    nS = (kSmemBudget - ctl - 2 * a_bytes) / s_bytes;
+    if (nS < 2) {
+      nA = 1;
+      nS = (kSmemBudget - ctl - a_bytes) / s_bytes;
+    }
+  } else if (!split && D <= ASSIGN_MAX_D) {
+    stream = true;
+    s_bytes = STAGE_BYTES_STREAM;
+    nS = (kSmemBudget - ctl) / s_bytes;
   }
   if (nS > 8) nS = 8;
   if (nS < 2) return false;
   if (nA_out) *nA_out = nA;
   if (nS_out) *nS_out = (int)nS;
   if (smem_out) *smem_out = (size_t)(nA * a_bytes + nS * s_bytes + ctl + 1024);
+  if (stream_out) *stream_out = stream;
   return true;
 }
 
@@ -546,13 +575,17 @@ fkm_status assign_prepare() {
   FKM_CUDA_TRY(cudaGetDevice(&dev));
   if (dev >= 0 && dev < 64 && done[dev]) return FKM_OK;
   const int lim = kSmemBudget + 1024;
-  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<true, false>,
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<true, false, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, false>,
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, false, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<true, true>,
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<true, true, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, true>,
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, true, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, false, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, true, true>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
   if (dev >= 0 && dev < 64) done[dev] = true;
   return FKM_OK;
@@ -561,7 +594,8 @@ fkm_status assign_prepare() {
 fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
   int nA = 0, nS = 0;
   size_t smem = 0;
-  if (!assign_smem_plan(a.D, a.split, &nA, &nS, &smem)) {
+  bool stream = false;
+  if (!assign_smem_plan(a.D, a.split, &nA, &nS, &smem, &stream)) {
     set_error("D=%d does not fit the assign kernel's shared memory", a.D);
     return FKM_ERR_UNSUPPORTED;
   }
@@ -606,15 +640,26 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
   const int sms = num_sms();
   const int grid = p.n_work < sms ? p.n_work : sms;
   FKM_TRY(assign_prepare());
-  if (a.dist) {
-    if (a.split)
-      assign_tc_kernel<true, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
+  if (stream) {
+    if (a.dist)
+      assign_tc_kernel<false, true, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                              taug, p);
     else
-      assign_tc_kernel<false, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
+      assign_tc_kernel<false, false, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                               taug, p);
+  } else if (a.dist) {
+    if (a.split)
+      assign_tc_kernel<true, true, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                              taug, p);
+    else
+      assign_tc_kernel<false, true, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                               taug, p);
   } else if (a.split) {
-    assign_tc_kernel<true, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
+    assign_tc_kernel<true, false, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                             taug, p);
   } else {
-    assign_tc_kernel<false, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl, taug, p);
+    assign_tc_kernel<false, false, false><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                              taug, p);
   }
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());

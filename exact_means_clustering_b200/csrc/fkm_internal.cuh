@@ -97,7 +97,9 @@ struct AssignArgs {
   float* dist = nullptr;  // comparison mode: write the [B, N, K] distances here
 };
 fkm_status launch_assign(const AssignArgs& a, cudaStream_t st);
-bool assign_smem_plan(int D, bool split, int* nA, int* nS, size_t* smem);
+// Largest D of 16-bit points (streamed point tiles); fp32 points: 128.
+constexpr int ASSIGN_MAX_D = 4096;
+bool assign_smem_plan(int D, bool split, int* nA, int* nS, size_t* smem, bool* stream = nullptr);
 fkm_status assign_prepare();
 
 // Per batch mean centroid m [B][D]; q(c - m) rows [B][Kp][Dq] (split rows

@@ -41,15 +41,20 @@ __global__ void seg_bounds_kernel(const int32_t* __restrict__ skeys, int64_t n, 
   if (i == n - 1 || skeys[i + 1] != k) segend[k] = (int32_t)(i + 1);
 }
 
+// Rows longer than 512 bytes are summed in slabs of columns, one launch per
+// slab: x, centers, sums64, the centroid rows and the mean point at the slab's
+// first column, D its width, Dfull the whole row length.
 struct SegParams {
   const void* x;
   const int32_t* skeys;
   const int32_t* svals;
   int64_t n;
-  int D;
+  int D;                 // columns in this slab
+  int Dfull;             // columns of a whole row (stride of centers / sums / centroid rows)
   int BK;
-  int64_t row_bytes;
-  int V;                 // 16-byte vectors per row
+  int64_t row_bytes;     // bytes between rows of x
+  int ebytes;            // bytes per element of x
+  int V;                 // 16-byte vectors per slab row
   double* sums64;
   float* centers;
   bool accumulate_all;   // out-of-core chunks: every run goes to sums64
@@ -136,12 +141,12 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
     const int64_t col0 = (int64_t)sub * E;
     if (interior) {
       const double n = (double)nk;
-      float* c = p.centers + (int64_t)key * p.D + col0;
+      float* c = p.centers + (int64_t)key * p.Dfull + col0;
 #pragma unroll
       for (int e = 0; e < E; ++e)
         if (col0 + e < p.D) c[e] = (float)(acc[e] / n);
     } else {
-      double* sd = p.sums64 + (int64_t)key * p.D + col0;
+      double* sd = p.sums64 + (int64_t)key * p.Dfull + col0;
 #pragma unroll
       for (int e = 0; e < E; ++e)
         if (col0 + e < p.D) atomicAdd(sd + e, acc[e]);
@@ -207,7 +212,7 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
   const int g = lane / LPR, sub = lane % LPR;
   const bool lane_has_vec = sub < p.V;
   const bool want_obj = p.oa.obj != nullptr;
-  const int64_t elem_bytes_ = p.row_bytes / p.D;
+  const int64_t elem_bytes_ = p.ebytes;
   const int64_t r = (int64_t)blockIdx.x * SEG_WARPS + wid;
   const int64_t nranges = ceil_div(p.n, SEG_RANGE);
   if (r >= nranges) return;
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     const int kg = ws.kv[ws.runs[run]].x;
     const int b = kg / p.oa.K, k = kg % p.oa.K;
     const char* row = static_cast<const char*>(p.oa.chat) +
-                      ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.D) * elem_bytes_;
+                      ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.Dfull) * elem_bytes_;
     chat_next = ldg_nc_v4(row + (int64_t)sub * 16);
   };
   prefetch_chat(0);
@@ -361,7 +366,8 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
       float2 c2[E / 2];
       Vec<DT>::widen2(chat_next, c2);
       if (p.oa.m) {   // the batch's mean centroid: a few KB, cache-resident
-        const float2* mb = reinterpret_cast<const float2*>(p.oa.m + (int64_t)b * p.D) + sub * (E / 2);
+        const float2* mb =
+            reinterpret_cast<const float2*>(p.oa.m + (int64_t)b * p.Dfull) + sub * (E / 2);
 #pragma unroll
         for (int e = 0; e < E / 2; ++e) c2[e] = __fadd2_rn(c2[e], mb[e]);
       }
@@ -428,24 +434,26 @@ __global__ void __launch_bounds__(256) objective_kernel(const void* __restrict__
   double acc = 0.0;
   for (int64_t i = r0 + warp; i < r0 + rows_per_block && i < N; i += 8) {
     const int id = ids[(int64_t)b * N + i];
-    if (id < 0 || id >= oa.K || lane >= V) continue;
-    float f[E], c[E];
-    Vec<DT>::widen(ldg_nc_v4(static_cast<const char*>(x) + ((int64_t)b * N + i) * row_bytes +
-                             lane * 16),
-                   f);
-    const char* crow = static_cast<const char*>(oa.chat) +
-                       ((int64_t)b * oa.chat_bstride + (int64_t)id * D) * (row_bytes / D);
-    Vec<DT>::widen(ldg_nc_v4(crow + lane * 16), c);
-    if (oa.m) {
-      const float* mb = oa.m + (int64_t)b * D + (int64_t)lane * E;
-#pragma unroll
-      for (int e = 0; e < E; ++e) c[e] += mb[e];
-    }
+    if (id < 0 || id >= oa.K) continue;
     float d2 = 0.0f;
+    for (int v = lane; v < V; v += 32) {   // the row's 16-byte vectors
+      float f[E], c[E];
+      Vec<DT>::widen(ldg_nc_v4(static_cast<const char*>(x) + ((int64_t)b * N + i) * row_bytes +
+                               (int64_t)v * 16),
+                     f);
+      const char* crow = static_cast<const char*>(oa.chat) +
+                         ((int64_t)b * oa.chat_bstride + (int64_t)id * D) * (row_bytes / D);
+      Vec<DT>::widen(ldg_nc_v4(crow + (int64_t)v * 16), c);
+      if (oa.m) {
+        const float* mb = oa.m + (int64_t)b * D + (int64_t)v * E;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float df = f[e] - c[e];
-      d2 = fmaf(df, df, d2);
+        for (int e = 0; e < E; ++e) c[e] += mb[e];
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float df = f[e] - c[e];
+        d2 = fmaf(df, df, d2);
+      }
     }
     acc += (double)d2;
   }
@@ -622,27 +630,31 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          bool accumulate_all, const ObjArgs& oa, cudaStream_t st) {
   if (n == 0) return FKM_OK;
   FKM_TRY(segsum_prepare());
-  SegParams sp;
-  sp.x = x;
-  sp.skeys = skeys;
-  sp.svals = svals;
-  sp.n = n;
-  sp.D = D;
-  sp.BK = BK;
-  sp.row_bytes = (int64_t)D * elem_bytes(dtype);
-  sp.V = (int)(sp.row_bytes / 16);
-  sp.sums64 = sums64;
-  sp.centers = centers;
-  sp.accumulate_all = accumulate_all;
-  sp.oa = oa;
-  if (sp.V > 32) {
-    set_error("rows of %lld bytes exceed the update kernel's 512-byte limit",
-              (long long)sp.row_bytes);
-    return FKM_ERR_UNSUPPORTED;
+  const int eb = elem_bytes(dtype);
+  const int slab = 512 / eb;   // columns per launch: 512-byte row pieces
+  for (int c0 = 0; c0 < D; c0 += slab) {
+    SegParams sp;
+    sp.x = static_cast<const char*>(x) + (int64_t)c0 * eb;
+    sp.skeys = skeys;
+    sp.svals = svals;
+    sp.n = n;
+    sp.D = D - c0 < slab ? D - c0 : slab;
+    sp.Dfull = D;
+    sp.BK = BK;
+    sp.row_bytes = (int64_t)D * eb;
+    sp.ebytes = eb;
+    sp.V = (int)((int64_t)sp.D * eb / 16);
+    sp.sums64 = sums64 + c0;
+    sp.centers = centers ? centers + c0 : nullptr;
+    sp.accumulate_all = accumulate_all;
+    sp.oa = oa;
+    if (oa.chat) sp.oa.chat = static_cast<const char*>(oa.chat) + (int64_t)c0 * eb;
+    if (oa.m) sp.oa.m = oa.m + c0;
+    if (dtype == FKM_BF16) FKM_TRY(run_segsum_dt<FKM_BF16>(sp, st));
+    else if (dtype == FKM_F16) FKM_TRY(run_segsum_dt<FKM_F16>(sp, st));
+    else FKM_TRY(run_segsum_dt<FKM_F32>(sp, st));
   }
-  if (dtype == FKM_BF16) return run_segsum_dt<FKM_BF16>(sp, st);
-  if (dtype == FKM_F16) return run_segsum_dt<FKM_F16>(sp, st);
-  return run_segsum_dt<FKM_F32>(sp, st);
+  return FKM_OK;
 }
 
 fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const int32_t* ids,

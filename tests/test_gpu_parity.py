@@ -455,3 +455,52 @@ def test_lloyd_host_injected_copy_failure(monkeypatch):
     assert n == 3
     assert torch.equal(ids, i2) and torch.equal(counts, n2)
     assert torch.allclose(centers, c2, rtol=1e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------------ large D
+# D above 256 (16-bit points): the assign kernel streams the point tile chunk
+# by chunk with the centroids (the accumulator persists across the D chunks),
+# and the segment sums run over 512-byte column slabs of each row.
+@pytest.mark.parametrize("dtype,B,N,K,D", [("bf16", 2, 3000, 300, 512), ("f16", 1, 2500, 257, 1024),
+                                           ("bf16", 1, 1500, 64, 2048), ("bf16", 1, 700, 40, 264)])
+def test_large_d(dtype, B, N, K, D):
+    w = datagen.Workload("large_d", B, N, D, K, dtype, K, sigma=0.5, iters=3, seed=D + N)
+    x, xt, c0 = problem(w)
+    c0t = torch.from_numpy(c0).cuda()
+    mir = _mirror(dtype)
+    # assign, teacher-forced, from the oracle's centroids after one iteration
+    c1 = oracle.lloyd(x, c0, 1, dtype=dtype, mirror=mir)["centers"].astype(np.float32)
+    ids = torch.empty(B, N, dtype=torch.int32, device="cuda")
+    inertia = torch.empty(B, dtype=torch.float64, device="cuda")
+    fkm.fkm_assign(xt, torch.from_numpy(c1).cuda(), ids, inertia)
+    g = ids.cpu().numpy()
+    check_assign(x, dtype, c1, g)
+    J = oracle.inertia(x, g, c1.astype(np.float64), dtype=dtype, mirror=mir)
+    for b in range(B):
+        assert rel(inertia[b].item(), J[b]) < 1e-4
+    # update, teacher-forced on those ids
+    c = torch.empty(B, K, D, device="cuda")
+    n = torch.empty(B, K, dtype=torch.int32, device="cuda")
+    fkm.fkm_update(xt, ids, torch.from_numpy(c1).cuda(), c, n)
+    check_update(x, dtype, g, c1, c.cpu().numpy(), n.cpu().numpy())
+    # the loop against the oracle's own run
+    i3, c3, n3 = _empty(B, N, K, D)
+    in3 = torch.empty(B, dtype=torch.float64, device="cuda")
+    assert fkm.fkm_lloyd(xt, c0t, 3, 0.0, i3, c3, n3, in3) == 3
+    ref = oracle.lloyd(x, c0, 3, dtype=dtype, mirror=mir)
+    for b in range(B):
+        agree = (i3[b].cpu().numpy() == ref["ids"][b]).mean()
+        assert agree > 0.999, agree
+        assert rel(in3[b].item(), ref["inertia"][b]) < 2e-3
+
+
+def test_large_d_host_streaming():
+    w = datagen.Workload("large_d_host", 1, 6000, 512, 100, "bf16", 100, sigma=0.5, iters=2, seed=9)
+    x, xt, c0 = problem(w)
+    ids, centers, counts = _empty(1, w.N, w.K, w.D)
+    fkm.fkm_lloyd_host(xt.cpu().pin_memory(), torch.from_numpy(c0).cuda(), 2, 0.0, 2048, ids,
+                       centers, counts)
+    i2, c2, n2 = _empty(1, w.N, w.K, w.D)
+    fkm.fkm_lloyd(xt, torch.from_numpy(c0).cuda(), 2, 0.0, i2, c2, n2)
+    assert (ids != i2).float().mean().item() <= 1e-3
+    assert torch.allclose(centers, c2, rtol=1e-4, atol=1e-4)
