@@ -127,6 +127,9 @@ CONFIGS = {
     # kernel streams the point tile with the centroids
     6: Workload("mixture_bf16_B1_N1048576_D2048_K1024", 1, 1 << 20, 2048, 1024, "bf16", 1024,
                 W_EQUAL, 0.0, 1.0, 0.5, 10, 0.0, 20260006),
+    # the README's "d=2048, k=1024, fp32" shape: split-bf16 operands, streamed
+    7: Workload("mixture_f32_B1_N262144_D2048_K1024", 1, 1 << 18, 2048, 1024, "f32", 1024,
+                W_EQUAL, 0.0, 1.0, 0.5, 10, 0.0, 20260007),
 }
 
 

@@ -117,9 +117,8 @@ static fkm_status validate_shape(int B, int N, int K, int D, int dtype) {
     set_error("D * sizeof(dtype) = %d is not a multiple of 16 bytes", D * s);
     return FKM_ERR_UNSUPPORTED;
   }
-  if ((dtype == FKM_F32 && D > 128) || D > ASSIGN_MAX_D) {
-    set_error("D = %d exceeds the supported maximum (%d for 16-bit points, 128 for fp32)", D,
-              ASSIGN_MAX_D);
+  if (D > ASSIGN_MAX_D) {
+    set_error("D = %d exceeds the supported maximum of %d", D, ASSIGN_MAX_D);
     return FKM_ERR_UNSUPPORTED;
   }
   if ((int64_t)B * N >= (int64_t(1) << 31) || (int64_t)B * K >= (int64_t(1) << 31) - 1) {

@@ -72,6 +72,9 @@ constexpr int STAGE_BYTES = B_CHUNK_BYTES + AUG_B_BYTES; // chunk + bias slot
 // streamed once per centroid tile (from L2 after the first) while the TMEM
 // accumulator persists across the D chunks.
 constexpr int STAGE_BYTES_STREAM = B_CHUNK_BYTES + A_CHUNK_BYTES + AUG_B_BYTES;
+// fp32 points (split hi / lo operands): a stage carries one centroid part (hi
+// or lo), the point hi chunk, and for the hi part also the point lo chunk.
+constexpr int STAGE_BYTES_STREAM_SPLIT = B_CHUNK_BYTES + 2 * A_CHUNK_BYTES + AUG_B_BYTES;
 
 struct AssignKParams {
   int B, N, Kp, K;
@@ -222,8 +225,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  constexpr int kStageBytes = kStreamA ? STAGE_BYTES_STREAM : STAGE_BYTES;
-  constexpr int kAugOff = kStreamA ? B_CHUNK_BYTES + A_CHUNK_BYTES : B_CHUNK_BYTES;
+  constexpr int kStageBytes =
+      kStreamA ? (kSplit ? STAGE_BYTES_STREAM_SPLIT : STAGE_BYTES_STREAM) : STAGE_BYTES;
+  constexpr int kAugOff =
+      kStreamA ? B_CHUNK_BYTES + (kSplit ? 2 : 1) * A_CHUNK_BYTES : B_CHUNK_BYTES;
   uint8_t* a_base = smem;
   uint8_t* aug_a = a_base + (kStreamA ? 0 : (size_t)p.nA * p.a_bytes);
   uint8_t* b_base = aug_a + AUG_A_BYTES;
@@ -306,14 +311,20 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
             const uint32_t spar = ((s_arms / p.nS) & 1) ^ 1;
             if (!ptx::mbar_wait_bounded(&ctl->b_empty[sb], spar, abort_flag, p.status, ST_TIMEOUT,
                                         kWaitTimeoutNs)) { ok = false; break; }
+            // streamed points: the hi part of a split chunk also needs the lo points
+            const bool lo_pts = kStreamA && kSplit && !(q & 1);
             ptx::mbar_arrive_expect_tx(&ctl->b_full[sb],
                                        B_CHUNK_BYTES + (kStreamA ? A_CHUNK_BYTES : 0) +
+                                           (lo_pts ? A_CHUNK_BYTES : 0) +
                                            (q == 0 ? AUG_B_BYTES : 0));
             uint8_t* sbuf = b_base + (size_t)sb * kStageBytes;
             ptx::tma_load_3d(sbuf, (kSplit && (q & 1)) ? &tm_cl : &tm_c, &ctl->b_full[sb],
                              dc * KC, kt * BN, b);
             if (kStreamA)   // the point chunk these products need
               ptx::tma_load_3d(sbuf + B_CHUNK_BYTES, &tm_x, &ctl->b_full[sb], dc * KC, mt * BM, b);
+            if (lo_pts)
+              ptx::tma_load_3d(sbuf + B_CHUNK_BYTES + A_CHUNK_BYTES, &tm_xl, &ctl->b_full[sb],
+                               dc * KC, mt * BM, b);
             if (q == 0)
               ptx::tma_load_3d(sbuf + kAugOff, &tm_aug, &ctl->b_full[sb], 0, kt * BN, b);
             ++s_arms;
@@ -371,7 +382,8 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
                 ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xa + 32 * k),
                                 ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc, 1u);
               if (kSplit) {   // xl . ch
-                const uint32_t xl = a_addr + (p.nD + dc) * A_CHUNK_BYTES;
+                const uint32_t xl = kStreamA ? b_addr + B_CHUNK_BYTES + A_CHUNK_BYTES
+                                             : a_addr + (p.nD + dc) * A_CHUNK_BYTES;
 #pragma unroll
                 for (int k = 0; k < KC / 16; ++k)
                   ptx::mma_f16_ss(d_tmem, ptx::umma_desc_sw128(xl + 32 * k),
@@ -536,8 +548,9 @@ constexpr int kSmemBudget = 232448 - 1024;  // opt-in maximum minus alignment sl
 }  // namespace
 
 // Shared-memory plan of the assign kernel for D (also used by validation).
-// The point tile stays resident (double-buffered when it fits) up to D = 256;
-// beyond that, 16-bit points are streamed chunk by chunk with the centroids.
+// The point tile stays resident (double-buffered when it fits) up to D = 256
+// (fp32 points: 128); beyond that it is streamed chunk by chunk with the
+// centroids.
 bool assign_smem_plan(int D, bool split, int* nA_out, int* nS_out, size_t* smem_out,
                       bool* stream_out) {
   const int nD = (int)ceil_div(D, KC);
@@ -546,16 +559,16 @@ bool assign_smem_plan(int D, bool split, int* nA_out, int* nS_out, size_t* smem_
   int nA = 0;
   long nS = 0, s_bytes = STAGE_BYTES;
   bool stream = false;
-  if (D <= 256) {
+  if (D <= (split ? 128 : 256)) {
     nA = 2;
     nS = (kSmemBudget - ctl - 2 * a_bytes) / s_bytes;
     if (nS < 2) {
       nA = 1;
       nS = (kSmemBudget - ctl - a_bytes) / s_bytes;
     }
-  } else if (!split && D <= ASSIGN_MAX_D) {
+  } else if (D <= ASSIGN_MAX_D) {
     stream = true;
-    s_bytes = STAGE_BYTES_STREAM;
+    s_bytes = split ? STAGE_BYTES_STREAM_SPLIT : STAGE_BYTES_STREAM;
     nS = (kSmemBudget - ctl) / s_bytes;
   }
   if (nS > 8) nS = 8;
@@ -586,6 +599,10 @@ fkm_status assign_prepare() {
   FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, false, true>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
   FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<false, true, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<true, false, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<true, true, true>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
   if (dev >= 0 && dev < 64) done[dev] = true;
   return FKM_OK;
@@ -641,7 +658,13 @@ fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
   const int grid = p.n_work < sms ? p.n_work : sms;
   FKM_TRY(assign_prepare());
   if (stream) {
-    if (a.dist)
+    if (a.split && a.dist)
+      assign_tc_kernel<true, true, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                             taug, p);
+    else if (a.split)
+      assign_tc_kernel<true, false, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
+                                                                              taug, p);
+    else if (a.dist)
       assign_tc_kernel<false, true, true><<<grid, ASSIGN_THREADS, smem, st>>>(tx, txl, tc, tcl,
                                                                               taug, p);
     else

@@ -97,7 +97,7 @@ struct AssignArgs {
   float* dist = nullptr;  // comparison mode: write the [B, N, K] distances here
 };
 fkm_status launch_assign(const AssignArgs& a, cudaStream_t st);
-// Largest D of 16-bit points (streamed point tiles); fp32 points: 128.
+// Largest D (point tiles streamed with the centroids above 256, fp32: 128).
 constexpr int ASSIGN_MAX_D = 4096;
 bool assign_smem_plan(int D, bool split, int* nA, int* nS, size_t* smem, bool* stream = nullptr);
 fkm_status assign_prepare();

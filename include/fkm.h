@@ -24,8 +24,8 @@
  *              before the GPU finishes.
  *   Limits     B, N, K, D >= 1; D * sizeof(dtype) a multiple of 16 bytes
  *              (D % 8 == 0 for bf16/fp16, D % 4 == 0 for fp32);
- *              D <= 4096 (fp32: D <= 128); B*N < 2^31; B*K < 2^31.  Above
- *              D = 256 the assign kernel streams the point tile in 64-column
+ *              D <= 4096; B*N < 2^31; B*K < 2^31.  Above D = 256 (fp32:
+ *              128) the assign kernel streams the point tile in 64-column
  *              chunks and the update sums 512-byte column slabs.
  *   Errors     Arguments are validated before anything is launched; a violation
  *              returns FKM_ERR_INVALID_ARG or FKM_ERR_UNSUPPORTED and launches

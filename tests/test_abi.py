@@ -65,7 +65,7 @@ def test_workspace_size_is_independent_of_n_times_k(fkm):
     ((1, 10, 4, 12, 2), 2),        # 24-byte rows: not a multiple of 16
     ((1, 10, 4, 6, 0), 2),         # 24-byte fp32 rows
     ((1, 10, 4, 4104, 2), 2),      # D too large for 16-bit points
-    ((1, 10, 4, 132, 0), 2),       # D too large for fp32 points
+    ((1, 10, 4, 4100, 0), 2),      # D too large for fp32 points
     ((2, 1 << 30, 4, 64, 2), 2),   # B*N >= 2^31
 ])
 def test_invalid_shapes_are_rejected(fkm, shape, code):

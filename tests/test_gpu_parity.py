@@ -458,11 +458,13 @@ def test_lloyd_host_injected_copy_failure(monkeypatch):
 
 
 # ------------------------------------------------------------------ large D
-# D above 256 (16-bit points): the assign kernel streams the point tile chunk
-# by chunk with the centroids (the accumulator persists across the D chunks),
-# and the segment sums run over 512-byte column slabs of each row.
+# D above 256 (fp32 points: 128): the assign kernel streams the point tile
+# chunk by chunk with the centroids (the accumulator persists across the D
+# chunks), and the segment sums run over 512-byte column slabs of each row.
 @pytest.mark.parametrize("dtype,B,N,K,D", [("bf16", 2, 3000, 300, 512), ("f16", 1, 2500, 257, 1024),
-                                           ("bf16", 1, 1500, 64, 2048), ("bf16", 1, 700, 40, 264)])
+                                           ("bf16", 1, 1500, 64, 2048), ("bf16", 1, 700, 40, 264),
+                                           ("f32", 1, 1200, 50, 132), ("f32", 2, 900, 70, 512),
+                                           ("f32", 1, 800, 30, 2048)])
 def test_large_d(dtype, B, N, K, D):
     w = datagen.Workload("large_d", B, N, D, K, dtype, K, sigma=0.5, iters=3, seed=D + N)
     x, xt, c0 = problem(w)
