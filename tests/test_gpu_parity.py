@@ -132,9 +132,11 @@ def test_assign_teacher_forced(wid, scale):
 
 
 # ------------------------------------------------------------------ update
+# K <= 2048 takes the one-pass counting sort, larger K the LSD radix sort
 @pytest.mark.parametrize("dtype,B,N,K,D", [("bf16", 2, 9000, 300, 128), ("f16", 3, 4097, 50, 64),
                                            ("f32", 1, 20000, 40, 64), ("f32", 2, 3000, 100, 128),
-                                           ("bf16", 1, 70000, 9, 256), ("bf16", 2, 1, 3, 8)])
+                                           ("bf16", 1, 70000, 9, 256), ("bf16", 2, 1, 3, 8),
+                                           ("bf16", 2, 30000, 3000, 64), ("f16", 1, 9000, 2049, 32)])
 def test_update_teacher_forced(dtype, B, N, K, D):
     rng = np.random.default_rng(N + K)
     w = datagen.Workload("t", B, N, D, K, dtype, 0, sigma=2.0, seed=N)
@@ -177,6 +179,7 @@ def test_update_rejects_bad_ids():
 @pytest.mark.parametrize("wid,scale", [(1, {}), (2, dict(B=4, N=8192, K=128)),
                                        (3, dict(B=4, N=7560, K=100)),
                                        (4, dict(N=60000, K=300)),
+                                       (4, dict(N=50000, K=2500, n_comp=2500)),   # radix sort
                                        (5, dict(N=40000, K=200, iters=3))])
 def test_lloyd_free_running(wid, scale):
     """(i) the reported objective is the oracle's objective of the GPU's own
