@@ -257,9 +257,11 @@ static ObjArgs obj_args(const Ws& w, const float* prev, double* obj) {
 
 // argsort + bounds + segment sums (+ objective) + finalize; prev -> next.
 // obj (device [B], zeroed here) receives the objective of ids against prev.
+// ids_valid: the ids were written by the assign kernel (all in [0, K)).
 static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, const float* prev,
                               float* next, int32_t* counts, bool requant, double* obj,
-                              cudaStream_t st, cudaEvent_t* ev = nullptr) {
+                              cudaStream_t st, cudaEvent_t* ev = nullptr,
+                              bool ids_valid = false) {
   const Layout& L = *w.L;
   SortArgs s;
   s.ids = ids;
@@ -278,18 +280,19 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   int32_t* segstart = w.at<int32_t>(L.segstart);
   int32_t* segend = w.at<int32_t>(L.segend);
   if (L.count_sort) {
-    FKM_TRY(launch_count_sort_ids(s, L.B, segstart, segend, st));
+    FKM_TRY(launch_count_sort_ids(s, L.B, segstart, segend, st, ids_valid));
   } else {
     FKM_TRY(launch_argsort_ids(s, st));
     FKM_TRY(launch_seg_bounds(s.keys_out, L.n_sort, BK, segstart, segend, st));
   }
   if (ev) FKM_TRY(record_stage(ev[2], st));
   if (obj) FKM_CUDA_TRY(cudaMemsetAsync(obj, 0, sizeof(double) * L.B, st));
+  const int range = segsum_range_rows(L.n_sort);
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK,
-                        w.at<double>(L.sums64), next, false, obj_args(w, prev, obj), st));
+                        w.at<double>(L.sums64), next, false, obj_args(w, prev, obj), st, range));
   if (ev) FKM_TRY(record_stage(ev[3], st));
   FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64), prev,
-                          next, counts, w.at<double>(L.shiftk), st));
+                          next, counts, w.at<double>(L.shiftk), st, range));
   // the next assign's operands: offsets of the new centroids from their mean
   if (requant)
     FKM_TRY(launch_prep_centroids(next, L.B, L.K, L.Kp, L.D, L.dtype, w.at<float>(L.mvec),
@@ -365,7 +368,7 @@ static fkm_status lloyd_iterations(const Ws& w, const void* x, int iters, int32_
     if (ev) FKM_TRY(record_stage(ev[0], st));
     FKM_TRY(step_assign(w, x, ids, st));
     if (ev) FKM_TRY(record_stage(ev[1], st));
-    FKM_TRY(step_update(w, x, ids, cur, nxt, counts, true, inertia, st, ev));
+    FKM_TRY(step_update(w, x, ids, cur, nxt, counts, true, inertia, st, ev, true));
     if (track_max) FKM_CUDA_TRY(cudaMemsetAsync(w.max_shift(), 0, sizeof(double), st));
     FKM_TRY(launch_batch_reduce(L.B, L.K, w.at<double>(L.shiftk), shift_dev,
                                 track_max ? w.max_shift() : nullptr, st));

@@ -137,8 +137,11 @@ size_t argsort_scratch_words(int64_t n);
 constexpr int CS_MAX_K = 2048;
 int64_t cs_hist_words(int B, int N, int K);
 size_t cs_scan_scratch_words(int B, int N, int K);
+// ids_valid: every id is known to lie in [0, K) (the assign kernel wrote
+// them), which allows the one-launch path for batches of at most SORT_TILE
+// points.
 fkm_status launch_count_sort_ids(SortArgs& a, int B, int32_t* segstart, int32_t* segend,
-                                 cudaStream_t st);
+                                 cudaStream_t st, bool ids_valid = false);
 fkm_status count_sort_prepare();
 
 fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
@@ -158,7 +161,11 @@ struct ObjArgs {
 };
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
-                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st);
+                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range = 0);
+// Rows per warp range of the segment sums for n sorted rows: SEG_RANGE for
+// large n, fewer (down to 32) when n is small, so a small problem still
+// spreads over many warps.  finalize must be given the same value.
+int segsum_range_rows(int64_t n);
 // Raises the segment-sum kernels' dynamic shared-memory limit once per device
 // (outside any stream capture).
 fkm_status segsum_prepare();
@@ -167,7 +174,8 @@ fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const
                             const ObjArgs& oa, cudaStream_t st);
 fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
                            const int32_t* counts_in, double* sums64, const float* prev,
-                           float* centers, int32_t* counts, double* shiftk, cudaStream_t st);
+                           float* centers, int32_t* counts, double* shiftk, cudaStream_t st,
+                           int range = SEG_RANGE);
 fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
                                double* max_shift, cudaStream_t st);
 

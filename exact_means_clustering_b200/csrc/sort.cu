@@ -366,6 +366,85 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_scatter_kernel(CsArgs a) {
   }
 }
 
+// Small batches (N <= SORT_TILE, every id valid): one block per batch does the
+// whole counting sort of that batch -- stable per-warp ranking as in the
+// scatter pass, the bin totals scanned inside the block, then the scatter --
+// and writes the batch's segment bounds.  Batch b's keys occupy positions
+// [b*N, (b+1)*N).  One launch instead of five.
+__global__ void __launch_bounds__(SORT_THREADS) cs_single_tile_kernel(CsArgs a) {
+  constexpr int NW = SORT_THREADS / 32;
+  constexpr int PER_WARP = SORT_TILE / NW;
+  extern __shared__ uint32_t cnt[];   // NW * (K + 1) per-warp counters, then K + 1 bin starts
+  __shared__ uint32_t sw[32];
+  const int KB = a.K + 1;
+  uint32_t* start = cnt + NW * KB;
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < NW * KB; i += SORT_THREADS) cnt[i] = 0;
+  const int64_t row0 = (int64_t)b * a.N;
+  int bin[SORT_ITEMS];
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    const int i = warp * PER_WARP + r * 32 + lane;
+    bin[r] = a.K + 1;
+    if (i < a.N) {
+      const int id = a.ids[row0 + i];
+      bin[r] = (id < 0 || id >= a.K) ? a.K : id;   // cannot happen for valid ids
+    }
+  }
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  uint32_t* wc = cnt + warp * KB;
+  uint32_t rank[SORT_ITEMS];
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    const unsigned peers = __match_any_sync(0xffffffffu, bin[r]);
+    uint32_t before = 0;
+    if (bin[r] <= a.K) before = wc[bin[r]];
+    rank[r] = before + __popc(peers & lt_mask);
+    __syncwarp();
+    if (bin[r] <= a.K && lane == __ffs(peers) - 1) wc[bin[r]] = before + __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per bin: earlier warps' counts become offsets; the bin total is kept
+  for (int k = threadIdx.x; k < KB; k += SORT_THREADS) {
+    uint32_t run = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t c = cnt[w * KB + k];
+      cnt[w * KB + k] = run;
+      run += c;
+    }
+    start[k] = run;
+  }
+  __syncthreads();
+  // exclusive scan of the bin totals: thread t owns bins [t*kpt, (t+1)*kpt)
+  const int kpt = (KB + SORT_THREADS - 1) / SORT_THREADS;
+  const int k0 = threadIdx.x * kpt;
+  uint32_t local = 0;
+  for (int k = k0; k < k0 + kpt && k < KB; ++k) local += start[k];
+  uint32_t run = (uint32_t)row0 + block_exclusive_scan(local, sw, nullptr);
+  for (int k = k0; k < k0 + kpt && k < KB; ++k) {
+    const uint32_t n = start[k];
+    start[k] = run;
+    if (k < a.K) {
+      a.segstart[(int64_t)b * a.K + k] = (int32_t)run;
+      a.segend[(int64_t)b * a.K + k] = (int32_t)(run + n);
+    }
+    run += n;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    if (bin[r] < a.K) {
+      const uint32_t pos = start[bin[r]] + wc[bin[r]] + rank[r];
+      a.keys_out[pos] = b * a.K + bin[r];
+      a.vals_out[pos] = (int32_t)(row0 + warp * PER_WARP + r * 32 + lane);
+    }
+  }
+}
+
 fkm_status device_scan(uint32_t* data, int64_t len, uint32_t* part, cudaStream_t st) {
   const int64_t nparts = ceil_div(len, kScanChunk);
   scan_reduce<<<(unsigned)nparts, kScanBlock, 0, st>>>(data, len, part);
@@ -401,12 +480,15 @@ fkm_status count_sort_prepare() {
   if (dev >= 0 && dev < 64 && done[dev]) return FKM_OK;
   const int b = (SORT_THREADS / 32) * (CS_MAX_K + 1) * 4;
   FKM_CUDA_TRY(cudaFuncSetAttribute(cs_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
+  const int b1 = (SORT_THREADS / 32 + 1) * (CS_MAX_K + 1) * 4;
+  FKM_CUDA_TRY(
+      cudaFuncSetAttribute(cs_single_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, b1));
   if (dev >= 0 && dev < 64) done[dev] = true;
   return FKM_OK;
 }
 
 fkm_status launch_count_sort_ids(SortArgs& s, int B, int32_t* segstart, int32_t* segend,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool ids_valid) {
   if (s.K > CS_MAX_K || s.n != (int64_t)B * s.N) {
     set_error("count sort: K = %d exceeds %d or n != B*N", s.K, CS_MAX_K);
     return FKM_ERR_INTERNAL;
@@ -428,6 +510,13 @@ fkm_status launch_count_sort_ids(SortArgs& s, int B, int32_t* segstart, int32_t*
   s.vals_out = s.vals0;
   if (s.n == 0) return FKM_OK;
   const unsigned tiles = (unsigned)((int64_t)B * a.tpb);
+  if (ids_valid && a.tpb == 1) {
+    const size_t smem = (size_t)(SORT_THREADS / 32 + 1) * (a.K + 1) * 4;
+    cs_single_tile_kernel<<<(unsigned)B, SORT_THREADS, smem, st>>>(a);
+    note_launch();
+    FKM_CUDA_TRY(cudaGetLastError());
+    return FKM_OK;
+  }
   cs_hist_kernel<<<tiles, SORT_THREADS, (a.K + 1) * 4, st>>>(a);
   FKM_TRY(device_scan(a.hist, cs_hist_words(B, s.N, s.K), s.hist_part, st));
   cs_scatter_kernel<<<tiles, SORT_THREADS, (SORT_THREADS / 32) * (a.K + 1) * 4, st>>>(a);

@@ -55,6 +55,7 @@ struct SegParams {
   int64_t row_bytes;     // bytes between rows of x
   int ebytes;            // bytes per element of x
   int V;                 // 16-byte vectors per slab row
+  int range;             // sorted rows per warp (<= SEG_RANGE)
   double* sums64;
   float* centers;
   bool accumulate_all;   // out-of-core chunks: every run goes to sums64
@@ -214,10 +215,10 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
   const bool want_obj = p.oa.obj != nullptr;
   const int64_t elem_bytes_ = p.ebytes;
   const int64_t r = (int64_t)blockIdx.x * SEG_WARPS + wid;
-  const int64_t nranges = ceil_div(p.n, SEG_RANGE);
+  const int64_t nranges = ceil_div(p.n, p.range);
   if (r >= nranges) return;
-  const int64_t j0 = r * SEG_RANGE;
-  const int nrows = (int)((j0 + SEG_RANGE < p.n) ? SEG_RANGE : p.n - j0);
+  const int64_t j0 = r * p.range;
+  const int nrows = (int)((j0 + p.range < p.n) ? p.range : p.n - j0);
 
   // ---- staging: all loads first, then the stores
   int2 e_[SEG_RANGE / 32];
@@ -477,6 +478,7 @@ struct FinParams {
   int32_t* counts;
   double* shiftk;
   const int32_t* counts_in;  // out-of-core: accumulated counts (segstart/end unused)
+  int range;                 // the segment sums' rows per warp range
 };
 
 // One warp per cluster.  When D is a multiple of 4 each lane moves four
@@ -493,7 +495,7 @@ __global__ void finalize_kernel(FinParams p) {
   } else {
     const int32_t s = p.segstart[key], t = p.segend[key];
     nk = t - s;
-    interior = nk > 0 && (s / SEG_RANGE) == ((t - 1) / SEG_RANGE);
+    interior = nk > 0 && (s / p.range) == ((t - 1) / p.range);
   }
   if (lane == 0 && p.counts) p.counts[key] = nk;
   double sh = 0.0;
@@ -565,7 +567,7 @@ __global__ void __launch_bounds__(256) batch_reduce_kernel(int K, const double* 
 
 template <int DT, int RPS>
 fkm_status run_segsum(const SegParams& sp, cudaStream_t st) {
-  const int64_t nranges = ceil_div(sp.n, SEG_RANGE);
+  const int64_t nranges = ceil_div(sp.n, sp.range);
   const int64_t blocks = ceil_div(nranges, SEG_WARPS);
   segsum_kernel<DT, RPS><<<(unsigned)blocks, SEG_WARPS * 32, SEG_SMEM_BYTES, st>>>(sp);
   note_launch();
@@ -601,6 +603,15 @@ fkm_status run_segsum_dt(const SegParams& sp, cudaStream_t st) {
 
 }  // namespace
 
+int segsum_range_rows(int64_t n) {
+  // about two rounds of the warps that fit on the GPU at once
+  const int64_t warps = (int64_t)num_sms() * SEG_WARPS * FKM_SEG_MIN_BLOCKS * 2;
+  int64_t r = round_up(ceil_div(n, warps), 32);
+  if (r < 32) r = 32;
+  if (r > SEG_RANGE) r = SEG_RANGE;
+  return (int)r;
+}
+
 fkm_status segsum_prepare() {
   static bool done[64] = {false};
   int dev = 0;
@@ -627,8 +638,9 @@ fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* s
 
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
-                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st) {
+                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range) {
   if (n == 0) return FKM_OK;
+  if (range <= 0) range = segsum_range_rows(n);
   FKM_TRY(segsum_prepare());
   const int eb = elem_bytes(dtype);
   const int slab = 512 / eb;   // columns per launch: 512-byte row pieces
@@ -644,6 +656,7 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
     sp.row_bytes = (int64_t)D * eb;
     sp.ebytes = eb;
     sp.V = (int)((int64_t)sp.D * eb / 16);
+    sp.range = range;
     sp.sums64 = sums64 + c0;
     sp.centers = centers ? centers + c0 : nullptr;
     sp.accumulate_all = accumulate_all;
@@ -676,8 +689,10 @@ fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const
 
 fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
                            const int32_t* counts_in, double* sums64, const float* prev,
-                           float* centers, int32_t* counts, double* shiftk, cudaStream_t st) {
+                           float* centers, int32_t* counts, double* shiftk, cudaStream_t st,
+                           int range) {
   FinParams fp;
+  fp.range = range;
   fp.B = B;
   fp.K = K;
   fp.D = D;

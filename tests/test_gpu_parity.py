@@ -294,6 +294,7 @@ def test_lloyd_init_may_alias_centers():
 @pytest.mark.parametrize("dtype,B,N,K,D", [
     ("bf16", 1, 1, 1, 8), ("bf16", 2, 5, 1, 8), ("f16", 1, 100, 300, 16),   # K > N: empties
     ("f32", 1, 129, 257, 4), ("bf16", 3, 128, 256, 256), ("f32", 2, 255, 2, 128),
+    ("bf16", 8, 4096, 2048, 64), ("f16", 5, 3000, 700, 32),   # batches of one sort tile
 ])
 def test_edge_shapes_free_running(dtype, B, N, K, D):
     w = datagen.Workload("edge", B, N, D, K, dtype, 0, sigma=1.0, iters=3, seed=B * N + K)
