@@ -437,6 +437,85 @@ def run_host(args, w):
     return 0
 
 
+def run_sharded(args, w):
+    """One workload split over the ranks (README "Multi-GPU Support"): rank r
+    holds rows [r*N/R, (r+1)*N/R) of every problem and runs the sharded Lloyd
+    loop (assign and partial update on its shard, an NCCL all-reduce of the
+    partial sums and counts, the same finalize everywhere).  Strong scaling:
+    the whole problem's iterations per second, the time the slowest rank's."""
+    import torch
+    import exact_means_clustering_b200 as fkm
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    x = datagen.points(w)
+    c0 = datagen.init_centroids(x, datagen.init_indices(w), w.dtype)
+    r0, r1 = (w.N * rank) // world, (w.N * (rank + 1)) // world
+    xs = np.ascontiguousarray(x[:, r0:r1])
+    del x
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[w.dtype]
+    xt = (torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16"
+          else torch.from_numpy(xs)).to(dev)
+    c0t = torch.from_numpy(c0).to(dev)
+    ws = fkm.workspace(fkm.fkm_workspace_size(w.B, r1 - r0, w.K, w.D, tdt), dev)
+
+    def step():
+        return fkm.lloyd_sharded(xt, c0t, w.iters, w.tol, ws=ws)[4]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        h0 = time.time()
+        e0.record()
+        n = 0
+        for _ in range(args.steps):
+            n += step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        clk.window(h0, time.time())
+    t_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        tt = torch.tensor([t_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms = tt.item()
+    value = n / (t_ms / 1e3)            # every rank ran the same n iterations of one problem
+    peaks, src = load_peaks()
+    peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    per_iter_s = t_ms / 1e3 / max(n, 1)
+    achieved = assign_flops(w) / world / per_iter_s / 1e12
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": dict(workload_config(w), sharded=True, rows_per_rank=r1 - r0),
+            "roofline": {"bound": "tensor", "kernel": "whole sharded iteration, per GPU",
+                         "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": achieved / peak_t, "traffic": None,
+                         "peak_source": f"{src} (bf16 sustained, MEASURED_PEAKS.json)",
+                         "note": "2*N*K*D / GPUs per whole iteration time: a lower bound on "
+                                 "the assign kernel's rate"},
+            "clocks": clk.summary()}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -447,6 +526,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-comparison", action="store_true")
+    ap.add_argument("--sharded", action="store_true",
+                    help="one problem split over the ranks' GPUs (strong scaling)")
     ap.add_argument("--oracle-iters", type=int, default=10)
     args = ap.parse_args()
 
@@ -458,6 +539,8 @@ def main():
         return run_reference(args, w)
     if w.host_resident:
         return run_host(args, w)
+    if args.sharded:
+        return run_sharded(args, w)
 
     import torch
     import exact_means_clustering_b200 as fkm

@@ -34,6 +34,8 @@ _SIG = {
     "fkm_workspace_size": ([_I, _I, _I, _I, _I, ctypes.POINTER(_Z)], _I),
     "fkm_selftest_wait_timeout": ([ctypes.c_uint64, _P, _Z, _P], _I),
     "fkm_centre_workspace_size": ([_I, _I, _I, ctypes.POINTER(_Z)], _I),
+    "fkm_partial_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_finalize_sums": ([_I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_centre": ([_I, _I, _I, _I, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
@@ -225,6 +227,73 @@ def fkm_assign_noalloc(x, centers, ids, stream=None):
     _check("fkm_assign_noalloc", lib().fkm_assign_noalloc(B, N, K, D, _dt(x), _ptr(x),
                                                           _ptr(centers), _ptr(ids),
                                                           _stream(stream)))
+
+
+def fkm_partial_update(x, ids, prev, sums, counts, obj=None, ws=None, stream=None):
+    """Add one shard's per-cluster sums / counts (and objective) to sums [B, K, D]
+    float64, counts [B, K] int32 (and obj [B] float64); see fkm.h."""
+    B, N, D = x.shape
+    K = prev.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    _check("fkm_partial_update",
+           lib().fkm_partial_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids), _ptr(prev), _ptr(sums),
+                                    _ptr(counts), _ptr(obj), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fkm_finalize_sums(sums, counts, prev, centers, shift=None, ws=None, stream=None):
+    """centers = sums / counts (prev where a cluster is empty); shift [B] optional."""
+    B, K, D = prev.shape
+    ws = ws if ws is not None else workspace(256 + 8 * B * K, prev.device)
+    _check("fkm_finalize_sums",
+           lib().fkm_finalize_sums(B, K, D, _ptr(sums), _ptr(counts), _ptr(prev), _ptr(centers),
+                                   _ptr(shift), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def reduce_partials(tensors, group=None):
+    """Sum the shards' partial sums / counts / objectives over the ranks of a
+    torch.distributed group (NCCL over NVLink for CUDA tensors): one
+    all-reduce each.  A no-op without an initialised group of 2+ ranks."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) < 2:
+        return
+    for t in tensors:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+
+
+def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None):
+    """Data-parallel Lloyd k-means over the ranks of a torch.distributed group
+    (README "Multi-GPU Support"): every rank passes its own contiguous shard
+    x [B, N_r, D] of the same B problems and the same init_centers [B, K, D];
+    per iteration each rank assigns its shard, forms its partial sums and
+    counts, the partials are all-reduced, and every rank forms the same
+    centroids.  Returns (ids of this shard [B, N_r], centers [B, K, D],
+    counts [B, K] of all shards, inertia [B] of all shards, n_iter)."""
+    B, N, D = x.shape
+    K = init_centers.shape[1]
+    dev = x.device
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), dev)
+    c = init_centers.to(dev, torch.float32).contiguous().clone()
+    ids = torch.empty(B, N, dtype=torch.int32, device=dev)
+    sums = torch.empty(B, K, D, dtype=torch.float64, device=dev)
+    counts = torch.empty(B, K, dtype=torch.int32, device=dev)
+    obj = torch.empty(B, dtype=torch.float64, device=dev)
+    shift = torch.empty(B, dtype=torch.float64, device=dev)
+    n_iter = 0
+    for t in range(max_iters):
+        fkm_assign(x, c, ids, ws=ws)
+        sums.zero_()
+        counts.zero_()
+        obj.zero_()
+        fkm_partial_update(x, ids, c, sums, counts, obj, ws=ws)
+        reduce_partials((sums, counts, obj), group)
+        nxt = torch.empty_like(c)
+        fkm_finalize_sums(sums, counts, c, nxt, shift, ws=ws)
+        c = nxt
+        n_iter = t + 1
+        if tol > 0.0 and shift.max().item() < tol:
+            break
+    fkm_sync_status(ws)
+    return ids, c, counts, obj, n_iter
 
 
 def fkm_centre_workspace_size_bytes(B, N, D) -> int:

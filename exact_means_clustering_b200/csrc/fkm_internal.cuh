@@ -61,6 +61,8 @@ fkm_status cuda_fail(cudaError_t e, const char* what);
 // Every buffer the library needs beyond the caller's inputs and outputs lives
 // in one caller-provided workspace, carved up by this layout.  Sizes depend on
 // B, N, K, D and dtype, never on N*K.
+struct Layout;
+fkm_status make_layout(int B, int N, int K, int D, int dtype, Layout* L);
 struct Layout {
   int B, N, K, D, dtype;
   int Kp;          // K rounded up to BN
@@ -172,10 +174,12 @@ fkm_status segsum_prepare();
 // Direct objective of a given assignment: obj[b] += sum_i ||x_i - chat_{ids_i}||^2.
 fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const int32_t* ids,
                             const ObjArgs& oa, cudaStream_t st);
+// clear_sums: zero sums64 after reading it (the library's own accumulators);
+// false leaves a caller's reduced sums untouched.
 fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
                            const int32_t* counts_in, double* sums64, const float* prev,
                            float* centers, int32_t* counts, double* shiftk, cudaStream_t st,
-                           int range = SEG_RANGE);
+                           int range = SEG_RANGE, bool clear_sums = true);
 fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
                                double* max_shift, cudaStream_t st);
 

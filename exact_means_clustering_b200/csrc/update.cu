@@ -479,6 +479,7 @@ struct FinParams {
   double* shiftk;
   const int32_t* counts_in;  // out-of-core: accumulated counts (segstart/end unused)
   int range;                 // the segment sums' rows per warp range
+  bool clear_sums;           // zero sums64 after use (the library's own accumulators)
 };
 
 // One warp per cluster.  When D is a multiple of 4 each lane moves four
@@ -513,8 +514,10 @@ __global__ void finalize_kernel(FinParams p) {
         const double2 a = s2[0], b = s2[1];
         const double n = (double)nk;
         v = make_float4((float)(a.x / n), (float)(a.y / n), (float)(b.x / n), (float)(b.y / n));
-        s2[0] = make_double2(0.0, 0.0);   // leave the accumulator clean for the next update
-        s2[1] = make_double2(0.0, 0.0);
+        if (p.clear_sums) {   // leave the accumulator clean for the next update
+          s2[0] = make_double2(0.0, 0.0);
+          s2[1] = make_double2(0.0, 0.0);
+        }
       }
       *reinterpret_cast<float4*>(p.centers + e) = v;
       const double d0 = (double)v.x - (double)pv.x, d1 = (double)v.y - (double)pv.y;
@@ -532,7 +535,7 @@ __global__ void finalize_kernel(FinParams p) {
         v = p.centers[e];
       } else {
         v = (float)(p.sums64[e] / (double)nk);
-        p.sums64[e] = 0.0;
+        if (p.clear_sums) p.sums64[e] = 0.0;
       }
       p.centers[e] = v;
       const double df = (double)v - (double)prev;
@@ -690,9 +693,10 @@ fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const
 fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
                            const int32_t* counts_in, double* sums64, const float* prev,
                            float* centers, int32_t* counts, double* shiftk, cudaStream_t st,
-                           int range) {
+                           int range, bool clear_sums) {
   FinParams fp;
   fp.range = range;
+  fp.clear_sums = clear_sums;
   fp.B = B;
   fp.K = K;
   fp.D = D;

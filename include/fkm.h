@@ -169,6 +169,36 @@ FKM_API fkm_status fkm_argsort_workspace_size(int64_t n, int n_keys, size_t* byt
 FKM_API fkm_status fkm_argsort(const int32_t* keys, int64_t n, int n_keys, int32_t* idx,
                        int32_t* sorted_keys, void* ws, size_t ws_bytes, void* stream);
 
+/* Data-parallel Lloyd over several GPUs ("Flash-KMeans" GitHub README,
+ * section "Multi-GPU Support"): the N points of every problem are split into
+ * contiguous shards, one per GPU.  One iteration on each GPU is
+ *   fkm_assign(shard, c)                        -> shard ids
+ *   fkm_partial_update(shard, ids, c)           -> += shard sums / counts / objective
+ *   all-reduce of sums, counts (and objective) across the GPUs (the caller's)
+ *   fkm_finalize_sums(reduced sums, counts, c)  -> the same new centroids everywhere
+ *
+ * fkm_partial_update: for the shard x [B, N, D] (this GPU's N points of each
+ * problem) and its ids [B, N], ADDS the per-cluster fp64 sums of the points
+ * to sums [B, K, D] (double), their counts to counts [B, K] (int32), and,
+ * when obj is non-null, the shard's objective sum ||x - c_hat||^2 against the
+ * centroids prev [B, K, D] the ids were assigned with to obj [B] (double).
+ * The caller zeroes sums / counts / obj once per iteration.  ws: a workspace
+ * of fkm_workspace_size(B, N, K, D, dtype) bytes.  All device pointers.
+ * An id outside [0, K) sets FKM_ERR_BAD_ID in the status word.  Async.
+ *
+ * fkm_finalize_sums: centers = sums / counts per cluster (IEEE division in
+ * fp64, rounded to fp32), prev for a cluster with no points; shift [B] (may
+ * be NULL) = sum_k ||centers - prev||^2.  sums and counts are not modified.
+ * ws: device scratch of at least 256 + 8 * B * K bytes.  centers must not
+ * alias prev.  Async. */
+FKM_API fkm_status fkm_partial_update(int B, int N, int K, int D, int dtype, const void* x,
+                                      const int32_t* ids, const float* prev, double* sums,
+                                      int32_t* counts, double* obj, void* ws, size_t ws_bytes,
+                                      void* stream);
+FKM_API fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
+                                     const int32_t* counts, const float* prev, float* centers,
+                                     double* shift, void* ws, size_t ws_bytes, void* stream);
+
 /* Centring ("Flash-KMeans" GitHub README, section "Centre your data"):
  * k-means is translation invariant, so points with a large common offset can
  * be clustered after subtracting their mean and the centroids shifted back
