@@ -36,6 +36,8 @@ _SIG = {
     "fkm_centre_workspace_size": ([_I, _I, _I, ctypes.POINTER(_Z)], _I),
     "fkm_partial_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_finalize_sums": ([_I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_partial_update_host": ([_I, _I, _I, _I, _I, _P, _P, _L, _P, _P, _P, _P, _P, _Z, _P],
+                                _I),
     "fkm_centre": ([_I, _I, _I, _I, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
@@ -240,6 +242,21 @@ def fkm_partial_update(x, ids, prev, sums, counts, obj=None, ws=None, stream=Non
                                     _ptr(counts), _ptr(obj), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=None, ws=None,
+                            stream=None):
+    """fkm_partial_update for a shard in pinned host memory x_host [B, N, D],
+    streamed in chunks of chunk_rows points; also writes the shard's ids."""
+    B, N, D = x_host.shape
+    K = centers.shape[1]
+    if ws is None:
+        ws = workspace(fkm_host_workspace_size(B, N, K, D, _dt(x_host), chunk_rows),
+                       centers.device)
+    _check("fkm_partial_update_host",
+           lib().fkm_partial_update_host(B, N, K, D, _dt(x_host), _ptr(x_host), _ptr(centers),
+                                         int(chunk_rows), _ptr(ids), _ptr(sums), _ptr(counts),
+                                         _ptr(obj), _ptr(ws), ws.numel(), _stream(stream)))
+
+
 def fkm_finalize_sums(sums, counts, prev, centers, shift=None, ws=None, stream=None):
     """centers = sums / counts (prev where a cluster is empty); shift [B] optional."""
     B, K, D = prev.shape
@@ -260,18 +277,28 @@ def reduce_partials(tensors, group=None):
         dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
 
 
-def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None):
+def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None, chunk_rows=None):
     """Data-parallel Lloyd k-means over the ranks of a torch.distributed group
     (README "Multi-GPU Support"): every rank passes its own contiguous shard
     x [B, N_r, D] of the same B problems and the same init_centers [B, K, D];
     per iteration each rank assigns its shard, forms its partial sums and
     counts, the partials are all-reduced, and every rank forms the same
-    centroids.  Returns (ids of this shard [B, N_r], centers [B, K, D],
-    counts [B, K] of all shards, inertia [B] of all shards, n_iter)."""
+    centroids.  A shard in pinned host memory (x on the CPU) is streamed to
+    init_centers' device in chunks of chunk_rows points every iteration, as
+    fkm_lloyd_host does.  Returns (ids of this shard [B, N_r], centers
+    [B, K, D], counts [B, K] of all shards, inertia [B] of all shards, n_iter)."""
     B, N, D = x.shape
     K = init_centers.shape[1]
-    dev = x.device
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), dev)
+    on_host = not x.is_cuda
+    dev = init_centers.device if on_host else x.device
+    if dev.type != "cuda":
+        raise ValueError("lloyd_sharded: init_centers must be on the GPU when x is on the host")
+    if on_host:
+        chunk_rows = int(chunk_rows or min(N, 1 << 20))
+        if ws is None:
+            ws = workspace(fkm_host_workspace_size(B, N, K, D, _dt(x), chunk_rows), dev)
+    elif ws is None:
+        ws = workspace(fkm_workspace_size(B, N, K, D, x.dtype), dev)
     c = init_centers.to(dev, torch.float32).contiguous().clone()
     ids = torch.empty(B, N, dtype=torch.int32, device=dev)
     sums = torch.empty(B, K, D, dtype=torch.float64, device=dev)
@@ -280,11 +307,14 @@ def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None):
     shift = torch.empty(B, dtype=torch.float64, device=dev)
     n_iter = 0
     for t in range(max_iters):
-        fkm_assign(x, c, ids, ws=ws)
         sums.zero_()
         counts.zero_()
         obj.zero_()
-        fkm_partial_update(x, ids, c, sums, counts, obj, ws=ws)
+        if on_host:
+            fkm_partial_update_host(x, c, chunk_rows, ids, sums, counts, obj, ws=ws)
+        else:
+            fkm_assign(x, c, ids, ws=ws)
+            fkm_partial_update(x, ids, c, sums, counts, obj, ws=ws)
         reduce_partials((sums, counts, obj), group)
         nxt = torch.empty_like(c)
         fkm_finalize_sums(sums, counts, c, nxt, shift, ws=ws)

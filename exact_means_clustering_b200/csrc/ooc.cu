@@ -133,10 +133,25 @@ int64_t injected_h2d_fault_chunk() {
   return -1;
 }
 
+// Partial mode (one shard of a data-parallel run): one pass over the chunks
+// with the given centroids, adding the per-cluster sums, counts and objective
+// to the caller's buffers instead of finalizing.
+struct HostPartial {
+  double* sums;
+  int32_t* counts;
+  double* obj;
+};
+
 }  // namespace
 }  // namespace fkm
 
 using namespace fkm;
+
+static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const void* x_host,
+                                  const float* init_centers, int max_iters, float tol,
+                                  int64_t chunk_rows, int32_t* ids, float* centers,
+                                  int32_t* counts, double* inertia, int* n_iter, void* ws,
+                                  size_t ws_bytes, void* stream, const HostPartial* part);
 
 extern "C" {
 
@@ -156,6 +171,33 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
                           const float* init_centers, int max_iters, float tol,
                           int64_t chunk_rows, int32_t* ids, float* centers, int32_t* counts,
                           double* inertia, int* n_iter, void* ws, size_t ws_bytes, void* stream) {
+  return lloyd_host_impl(B, N, K, D, dtype, x_host, init_centers, max_iters, tol, chunk_rows, ids,
+                         centers, counts, inertia, n_iter, ws, ws_bytes, stream, nullptr);
+}
+
+fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype, const void* x_host,
+                                   const float* centers, int64_t chunk_rows, int32_t* ids,
+                                   double* sums, int32_t* counts, double* obj, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!sums || (reinterpret_cast<uintptr_t>(sums) & 15) ||
+      (obj && (reinterpret_cast<uintptr_t>(obj) & 15))) {
+    set_error("sums must be non-null; sums and obj 16-byte aligned");
+    return FKM_ERR_INVALID_ARG;
+  }
+  HostPartial part{sums, counts, obj};
+  int n_iter = 0;
+  return lloyd_host_impl(B, N, K, D, dtype, x_host, centers, 1, 0.0f, chunk_rows, ids,
+                         const_cast<float*>(centers), counts, obj, &n_iter, ws, ws_bytes, stream,
+                         &part);
+}
+
+}  // extern "C"
+
+static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const void* x_host,
+                                  const float* init_centers, int max_iters, float tol,
+                                  int64_t chunk_rows, int32_t* ids, float* centers,
+                                  int32_t* counts, double* inertia, int* n_iter, void* ws,
+                                  size_t ws_bytes, void* stream, const HostPartial* part) {
   HostLayout L;
   FKM_TRY(make_host_layout(B, N, K, D, dtype, chunk_rows, &L));
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15) || ws_bytes < L.total) {
@@ -191,8 +233,8 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
   const size_t cbytes = (size_t)B * K * D * sizeof(float);
   float* cA = static_cast<float*>(at(L.cbuf));
   float* cB = cA + (size_t)B * K * D;
-  double* sums64 = static_cast<double*>(at(L.sums64));
-  int32_t* counts_acc = static_cast<int32_t*>(at(L.counts_acc));
+  double* sums64 = part ? part->sums : static_cast<double*>(at(L.sums64));
+  int32_t* counts_acc = part ? part->counts : static_cast<int32_t*>(at(L.counts_acc));
 
   StreamSet ss;
   FKM_CUDA_TRY(cudaStreamCreateWithFlags(&ss.copy, cudaStreamNonBlocking));
@@ -204,7 +246,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
   FKM_TRY(assign_prepare());
 
   FKM_CUDA_TRY(cudaMemsetAsync(status, 0, 256, st));
-  FKM_CUDA_TRY(cudaMemsetAsync(sums64, 0, (size_t)B * K * D * 8, st));
+  if (!part) FKM_CUDA_TRY(cudaMemsetAsync(sums64, 0, (size_t)B * K * D * 8, st));
   FKM_CUDA_TRY(cudaMemcpyAsync(cA, init_centers, cbytes, cudaMemcpyDeviceToDevice, st));
   float* mvec = static_cast<float*>(at(L.mvec));
   FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, mvec, at(L.cq),
@@ -219,8 +261,10 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
   for (int t = 0; t < max_iters; ++t) {
     float* cur = (t & 1) ? cB : cA;
     float* nxt = (t & 1) ? cA : cB;
-    FKM_CUDA_TRY(cudaMemsetAsync(counts_acc, 0, (size_t)B * K * 4, st));
-    if (inertia) FKM_CUDA_TRY(cudaMemsetAsync(inertia, 0, (size_t)B * 8, st));
+    if (!part) {   // a partial pass adds to the caller's buffers
+      FKM_CUDA_TRY(cudaMemsetAsync(counts_acc, 0, (size_t)B * K * 4, st));
+      if (inertia) FKM_CUDA_TRY(cudaMemsetAsync(inertia, 0, (size_t)B * 8, st));
+    }
     for (int b = 0; b < B; ++b) {
       for (int c = 0; c < L.chunks_per_batch; ++c, ++chunk_no) {
         const int buf = (int)(chunk_no & 1);
@@ -296,6 +340,10 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
         FKM_CUDA_TRY(cudaEventRecord(ss.freed[buf], st));
       }
     }
+    if (part) {
+      done = 1;
+      break;
+    }
     FKM_TRY(launch_finalize(B, K, D, nullptr, nullptr, counts_acc, sums64, cur, nxt, counts,
                             static_cast<double*>(at(L.shiftk)), st));
     FKM_TRY(launch_prep_centroids(nxt, B, K, L.Kp, D, dtype, mvec, at(L.cq),
@@ -312,7 +360,7 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
     }
   }
   float* last = (done & 1) ? cB : cA;
-  FKM_CUDA_TRY(cudaMemcpyAsync(centers, last, cbytes, cudaMemcpyDeviceToDevice, st));
+  if (!part) FKM_CUDA_TRY(cudaMemcpyAsync(centers, last, cbytes, cudaMemcpyDeviceToDevice, st));
   int host_status = 0;
   FKM_CUDA_TRY(cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, st));
   FKM_CUDA_TRY(cudaStreamSynchronize(st));
@@ -328,5 +376,3 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
   }
   return FKM_OK;
 }
-
-}  // extern "C"

@@ -48,7 +48,16 @@ __global__ void __launch_bounds__(1024) center_kernel(const float* __restrict__ 
   double s = 0.0;
   if (d < D) {
     const float* p = c + (int64_t)b * K * D + d;
-    for (int k = w; k < K; k += 32) s += (double)p[(int64_t)k * D];
+    int k = w;
+    // eight rows' loads in flight at once, added in the same ascending order
+    for (; k + 7 * 32 < K; k += 8 * 32) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = p[(int64_t)(k + 32 * j) * D];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += (double)v[j];
+    }
+    for (; k < K; k += 32) s += (double)p[(int64_t)k * D];
   }
   part[w][lane] = s;
   __syncthreads();
@@ -90,7 +99,21 @@ __device__ __forceinline__ void bias_parts(double v, bool f16, uint16_t out[3]) 
   }
 }
 
-// one warp per padded centroid row
+// q(v) in the points' 16-bit type, as raw bits and as the value it rounds to
+__device__ __forceinline__ uint16_t q16(float v, bool bf, float* back) {
+  if (bf) {
+    const __nv_bfloat16 q = __float2bfloat16_rn(v);
+    *back = __bfloat162float(q);
+    return __bfloat16_as_ushort(q);
+  }
+  const __half q = __float2half_rn(v);
+  *back = __half2float(q);
+  return __half_as_ushort(q);
+}
+
+// one warp per padded centroid row; each lane takes four consecutive
+// elements at a time (D is a multiple of 4 for every dtype: the rows of x
+// are 16-byte multiples)
 __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* __restrict__ m,
                                       int B, int K, int Kp, int D, int dtype,
                                       void* __restrict__ cq, uint16_t* __restrict__ caug) {
@@ -104,30 +127,42 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
   double acc = 0.0;
   if (dtype == FKM_F32) {
     const int Dp = (D + 7) & ~7;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(cq) + row * (int64_t)(2 * Dp);
-    for (int d = lane; d < D; d += 32) {
-      const float v = real ? src[d] - mb[d] : 0.0f;
-      __nv_bfloat16 h = __float2bfloat16_rn(v);
-      __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-      out[d] = h;
-      out[Dp + d] = l;
-      acc += (double)v * ((double)v + 2.0 * (double)mb[d]);
-    }
-  } else if (dtype == FKM_BF16) {
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(cq) + row * (int64_t)D;
-    for (int d = lane; d < D; d += 32) {
-      __nv_bfloat16 q = __float2bfloat16_rn(real ? src[d] - mb[d] : 0.0f);
-      out[d] = q;
-      const double f = (double)__bfloat162float(q);
-      acc += f * (f + 2.0 * (double)mb[d]);
+    uint16_t* out = static_cast<uint16_t*>(cq) + row * (int64_t)(2 * Dp);
+    for (int d = 4 * lane; d < D; d += 128) {
+      const float4 mm = *reinterpret_cast<const float4*>(mb + d);
+      const float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
+      const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
+      const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
+      uint16_t hb[4], lb[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float hf, lf;
+        hb[j] = q16(v[j], true, &hf);
+        lb[j] = q16(v[j] - hf, true, &lf);
+        acc += (double)v[j] * ((double)v[j] + 2.0 * (double)mv[j]);
+      }
+      *reinterpret_cast<uint2*>(out + d) =
+          make_uint2(hb[0] | ((uint32_t)hb[1] << 16), hb[2] | ((uint32_t)hb[3] << 16));
+      *reinterpret_cast<uint2*>(out + Dp + d) =
+          make_uint2(lb[0] | ((uint32_t)lb[1] << 16), lb[2] | ((uint32_t)lb[3] << 16));
     }
   } else {
-    __half* out = static_cast<__half*>(cq) + row * (int64_t)D;
-    for (int d = lane; d < D; d += 32) {
-      __half q = __float2half_rn(real ? src[d] - mb[d] : 0.0f);
-      out[d] = q;
-      const double f = (double)__half2float(q);
-      acc += f * (f + 2.0 * (double)mb[d]);
+    const bool bf = dtype == FKM_BF16;
+    uint16_t* out = static_cast<uint16_t*>(cq) + row * (int64_t)D;
+    for (int d = 4 * lane; d < D; d += 128) {
+      const float4 mm = *reinterpret_cast<const float4*>(mb + d);
+      const float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
+      const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
+      const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
+      uint16_t qb[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float f;
+        qb[j] = q16(v[j], bf, &f);
+        acc += (double)f * ((double)f + 2.0 * (double)mv[j]);
+      }
+      *reinterpret_cast<uint2*>(out + d) =
+          make_uint2(qb[0] | ((uint32_t)qb[1] << 16), qb[2] | ((uint32_t)qb[3] << 16));
     }
   }
   acc = warp_sum(acc);

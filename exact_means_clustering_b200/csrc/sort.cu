@@ -11,8 +11,9 @@
 //   upsweep    tile histograms (4096 keys per 256-thread tile), digit-major
 //   scan       exclusive scan of the histogram matrix: global base per
 //              (digit, tile)
-//   downsweep  stable rank of every key inside its tile (warp match_any
-//              ranking), keys and values staged in shared memory in sorted
+//   downsweep  stable rank of every key inside its tile (warp multisplit:
+//              the lanes holding the same digit found with one ballot per
+//              digit bit), keys and values staged in shared memory in sorted
 //              order, then written out in contiguous runs per digit.
 // The first pass forms the keys from the ids on the fly and validates them:
 // an id outside [0, K) sets ST_BAD_ID and gets the sentinel key B*K, which
@@ -30,6 +31,28 @@
 
 namespace fkm {
 namespace {
+
+// Lanes of the warp whose value equals this lane's, for values in
+// [0, 2^nbits): one ballot per bit, keeping the lanes that agree on it.  The
+// hardware match instruction gives the same mask, but its cost grows with
+// the number of distinct values in the warp, and with ~32 distinct cluster
+// ids per warp it saturated its pipe in the sort kernels.
+__device__ __forceinline__ unsigned warp_peers(unsigned v, int nbits) {
+  unsigned m = 0xffffffffu;
+  for (int i = 0; i < nbits; ++i) {
+    const unsigned bit = (v >> i) & 1u;
+    const unsigned bal = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? bal : ~bal;
+  }
+  return m;
+}
+
+// Bits needed for the values 0..vmax.
+__host__ __device__ __forceinline__ int value_bits(unsigned vmax) {
+  int b = 1;
+  while (b < 32 && (vmax >> b)) ++b;
+  return b;
+}
 
 constexpr int kScanBlock = 1024;
 constexpr int kScanItems = 4;
@@ -66,7 +89,7 @@ template <bool kFirst>
 __global__ void __launch_bounds__(SORT_THREADS) radix_upsweep(KeySrc s, int64_t n, int shift,
                                                               int n_tiles, uint32_t* hist) {
   __shared__ uint32_t h[SORT_THREADS / 32][RADIX_BINS];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < (SORT_THREADS / 32) * RADIX_BINS; i += SORT_THREADS)
     (&h[0][0])[i] = 0;
   __syncthreads();
@@ -80,8 +103,7 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_upsweep(KeySrc s, int64_t 
       load_key<kFirst>(s, j, key, val);
       digit = (key >> shift) & (RADIX_BINS - 1);
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, digit);
-    if (digit < RADIX_BINS && lane == __ffs(peers) - 1) atomicAdd(&h[warp][digit], __popc(peers));
+    if (digit < RADIX_BINS) atomicAdd(&h[warp][digit], 1u);
   }
   __syncthreads();
   for (int d = threadIdx.x; d < RADIX_BINS; d += SORT_THREADS) {
@@ -205,7 +227,7 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_downsweep(KeySrc s, int64_
       d = (key[r] >> shift) & (RADIX_BINS - 1);
     }
     dig[r] = d;
-    const unsigned peers = __match_any_sync(0xffffffffu, d);
+    const unsigned peers = warp_peers((unsigned)d, 9);   // digits 0..RADIX_BINS
     const uint32_t before = cnt[warp][d];
     rank[r] = before + __popc(peers & lt_mask);
     __syncwarp();
@@ -265,7 +287,6 @@ struct CsArgs {
 __global__ void __launch_bounds__(SORT_THREADS) cs_hist_kernel(CsArgs a) {
   extern __shared__ uint32_t h[];   // K + 1
   const int tg = blockIdx.x, b = tg / a.tpb, t = tg % a.tpb;
-  const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i <= a.K; i += SORT_THREADS) h[i] = 0;
   __syncthreads();
   const int64_t row0 = (int64_t)b * a.N + (int64_t)t * SORT_TILE;
@@ -289,8 +310,7 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_hist_kernel(CsArgs a) {
         bin = id[it];
       }
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, bin);
-    if (bin <= a.K && lane == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+    if (bin <= a.K) atomicAdd(&h[bin], 1u);
   }
   if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(a.status, ST_BAD_ID);
   for (int k = threadIdx.x; k < a.K; k += SORT_THREADS)
@@ -299,7 +319,7 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_hist_kernel(CsArgs a) {
 }
 
 // Stable scatter of one tile: warp w ranks rows [512 w, 512 w + 512) of the
-// tile in order with per-warp bin counters (match_any), the counters are
+// tile in order with per-warp bin counters (warp multisplit), the counters are
 // turned into output positions (scanned base + earlier warps' counts), and
 // every row writes its key and index.  Tile 0 of each batch also writes that
 // batch's segment bounds.
@@ -325,11 +345,12 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_scatter_kernel(CsArgs a) {
   }
   __syncthreads();
   const unsigned lt_mask = (1u << lane) - 1u;
+  const int nbits = value_bits((unsigned)a.K + 1);   // bins 0..K+1
   uint32_t* wc = cnt + warp * KB;
   uint32_t rank[SORT_ITEMS];
 #pragma unroll
   for (int r = 0; r < SORT_ITEMS; ++r) {
-    const unsigned peers = __match_any_sync(0xffffffffu, bin[r]);
+    const unsigned peers = warp_peers((unsigned)bin[r], nbits);
     uint32_t before = 0;
     if (bin[r] <= a.K) before = wc[bin[r]];
     rank[r] = before + __popc(peers & lt_mask);
@@ -394,11 +415,12 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_single_tile_kernel(CsArgs a) 
   }
   __syncthreads();
   const unsigned lt_mask = (1u << lane) - 1u;
+  const int nbits = value_bits((unsigned)a.K + 1);   // bins 0..K+1
   uint32_t* wc = cnt + warp * KB;
   uint32_t rank[SORT_ITEMS];
 #pragma unroll
   for (int r = 0; r < SORT_ITEMS; ++r) {
-    const unsigned peers = __match_any_sync(0xffffffffu, bin[r]);
+    const unsigned peers = warp_peers((unsigned)bin[r], nbits);
     uint32_t before = 0;
     if (bin[r] <= a.K) before = wc[bin[r]];
     rank[r] = before + __popc(peers & lt_mask);

@@ -199,6 +199,21 @@ FKM_API fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
                                      const int32_t* counts, const float* prev, float* centers,
                                      double* shift, void* ws, size_t ws_bytes, void* stream);
 
+/* fkm_partial_update_host: the same shard step for a shard that stays in HOST
+ * memory (pinned), as fkm_lloyd_host streams it: each chunk of chunk_rows
+ * points is copied to the device, assigned against centers [B, K, D] (fp32,
+ * device) and folded into sums / counts / obj exactly as fkm_partial_update
+ * adds them; ids [B, N] (device) receive the shard's assignments.  ws: a
+ * workspace of fkm_host_workspace_size(B, N, K, D, dtype, chunk_rows) bytes.
+ * sums, counts, obj as in fkm_partial_update (the caller zeroes them once per
+ * iteration; obj may be NULL).  Synchronous, like fkm_lloyd_host, and
+ * FKM_FAULT_INJECT applies to its chunk copies in the same way. */
+FKM_API fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype,
+                                           const void* x_host, const float* centers,
+                                           int64_t chunk_rows, int32_t* ids, double* sums,
+                                           int32_t* counts, double* obj, void* ws,
+                                           size_t ws_bytes, void* stream);
+
 /* Centring ("Flash-KMeans" GitHub README, section "Centre your data"):
  * k-means is translation invariant, so points with a large common offset can
  * be clustered after subtracting their mean and the centroids shifted back

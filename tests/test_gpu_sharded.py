@@ -70,3 +70,57 @@ def test_sharded_loop_tol_stops_like_lloyd():
     c2 = torch.empty(w.B, w.K, w.D, device="cuda")
     n2 = torch.empty(w.B, w.K, dtype=torch.int32, device="cuda")
     assert n == fkm.fkm_lloyd(xt, c0t, 40, 1e-2, i2, c2, n2)
+
+
+@pytest.mark.parametrize("dtype,B,N,K,D,cut,chunk", [("bf16", 2, 9000, 300, 128, 5000, 2048),
+                                                     ("f32", 1, 6000, 100, 96, 777, 1000)])
+def test_host_shard_partials_match_device_partials(dtype, B, N, K, D, cut, chunk):
+    """Shards kept in pinned host memory and streamed in chunks give the same
+    ids, counts and (up to fp64 summation order) sums and objective as the
+    device-resident shard step."""
+    w = datagen.Workload("host-shards", B, N, D, K, dtype, K, sigma=0.5, iters=1, seed=N + D)
+    x, xt, c0 = problem(w)
+    c = torch.from_numpy(c0).cuda()
+    ref = [torch.zeros(B, K, D, dtype=torch.float64, device="cuda"),
+           torch.zeros(B, K, dtype=torch.int32, device="cuda"),
+           torch.zeros(B, dtype=torch.float64, device="cuda")]
+    got = [torch.zeros_like(t) for t in ref]
+    ids_ref = torch.empty(B, N, dtype=torch.int32, device="cuda")
+    fkm.fkm_assign(xt, c, ids_ref)
+    ids = torch.full((B, N), -1, dtype=torch.int32, device="cuda")
+    for a, b in ((0, cut), (cut, N)):
+        fkm.fkm_partial_update(xt[:, a:b].clone(), ids_ref[:, a:b].clone(), c, *ref)
+        xh = xt[:, a:b].cpu().pin_memory()
+        part_ids = torch.empty(B, b - a, dtype=torch.int32, device="cuda")
+        fkm.fkm_partial_update_host(xh, c, chunk, part_ids, *got)
+        ids[:, a:b] = part_ids
+    assert torch.equal(ids, ids_ref)
+    assert torch.equal(got[1], ref[1])
+    # the segment sums add up to 16 rows in fp32 before each fp64 fold; a fold
+    # of <= 16 values rounds by <= 16 * 2^-24 * 16 max|x|, so a cluster of n
+    # points differs by <= n * 2^-20 * max|x| per side between two groupings
+    bound = 2.0 ** -19 * got[1].double().unsqueeze(-1) * xt.abs().max().double()
+    assert ((got[0] - ref[0]).abs() <= bound + 1e-12).all()
+    assert torch.allclose(got[2], ref[2], rtol=1e-6)
+    cen = torch.empty_like(c)
+    fkm.fkm_finalize_sums(got[0], got[1], c, cen)
+    check_update(x, dtype, ids.cpu().numpy(), c0, cen.cpu().numpy(), got[1].cpu().numpy())
+
+
+def test_sharded_loop_from_host_matches_lloyd_host():
+    w = datagen.CONFIGS[2].scaled(B=2, N=8192, K=256, iters=3)
+    x, xt, c0 = problem(w)
+    c0t = torch.from_numpy(c0).cuda()
+    xh = xt.cpu().pin_memory()
+    ids, cen, cnt, inertia, n = fkm.lloyd_sharded(xh, c0t, 3, chunk_rows=3000)
+    i2 = torch.empty(w.B, w.N, dtype=torch.int32, device="cuda")
+    c2 = torch.empty(w.B, w.K, w.D, device="cuda")
+    n2 = torch.empty(w.B, w.K, dtype=torch.int32, device="cuda")
+    in2 = torch.empty(w.B, dtype=torch.float64, device="cuda")
+    assert n == fkm.fkm_lloyd_host(xh, c0t, 3, 0.0, 3000, i2, c2, n2, in2) == 3
+    # the fp64 atomics of runs that cross a segment-sum range may round in
+    # another order, so a near tie may still flip
+    assert (ids != i2).float().mean().item() <= 1e-4
+    assert (cnt - n2).abs().sum().item() <= 2 * (ids != i2).sum().item()
+    assert torch.allclose(cen, c2, rtol=1e-6, atol=1e-6)
+    assert torch.allclose(inertia, in2, rtol=1e-6)
