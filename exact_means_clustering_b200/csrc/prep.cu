@@ -111,24 +111,25 @@ __device__ __forceinline__ uint16_t q16(float v, bool bf, float* back) {
   return __half_as_ushort(q);
 }
 
-// one warp per padded centroid row; each lane takes four consecutive
-// elements at a time (D is a multiple of 4 for every dtype: the rows of x
-// are 16-byte multiples)
+// Four padded centroid rows per warp, eight lanes per row; each lane takes
+// four consecutive elements at a time (D is a multiple of 4 for every dtype:
+// the rows of x are 16-byte multiples).
 __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* __restrict__ m,
                                       int B, int K, int Kp, int D, int dtype,
                                       void* __restrict__ cq, uint16_t* __restrict__ caug) {
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= (int64_t)B * Kp) return;
-  const int b = (int)(row / Kp), k = (int)(row % Kp);
-  const bool real = k < K;
+  const int lane = threadIdx.x & 31, l8 = lane & 7;
+  const int64_t row =
+      ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
+  const bool valid = row < (int64_t)B * Kp;
+  const int b = valid ? (int)(row / Kp) : 0, k = valid ? (int)(row % Kp) : 0;
+  const bool real = valid && k < K;
   const float* src = c + ((int64_t)b * K + k) * D;
   const float* mb = m + (int64_t)b * D;
   double acc = 0.0;
   if (dtype == FKM_F32) {
     const int Dp = (D + 7) & ~7;
     uint16_t* out = static_cast<uint16_t*>(cq) + row * (int64_t)(2 * Dp);
-    for (int d = 4 * lane; d < D; d += 128) {
+    for (int d = 4 * l8; valid && d < D; d += 32) {
       const float4 mm = *reinterpret_cast<const float4*>(mb + d);
       const float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
       const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
@@ -149,7 +150,7 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
   } else {
     const bool bf = dtype == FKM_BF16;
     uint16_t* out = static_cast<uint16_t*>(cq) + row * (int64_t)D;
-    for (int d = 4 * lane; d < D; d += 128) {
+    for (int d = 4 * l8; valid && d < D; d += 32) {
       const float4 mm = *reinterpret_cast<const float4*>(mb + d);
       const float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
       const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
@@ -165,12 +166,20 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
           make_uint2(qb[0] | ((uint32_t)qb[1] << 16), qb[2] | ((uint32_t)qb[3] << 16));
     }
   }
-  acc = warp_sum(acc);
+  // sum over the row's eight lanes; the butterfly leaves every lane the same
+  // value (each level adds the same two operands on both sides)
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   // the bias slab: [-n/2 in three parts, 0 x 13]; padding rows are all zero
-  // (the assign kernel masks their columns)
+  // (the assign kernel masks their columns); lane l8 writes entries 2 l8, 2 l8 + 1
   uint16_t parts[3] = {0, 0, 0};
   if (real) bias_parts(-0.5 * acc, dtype == FKM_F16, parts);
-  if (lane < AUG_SLAB) caug[row * AUG_SLAB + lane] = lane < 3 ? parts[lane] : (uint16_t)0;
+  if (valid) {
+    const int e = 2 * l8;
+    const uint32_t lo = e == 0 ? parts[0] : e == 2 ? parts[2] : 0u;
+    const uint32_t hi = e == 0 ? parts[1] : 0u;
+    *reinterpret_cast<uint32_t*>(caug + row * AUG_SLAB + e) = lo | (hi << 16);
+  }
 }
 
 // one warp per point row; xn[row] = ||x - m[batch]||^2 when m is given
@@ -233,8 +242,8 @@ fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int
   center_kernel<<<dim3((unsigned)B, (unsigned)ceil_div(D, 32)), 1024, 0, st>>>(centers, B, K, D,
                                                                               m);
   const int64_t rows = (int64_t)B * Kp;
-  const int wpb = 8;
-  prep_centroids_kernel<<<(unsigned)ceil_div(rows, wpb), wpb * 32, 0, st>>>(
+  const int wpb = 8;   // 4 rows per warp
+  prep_centroids_kernel<<<(unsigned)ceil_div(rows, 4 * wpb), wpb * 32, 0, st>>>(
       centers, m, B, K, Kp, D, dtype, cq, static_cast<uint16_t*>(caug));
   note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());

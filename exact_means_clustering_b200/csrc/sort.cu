@@ -318,16 +318,35 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_hist_kernel(CsArgs a) {
   if (threadIdx.x == 0) a.hist[(int64_t)a.B * a.K * a.tpb + tg] = h[a.K];
 }
 
+// Shared memory of the scatter pass, in 32-bit words: the per-warp bin
+// counters, which the staged (key, row) pairs of the tile reuse once every
+// row knows its place, then the bins' tile starts and their global shifts.
+__host__ __device__ __forceinline__ int cs_scatter_stage_words(int K) {
+  const int counters = (SORT_THREADS / 32) * (K + 1);
+  return counters > 2 * SORT_TILE ? counters : 2 * SORT_TILE;
+}
+__host__ __device__ __forceinline__ size_t cs_scatter_smem_bytes(int K) {
+  return ((size_t)cs_scatter_stage_words(K) + 2 * (size_t)(K + 1)) * 4;
+}
+
 // Stable scatter of one tile: warp w ranks rows [512 w, 512 w + 512) of the
-// tile in order with per-warp bin counters (warp multisplit), the counters are
-// turned into output positions (scanned base + earlier warps' counts), and
-// every row writes its key and index.  Tile 0 of each batch also writes that
-// batch's segment bounds.
-__global__ void __launch_bounds__(SORT_THREADS) cs_scatter_kernel(CsArgs a) {
+// tile in order with per-warp bin counters (warp multisplit).  The counters
+// become offsets inside each bin (earlier warps first), a block scan of the
+// bin totals gives each bin's start in the tile's sorted order, and every row
+// stages its key and index at its sorted place in shared memory.  The staged
+// tile is then written out in order, so the rows of a bin (consecutive in the
+// output) leave as contiguous runs instead of one scattered word per row.
+// Tile 0 of each batch also writes that batch's segment bounds.  Four blocks
+// per SM keep a 32-batch grid of 16 tiles each (512 blocks) in one wave.
+__global__ void __launch_bounds__(SORT_THREADS, 4) cs_scatter_kernel(CsArgs a) {
   constexpr int NW = SORT_THREADS / 32;
   constexpr int PER_WARP = SORT_TILE / NW;
-  extern __shared__ uint32_t cnt[];   // NW * (K + 1)
+  extern __shared__ uint32_t smem[];
+  __shared__ uint32_t sw[32];
   const int KB = a.K + 1;
+  uint32_t* cnt = smem;                                   // NW * KB, then the staged tile
+  uint32_t* start = smem + cs_scatter_stage_words(a.K);   // KB: bin start in the tile
+  int32_t* shift = reinterpret_cast<int32_t*>(start + KB);  // KB: global - tile position
   const int tg = blockIdx.x, b = tg / a.tpb, t = tg % a.tpb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < NW * KB; i += SORT_THREADS) cnt[i] = 0;
@@ -347,36 +366,69 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_scatter_kernel(CsArgs a) {
   const unsigned lt_mask = (1u << lane) - 1u;
   const int nbits = value_bits((unsigned)a.K + 1);   // bins 0..K+1
   uint32_t* wc = cnt + warp * KB;
-  uint32_t rank[SORT_ITEMS];
+  // after ranking, bin[r] holds the bin in its low 16 bits and the row's rank
+  // among the warp's rows of that bin (< SORT_TILE) in its high 16 bits
 #pragma unroll
   for (int r = 0; r < SORT_ITEMS; ++r) {
     const unsigned peers = warp_peers((unsigned)bin[r], nbits);
     uint32_t before = 0;
     if (bin[r] <= a.K) before = wc[bin[r]];
-    rank[r] = before + __popc(peers & lt_mask);
+    const uint32_t rank = before + __popc(peers & lt_mask);
     __syncwarp();
     if (bin[r] <= a.K && lane == __ffs(peers) - 1) wc[bin[r]] = before + __popc(peers);
     __syncwarp();
+    bin[r] |= (int)(rank << 16);
   }
   __syncthreads();
-  for (int k = threadIdx.x; k < KB; k += SORT_THREADS) {
-    uint32_t base = k < a.K ? a.hist[((int64_t)b * a.K + k) * a.tpb + t]
-                            : a.hist[(int64_t)a.B * a.K * a.tpb + tg];
+  // per bin: earlier warps' counts become offsets inside the bin; thread t
+  // owns bins [t*kpt, (t+1)*kpt) and scans their totals across the block
+  const int kpt = (KB + SORT_THREADS - 1) / SORT_THREADS;
+  const int k0 = threadIdx.x * kpt;
+  uint32_t local = 0;
+  for (int k = k0; k < k0 + kpt && k < KB; ++k) {
+    uint32_t run = 0;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const uint32_t c = cnt[w * KB + k];
-      cnt[w * KB + k] = base;
-      base += c;
+      cnt[w * KB + k] = run;
+      run += c;
+    }
+    start[k] = run;
+    local += run;
+  }
+  uint32_t pos = block_exclusive_scan(local, sw, nullptr);
+  for (int k = k0; k < k0 + kpt && k < KB; ++k) {
+    const uint32_t n = start[k];
+    const uint32_t g = k < a.K ? a.hist[((int64_t)b * a.K + k) * a.tpb + t]
+                               : a.hist[(int64_t)a.B * a.K * a.tpb + tg];
+    start[k] = pos;
+    shift[k] = (int32_t)(g - pos);
+    pos += n;
+  }
+  __syncthreads();
+  // each row's place in the tile's sorted order (bin[r] becomes it)
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    const int k = bin[r] & 0xffff;
+    bin[r] = k <= a.K ? (int)(start[k] + wc[k] + ((uint32_t)bin[r] >> 16)) | (k << 16) : -1;
+  }
+  __syncthreads();   // the counters are dead: the staged tile takes their place
+  int32_t* sk = reinterpret_cast<int32_t*>(smem);
+  int32_t* sv = sk + SORT_TILE;
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    if (bin[r] >= 0) {
+      const int lp = bin[r] & 0xffff;
+      sk[lp] = bin[r] >> 16;
+      sv[lp] = (int32_t)(row0 + warp * PER_WARP + r * 32 + lane);
     }
   }
   __syncthreads();
-#pragma unroll
-  for (int r = 0; r < SORT_ITEMS; ++r) {
-    if (bin[r] <= a.K) {
-      const uint32_t pos = wc[bin[r]] + rank[r];
-      a.keys_out[pos] = bin[r] < a.K ? b * a.K + bin[r] : a.B * a.K;
-      a.vals_out[pos] = (int32_t)(row0 + warp * PER_WARP + r * 32 + lane);
-    }
+  for (int j = threadIdx.x; j < nrows; j += SORT_THREADS) {
+    const int k = sk[j];
+    const int64_t g = (int64_t)j + shift[k];
+    a.keys_out[g] = k < a.K ? b * a.K + k : a.B * a.K;
+    a.vals_out[g] = sv[j];
   }
   if (t == 0) {
     for (int k = threadIdx.x; k < a.K; k += SORT_THREADS) {
@@ -500,7 +552,7 @@ fkm_status count_sort_prepare() {
   int dev = 0;
   FKM_CUDA_TRY(cudaGetDevice(&dev));
   if (dev >= 0 && dev < 64 && done[dev]) return FKM_OK;
-  const int b = (SORT_THREADS / 32) * (CS_MAX_K + 1) * 4;
+  const int b = (int)cs_scatter_smem_bytes(CS_MAX_K);
   FKM_CUDA_TRY(cudaFuncSetAttribute(cs_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, b));
   const int b1 = (SORT_THREADS / 32 + 1) * (CS_MAX_K + 1) * 4;
   FKM_CUDA_TRY(
@@ -541,7 +593,7 @@ fkm_status launch_count_sort_ids(SortArgs& s, int B, int32_t* segstart, int32_t*
   }
   cs_hist_kernel<<<tiles, SORT_THREADS, (a.K + 1) * 4, st>>>(a);
   FKM_TRY(device_scan(a.hist, cs_hist_words(B, s.N, s.K), s.hist_part, st));
-  cs_scatter_kernel<<<tiles, SORT_THREADS, (SORT_THREADS / 32) * (a.K + 1) * 4, st>>>(a);
+  cs_scatter_kernel<<<tiles, SORT_THREADS, cs_scatter_smem_bytes(a.K), st>>>(a);
   note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
