@@ -49,13 +49,13 @@ __global__ void __launch_bounds__(1024) center_kernel(const float* __restrict__ 
   if (d < D) {
     const float* p = c + (int64_t)b * K * D + d;
     int k = w;
-    // eight rows' loads in flight at once, added in the same ascending order
-    for (; k + 7 * 32 < K; k += 8 * 32) {
-      float v[8];
+    // sixteen rows' loads in flight at once, added in the same ascending order
+    for (; k + 15 * 32 < K; k += 16 * 32) {
+      float v[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = p[(int64_t)(k + 32 * j) * D];
+      for (int j = 0; j < 16; ++j) v[j] = p[(int64_t)(k + 32 * j) * D];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s += (double)v[j];
+      for (int j = 0; j < 16; ++j) s += (double)v[j];
     }
     for (; k < K; k += 32) s += (double)p[(int64_t)k * D];
   }

@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_upsweep(KeySrc s, int64_t 
   }
 }
 
-// --- device-wide exclusive scan of uint32 (three phases) ---
+// --- device-wide exclusive scan of uint32: chunk totals, then every chunk scans itself ---
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* sh_warp,
                                                          uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -157,22 +157,15 @@ __global__ void __launch_bounds__(kScanBlock) scan_reduce(const uint32_t* in, in
   if (threadIdx.x == 0) part[blockIdx.x] = tot;
 }
 
-__global__ void __launch_bounds__(kScanBlock) scan_parts(uint32_t* part, int64_t nparts) {
-  __shared__ uint32_t sw[32];
-  uint32_t carry = 0;
-  for (int64_t b0 = 0; b0 < nparts; b0 += kScanBlock) {
-    const int64_t j = b0 + threadIdx.x;
-    uint32_t v = j < nparts ? part[j] : 0;
-    uint32_t tot;
-    uint32_t ex = block_exclusive_scan(v, sw, &tot);
-    if (j < nparts) part[j] = carry + ex;
-    carry += tot;
-  }
-}
-
+// Chunk i adds the totals of chunks 0..i-1 itself (a block sum over at most
+// a few thousand words in L2), so no separate pass scans the chunk totals.
 __global__ void __launch_bounds__(kScanBlock) scan_apply(uint32_t* data, int64_t len,
                                                          const uint32_t* part) {
   __shared__ uint32_t sw[32];
+  uint32_t earlier = 0;
+  for (int64_t j = threadIdx.x; j < (int64_t)blockIdx.x; j += kScanBlock) earlier += part[j];
+  uint32_t carry;
+  block_exclusive_scan(earlier, sw, &carry);
   const int64_t base = (int64_t)blockIdx.x * kScanChunk;
   // blocked arrangement: thread t owns kScanItems consecutive entries
   uint32_t v[kScanItems];
@@ -183,7 +176,7 @@ __global__ void __launch_bounds__(kScanBlock) scan_apply(uint32_t* data, int64_t
     v[i] = j < len ? data[j] : 0;
     t += v[i];
   }
-  uint32_t ex = block_exclusive_scan(t, sw, nullptr) + part[blockIdx.x];
+  uint32_t ex = block_exclusive_scan(t, sw, nullptr) + carry;
 #pragma unroll
   for (int i = 0; i < kScanItems; ++i) {
     int64_t j = base + (int64_t)threadIdx.x * kScanItems + i;
@@ -522,9 +515,8 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_single_tile_kernel(CsArgs a) 
 fkm_status device_scan(uint32_t* data, int64_t len, uint32_t* part, cudaStream_t st) {
   const int64_t nparts = ceil_div(len, kScanChunk);
   scan_reduce<<<(unsigned)nparts, kScanBlock, 0, st>>>(data, len, part);
-  scan_parts<<<1, kScanBlock, 0, st>>>(part, nparts);
   scan_apply<<<(unsigned)nparts, kScanBlock, 0, st>>>(data, len, part);
-  note_launch(3);
+  note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
 }

@@ -75,6 +75,27 @@ def test_argsort_rejects_bad_keys():
     assert e.value.code == 7
 
 
+@pytest.mark.parametrize("n,n_keys", [(3 * 4096 + 77, 300), (2 * 4096 + 5, 2048),
+                                      (2 * 4096 + 5, 2049), (20011, 5000)])
+def test_argsort_rejected_keys_sort_last_in_index_order(n, n_keys):
+    """Keys outside [0, n_keys), spread over several sort tiles, go after
+    every valid key, themselves in index order (both the counting sort and
+    the radix sort), and raise FKM_ERR_BAD_ID."""
+    rng = np.random.default_rng(7 * n + n_keys)
+    keys = rng.integers(0, n_keys, size=n).astype(np.int32)
+    bad = rng.random(n) < 0.01
+    keys[bad] = np.where(rng.random(bad.sum()) < 0.5, -3, n_keys + 11).astype(np.int32)
+    t = torch.from_numpy(keys).cuda()
+    idx = torch.empty_like(t)
+    ws = fkm.workspace(fkm.fkm_argsort_workspace_size(n, n_keys))
+    fkm.fkm_argsort(t, n_keys, idx, ws=ws)
+    with pytest.raises(fkm.FkmError) as e:
+        fkm.fkm_sync_status(ws)
+    assert e.value.code == 7
+    mapped = np.where(bad, n_keys, keys).astype(np.int32)
+    assert np.array_equal(idx.cpu().numpy(), oracle.argsort_stable(mapped, n_keys + 1))
+
+
 # ------------------------------------------------------------------ assign
 def _grid(rng, B, N, K, D, dup=True):
     """Integer centroids and points: every product and sum is exact in fp32,
