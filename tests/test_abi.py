@@ -88,6 +88,26 @@ def test_null_pointers_rejected_before_any_launch(fkm):
     assert rc == 4
 
 
+def test_shard_calls_validate_before_any_launch(fkm):
+    L = fkm.lib()
+    ws = ctypes.create_string_buffer(1 << 20)
+    a = (ctypes.addressof(ws) + 15) & ~15
+    # fkm_partial_update: x is required
+    assert L.fkm_partial_update(1, 16, 4, 64, 2, None, a, a, a, a, None, a, 1 << 19, None) == 1
+    # fkm_finalize_sums: centers may not alias prev; the scratch must hold 256 + 8*B*K bytes
+    assert L.fkm_finalize_sums(1, 4, 64, a, a + 4096, a + 8192, a + 8192, None, a + 16384,
+                               1024, None) == 1
+    assert L.fkm_finalize_sums(1, 4, 64, a, a + 4096, a + 8192, a + 12288, None, a + 16384,
+                               200, None) == 4
+    # fkm_partial_update_host: sums are required and 16-byte aligned; the host workspace
+    # is sized by fkm_host_workspace_size
+    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, None, a, None, a, 1 << 19,
+                                     None) == 1
+    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a + 8, a, None, a, 1 << 19,
+                                     None) == 1
+    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a, a, None, a, 64, None) == 4
+
+
 def test_status_strings_and_version(fkm):
     L = fkm.lib()
     assert L.fkm_status_string(0) == b"ok"
