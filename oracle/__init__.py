@@ -12,6 +12,10 @@ Parity pins: every function here is pinned by ``tests/test_oracle.py``
 (the pages' argsort example, brute force on tiny inputs, closed forms for
 K = 1 and K = N, the D = 1 nearest-neighbour rule, exact integer-grid cases,
 translation invariance, monotone objective, fixed point, storage rounding).
+The dot-product and cosine functions are pinned against the Euclidean ones
+where the metrics coincide (unit-norm points and centroids; centroids of
+equal norm), by scale invariance, and by the spherical objective's monotone
+ascent.
 """
 from __future__ import annotations
 
@@ -63,8 +67,15 @@ def _load():
                                 ctypes.c_double, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]
         L.orc_argsort_stable.argtypes = [_P, _I, _I, _P]
         L.orc_centre.argtypes = [_I, _I, _I, _P, ctypes.c_int, _P, _P, _P]
+        _c = ctypes.c_int
+        L.orc_assign_sim.argtypes = [_I, _I, _I, _I, _P, _c, _P, _c, _c, _P, _P, _P]
+        L.orc_similarity.argtypes = [_I, _I, _I, _I, _P, _c, _P, _P, _c, _P]
+        L.orc_update_sim.argtypes = [_I, _I, _I, _I, _P, _c, _P, _P, _c, _P, _P, _P]
+        L.orc_lloyd_sim.argtypes = [_I, _I, _I, _I, _P, _c, _P, _c, ctypes.c_double, _c, _c,
+                                    _P, _P, _P, _P, _P, _P, _P]
         for f in ("orc_assign", "orc_inertia", "orc_update", "orc_lloyd", "orc_argsort_stable",
-                  "orc_centre"):
+                  "orc_centre", "orc_assign_sim", "orc_similarity", "orc_update_sim",
+                  "orc_lloyd_sim"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -187,6 +198,82 @@ def lloyd(x, c0, max_iters, tol=0.0, dtype="f32", mirror=None):
                            ctypes.byref(n_iter), _ptr(J_hist), _ptr(sh_hist))
     if rc:
         raise RuntimeError("orc_lloyd failed")
+    n = n_iter.value
+    return dict(ids=ids, centers=centers, counts=counts, inertia=inert, n_iter=n,
+                J_hist=J_hist[:n], shift_hist=sh_hist[:n])
+
+
+# ---- dot-product and cosine k-means (see oracle.c for the readings) ----
+METRIC_CODE = {"dot": 1, "cosine": 2}
+
+
+def assign_sim(x, c, metric, dtype="f32", mirror=None):
+    """Most similar centroid per point under ``metric`` ('dot' or 'cosine'):
+    returns (ids int32 [B,N], s1 best score, s2 second-best score [B,N])."""
+    x, code = _x3(x, dtype)
+    B, N, D = x.shape
+    c = _c3(c, B)
+    K = c.shape[1]
+    ids = np.empty((B, N), np.int32)
+    s1 = np.empty((B, N), np.float64)
+    s2 = np.empty((B, N), np.float64)
+    rc = _load().orc_assign_sim(B, N, K, D, _ptr(x), code, _ptr(c), METRIC_CODE[metric],
+                                _mirror(mirror), _ptr(ids), _ptr(s1), _ptr(s2))
+    if rc:
+        raise RuntimeError("orc_assign_sim failed")
+    return ids, s1, s2
+
+
+def similarity(x, ids, c, metric, dtype="f32"):
+    """Objective of an assignment: J [B] = sum_i x_i . v_{ids_i}, v = c (dot) or c/||c||."""
+    x, code = _x3(x, dtype)
+    B, N, D = x.shape
+    c = _c3(c, B)
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(B, N)
+    J = np.empty(B, np.float64)
+    rc = _load().orc_similarity(B, N, c.shape[1], D, _ptr(x), code, _ptr(ids), _ptr(c),
+                                METRIC_CODE[metric], _ptr(J))
+    if rc:
+        raise RuntimeError("orc_similarity failed (id out of range?)")
+    return J
+
+
+def update_sim(x, ids, c_prev, metric, dtype="f32"):
+    """Update under ``metric``: returns (c_new float64 [B,K,D], counts [B,K], shift [B])."""
+    x, code = _x3(x, dtype)
+    B, N, D = x.shape
+    c_prev = _c3(c_prev, B)
+    K = c_prev.shape[1]
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(B, N)
+    c_new = np.empty_like(c_prev)
+    counts = np.empty((B, K), np.int64)
+    shift = np.empty(B, np.float64)
+    rc = _load().orc_update_sim(B, N, K, D, _ptr(x), code, _ptr(ids), _ptr(c_prev),
+                                METRIC_CODE[metric], _ptr(c_new), _ptr(counts), _ptr(shift))
+    if rc:
+        raise RuntimeError("orc_update_sim failed (id out of range?)")
+    return c_new, counts, shift
+
+
+def lloyd_sim(x, c0, max_iters, metric, tol=0.0, dtype="f32", mirror=None):
+    """Lloyd run under ``metric``; the same dict as lloyd()."""
+    x, code = _x3(x, dtype)
+    B, N, D = x.shape
+    c0 = _c3(c0, B)
+    K = c0.shape[1]
+    ids = np.empty((B, N), np.int32)
+    centers = np.empty_like(c0)
+    counts = np.empty((B, K), np.int64)
+    inert = np.empty(B, np.float64)
+    n_iter = ctypes.c_int(0)
+    J_hist = np.full((max_iters, B), np.nan)
+    sh_hist = np.full((max_iters, B), np.nan)
+    rc = _load().orc_lloyd_sim(B, N, K, D, _ptr(x), code, _ptr(c0), max_iters, float(tol),
+                               METRIC_CODE[metric], _mirror(mirror), _ptr(ids), _ptr(centers),
+                               _ptr(counts), _ptr(inert), ctypes.byref(n_iter), _ptr(J_hist),
+                               _ptr(sh_hist))
+    if rc:
+        raise RuntimeError("orc_lloyd_sim failed")
     n = n_iter.value
     return dict(ids=ids, centers=centers, counts=counts, inertia=inert, n_iter=n,
                 J_hist=J_hist[:n], shift_hist=sh_hist[:n])

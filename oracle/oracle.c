@@ -355,6 +355,176 @@ int orc_lloyd(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xdt
   return rc;
 }
 
+/* ---------- dot-product and cosine k-means ----------
+ * The README lists cosine and dot-product k-means beside the Euclidean one
+ * ("Flash-KMeans" GitHub README, section "Usage", the CuTe backend note) but
+ * defines neither; the plainest readings are taken:
+ *   dot      a_i = argmax_k x_i . c_k; c_k = mean of its points (as above);
+ *            objective J = sum_i x_i . c_{a_i}
+ *   cosine   a_i = argmax_k x_i . u_k with u_k = c_k / ||c_k|| (the point's
+ *            own norm does not move its argmax); c_k = s_k / ||s_k||, the
+ *            direction of its points' sum (spherical k-means; for unit-norm
+ *            points the sum of directions); objective J = sum_i x_i . u_{a_i}
+ * Ties go to the lowest index, an empty cluster (or one whose sum is the zero
+ * vector) keeps its previous centroid, and shift is as above.  In mirror mode
+ * the assignment measures against c_hat = m + q(fp32(v - m)) of v = c (dot)
+ * or v = u (cosine), u = fp32(c_d / ||c||) with ||c|| in fp64 and m the mean
+ * of the v rows, as orc_chat forms it; the objective uses the plain c or u. */
+enum { ORC_EUCLID = 0, ORC_DOT = 1, ORC_COSINE = 2 };
+
+/* u = fp32(c / ||c||) row by row (a zero row stays zero) */
+static void orc_unit_rows(const double* c, int64_t rows, int64_t D, double* u) {
+  for (int64_t r = 0; r < rows; ++r) {
+    double nn = 0.0;
+    for (int64_t d = 0; d < D; ++d) {
+      const double v = (double)(float)c[r * D + d];
+      nn += v * v;
+    }
+    const double n = sqrt(nn);
+    for (int64_t d = 0; d < D; ++d)
+      u[r * D + d] = n > 0.0 ? (double)(float)((double)(float)c[r * D + d] / n) : 0.0;
+  }
+}
+
+/* the vectors a metric scores against, before any mirroring: c or u */
+static int orc_metric_rows(const double* c, int64_t rows, int64_t D, int metric, double* out) {
+  if (metric == ORC_COSINE) orc_unit_rows(c, rows, D, out);
+  else if (metric == ORC_DOT) memcpy(out, c, sizeof(double) * (size_t)(rows * D));
+  else return -1;
+  return 0;
+}
+
+/* ids = argmax_k x_i . c_hat_k (lowest k on ties), s1 the best score, s2 the
+ * second best over the other centroids (-inf when K == 1).  Returns 0 or -1. */
+int orc_assign_sim(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xdt,
+                   const double* c, int metric, int mirror, int32_t* ids, double* s1,
+                   double* s2) {
+  if (B < 1 || N < 0 || K < 1 || D < 1 || !x || !c) return -1;
+  double* v = (double*)malloc(sizeof(double) * (size_t)(B * K * D));
+  double* ch = (double*)malloc(sizeof(double) * (size_t)(B * K * D));
+  if (!v || !ch || orc_metric_rows(c, B * K, D, metric, v)) { free(v); free(ch); return -1; }
+  orc_chat(v, B, K, D, mirror, ch);
+  for (int64_t b = 0; b < B; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+      double best = -INFINITY, second = -INFINITY;
+      int64_t arg = 0;
+      for (int64_t k = 0; k < K; ++k) {
+        const double* ck = ch + (b * K + k) * D;
+        double sc = 0.0;
+        for (int64_t d = 0; d < D; ++d) sc += orc_read(x, xdt, (b * N + i) * D + d) * ck[d];
+        if (sc > best) { second = best; best = sc; arg = k; }
+        else if (sc > second) { second = sc; }
+      }
+      if (ids) ids[b * N + i] = (int32_t)arg;
+      if (s1) s1[b * N + i] = best;
+      if (s2) s2[b * N + i] = second;
+    }
+  }
+  free(v);
+  free(ch);
+  return 0;
+}
+
+/* J[b] = sum_i x_i . v_{ids_i} (point order), v = c (dot) or u (cosine). */
+int orc_similarity(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xdt,
+                   const int32_t* ids, const double* c, int metric, double* J) {
+  if (B < 1 || N < 0 || K < 1 || D < 1 || !x || !c || !ids || !J) return -1;
+  double* v = (double*)malloc(sizeof(double) * (size_t)(B * K * D));
+  if (!v || orc_metric_rows(c, B * K, D, metric, v)) { free(v); return -1; }
+  int bad = 0;
+  for (int64_t b = 0; b < B; ++b) {
+    double Jb = 0.0;
+    for (int64_t i = 0; i < N; ++i) {
+      const int64_t k = ids[b * N + i];
+      if (k < 0 || k >= K) { bad = 1; continue; }
+      for (int64_t d = 0; d < D; ++d)
+        Jb += orc_read(x, xdt, (b * N + i) * D + d) * v[(b * K + k) * D + d];
+    }
+    J[b] = Jb;
+  }
+  free(v);
+  return bad ? -1 : 0;
+}
+
+/* The update of a metric: the mean for dot (orc_update); for cosine the mean
+ * scaled to unit length, s_k / ||s_k||, unless the cluster is empty or its sum
+ * is zero (then the previous centroid stays).  shift as in orc_update. */
+int orc_update_sim(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xdt,
+                   const int32_t* ids, const double* c_prev, int metric, double* c_new,
+                   int64_t* counts, double* shift) {
+  if (metric != ORC_DOT && metric != ORC_COSINE) return -1;
+  int64_t* n = (int64_t*)malloc(sizeof(int64_t) * (size_t)(B * K));
+  if (!n) return -1;
+  int rc = orc_update(B, N, K, D, x, xdt, ids, c_prev, c_new, n, NULL);
+  if (!rc) {
+    for (int64_t b = 0; b < B; ++b) {
+      double sh = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        double* ck = c_new + (b * K + k) * D;
+        if (metric == ORC_COSINE && n[b * K + k] > 0) {
+          double nn = 0.0;
+          for (int64_t d = 0; d < D; ++d) nn += ck[d] * ck[d];
+          if (nn > 0.0) {
+            const double r = sqrt(nn);
+            for (int64_t d = 0; d < D; ++d) ck[d] /= r;
+          } else {
+            memcpy(ck, c_prev + (b * K + k) * D, sizeof(double) * (size_t)D);
+          }
+        }
+        for (int64_t d = 0; d < D; ++d) {
+          const double df = ck[d] - c_prev[(b * K + k) * D + d];
+          sh += df * df;
+        }
+        if (counts) counts[b * K + k] = n[b * K + k];
+      }
+      if (shift) shift[b] = sh;
+    }
+  }
+  free(n);
+  return rc;
+}
+
+/* The Lloyd loop of a metric, as orc_lloyd: inertia is the objective J of the
+ * last assignment against the centroids it used; J_hist / shift_hist record
+ * every iteration. */
+int orc_lloyd_sim(int64_t B, int64_t N, int64_t K, int64_t D, const void* x, int xdt,
+                  const double* c0, int max_iters, double tol, int metric, int mirror,
+                  int32_t* ids, double* centers, int64_t* counts, double* inertia, int* n_iter,
+                  double* J_hist, double* shift_hist) {
+  if (B < 1 || N < 0 || K < 1 || D < 1 || max_iters < 1 || !x || !c0 || !ids || !centers)
+    return -1;
+  const int64_t nc = B * K * D;
+  double* cur = (double*)malloc(sizeof(double) * (size_t)nc);
+  double* nxt = (double*)malloc(sizeof(double) * (size_t)nc);
+  double* J = (double*)malloc(sizeof(double) * (size_t)B);
+  double* sh = (double*)malloc(sizeof(double) * (size_t)B);
+  if (!cur || !nxt || !J || !sh) { free(cur); free(nxt); free(J); free(sh); return -1; }
+  memcpy(cur, c0, sizeof(double) * (size_t)nc);
+  int rc = 0, t = 0;
+  for (t = 0; t < max_iters; ++t) {
+    rc = orc_assign_sim(B, N, K, D, x, xdt, cur, metric, mirror, ids, NULL, NULL);
+    if (!rc) rc = orc_similarity(B, N, K, D, x, xdt, ids, cur, metric, J);
+    if (!rc) rc = orc_update_sim(B, N, K, D, x, xdt, ids, cur, metric, nxt, counts, sh);
+    if (rc) break;
+    double* tmp = cur; cur = nxt; nxt = tmp;
+    double mx = 0.0;
+    for (int64_t b = 0; b < B; ++b) {
+      if (J_hist) J_hist[(int64_t)t * B + b] = J[b];
+      if (shift_hist) shift_hist[(int64_t)t * B + b] = sh[b];
+      if (sh[b] > mx) mx = sh[b];
+    }
+    if (mx < tol) { t += 1; break; }
+  }
+  if (!rc) {
+    memcpy(centers, cur, sizeof(double) * (size_t)nc);
+    if (inertia) memcpy(inertia, J, sizeof(double) * (size_t)B);
+    if (n_iter) *n_iter = t;
+  }
+  free(cur); free(nxt); free(J); free(sh);
+  return rc;
+}
+
 /* ---------- stable argsort of small non-negative integer keys ---------- */
 /* idx[r] = the index of the r-th smallest key; equal keys keep index order. */
 int orc_argsort_stable(const int64_t* keys, int64_t n, int64_t n_keys, int64_t* idx) {

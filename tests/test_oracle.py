@@ -460,3 +460,170 @@ def test_centre_is_translation_free():
     a, _ = oracle.centre(x, "f32")
     b, _ = oracle.centre(x + t, "f32")
     assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------- dot-product and cosine
+def _unit_centroids(D, K, rng):
+    """K distinct rows of exactly unit norm in fp32: signed axis vectors and
+    (+-1/2, +-1/2, +-1/2, +-1/2) on a random choice of four axes."""
+    rows = set()
+    while len(rows) < K:
+        v = np.zeros(D)
+        if rng.random() < 0.5:
+            v[rng.integers(D)] = rng.choice([-1.0, 1.0])
+        else:
+            v[rng.choice(D, 4, replace=False)] = rng.choice([-0.5, 0.5], 4)
+        rows.add(tuple(v))
+    return np.array(sorted(rows))
+
+
+def _clear_of_ties(d1, d2, eps=1e-9):
+    return (d2 - d1) > eps
+
+
+def test_cosine_equals_euclid_on_unit_centroids():
+    """||x - c||^2 = ||x||^2 + 1 - 2 x.c for unit c: nearest = most similar."""
+    rng = np.random.default_rng(21)
+    B, N, K, D = 2, 300, 12, 8
+    x = rng.standard_normal((B, N, D)).astype(np.float32)
+    c = np.stack([_unit_centroids(D, K, rng) for _ in range(B)])
+    ids_e, d1, d2, _ = oracle.assign(x, c)
+    ok = _clear_of_ties(d1, d2)
+    for metric in ("cosine", "dot"):
+        ids_s, s1, s2 = oracle.assign_sim(x, c, metric)
+        assert ok.mean() > 0.99
+        assert np.array_equal(ids_s[ok], ids_e[ok])
+        assert np.all(s1 >= s2)
+
+
+def test_dot_equals_euclid_for_equal_norm_centroids():
+    rng = np.random.default_rng(22)
+    B, N, K, D = 1, 400, 10, 8
+    x = rng.standard_normal((B, N, D)).astype(np.float32)
+    c = 3.0 * _unit_centroids(D, K, rng)[None]       # every row of norm exactly 3
+    ids_e, d1, d2, _ = oracle.assign(x, c)
+    ids_s, _, _ = oracle.assign_sim(x, c, "dot")
+    ok = _clear_of_ties(d1, d2)
+    assert np.array_equal(ids_s[ok], ids_e[ok])
+
+
+def test_sim_assign_matches_numpy_argmax_tiny():
+    rng = np.random.default_rng(23)
+    x = rng.standard_normal((1, 40, 5)).astype(np.float32)
+    c = rng.standard_normal((1, 7, 5))
+    xd = x[0].astype(np.float64)
+    dot = xd @ c[0].T
+    u = (c[0] / np.linalg.norm(c[0], axis=1, keepdims=True)).astype(np.float32).astype(np.float64)
+    cos = xd @ u.T
+    assert np.array_equal(oracle.assign_sim(x, c, "dot")[0][0], dot.argmax(1))
+    assert np.array_equal(oracle.assign_sim(x, c, "cosine")[0][0], cos.argmax(1))
+
+
+def test_sim_assign_mirror_scores_against_the_centred_rounded_operand():
+    rng = np.random.default_rng(24)
+    x = rng.standard_normal((1, 60, 16)).astype(np.float32)
+    c = rng.standard_normal((1, 9, 16)) + 5.0
+    xd = x[0].astype(np.float64)
+    ch = oracle.chat(c, "bf16")[0]
+    assert np.array_equal(oracle.assign_sim(x, c, "dot", mirror="bf16")[0][0],
+                          (xd @ ch.T).argmax(1))
+    u = (c[0] / np.linalg.norm(c[0], axis=1, keepdims=True)).astype(np.float32)
+    chu = oracle.chat(u.astype(np.float64)[None], "bf16")[0]
+    assert np.array_equal(oracle.assign_sim(x, c, "cosine", mirror="bf16")[0][0],
+                          (xd @ chu.T).argmax(1))
+
+
+def test_cosine_assign_is_scale_invariant():
+    """Scaling points and centroid rows by powers of two (exact in fp32)
+    leaves every cosine assignment unchanged."""
+    rng = np.random.default_rng(25)
+    x = rng.standard_normal((2, 200, 12)).astype(np.float32)
+    c = rng.standard_normal((2, 9, 12))
+    ids0, _, _ = oracle.assign_sim(x, c, "cosine")
+    xs = (x * (2.0 ** rng.integers(-3, 4, size=(2, 200, 1)))).astype(np.float32)
+    cs = c * 2.0 ** rng.integers(-3, 4, size=(2, 9, 1))
+    assert np.array_equal(oracle.assign_sim(xs, cs, "cosine")[0], ids0)
+
+
+def test_sim_ties_go_to_lowest_index():
+    x = np.array([[[1.0, 2.0]]], np.float32)
+    c = np.array([[[0.0, 1.0], [2.0, 0.0], [0.0, 1.0]]])   # dot: 2, 2, 2
+    assert oracle.assign_sim(x, c, "dot")[0][0, 0] == 0
+    c2 = np.array([[[0.0, 5.0], [0.0, 1.0]]])              # cosine: equal directions
+    assert oracle.assign_sim(x, c2, "cosine")[0][0, 0] == 0
+
+
+def test_update_sim_dot_is_the_mean_cosine_the_unit_sum():
+    rng = np.random.default_rng(26)
+    B, N, K, D = 2, 300, 8, 6
+    x = rng.standard_normal((B, N, D)).astype(np.float32)
+    ids = rng.integers(0, K - 1, size=(B, N)).astype(np.int32)     # cluster K-1 empty
+    ids[0, :2] = K - 2
+    ids[0, 2:][ids[0, 2:] == K - 2] = 0
+    x[0, 1] = -x[0, 0]                                             # cluster K-2: zero sum
+    c_prev = rng.standard_normal((B, K, D))
+    cd, nd, shd = oracle.update_sim(x, ids, c_prev, "dot")
+    cc, nc, shc = oracle.update_sim(x, ids, c_prev, "cosine")
+    for b in range(B):
+        assert np.array_equal(nd[b], np.bincount(ids[b], minlength=K))
+        assert np.array_equal(nc[b], nd[b])
+        for k in range(K):
+            m = ids[b] == k
+            s = x[b][m].astype(np.float64).sum(0)
+            if not m.any() or not s.any():
+                assert np.array_equal(cc[b, k], c_prev[b, k])
+            else:
+                assert np.allclose(cd[b, k], s / m.sum(), rtol=1e-13)
+                assert np.isclose(np.linalg.norm(cc[b, k]), 1.0, rtol=1e-14)
+                assert np.allclose(cc[b, k] * np.linalg.norm(s), s, rtol=1e-12, atol=1e-12)
+        assert np.isclose(shc[b], np.sum((cc[b] - c_prev[b]) ** 2), rtol=1e-13)
+
+
+def test_similarity_closed_forms():
+    """Dot: J = sum_k s_k . c_k over the cluster sums.  Cosine, against the
+    centroids the update just formed: J = sum_k ||s_k||."""
+    rng = np.random.default_rng(27)
+    B, N, K, D = 2, 250, 7, 5
+    x = rng.standard_normal((B, N, D)).astype(np.float32)
+    ids = rng.integers(0, K, size=(B, N)).astype(np.int32)
+    c = rng.standard_normal((B, K, D))
+    sums = np.zeros((B, K, D))
+    for b in range(B):
+        np.add.at(sums[b], ids[b], x[b].astype(np.float64))
+    assert np.allclose(oracle.similarity(x, ids, c, "dot"), np.einsum("bkd,bkd->b", sums, c),
+                       rtol=1e-12)
+    cc, _, _ = oracle.update_sim(x, ids, c, "cosine")
+    # the update's rows are unit length in fp64; the objective rounds them to fp32 first
+    J = oracle.similarity(x, ids, cc, "cosine")
+    assert np.allclose(J, np.linalg.norm(sums, axis=2).sum(1), rtol=1e-6)
+
+
+def test_spherical_lloyd_objective_never_decreases():
+    """Assignment maximises each point's similarity and the unit sum maximises
+    each cluster's, so J can only grow (pure mode)."""
+    rng = np.random.default_rng(28)
+    w = datagen.CONFIGS[1].scaled(B=2, N=600, K=9, iters=8)
+    x = datagen.points(w)
+    c0 = datagen.init_centroids(x, datagen.init_indices(w), w.dtype)
+    r = oracle.lloyd_sim(x, c0, 8, "cosine", dtype=w.dtype)
+    J = r["J_hist"]
+    assert np.all(np.diff(J, axis=0) >= -1e-9 * np.abs(J[1:]))
+    assert np.all(r["counts"].sum(1) == w.N)
+    assert np.allclose(np.linalg.norm(r["centers"], axis=2)[r["counts"] > 0], 1.0, rtol=1e-12)
+
+
+@pytest.mark.parametrize("metric", ["dot", "cosine"])
+def test_lloyd_sim_wiring_matches_step_chain(metric):
+    rng = np.random.default_rng(29)
+    x = rng.standard_normal((2, 120, 6)).astype(np.float32)
+    c0 = x[:, :5].astype(np.float64)
+    r = oracle.lloyd_sim(x, c0, 2, metric)
+    c = c0
+    for _ in range(2):
+        ids, _, _ = oracle.assign_sim(x, c, metric)
+        J = oracle.similarity(x, ids, c, metric)
+        c, counts, _ = oracle.update_sim(x, ids, c, metric)
+    assert np.array_equal(r["ids"], ids)
+    assert np.array_equal(r["centers"], c)
+    assert np.array_equal(r["inertia"], J)
+    assert r["n_iter"] == 2
