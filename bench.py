@@ -177,10 +177,11 @@ def over_ranks(torch, dist, dev, t_ms, n_iters):
     return t.item(), int(n.item())
 
 
-def oracle_sample(w, iters, rows=None):
+def oracle_sample(w, iters, rows=None, metric="euclid"):
     """The fp64 oracle on batch 0 of the workload (its first `rows` points when
-    given) for `iters` Lloyd iterations.  Returns (seconds, scale, description):
-    the whole problem's iteration costs `scale` times the sample's."""
+    given) for `iters` Lloyd iterations under `metric`.  Returns (seconds,
+    scale, description): the whole problem's iteration costs `scale` times the
+    sample's."""
     import oracle
     n = w.N if rows is None else max(min(int(rows), w.N), w.K)
     ws = w.scaled(B=1, N=n)
@@ -188,7 +189,10 @@ def oracle_sample(w, iters, rows=None):
     c0 = datagen.init_centroids(x, datagen.init_indices(ws), ws.dtype)
     mir = w.dtype if w.dtype != "f32" else None
     t0 = time.perf_counter()
-    oracle.lloyd(x, c0, iters, 0.0, dtype=w.dtype, mirror=mir)
+    if metric == "euclid":
+        oracle.lloyd(x, c0, iters, 0.0, dtype=w.dtype, mirror=mir)
+    else:
+        oracle.lloyd_sim(x, c0, iters, metric, 0.0, dtype=w.dtype, mirror=mir)
     dt = time.perf_counter() - t0
     scale = w.B * (w.N / n)
     part = "" if n == w.N else f"first {n} points of "
@@ -248,16 +252,16 @@ def comparison(fkm, torch, w, xt, c0t, ws, stream, dev, reps=3):
     return out
 
 
-def cpu_baseline(w, max_iters, budget_s=15.0):
+def cpu_baseline(w, max_iters, budget_s=15.0, metric="euclid"):
     """The oracle's iteration rate on a bounded sample of the workload: a probe
     on a few thousand points of batch 0 sizes the sample (points of batch 0,
     and iterations up to max_iters) to about budget_s seconds of CPU work."""
     probe_rows = max(w.K, min(w.N, 4096))
-    t_probe, _, _ = oracle_sample(w, 1, probe_rows)
+    t_probe, _, _ = oracle_sample(w, 1, probe_rows, metric)
     per_row = max(t_probe, 1e-6) / probe_rows
     rows = int(min(w.N, max(probe_rows, budget_s / per_row)))
     iters = int(max(1, min(max_iters, budget_s / (per_row * rows))))
-    dt, scale, desc = oracle_sample(w, iters, rows)
+    dt, scale, desc = oracle_sample(w, iters, rows, metric)
     return iters / (dt * scale), desc
 
 
@@ -529,6 +533,8 @@ def main():
     ap.add_argument("--sharded", action="store_true",
                     help="one problem split over the ranks' GPUs (strong scaling)")
     ap.add_argument("--oracle-iters", type=int, default=10)
+    ap.add_argument("--metric", default="euclid", choices=["euclid", "dot", "cosine"],
+                    help="similarity of the clustering (dot and cosine k-means: fkm_lloyd_metric)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -572,9 +578,15 @@ def main():
     ws = fkm.workspace(fkm.fkm_workspace_size(B, N, K, D, tdt), dev)
     stream = torch.cuda.current_stream(dev)
 
+    def lloyd(xs, cs):
+        if args.metric == "euclid":
+            return fkm.fkm_lloyd(xs, cs, wr.iters, wr.tol, ids, centers, counts, inertia, ws=ws,
+                                 stream=stream)
+        return fkm.fkm_lloyd_metric(xs, cs, wr.iters, wr.tol, ids, centers, counts, args.metric,
+                                    inertia, ws=ws, stream=stream)
+
     def step():
-        return fkm.fkm_lloyd(xt, c0t, wr.iters, wr.tol, ids, centers, counts, inertia, ws=ws,
-                             stream=stream)
+        return lloyd(xt, c0t)
 
     def barrier():
         if dist is not None:
@@ -632,7 +644,9 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": wr.dtype, "data": "synthetic", "config": workload_config(wr),
+            "dtype": wr.dtype, "data": "synthetic",
+            "config": dict(workload_config(wr), **({} if args.metric == "euclid"
+                                                    else {"metric": args.metric})),
             "roofline": roofline,
             "stages_ms_per_iter": {k: prof[k] / it for k in fkm.STAGES},
             "assign_tflops": tflops,
@@ -644,7 +658,7 @@ def main():
     # --- the pages' comparison point (not the method): materialised distances
     # + argmin read-back, and the scatter-atomic update, against the fused
     # calls on the same inputs (outside the timed region)
-    if not args.no_comparison:
+    if not args.no_comparison and args.metric == "euclid":
         line["comparison"] = comparison(fkm, torch, wr, xt, c0t, ws, stream, dev)
 
     # --- end to end through the C ABI with host buffers.  Every step copies its
@@ -676,8 +690,7 @@ def main():
         def e2e_step(k):
             s = k % 2
             stream.wait_event(ready[s])
-            n_it = fkm.fkm_lloyd(x_e[s], c_e[s], wr.iters, wr.tol, ids, centers, counts, inertia,
-                                 ws=ws, stream=stream)
+            n_it = lloyd(x_e[s], c_e[s])
             done[s].record(stream)
             ids_h.copy_(ids, non_blocking=True)
             cen_h.copy_(centers, non_blocking=True)
@@ -712,7 +725,7 @@ def main():
 
     # --- the oracle on this host's cores (rank 0, one GPU only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        value_c, desc = cpu_baseline(wr, args.oracle_iters)
+        value_c, desc = cpu_baseline(wr, args.oracle_iters, metric=args.metric)
         line["cpu_baseline"] = {"value": value_c, "unit": UNIT, "cores": cpu_cores(),
                                 "kind": "oracle", "sample": desc}
 

@@ -27,6 +27,7 @@ STATUS_NAMES = {0: "FKM_OK", 1: "FKM_ERR_INVALID_ARG", 2: "FKM_ERR_UNSUPPORTED",
                 3: "FKM_ERR_CUDA", 4: "FKM_ERR_WORKSPACE_TOO_SMALL", 5: "FKM_ERR_TIMEOUT",
                 6: "FKM_ERR_INTERNAL", 7: "FKM_ERR_BAD_ID"}
 DTYPES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+METRICS = {"euclid": 0, "dot": 1, "cosine": 2}
 
 # every entry point of include/fkm.h: name -> (argtypes, restype)
 _P, _I, _L, _Z, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -43,6 +44,10 @@ _SIG = {
     "fkm_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_lloyd": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _P, _P, ctypes.POINTER(_I), _P, _Z,
                    _P], _I),
+    "fkm_assign_metric": ([_I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_update_metric": ([_I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_lloyd_metric": ([_I, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _P, _P,
+                          ctypes.POINTER(_I), _P, _Z, _P], _I),
     "fkm_host_workspace_size": ([_I, _I, _I, _I, _I, _L, ctypes.POINTER(_Z)], _I),
     "fkm_lloyd_host": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _L, _P, _P, _P, _P,
                         ctypes.POINTER(_I), _P, _Z, _P], _I),
@@ -170,6 +175,47 @@ def fkm_lloyd(x, init_centers, max_iters, tol, ids, centers, counts, inertia=Non
                                         float(tol), _ptr(ids), _ptr(centers), _ptr(counts),
                                         _ptr(inertia), ctypes.byref(n_iter), _ptr(ws), ws.numel(),
                                         _stream(stream)))
+    return n_iter.value
+
+
+def _metric(metric) -> int:
+    if isinstance(metric, str):
+        return METRICS[metric]
+    return int(metric)
+
+
+def fkm_assign_metric(x, centers, ids, metric, ws=None, stream=None):
+    """ids = the most similar centroid under metric ('euclid', 'dot', 'cosine')."""
+    B, N, D = x.shape
+    K = centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    _check("fkm_assign_metric",
+           lib().fkm_assign_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(centers),
+                                   _ptr(ids), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fkm_update_metric(x, ids, prev_centers, centers, counts, metric, shift=None, objective=None,
+                      ws=None, stream=None):
+    B, N, D = x.shape
+    K = prev_centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    _check("fkm_update_metric",
+           lib().fkm_update_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(ids),
+                                   _ptr(prev_centers), _ptr(centers), _ptr(counts), _ptr(shift),
+                                   _ptr(objective), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fkm_lloyd_metric(x, init_centers, max_iters, tol, ids, centers, counts, metric,
+                     objective=None, ws=None, stream=None) -> int:
+    B, N, D = x.shape
+    K = init_centers.shape[1]
+    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    n_iter = ctypes.c_int(0)
+    _check("fkm_lloyd_metric",
+           lib().fkm_lloyd_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x),
+                                  _ptr(init_centers), max_iters, float(tol), _ptr(ids),
+                                  _ptr(centers), _ptr(counts), _ptr(objective),
+                                  ctypes.byref(n_iter), _ptr(ws), ws.numel(), _stream(stream)))
     return n_iter.value
 
 
@@ -381,12 +427,14 @@ def fkm_version() -> str:
 
 
 # ---------------------------------------------------------------- wrapper
-def batch_kmeans_Euclid(x: torch.Tensor, n_clusters: int, max_iters: int = 100, tol: float = 0.0,
-                        init_centroids: torch.Tensor | None = None, seed: int = 0):
-    """Exact batched Lloyd k-means.  x: [B, N, D] (or [N, D]) CUDA tensor in
-    float32 / float16 / bfloat16.  Returns (cluster_ids int32 [B, N], centers
-    float32 [B, K, D], n_iter).  Default initial centroids: per batch, the
-    points at the first K positions of a seeded random permutation."""
+def batch_kmeans(x: torch.Tensor, n_clusters: int, max_iters: int = 100, tol: float = 0.0,
+                 init_centroids: torch.Tensor | None = None, seed: int = 0,
+                 metric: str = "euclid"):
+    """Exact batched Lloyd k-means under metric 'euclid', 'dot' or 'cosine'
+    (fkm.h, fkm_metric).  x: [B, N, D] (or [N, D]) CUDA tensor in float32 /
+    float16 / bfloat16.  Returns (cluster_ids int32 [B, N], centers float32
+    [B, K, D], n_iter).  Default initial centroids: per batch, the points at
+    the first K positions of a seeded random permutation."""
     squeeze = x.dim() == 2
     if squeeze:
         x = x.unsqueeze(0)
@@ -403,10 +451,20 @@ def batch_kmeans_Euclid(x: torch.Tensor, n_clusters: int, max_iters: int = 100, 
     ids = torch.empty(B, N, dtype=torch.int32, device=dev)
     centers = torch.empty(B, K, D, dtype=torch.float32, device=dev)
     counts = torch.empty(B, K, dtype=torch.int32, device=dev)
-    n_iter = fkm_lloyd(x, init, max_iters, tol, ids, centers, counts)
+    if _metric(metric) == METRICS["euclid"]:
+        n_iter = fkm_lloyd(x, init, max_iters, tol, ids, centers, counts)
+    else:
+        n_iter = fkm_lloyd_metric(x, init, max_iters, tol, ids, centers, counts, metric)
     if squeeze:
         return ids[0], centers[0], n_iter
     return ids, centers, n_iter
+
+
+def batch_kmeans_Euclid(x: torch.Tensor, n_clusters: int, max_iters: int = 100, tol: float = 0.0,
+                        init_centroids: torch.Tensor | None = None, seed: int = 0):
+    """Exact batched Lloyd k-means (Euclidean), the README's call shape; see
+    batch_kmeans."""
+    return batch_kmeans(x, n_clusters, max_iters, tol, init_centroids, seed, "euclid")
 
 
 # ---------------------------------------------------------------- class API

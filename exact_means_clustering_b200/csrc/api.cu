@@ -181,6 +181,9 @@ fkm_status make_layout(int B, int N, int K, int D, int dtype, Layout* L) {
   l.shiftk = take(BK * 8);
   l.cbuf = take(2 * BK * D * 4);
   l.scal = take((size_t)B * 8 * 2 + 64);
+  l.cnorm = take(BK * 8);
+  l.objk = take(BK * 8);
+  l.metric = FKM_METRIC_EUCLID;
   l.total = off;
   *L = l;
   return FKM_OK;
@@ -286,17 +289,29 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
     FKM_TRY(launch_seg_bounds(s.keys_out, L.n_sort, BK, segstart, segend, st));
   }
   if (ev) FKM_TRY(record_stage(ev[2], st));
-  if (obj) FKM_CUDA_TRY(cudaMemsetAsync(obj, 0, sizeof(double) * L.B, st));
+  const bool euclid = L.metric == FKM_METRIC_EUCLID;
+  if (obj && euclid) FKM_CUDA_TRY(cudaMemsetAsync(obj, 0, sizeof(double) * L.B, st));
   const int range = segsum_range_rows(L.n_sort);
+  // the Euclidean objective is summed with the rows; the similarity ones come
+  // from the cluster sums in the finalize step
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK,
-                        w.at<double>(L.sums64), next, false, obj_args(w, prev, obj), st, range));
+                        w.at<double>(L.sums64), next, false,
+                        obj_args(w, prev, euclid ? obj : nullptr), st, range));
   if (ev) FKM_TRY(record_stage(ev[3], st));
-  FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64), prev,
-                          next, counts, w.at<double>(L.shiftk), st, range));
+  if (euclid) {
+    FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64),
+                            prev, next, counts, w.at<double>(L.shiftk), st, range));
+  } else {
+    FKM_TRY(launch_finalize_sim(L.B, L.K, L.D, L.metric, segstart, segend,
+                                w.at<double>(L.sums64), prev, next, counts,
+                                w.at<double>(L.shiftk), w.at<double>(L.objk), st, range));
+    if (obj) FKM_TRY(launch_batch_reduce(L.B, L.K, w.at<double>(L.objk), obj, nullptr, st));
+  }
   // the next assign's operands: offsets of the new centroids from their mean
   if (requant)
     FKM_TRY(launch_prep_centroids(next, L.B, L.K, L.Kp, L.D, L.dtype, w.at<float>(L.mvec),
-                                  w.at<void>(L.cq), w.at<void>(L.caug), st));
+                                  w.at<void>(L.cq), w.at<void>(L.caug), st, L.metric,
+                                  w.at<double>(L.cnorm)));
   return FKM_OK;
 }
 
@@ -320,7 +335,7 @@ static fkm_status read_status(const Ws& w, cudaStream_t st) {
 
 // ---- CUDA graph of a tol = 0 Lloyd loop, cached for identical calls ----
 struct GraphKey {
-  int B, N, K, D, dtype, iters;
+  int B, N, K, D, dtype, metric, iters;
   const void* x;
   const float* init;
   int32_t* ids;
@@ -408,10 +423,21 @@ fkm_status fkm_workspace_size(int B, int N, int K, int D, int dtype, size_t* byt
   return FKM_OK;
 }
 
-fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, const float* centers,
-                      int32_t* ids, double* inertia, void* ws, size_t ws_bytes, void* stream) {
+static fkm_status check_metric(int metric) {
+  if (metric != FKM_METRIC_EUCLID && metric != FKM_METRIC_DOT && metric != FKM_METRIC_COSINE) {
+    set_error("metric %d is not one of FKM_METRIC_EUCLID, _DOT, _COSINE", metric);
+    return FKM_ERR_INVALID_ARG;
+  }
+  return FKM_OK;
+}
+
+static fkm_status assign_impl(int metric, int B, int N, int K, int D, int dtype, const void* x,
+                              const float* centers, int32_t* ids, double* inertia, void* ws,
+                              size_t ws_bytes, void* stream) {
+  FKM_TRY(check_metric(metric));
   Layout L;
   FKM_TRY(make_layout(B, N, K, D, dtype, &L));
+  L.metric = metric;
   FKM_TRY(check_ws(L, ws, ws_bytes));
   FKM_TRY(check_ptr(x, "x"));
   FKM_TRY(check_ptr(centers, "centers"));
@@ -420,7 +446,8 @@ fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Ws w{ws, &L};
   FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
-                                w.at<void>(L.cq), w.at<void>(L.caug), st));
+                                w.at<void>(L.cq), w.at<void>(L.caug), st, metric,
+                                w.at<double>(L.cnorm)));
   if (L.split)
     FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, w.at<void>(L.xs), nullptr, st));
   FKM_TRY(step_assign(w, x, ids, st));
@@ -431,11 +458,14 @@ fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, cons
   return FKM_OK;
 }
 
-fkm_status fkm_update(int B, int N, int K, int D, int dtype, const void* x, const int32_t* ids,
-                      const float* prev_centers, float* centers, int32_t* counts, double* shift,
-                      double* inertia, void* ws, size_t ws_bytes, void* stream) {
+static fkm_status update_impl(int metric, int B, int N, int K, int D, int dtype, const void* x,
+                              const int32_t* ids, const float* prev_centers, float* centers,
+                              int32_t* counts, double* shift, double* inertia, void* ws,
+                              size_t ws_bytes, void* stream) {
+  FKM_TRY(check_metric(metric));
   Layout L;
   FKM_TRY(make_layout(B, N, K, D, dtype, &L));
+  L.metric = metric;
   FKM_TRY(check_ws(L, ws, ws_bytes));
   FKM_TRY(check_ptr(x, "x"));
   FKM_TRY(check_ptr(ids, "ids"));
@@ -451,7 +481,7 @@ fkm_status fkm_update(int B, int N, int K, int D, int dtype, const void* x, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Ws w{ws, &L};
   FKM_CUDA_TRY(cudaMemsetAsync(w.at<double>(L.sums64), 0, (size_t)B * K * D * 8, st));
-  if (inertia && !L.split)  // the objective measures against q(prev), the assign operand
+  if (inertia && !L.split && metric == FKM_METRIC_EUCLID)  // against q(prev), the assign operand
     FKM_TRY(launch_prep_centroids(prev_centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),
                                   w.at<void>(L.cq), w.at<void>(L.caug), st));
   FKM_TRY(step_update(w, x, ids, prev_centers, centers, counts, false, inertia, st));
@@ -459,12 +489,14 @@ fkm_status fkm_update(int B, int N, int K, int D, int dtype, const void* x, cons
   return FKM_OK;
 }
 
-fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
-                     const float* init_centers, int max_iters, float tol, int32_t* ids,
-                     float* centers, int32_t* counts, double* inertia, int* n_iter, void* ws,
-                     size_t ws_bytes, void* stream) {
+static fkm_status lloyd_impl(int metric, int B, int N, int K, int D, int dtype, const void* x,
+                             const float* init_centers, int max_iters, float tol, int32_t* ids,
+                             float* centers, int32_t* counts, double* inertia, int* n_iter,
+                             void* ws, size_t ws_bytes, void* stream) {
+  FKM_TRY(check_metric(metric));
   Layout L;
   FKM_TRY(make_layout(B, N, K, D, dtype, &L));
+  L.metric = metric;
   FKM_TRY(check_ws(L, ws, ws_bytes));
   FKM_TRY(check_ptr(x, "x"));
   FKM_TRY(check_ptr(init_centers, "init_centers"));
@@ -490,7 +522,7 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
   FKM_CUDA_TRY(cudaMemcpyAsync(cA, init_centers, cbytes, cudaMemcpyDeviceToDevice, st));
   if (L.split) FKM_TRY(launch_points_prep(x, L.n_sort, D, dtype, w.at<void>(L.xs), nullptr, st));
   FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, w.at<float>(L.mvec), w.at<void>(L.cq),
-                                w.at<void>(L.caug), st));
+                                w.at<void>(L.caug), st, metric, w.at<double>(L.cnorm)));
 
   // kernel attributes are set here, before any stream capture
   FKM_TRY(assign_prepare());
@@ -510,7 +542,8 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
     cudaGetDevice(&dev);
     GraphKey key;
     memset(&key, 0, sizeof(key));
-    key.B = B; key.N = N; key.K = K; key.D = D; key.dtype = dtype; key.iters = max_iters;
+    key.B = B; key.N = N; key.K = K; key.D = D; key.dtype = dtype; key.metric = metric;
+    key.iters = max_iters;
     key.x = x; key.init = init_centers; key.ids = ids; key.centers = centers;
     key.counts = counts; key.inertia = inertia; key.ws = ws; key.st = st; key.dev = dev;
     key.prof_gen = prof ? g_prof.gen : -1;
@@ -576,6 +609,49 @@ fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
   fkm_status rs = read_status(w, st);
   if (prof) prof_collect(done);
   return rs;
+}
+
+fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, const float* centers,
+                      int32_t* ids, double* inertia, void* ws, size_t ws_bytes, void* stream) {
+  return assign_impl(FKM_METRIC_EUCLID, B, N, K, D, dtype, x, centers, ids, inertia, ws, ws_bytes,
+                     stream);
+}
+
+fkm_status fkm_update(int B, int N, int K, int D, int dtype, const void* x, const int32_t* ids,
+                      const float* prev_centers, float* centers, int32_t* counts, double* shift,
+                      double* inertia, void* ws, size_t ws_bytes, void* stream) {
+  return update_impl(FKM_METRIC_EUCLID, B, N, K, D, dtype, x, ids, prev_centers, centers, counts,
+                     shift, inertia, ws, ws_bytes, stream);
+}
+
+fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* x,
+                     const float* init_centers, int max_iters, float tol, int32_t* ids,
+                     float* centers, int32_t* counts, double* inertia, int* n_iter, void* ws,
+                     size_t ws_bytes, void* stream) {
+  return lloyd_impl(FKM_METRIC_EUCLID, B, N, K, D, dtype, x, init_centers, max_iters, tol, ids,
+                    centers, counts, inertia, n_iter, ws, ws_bytes, stream);
+}
+
+fkm_status fkm_assign_metric(int B, int N, int K, int D, int dtype, int metric, const void* x,
+                             const float* centers, int32_t* ids, void* ws, size_t ws_bytes,
+                             void* stream) {
+  return assign_impl(metric, B, N, K, D, dtype, x, centers, ids, nullptr, ws, ws_bytes, stream);
+}
+
+fkm_status fkm_update_metric(int B, int N, int K, int D, int dtype, int metric, const void* x,
+                             const int32_t* ids, const float* prev_centers, float* centers,
+                             int32_t* counts, double* shift, double* objective, void* ws,
+                             size_t ws_bytes, void* stream) {
+  return update_impl(metric, B, N, K, D, dtype, x, ids, prev_centers, centers, counts, shift,
+                     objective, ws, ws_bytes, stream);
+}
+
+fkm_status fkm_lloyd_metric(int B, int N, int K, int D, int dtype, int metric, const void* x,
+                            const float* init_centers, int max_iters, float tol, int32_t* ids,
+                            float* centers, int32_t* counts, double* objective, int* n_iter,
+                            void* ws, size_t ws_bytes, void* stream) {
+  return lloyd_impl(metric, B, N, K, D, dtype, x, init_centers, max_iters, tol, ids, centers,
+                    counts, objective, n_iter, ws, ws_bytes, stream);
 }
 
 fkm_status fkm_profile(int enable) {

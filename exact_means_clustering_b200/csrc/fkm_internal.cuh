@@ -75,7 +75,8 @@ struct Layout {
   int key_bits;
   bool count_sort;  // one-pass counting sort (K <= CS_MAX_K) instead of LSD radix
   size_t status, mvec, cq, caug, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
-      segstart, segend, sums64, shiftk, cbuf, scal, total;
+      segstart, segend, sums64, shiftk, cbuf, scal, cnorm, objk, total;
+  int metric;  // FKM_METRIC_*; set by the caller after make_layout (default Euclidean)
 };
 
 fkm_status make_layout(int B, int N, int K, int D, int dtype, Layout* L);
@@ -109,8 +110,11 @@ fkm_status assign_prepare();
 // centroid the bias slab [B][Kp][16]: -n/2 as three 16-bit parts, n =
 // ||q(c-m)||^2 + 2 m.q(c-m) (zero on padding rows).
 constexpr int AUG_SLAB = 16;
+// metric: FKM_METRIC_EUCLID (bias slab -n/2), FKM_METRIC_DOT (zero bias) or
+// FKM_METRIC_COSINE (rows scaled to unit length first, norms into cnorm [B*K]).
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
-                                 float* m, void* cq, void* caug, cudaStream_t st);
+                                 float* m, void* cq, void* caug, cudaStream_t st,
+                                 int metric = FKM_METRIC_EUCLID, double* cnorm = nullptr);
 // fp32 points: split rows into xs; xn (optional) = ||x - m[row / N]||^2
 // (||x||^2 when m is null).
 fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,
@@ -182,6 +186,12 @@ fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const i
                            int range = SEG_RANGE, bool clear_sums = true);
 fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
                                double* max_shift, cudaStream_t st);
+// dot-product / cosine k-means: new centroids, per-cluster shift and
+// objective share (objk [B*K]) from the segment sums; sums64 left zeroed.
+fkm_status launch_finalize_sim(int B, int K, int D, int metric, const int32_t* segstart,
+                               const int32_t* segend, double* sums64, const float* prev,
+                               float* centers, int32_t* counts, double* shiftk, double* objk,
+                               cudaStream_t st, int range);
 
 fkm_status launch_baseline_argmin(const float* dist, int64_t rows, int K, int32_t* ids,
                                   cudaStream_t st);

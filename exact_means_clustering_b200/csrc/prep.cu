@@ -17,6 +17,12 @@
 //    norms).  Padding rows k >= K are zero (their columns are masked).  For
 //    fp32 points delta is split into bf16 hi and lo = bf16(delta - hi), rows
 //    [hi | lo], and the norm term uses the fp32 delta.
+//  dot-product and cosine k-means (the README lists both beside the
+//    Euclidean one): the score is x.c_hat, and x.m is the same for every
+//    centroid of a point, so the argmax of x.q(delta) alone picks the most
+//    similar centroid -- the bias slab is zero.  For cosine the rows are
+//    first scaled to unit length, u = fp32(c / ||c||) with the norm in fp64,
+//    and m, delta and q() are formed from u.
 //  points_prep: for fp32 points, the bf16 [hi | lo] split rows the tensor
 //    cores consume (each half padded to a multiple of 8 elements); optionally
 //    ||x - m||^2 per point (fp64 sum rounded to fp32), which only the
@@ -35,19 +41,44 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
+// A centroid element as the assignment sees it: c itself, or for cosine
+// k-means c / ||c|| rounded to fp32 (a zero row stays zero).
+__device__ __forceinline__ float metric_elem(float c, const double* cn, int64_t row) {
+  if (!cn) return c;
+  const double n = cn[row];
+  return n > 0.0 ? (float)((double)c / n) : 0.0f;
+}
+
+// ||c|| of every centroid row (fp64 sum of squares); one warp per row.
+__global__ void row_norms_kernel(const float* __restrict__ c, int64_t rows, int D,
+                                 double* __restrict__ cn) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  double s = 0.0;
+  for (int d = lane; d < D; d += 32) {
+    const double v = (double)c[row * D + d];
+    s += v * v;
+  }
+  s = warp_sum(s);
+  if (lane == 0) cn[row] = sqrt(s);
+}
+
 // m[b][d] = fp32(S / K) with S summed in fp64 in a fixed order that does not
 // depend on the launch: 32 partial sums P_w = sum over k = w, w+32, w+64, ...
 // (each in ascending k), then S = P_0 + P_1 + ... + P_31 in that order.
 // Block (b, 32-dimension group) of 32 warps: warp w forms P_w for the 32
 // dimensions of its lanes (coalesced rows), warp 0 adds the partials.
 __global__ void __launch_bounds__(1024) center_kernel(const float* __restrict__ c, int B, int K,
-                                                      int D, float* __restrict__ m) {
+                                                      int D, float* __restrict__ m,
+                                                      const double* __restrict__ cn) {
   __shared__ double part[32][33];
   const int b = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int d = blockIdx.y * 32 + lane;
   double s = 0.0;
   if (d < D) {
     const float* p = c + (int64_t)b * K * D + d;
+    const int64_t row0 = (int64_t)b * K;
     int k = w;
     // sixteen rows' loads in flight at once, added in the same ascending order
     for (; k + 15 * 32 < K; k += 16 * 32) {
@@ -55,9 +86,9 @@ __global__ void __launch_bounds__(1024) center_kernel(const float* __restrict__ 
 #pragma unroll
       for (int j = 0; j < 16; ++j) v[j] = p[(int64_t)(k + 32 * j) * D];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) s += (double)v[j];
+      for (int j = 0; j < 16; ++j) s += (double)metric_elem(v[j], cn, row0 + k + 32 * j);
     }
-    for (; k < K; k += 32) s += (double)p[(int64_t)k * D];
+    for (; k < K; k += 32) s += (double)metric_elem(p[(int64_t)k * D], cn, row0 + k);
   }
   part[w][lane] = s;
   __syncthreads();
@@ -116,7 +147,8 @@ __device__ __forceinline__ uint16_t q16(float v, bool bf, float* back) {
 // the rows of x are 16-byte multiples).
 __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* __restrict__ m,
                                       int B, int K, int Kp, int D, int dtype,
-                                      void* __restrict__ cq, uint16_t* __restrict__ caug) {
+                                      void* __restrict__ cq, uint16_t* __restrict__ caug,
+                                      const double* __restrict__ cn, bool bias) {
   const int lane = threadIdx.x & 31, l8 = lane & 7;
   const int64_t row =
       ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
@@ -131,7 +163,12 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
     uint16_t* out = static_cast<uint16_t*>(cq) + row * (int64_t)(2 * Dp);
     for (int d = 4 * l8; valid && d < D; d += 32) {
       const float4 mm = *reinterpret_cast<const float4*>(mb + d);
-      const float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
+      float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
+      if (real && cn) {
+        const int64_t r = (int64_t)b * K + k;
+        cv = make_float4(metric_elem(cv.x, cn, r), metric_elem(cv.y, cn, r),
+                         metric_elem(cv.z, cn, r), metric_elem(cv.w, cn, r));
+      }
       const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
       const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
       uint16_t hb[4], lb[4];
@@ -152,7 +189,12 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
     uint16_t* out = static_cast<uint16_t*>(cq) + row * (int64_t)D;
     for (int d = 4 * l8; valid && d < D; d += 32) {
       const float4 mm = *reinterpret_cast<const float4*>(mb + d);
-      const float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
+      float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
+      if (real && cn) {
+        const int64_t r = (int64_t)b * K + k;
+        cv = make_float4(metric_elem(cv.x, cn, r), metric_elem(cv.y, cn, r),
+                         metric_elem(cv.z, cn, r), metric_elem(cv.w, cn, r));
+      }
       const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
       const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
       uint16_t qb[4];
@@ -173,7 +215,7 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
   // the bias slab: [-n/2 in three parts, 0 x 13]; padding rows are all zero
   // (the assign kernel masks their columns); lane l8 writes entries 2 l8, 2 l8 + 1
   uint16_t parts[3] = {0, 0, 0};
-  if (real) bias_parts(-0.5 * acc, dtype == FKM_F16, parts);
+  if (real && bias) bias_parts(-0.5 * acc, dtype == FKM_F16, parts);
   if (valid) {
     const int e = 2 * l8;
     const uint32_t lo = e == 0 ? parts[0] : e == 2 ? parts[2] : 0u;
@@ -238,13 +280,22 @@ __global__ void points_prep_kernel(const void* __restrict__ x, int64_t rows, int
 }  // namespace
 
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
-                                 float* m, void* cq, void* caug, cudaStream_t st) {
+                                 float* m, void* cq, void* caug, cudaStream_t st, int metric,
+                                 double* cnorm) {
+  const double* cn = nullptr;
+  if (metric == FKM_METRIC_COSINE) {
+    const int64_t rows = (int64_t)B * K;
+    row_norms_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(centers, rows, D, cnorm);
+    note_launch();
+    cn = cnorm;
+  }
   center_kernel<<<dim3((unsigned)B, (unsigned)ceil_div(D, 32)), 1024, 0, st>>>(centers, B, K, D,
-                                                                              m);
+                                                                              m, cn);
   const int64_t rows = (int64_t)B * Kp;
   const int wpb = 8;   // 4 rows per warp
   prep_centroids_kernel<<<(unsigned)ceil_div(rows, 4 * wpb), wpb * 32, 0, st>>>(
-      centers, m, B, K, Kp, D, dtype, cq, static_cast<uint16_t*>(caug));
+      centers, m, B, K, Kp, D, dtype, cq, static_cast<uint16_t*>(caug), cn,
+      metric == FKM_METRIC_EUCLID);
   note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;

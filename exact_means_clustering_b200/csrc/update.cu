@@ -547,6 +547,89 @@ __global__ void finalize_kernel(FinParams p) {
   if (lane == 0) p.shiftk[key] = sh;
 }
 
+// Finalize for dot-product and cosine k-means (one warp per cluster).  The
+// new centroid is the mean of the cluster's points (dot), or its direction
+// scaled to unit length (cosine: the mean's direction is the sum's); an empty
+// cluster, or a cosine cluster whose sum is zero, keeps prev.  objk[key] is
+// the cluster's share of the objective of the assignment just summed,
+// s_k . c~ with c~ = prev (dot) or prev / ||prev|| (cosine), s_k the sum of
+// its points: the fp64 sums of a crossing run, or n times the mean the
+// segment sums wrote for an interior one.
+struct FinSimParams {
+  int B, K, D, metric, range;
+  const int32_t* segstart;
+  const int32_t* segend;
+  double* sums64;
+  const float* prev;
+  float* centers;
+  int32_t* counts;
+  double* shiftk;
+  double* objk;
+  bool clear_sums;
+};
+
+__global__ void finalize_sim_kernel(FinSimParams p) {
+  const int64_t key = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (key >= (int64_t)p.B * p.K) return;
+  const int32_t s0 = p.segstart[key], t0 = p.segend[key];
+  const int32_t nk = t0 - s0;
+  const bool interior = nk > 0 && (s0 / p.range) == ((t0 - 1) / p.range);
+  const bool cosine = p.metric == FKM_METRIC_COSINE;
+  const double n = (double)nk;
+  // pass 1: ||mean||^2, ||prev||^2 and sum . prev
+  double vv = 0.0, pp = 0.0, sp = 0.0;
+  for (int d = lane; d < p.D; d += 32) {
+    const int64_t e = key * p.D + d;
+    const double pv = (double)p.prev[e];
+    pp += pv * pv;
+    if (nk > 0) {
+      double sd;
+      float v;
+      if (interior) {
+        v = p.centers[e];
+        sd = (double)v * n;
+      } else {
+        sd = p.sums64[e];
+        v = (float)(sd / n);
+      }
+      vv += (double)v * (double)v;
+      sp += sd * pv;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    vv += __shfl_xor_sync(0xffffffffu, vv, o);
+    pp += __shfl_xor_sync(0xffffffffu, pp, o);
+    sp += __shfl_xor_sync(0xffffffffu, sp, o);
+  }
+  const double pn = sqrt(pp), vn = sqrt(vv);
+  const double obj = cosine ? (pn > 0.0 ? sp / pn : 0.0) : sp;
+  const bool keep = nk == 0 || (cosine && !(vv > 0.0));
+  // pass 2: the new centroid and its shift
+  double sh = 0.0;
+  for (int d = lane; d < p.D; d += 32) {
+    const int64_t e = key * p.D + d;
+    const float pv = p.prev[e];
+    float out = pv;
+    if (!keep) {
+      const float v = interior ? p.centers[e] : (float)(p.sums64[e] / n);
+      out = cosine ? (float)((double)v / vn) : v;
+    }
+    if (nk > 0 && !interior && p.clear_sums) p.sums64[e] = 0.0;
+    p.centers[e] = out;
+    const double df = (double)out - (double)pv;
+    sh += df * df;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sh += __shfl_xor_sync(0xffffffffu, sh, o);
+  if (lane == 0) {
+    p.shiftk[key] = sh;
+    p.objk[key] = obj;
+    if (p.counts) p.counts[key] = nk;
+  }
+}
+
 // one block per batch; fixed-order tree sum
 __global__ void __launch_bounds__(256) batch_reduce_kernel(int K, const double* __restrict__ shiftk,
                                                            double* shift_out, double* max_shift) {
@@ -711,6 +794,32 @@ fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const i
   const int64_t keys = (int64_t)B * K;
   const int wpb = 8;
   finalize_kernel<<<(unsigned)ceil_div(keys, wpb), wpb * 32, 0, st>>>(fp);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+fkm_status launch_finalize_sim(int B, int K, int D, int metric, const int32_t* segstart,
+                               const int32_t* segend, double* sums64, const float* prev,
+                               float* centers, int32_t* counts, double* shiftk, double* objk,
+                               cudaStream_t st, int range) {
+  FinSimParams fp;
+  fp.B = B;
+  fp.K = K;
+  fp.D = D;
+  fp.metric = metric;
+  fp.range = range;
+  fp.segstart = segstart;
+  fp.segend = segend;
+  fp.sums64 = sums64;
+  fp.prev = prev;
+  fp.centers = centers;
+  fp.counts = counts;
+  fp.shiftk = shiftk;
+  fp.objk = objk;
+  fp.clear_sums = true;
+  const int64_t keys = (int64_t)B * K;
+  finalize_sim_kernel<<<(unsigned)ceil_div(keys, 8), 256, 0, st>>>(fp);
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;

@@ -66,6 +66,21 @@ typedef enum {
 /* storage type of the points */
 typedef enum { FKM_F32 = 0, FKM_F16 = 1, FKM_BF16 = 2 } fkm_dtype;
 
+/* The similarity a run clusters by (fkm_assign_metric, fkm_update_metric,
+ * fkm_lloyd_metric; the calls without the suffix are Euclidean).  The README
+ * lists cosine and dot-product k-means beside the Euclidean one ("Flash-KMeans"
+ * GitHub README, section "Usage", the CuTe backend note) without defining
+ * them; the plain readings are taken:
+ *   FKM_METRIC_EUCLID   nearest centroid, c_k = mean of its points
+ *   FKM_METRIC_DOT      a_i = argmax_k x_i . c_k, c_k = mean of its points,
+ *                       objective sum_i x_i . c_{a_i}
+ *   FKM_METRIC_COSINE   a_i = argmax_k x_i . c_k / ||c_k||, c_k = s_k / ||s_k||
+ *                       (unit direction of its points' sum s_k; spherical
+ *                       k-means), objective sum_i x_i . c_{a_i} / ||c_{a_i}||
+ * Ties go to the lowest index; an empty cluster, or one whose sum is zero,
+ * keeps its previous centroid. */
+typedef enum { FKM_METRIC_EUCLID = 0, FKM_METRIC_DOT = 1, FKM_METRIC_COSINE = 2 } fkm_metric;
+
 /* Bytes of device workspace fkm_assign / fkm_update / fkm_lloyd need for this
  * shape (one size serves all three).  Host-only: makes no CUDA call.
  * Returns FKM_ERR_INVALID_ARG / FKM_ERR_UNSUPPORTED for shapes the library
@@ -134,6 +149,36 @@ FKM_API fkm_status fkm_lloyd(int B, int N, int K, int D, int dtype, const void* 
                      const float* init_centers, int max_iters, float tol, int32_t* ids,
                      float* centers, int32_t* counts, double* inertia, int* n_iter, void* ws,
                      size_t ws_bytes, void* stream);
+
+/* Dot-product and cosine k-means (fkm_metric above), with the same shapes,
+ * layouts, workspace (fkm_workspace_size), validation and stream behaviour
+ * as fkm_assign / fkm_update / fkm_lloyd; metric FKM_METRIC_EUCLID gives
+ * exactly those calls (without fkm_assign's optional objective).
+ *   assign   ids = argmax_k x . c_hat_k over the tensor-core operands
+ *            c_hat = m + q(v - m), v = c (dot) or fp32(c / ||c||) (cosine),
+ *            m the mean of the v rows; x . m is the same for every k, so the
+ *            bias product is zero and the epilogue compares x . q(v - m).
+ *   update   centers = the mean of each cluster's points (dot), or its unit
+ *            direction (cosine); empty or zero-sum clusters keep prev.
+ *            objective [B] (may be NULL) = sum_i x_i . c~_{ids_i}, c~ = prev or
+ *            prev / ||prev||: the objective of the assignment, formed from the
+ *            cluster sums.  shift as in fkm_update.
+ *   lloyd    the loop of the two; objective [B] is that of the last
+ *            assignment, against the centroids it used; tol compares the
+ *            centroid shift as in fkm_lloyd.
+ * An unknown metric returns FKM_ERR_INVALID_ARG before any launch. */
+FKM_API fkm_status fkm_assign_metric(int B, int N, int K, int D, int dtype, int metric,
+                                     const void* x, const float* centers, int32_t* ids, void* ws,
+                                     size_t ws_bytes, void* stream);
+FKM_API fkm_status fkm_update_metric(int B, int N, int K, int D, int dtype, int metric,
+                                     const void* x, const int32_t* ids, const float* prev_centers,
+                                     float* centers, int32_t* counts, double* shift,
+                                     double* objective, void* ws, size_t ws_bytes, void* stream);
+FKM_API fkm_status fkm_lloyd_metric(int B, int N, int K, int D, int dtype, int metric,
+                                    const void* x, const float* init_centers, int max_iters,
+                                    float tol, int32_t* ids, float* centers, int32_t* counts,
+                                    double* objective, int* n_iter, void* ws, size_t ws_bytes,
+                                    void* stream);
 
 /* Device workspace for fkm_lloyd_host with chunks of `chunk_rows` points. */
 FKM_API fkm_status fkm_host_workspace_size(int B, int N, int K, int D, int dtype, int64_t chunk_rows,

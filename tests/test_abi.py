@@ -108,6 +108,17 @@ def test_shard_calls_validate_before_any_launch(fkm):
     assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a, a, None, a, 64, None) == 4
 
 
+def test_metric_calls_reject_unknown_metric(fkm):
+    L = fkm.lib()
+    ws = ctypes.create_string_buffer(1 << 20)
+    a = (ctypes.addressof(ws) + 15) & ~15
+    assert L.fkm_assign_metric(1, 16, 4, 64, 2, 3, a, a, a, a, 1 << 19, None) == 1
+    assert L.fkm_assign_metric(1, 16, 4, 64, 2, -1, a, a, a, a, 1 << 19, None) == 1
+    assert b"metric" in L.fkm_last_error()
+    # a known metric still validates its pointers first
+    assert L.fkm_assign_metric(1, 16, 4, 64, 2, 2, None, a, a, a, 1 << 19, None) == 1
+
+
 def test_status_strings_and_version(fkm):
     L = fkm.lib()
     assert L.fkm_status_string(0) == b"ok"
