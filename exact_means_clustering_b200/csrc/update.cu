@@ -577,6 +577,69 @@ __global__ void finalize_sim_kernel(FinSimParams p) {
   const bool interior = nk > 0 && (s0 / p.range) == ((t0 - 1) / p.range);
   const bool cosine = p.metric == FKM_METRIC_COSINE;
   const double n = (double)nk;
+  if (p.D <= 128 && (p.D & 3) == 0) {
+    // one 16-byte piece per lane holds the whole cluster: one pass of loads
+    const int d = 4 * lane;
+    const bool on = d < p.D;
+    const int64_t e = key * p.D + d;
+    float4 pv = make_float4(0.f, 0.f, 0.f, 0.f), v = pv;
+    double sd[4] = {0.0, 0.0, 0.0, 0.0};
+    if (on) {
+      pv = *reinterpret_cast<const float4*>(p.prev + e);
+      if (nk > 0 && interior) {
+        v = *reinterpret_cast<const float4*>(p.centers + e);
+        sd[0] = (double)v.x * n;
+        sd[1] = (double)v.y * n;
+        sd[2] = (double)v.z * n;
+        sd[3] = (double)v.w * n;
+      } else if (nk > 0) {
+        double2* s2 = reinterpret_cast<double2*>(p.sums64 + e);
+        const double2 a = s2[0], b = s2[1];
+        sd[0] = a.x;
+        sd[1] = a.y;
+        sd[2] = b.x;
+        sd[3] = b.y;
+        v = make_float4((float)(a.x / n), (float)(a.y / n), (float)(b.x / n), (float)(b.y / n));
+        if (p.clear_sums) {
+          s2[0] = make_double2(0.0, 0.0);
+          s2[1] = make_double2(0.0, 0.0);
+        }
+      }
+    }
+    const float vv4[4] = {v.x, v.y, v.z, v.w}, pv4[4] = {pv.x, pv.y, pv.z, pv.w};
+    double vv = 0.0, pp = 0.0, sp = 0.0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      vv += (double)vv4[j] * (double)vv4[j];
+      pp += (double)pv4[j] * (double)pv4[j];
+      sp += sd[j] * (double)pv4[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      vv += __shfl_xor_sync(0xffffffffu, vv, o);
+      pp += __shfl_xor_sync(0xffffffffu, pp, o);
+      sp += __shfl_xor_sync(0xffffffffu, sp, o);
+    }
+    const double pn = sqrt(pp), vn = sqrt(vv);
+    const bool keep = nk == 0 || (cosine && !(vv > 0.0));
+    float o4[4];
+    double sh = 0.0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      o4[j] = keep ? pv4[j] : cosine ? (float)((double)vv4[j] / vn) : vv4[j];
+      const double df = (double)o4[j] - (double)pv4[j];
+      sh += df * df;
+    }
+    if (on) *reinterpret_cast<float4*>(p.centers + e) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sh += __shfl_xor_sync(0xffffffffu, sh, o);
+    if (lane == 0) {
+      p.shiftk[key] = sh;
+      p.objk[key] = cosine ? (pn > 0.0 ? sp / pn : 0.0) : sp;
+      if (p.counts) p.counts[key] = nk;
+    }
+    return;
+  }
   // pass 1: ||mean||^2, ||prev||^2 and sum . prev
   double vv = 0.0, pp = 0.0, sp = 0.0;
   for (int d = lane; d < p.D; d += 32) {
