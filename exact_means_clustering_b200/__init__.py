@@ -347,6 +347,33 @@ def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None, chun
         ws = workspace(fkm_workspace_size(B, N, K, D, x.dtype), dev)
     c = init_centers.to(dev, torch.float32).contiguous().clone()
     ids = torch.empty(B, N, dtype=torch.int32, device=dev)
+
+    def partials(c, sums, counts, obj):
+        if on_host:
+            fkm_partial_update_host(x, c, chunk_rows, ids, sums, counts, obj, ws=ws)
+        else:
+            fkm_assign(x, c, ids, ws=ws)
+            fkm_partial_update(x, ids, c, sums, counts, obj, ws=ws)
+
+    def finalize(sums, counts, c, nxt, shift):
+        fkm_finalize_sums(sums, counts, c, nxt, shift, ws=ws)
+
+    c, counts, obj, n_iter = sharded_loop(partials, finalize, c, max_iters, tol, group)
+    fkm_sync_status(ws)
+    return ids, c, counts, obj, n_iter
+
+
+def sharded_loop(partials, finalize, c, max_iters, tol=0.0, group=None):
+    """The rank-side control of the data-parallel loop, independent of where
+    the shard lives: per iteration partials(c, sums, counts, obj) adds this
+    rank's shard into zeroed sums [B, K, D] float64, counts [B, K] int32 and
+    obj [B] float64; reduce_partials sums them over the group; finalize(sums,
+    counts, c, nxt, shift) forms the next centroids and the shift [B].  The
+    stop test (max shift < tol) reads reduced values only, so every rank takes
+    the same number of iterations and the same collectives.  Returns (centers,
+    counts and objective of all shards, n_iter)."""
+    B, K, D = c.shape
+    dev = c.device
     sums = torch.empty(B, K, D, dtype=torch.float64, device=dev)
     counts = torch.empty(B, K, dtype=torch.int32, device=dev)
     obj = torch.empty(B, dtype=torch.float64, device=dev)
@@ -356,20 +383,15 @@ def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None, chun
         sums.zero_()
         counts.zero_()
         obj.zero_()
-        if on_host:
-            fkm_partial_update_host(x, c, chunk_rows, ids, sums, counts, obj, ws=ws)
-        else:
-            fkm_assign(x, c, ids, ws=ws)
-            fkm_partial_update(x, ids, c, sums, counts, obj, ws=ws)
+        partials(c, sums, counts, obj)
         reduce_partials((sums, counts, obj), group)
         nxt = torch.empty_like(c)
-        fkm_finalize_sums(sums, counts, c, nxt, shift, ws=ws)
+        finalize(sums, counts, c, nxt, shift)
         c = nxt
         n_iter = t + 1
         if tol > 0.0 and shift.max().item() < tol:
             break
-    fkm_sync_status(ws)
-    return ids, c, counts, obj, n_iter
+    return c, counts, obj, n_iter
 
 
 def fkm_centre_workspace_size_bytes(B, N, D) -> int:

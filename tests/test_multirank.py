@@ -64,3 +64,79 @@ def test_two_gloo_ranks():
         assert reduced == (24 * 3.0, 6 * 3, [1.5, 2.0])   # partials summed over ranks
     assert out[0][3] != out[1][3]                 # own seeds ...
     assert out[0][4] != out[1][4]                 # ... and so own points
+
+
+# ---- the sharded loop's control over two ranks, with CPU stand-ins for the
+# shard step and the finalize (the GPU calls they replace are covered by
+# tests/test_gpu_sharded.py)
+def _cpu_steps(x):
+    def partials(c, sums, counts, obj):
+        for b in range(x.shape[0]):
+            d = torch.cdist(x[b], c[b].double()) ** 2
+            dmin, ids = d.min(1)
+            sums[b].index_add_(0, ids, x[b])
+            counts[b] += torch.bincount(ids, minlength=c.shape[1]).to(torch.int32)
+            obj[b] += dmin.sum()
+
+    def finalize(sums, counts, c, nxt, shift):
+        n = counts.unsqueeze(-1).double()
+        new = torch.where(n > 0, sums / n.clamp(min=1), c.double())
+        nxt.copy_(new.float())
+        shift.copy_(((nxt.double() - c.double()) ** 2).sum((1, 2)))
+
+    return partials, finalize
+
+
+def _problem(seed=5, B=2, N=600, K=7, D=4):
+    g = torch.Generator().manual_seed(seed)
+    means = torch.randn(B, K, D, generator=g, dtype=torch.float64) * 4
+    lab = torch.randint(0, K, (B, N), generator=g)
+    x = torch.gather(means, 1, lab.unsqueeze(-1).expand(B, N, D)) + \
+        torch.randn(B, N, D, generator=g, dtype=torch.float64)
+    return x, x[:, :K].float().contiguous()
+
+
+def _sharded_rank(rank, world, port, tol, q):
+    sys.path.insert(0, ROOT)
+    import exact_means_clustering_b200 as fkm
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        x, c0 = _problem()
+        n = x.shape[1] // world
+        shard = x[:, rank * n:(rank + 1) * n]
+        c, counts, obj, n_iter = fkm.sharded_loop(*_cpu_steps(shard), c0.clone(), 30, tol)
+        q.put((rank, c.numpy(), counts.numpy(), obj.numpy(), n_iter))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("tol", [0.0, 1e-6])
+def test_sharded_loop_two_gloo_ranks_match_one_rank(tol):
+    """Two ranks holding halves of every problem reach the same centroids,
+    counts and objective as one rank holding all of it, and stop after the
+    same number of iterations."""
+    sys.path.insert(0, ROOT)
+    import exact_means_clustering_b200 as fkm
+    x, c0 = _problem()
+    c1, k1, o1, n1 = fkm.sharded_loop(*_cpu_steps(x), c0.clone(), 30, tol)
+    if tol > 0:
+        assert n1 < 30                       # the stop test fired
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_rank, args=(r, world, port, tol, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, c, k, o, n in out:
+        assert n == n1
+        assert np.array_equal(k, k1.numpy())
+        assert np.allclose(c, c1.numpy(), rtol=1e-6, atol=1e-6)
+        assert np.allclose(o, o1.numpy(), rtol=1e-9)
+    assert np.array_equal(out[0][1], out[1][1])   # every rank forms the same centroids
