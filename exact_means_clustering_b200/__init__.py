@@ -95,11 +95,20 @@ def _check(fn, code):
         raise FkmError(fn, code, lib().fkm_last_error().decode(errors="replace"))
 
 
-def _ptr(t):
+def _ptr(t, dtype=None):
+    """Address of a tensor's data for the C calls, which read every array as
+    dense row-major memory of a fixed type: a strided view or a wrong dtype
+    would be misread, so both are refused here.  Raw integer addresses and
+    None (an optional argument left out) pass through."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_contiguous():
+        raise ValueError(f"a {tuple(t.shape)} tensor passed to the library is not contiguous "
+                         "(call .contiguous())")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"expected a {dtype} tensor, got {t.dtype}")
     return t.data_ptr()
 
 
@@ -150,8 +159,8 @@ def fkm_assign(x, centers, ids, inertia=None, ws=None, stream=None):
     B, N, D = x.shape
     K = centers.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_assign", lib().fkm_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers), _ptr(ids),
-                                          _ptr(inertia), _ptr(ws), ws.numel(), _stream(stream)))
+    _check("fkm_assign", lib().fkm_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers, torch.float32), _ptr(ids, torch.int32),
+                                          _ptr(inertia, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def fkm_update(x, ids, prev_centers, centers, counts, shift=None, inertia=None, ws=None,
@@ -159,9 +168,9 @@ def fkm_update(x, ids, prev_centers, centers, counts, shift=None, inertia=None, 
     B, N, D = x.shape
     K = prev_centers.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_update", lib().fkm_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids),
-                                          _ptr(prev_centers), _ptr(centers), _ptr(counts),
-                                          _ptr(shift), _ptr(inertia), _ptr(ws), ws.numel(),
+    _check("fkm_update", lib().fkm_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids, torch.int32),
+                                          _ptr(prev_centers, torch.float32), _ptr(centers, torch.float32), _ptr(counts, torch.int32),
+                                          _ptr(shift, torch.float64), _ptr(inertia, torch.float64), _ptr(ws), ws.numel(),
                                           _stream(stream)))
 
 
@@ -171,9 +180,9 @@ def fkm_lloyd(x, init_centers, max_iters, tol, ids, centers, counts, inertia=Non
     K = init_centers.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
     n_iter = ctypes.c_int(0)
-    _check("fkm_lloyd", lib().fkm_lloyd(B, N, K, D, _dt(x), _ptr(x), _ptr(init_centers), max_iters,
-                                        float(tol), _ptr(ids), _ptr(centers), _ptr(counts),
-                                        _ptr(inertia), ctypes.byref(n_iter), _ptr(ws), ws.numel(),
+    _check("fkm_lloyd", lib().fkm_lloyd(B, N, K, D, _dt(x), _ptr(x), _ptr(init_centers, torch.float32), max_iters,
+                                        float(tol), _ptr(ids, torch.int32), _ptr(centers, torch.float32), _ptr(counts, torch.int32),
+                                        _ptr(inertia, torch.float64), ctypes.byref(n_iter), _ptr(ws), ws.numel(),
                                         _stream(stream)))
     return n_iter.value
 
@@ -190,8 +199,8 @@ def fkm_assign_metric(x, centers, ids, metric, ws=None, stream=None):
     K = centers.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
     _check("fkm_assign_metric",
-           lib().fkm_assign_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(centers),
-                                   _ptr(ids), _ptr(ws), ws.numel(), _stream(stream)))
+           lib().fkm_assign_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(centers, torch.float32),
+                                   _ptr(ids, torch.int32), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def fkm_update_metric(x, ids, prev_centers, centers, counts, metric, shift=None, objective=None,
@@ -200,9 +209,9 @@ def fkm_update_metric(x, ids, prev_centers, centers, counts, metric, shift=None,
     K = prev_centers.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
     _check("fkm_update_metric",
-           lib().fkm_update_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(ids),
-                                   _ptr(prev_centers), _ptr(centers), _ptr(counts), _ptr(shift),
-                                   _ptr(objective), _ptr(ws), ws.numel(), _stream(stream)))
+           lib().fkm_update_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(ids, torch.int32),
+                                   _ptr(prev_centers, torch.float32), _ptr(centers, torch.float32), _ptr(counts, torch.int32), _ptr(shift, torch.float64),
+                                   _ptr(objective, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def fkm_lloyd_metric(x, init_centers, max_iters, tol, ids, centers, counts, metric,
@@ -213,8 +222,8 @@ def fkm_lloyd_metric(x, init_centers, max_iters, tol, ids, centers, counts, metr
     n_iter = ctypes.c_int(0)
     _check("fkm_lloyd_metric",
            lib().fkm_lloyd_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x),
-                                  _ptr(init_centers), max_iters, float(tol), _ptr(ids),
-                                  _ptr(centers), _ptr(counts), _ptr(objective),
+                                  _ptr(init_centers, torch.float32), max_iters, float(tol), _ptr(ids, torch.int32),
+                                  _ptr(centers, torch.float32), _ptr(counts, torch.int32), _ptr(objective, torch.float64),
                                   ctypes.byref(n_iter), _ptr(ws), ws.numel(), _stream(stream)))
     return n_iter.value
 
@@ -233,9 +242,9 @@ def fkm_lloyd_host(x_host, init_centers, max_iters, tol, chunk_rows, ids, center
         ws = workspace(fkm_host_workspace_size(B, N, K, D, dt, chunk_rows), init_centers.device)
     n_iter = ctypes.c_int(0)
     _check("fkm_lloyd_host",
-           lib().fkm_lloyd_host(B, N, K, D, dt, _ptr(x_host), _ptr(init_centers), max_iters,
-                                float(tol), int(chunk_rows), _ptr(ids), _ptr(centers),
-                                _ptr(counts), _ptr(inertia), ctypes.byref(n_iter), _ptr(ws),
+           lib().fkm_lloyd_host(B, N, K, D, dt, _ptr(x_host), _ptr(init_centers, torch.float32), max_iters,
+                                float(tol), int(chunk_rows), _ptr(ids, torch.int32), _ptr(centers, torch.float32),
+                                _ptr(counts, torch.int32), _ptr(inertia, torch.float64), ctypes.byref(n_iter), _ptr(ws),
                                 ws.numel(), _stream(stream)))
     return n_iter.value
 
@@ -243,7 +252,7 @@ def fkm_lloyd_host(x_host, init_centers, max_iters, tol, chunk_rows, ids, center
 def fkm_argsort(keys, n_keys, idx, sorted_keys=None, ws=None, stream=None):
     n = keys.numel()
     ws = ws if ws is not None else workspace(fkm_argsort_workspace_size(n, n_keys), keys.device)
-    _check("fkm_argsort", lib().fkm_argsort(_ptr(keys), n, n_keys, _ptr(idx), _ptr(sorted_keys),
+    _check("fkm_argsort", lib().fkm_argsort(_ptr(keys, torch.int32), n, n_keys, _ptr(idx, torch.int32), _ptr(sorted_keys, torch.int32),
                                             _ptr(ws), ws.numel(), _stream(stream)))
 
 
@@ -252,8 +261,8 @@ def fkm_baseline_assign(x, centers, dist, ids, ws=None, stream=None):
     K = centers.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
     _check("fkm_baseline_assign",
-           lib().fkm_baseline_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers), _ptr(dist),
-                                     _ptr(ids), _ptr(ws), ws.numel(), _stream(stream)))
+           lib().fkm_baseline_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers, torch.float32), _ptr(dist),
+                                     _ptr(ids, torch.int32), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def fkm_baseline_update(x, ids, prev_centers, centers, counts, ws=None, stream=None):
@@ -261,8 +270,8 @@ def fkm_baseline_update(x, ids, prev_centers, centers, counts, ws=None, stream=N
     K = prev_centers.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
     _check("fkm_baseline_update",
-           lib().fkm_baseline_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids), _ptr(prev_centers),
-                                     _ptr(centers), _ptr(counts), _ptr(ws), ws.numel(),
+           lib().fkm_baseline_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids, torch.int32), _ptr(prev_centers, torch.float32),
+                                     _ptr(centers, torch.float32), _ptr(counts, torch.int32), _ptr(ws), ws.numel(),
                                      _stream(stream)))
 
 
@@ -273,7 +282,7 @@ def fkm_assign_noalloc(x, centers, ids, stream=None):
     B, N, D = x.shape
     K = centers.shape[1]
     _check("fkm_assign_noalloc", lib().fkm_assign_noalloc(B, N, K, D, _dt(x), _ptr(x),
-                                                          _ptr(centers), _ptr(ids),
+                                                          _ptr(centers, torch.float32), _ptr(ids, torch.int32),
                                                           _stream(stream)))
 
 
@@ -284,8 +293,8 @@ def fkm_partial_update(x, ids, prev, sums, counts, obj=None, ws=None, stream=Non
     K = prev.shape[1]
     ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
     _check("fkm_partial_update",
-           lib().fkm_partial_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids), _ptr(prev), _ptr(sums),
-                                    _ptr(counts), _ptr(obj), _ptr(ws), ws.numel(), _stream(stream)))
+           lib().fkm_partial_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids, torch.int32), _ptr(prev, torch.float32), _ptr(sums, torch.float64),
+                                    _ptr(counts, torch.int32), _ptr(obj, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=None, ws=None,
@@ -298,9 +307,9 @@ def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=
         ws = workspace(fkm_host_workspace_size(B, N, K, D, _dt(x_host), chunk_rows),
                        centers.device)
     _check("fkm_partial_update_host",
-           lib().fkm_partial_update_host(B, N, K, D, _dt(x_host), _ptr(x_host), _ptr(centers),
-                                         int(chunk_rows), _ptr(ids), _ptr(sums), _ptr(counts),
-                                         _ptr(obj), _ptr(ws), ws.numel(), _stream(stream)))
+           lib().fkm_partial_update_host(B, N, K, D, _dt(x_host), _ptr(x_host), _ptr(centers, torch.float32),
+                                         int(chunk_rows), _ptr(ids, torch.int32), _ptr(sums, torch.float64), _ptr(counts, torch.int32),
+                                         _ptr(obj, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def fkm_finalize_sums(sums, counts, prev, centers, shift=None, ws=None, stream=None):
@@ -308,8 +317,8 @@ def fkm_finalize_sums(sums, counts, prev, centers, shift=None, ws=None, stream=N
     B, K, D = prev.shape
     ws = ws if ws is not None else workspace(256 + 8 * B * K, prev.device)
     _check("fkm_finalize_sums",
-           lib().fkm_finalize_sums(B, K, D, _ptr(sums), _ptr(counts), _ptr(prev), _ptr(centers),
-                                   _ptr(shift), _ptr(ws), ws.numel(), _stream(stream)))
+           lib().fkm_finalize_sums(B, K, D, _ptr(sums, torch.float64), _ptr(counts, torch.int32), _ptr(prev, torch.float32), _ptr(centers, torch.float32),
+                                   _ptr(shift, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def reduce_partials(tensors, group=None):
@@ -408,7 +417,7 @@ def fkm_centre(x, mu=None, out=None, ws=None, stream=None):
     out = out if out is not None else torch.empty_like(x)
     if ws is None:
         ws = workspace(fkm_centre_workspace_size_bytes(B, N, D), x.device)
-    _check("fkm_centre", lib().fkm_centre(B, N, D, _dt(x), _ptr(x), _ptr(mu), _ptr(out), _ptr(ws),
+    _check("fkm_centre", lib().fkm_centre(B, N, D, _dt(x), _ptr(x), _ptr(mu, torch.float32), _ptr(out), _ptr(ws),
                                           ws.numel(), _stream(stream)))
     return out, mu
 

@@ -132,3 +132,22 @@ def test_argsort_workspace_size(fkm):
     assert 0 < a < b
     with pytest.raises(fkm.FkmError):
         fkm.fkm_argsort_workspace_size(-1, 4)
+
+
+def test_binding_refuses_strided_views_and_wrong_dtypes(fkm):
+    """The C calls read dense row-major arrays of fixed types, so the binding
+    refuses a strided view or a wrong dtype before any call."""
+    import torch
+    x = torch.zeros(2, 64, 16, dtype=torch.bfloat16)
+    c = torch.zeros(2, 4, 16)
+    ids = torch.zeros(2, 64, dtype=torch.int32)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="contiguous"):
+        fkm.fkm_assign(x[:, ::2], c, ids[:, ::2], ws=ws)
+    with pytest.raises(TypeError, match="float32"):
+        fkm.fkm_assign(x, c.double(), ids, ws=ws)
+    with pytest.raises(TypeError, match="int32"):
+        fkm.fkm_assign(x, c, ids.long(), ws=ws)
+    with pytest.raises(TypeError, match="float64"):
+        fkm.fkm_partial_update(x, ids, c, torch.zeros(2, 4, 16), torch.zeros(2, 4, dtype=torch.int32),
+                               ws=ws)
