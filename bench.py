@@ -541,6 +541,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = datagen.CONFIGS[args.config]
+    if args.metric != "euclid" and (w.host_resident or args.sharded or args.impl == "reference"):
+        print("bench.py: --metric dot/cosine runs on device-resident workloads with --impl fkm "
+              "only (the host-streamed and sharded runs are Euclidean)", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args, w)
     if w.host_resident:
