@@ -32,10 +32,8 @@
  *     update that followed it;
  *   - "mirror" mode: the assign step measures distances to
  *         c_hat = m + q(fp32(fp32(c) - m)),
- *     with m the batch's mean centroid (fp64 sum of the fp32 centroids in a
- *     fixed order: 32 partial sums over k = w, w+32, ... in ascending k, then
- *     the partials in order w = 0..31; divided by K, rounded to fp32) and q()
- *     round-to-nearest-
+ *     with m the batch's mean centroid (the fp64 sum of the fp32 centroids
+ *     in index order, divided by K, rounded to fp32) and q() round-to-nearest-
  *     even to the points' storage type (bf16 or fp16).  That is the precision
  *     contract "assignment operands are in the input dtype", applied to the
  *     centroids' offsets from their mean: k-means is translation invariant,
@@ -116,12 +114,9 @@ void orc_chat(const double* c, int64_t B, int64_t K, int64_t D, int mirror, doub
   }
   for (int64_t b = 0; b < B; ++b)
     for (int64_t d = 0; d < D; ++d) {
+      /* the plain mean: fp64 sum over k = 0 .. K-1 in index order */
       double s = 0.0;
-      for (int64_t w = 0; w < 32; ++w) {
-        double part = 0.0;
-        for (int64_t k = w; k < K; k += 32) part += (double)(float)c[(b * K + k) * D + d];
-        s += part;
-      }
+      for (int64_t k = 0; k < K; ++k) s += (double)(float)c[(b * K + k) * D + d];
       const float m = (float)(s / (double)K);
       for (int64_t k = 0; k < K; ++k) {
         const int64_t e = (b * K + k) * D + d;
