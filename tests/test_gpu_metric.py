@@ -1,7 +1,6 @@
 """Dot-product and cosine k-means (fkm.h, fkm_metric) on the GPU against the
 oracle: teacher-forced assign and update, the loop's objective, a
 free-running loop, and the Euclidean metric through the same entry points."""
-import math
 
 import numpy as np
 import pytest
@@ -10,77 +9,16 @@ import torch
 import datagen
 import exact_means_clustering_b200 as fkm
 import oracle
-from parity import problem, rel
+from parity import (check_assign_sim, check_free_running, check_update_sim, problem, rel,
+                    scored)
 
 pytestmark = pytest.mark.gpu
-
-
-def _scored(c, metric):
-    """The vectors a metric scores against: c, or its rows rounded to fp32 after
-    scaling to unit length."""
-    v = c.astype(np.float64)
-    if metric == "cosine":
-        n = np.linalg.norm(v, axis=-1, keepdims=True)
-        v = np.where(n > 0, v / np.where(n > 0, n, 1), 0).astype(np.float32).astype(np.float64)
-    return v
-
-
-def check_assign_sim(x, dtype, c, gpu_ids, metric):
-    """A point may differ from the oracle only at a near tie: the oracle's best
-    score beats the score of the GPU's choice by at most 1e-4 (||x||^2 +
-    ||c_hat||^2); at most ceil(1e-4 points) such points."""
-    mir = dtype if dtype != "f32" else None
-    bad = pts = 0
-    for b in range(x.shape[0]):
-        ids, s1, _ = oracle.assign_sim(x[b][None], c[b][None].astype(np.float64), metric,
-                                       dtype=dtype, mirror=mir)
-        ids, s1, gb = ids[0], s1[0], gpu_ids[b]
-        pts += len(gb)
-        mism = np.nonzero(ids != gb)[0]
-        if len(mism) == 0:
-            continue
-        ch = oracle.chat(_scored(c[b], metric)[None], mir)[0]
-        xf = datagen.widen(x[b][mism], dtype).astype(np.float64)
-        s_gpu = (xf * ch[gb[mism]]).sum(1)
-        band = 1e-4 * ((xf ** 2).sum(1) + (ch[ids[mism]] ** 2).sum(1))
-        over = s1[mism] - s_gpu > band
-        assert not over.any(), f"batch {b}: {over.sum()} points outside the near-tie band"
-        bad += len(mism)
-    assert bad <= math.ceil(1e-4 * pts), f"{bad} near-tie flips of {pts}"
-
-
-def check_update_sim(x, dtype, ids, prev, gpu_centers, gpu_counts, metric):
-    """counts exact; clusters that keep prev bit-identical; the mean (dot)
-    within 1e-5 of the cluster's mean |x|, the unit direction (cosine) within
-    1e-5 of the cluster's sum of |x| over the length of its sum."""
-    c_ref, n_ref, _ = oracle.update_sim(x, ids, prev.astype(np.float64), metric, dtype=dtype)
-    assert np.array_equal(gpu_counts.astype(np.int64), n_ref), "counts differ"
-    B, K, D = prev.shape
-    for b in range(B):
-        xf = datagen.widen(x[b], dtype).astype(np.float64)
-        absum = np.zeros((K, D))
-        s = np.zeros((K, D))
-        np.add.at(absum, ids[b], np.abs(xf))
-        np.add.at(s, ids[b], xf)
-        kept = (n_ref[b] == 0) | ((metric == "cosine") & ~s.any(1))
-        assert np.array_equal(gpu_centers[b][kept], prev[b][kept]), "kept clusters moved"
-        occ = ~kept
-        if metric == "dot":
-            tol = 1e-5 * absum / np.maximum(n_ref[b], 1)[:, None] + 1e-30
-        else:
-            tol = 1e-5 * absum / np.maximum(np.linalg.norm(s, axis=1), 1e-300)[:, None] + 2e-7
-        err = np.abs(gpu_centers[b].astype(np.float64) - c_ref[b])
-        assert np.all(err[occ] <= tol[occ]), \
-            f"batch {b}: centroid error {(err[occ] / tol[occ]).max():.2f}x tolerance"
-        if metric == "cosine":
-            nrm = np.linalg.norm(gpu_centers[b][occ].astype(np.float64), axis=1)
-            assert np.allclose(nrm, 1.0, atol=1e-6)
 
 
 def check_objective(x, dtype, ids, c, gpu_obj, metric):
     """sum_i x_i . c~_{ids_i} within 1e-6 of sum_i |x_i| . |c~_{ids_i}|."""
     ref = oracle.similarity(x, ids, c.astype(np.float64), metric, dtype=dtype)
-    v = np.abs(_scored(c, metric))
+    v = np.abs(scored(c, metric))
     for b in range(x.shape[0]):
         xf = np.abs(datagen.widen(x[b], dtype).astype(np.float64))
         scale = (xf * v[b][ids[b]]).sum()
@@ -151,9 +89,9 @@ def test_loop_objective_is_that_of_the_last_assignment(metric):
 @pytest.mark.parametrize("cfg,B,N,K", [(1, None, None, None), (2, 2, 8192, 256)])
 def test_loop_free_running_against_oracle(metric, cfg, B, N, K):
     """(i) the reported objective is the oracle's objective of the GPU's own
-    last assignment against the centroids it was made with; (ii) the run
-    matches the oracle's free-running one (1e-4 when the final assignments
-    agree; a run that took another path at a near tie is held to 2e-3)."""
+    last assignment against the centroids it was made with; (ii) the loop,
+    walked iteration by iteration against the oracle (check_free_running),
+    ends within 1e-4 of its objective."""
     it = 5
     w = datagen.CONFIGS[cfg].scaled(B=B, N=N, K=K, iters=it) if B else \
         datagen.CONFIGS[cfg].scaled(iters=it)
@@ -176,15 +114,13 @@ def test_loop_free_running_against_oracle(metric, cfg, B, N, K):
     assert torch.equal(ids_t, ids)
     g_ids, g_obj = ids.cpu().numpy(), obj.cpu().numpy()
     check_objective(x, w.dtype, g_ids, c_prev.cpu().numpy(), g_obj, metric)
-    mir = w.dtype if w.dtype != "f32" else None
-    r = oracle.lloyd_sim(x, c0, it, metric, dtype=w.dtype, mirror=mir)
-    for b in range(w.B):
-        agree = (g_ids[b] == r["ids"][b]).mean()
-        if agree >= 1 - 1e-4:
-            assert rel(g_obj[b], r["inertia"][b]) < 1e-4
-        else:
-            print(f"batch {b}: another path at a near tie, {agree:.5f} of ids agree")
-            assert agree > 0.98 and rel(g_obj[b], r["inertia"][b]) < 2e-3
+
+    def prefix(t):
+        i, ce, n, _ = run(t)
+        return i.cpu().numpy(), ce.cpu().numpy(), n.cpu().numpy()
+
+    check_free_running(x, w.dtype, c0, it, 0.0, prefix, lambda: (g_ids, g_obj, it),
+                       f"{metric} workload {cfg}", metric=metric)
 
 
 def test_euclid_metric_is_the_plain_loop():
