@@ -1,11 +1,12 @@
 // fkm_assign_noalloc: the assign step for callers that cannot allocate.
 //
 // Some callers are not allowed to allocate device memory at the point where
-// they need an assignment: code running inside a CUDA stream capture owned by
-// a framework that forbids allocations while capturing, real-time or embedded
-// services that reserve all memory up front in fixed pools, plugins handed
-// only their inputs and outputs by a host application.  They cannot call
-// cudaMalloc for the workspace that fkm_assign expects.
+// they need an assignment: code whose device memory is owned by a framework
+// allocator that must not be bypassed there, real-time or embedded services
+// that reserve all memory up front in fixed pools (a cudaMalloc mid-run can
+// stall or fail), plugins handed only their inputs and outputs by a host
+// application.  They cannot call cudaMalloc for the workspace that
+// fkm_assign expects.
 //
 // This entry point keeps its scratch (the per-batch mean centroid, the
 // centroid offsets rounded to the points' 16-bit type, their bias slabs, and
@@ -13,7 +14,10 @@
 // device array of FKM_NOALLOC_SCRATCH_BYTES.  Every GPU that loads the library
 // holds that array until the process exits.  The host-side name of the array
 // is only a stand-in: its device address is fetched with cudaGetSymbolAddress,
-// once per device, with that device current, on the first call made on it.
+// once per device, with that device current, on the first call made on it
+// (the address is cached for the life of the process, so a device reset
+// while the library is loaded is not supported).  fkm_assign_noalloc_status
+// reads and clears the array's status word.
 #include <cstring>
 #include <mutex>
 
@@ -111,4 +115,23 @@ extern "C" fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, 
   a.ids = ids;
   a.status = status;
   return launch_assign(a, st);
+}
+
+extern "C" fkm_status fkm_assign_noalloc_status(void* stream) {
+  void* base = nullptr;
+  FKM_TRY(scratch_for_current_device(&base));
+  int* status = static_cast<int*>(base);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  FKM_CUDA_TRY(cudaMemcpyAsync(&host, status, sizeof(int), cudaMemcpyDeviceToHost, st));
+  FKM_CUDA_TRY(cudaStreamSynchronize(st));
+  if (host == 0) return FKM_OK;
+  FKM_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  FKM_CUDA_TRY(cudaStreamSynchronize(st));
+  if (host & ST_TIMEOUT) {
+    set_error("a device-side bounded wait of fkm_assign_noalloc ran out (status 0x%x)", host);
+    return FKM_ERR_TIMEOUT;
+  }
+  set_error("fkm_assign_noalloc device status 0x%x", host);
+  return FKM_ERR_INTERNAL;
 }

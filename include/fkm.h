@@ -306,10 +306,10 @@ FKM_API long long fkm_kernel_launches(void);
 
 /* fkm_assign for callers that cannot allocate device memory.  The paper has no
  * counterpart: this is an interface for code that must not call cudaMalloc at
- * the point it needs an assignment -- inside a stream capture owned by a
- * framework that forbids allocating while capturing, in services that reserve
- * all device memory up front, or in plugins that are handed only their inputs
- * and outputs.  Same result as fkm_assign with inertia = NULL, but the
+ * the point it needs an assignment -- code whose device memory belongs to a
+ * framework allocator that must not be bypassed there, services that reserve
+ * all device memory up front in fixed pools, or plugins that are handed only
+ * their inputs and outputs.  Same result as fkm_assign with inertia = NULL, but the
  * scratch (the mean centroids, the rounded centroid offsets, their norm terms
  * and a status word) lives in a
  * file-scope device array of FKM_NOALLOC_SCRATCH_BYTES that every GPU loading
@@ -318,17 +318,28 @@ FKM_API long long fkm_kernel_launches(void);
  *   x        device [B,N,D] bf16 or fp16 (fp32 points are rejected: their
  *            split operands need scratch proportional to N)
  *   centers  device [B,K,D] float32;  ids device [B,N] int32 (out)
- * Limit: 256 + B*(4*D + Kp*(2*D + 4)) bytes (each part rounded to 256-byte
- * blocks) must fit in FKM_NOALLOC_SCRATCH_BYTES, Kp = K rounded up to 256;
- * larger shapes return FKM_ERR_UNSUPPORTED.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) and raises the kernel's shared-memory
- * limit; make that first call before any stream capture.  All calls share
- * the one array, which keeps the last call's contents: calls that can overlap
- * on the GPU (other streams, other threads) race with each other, so
- * serialise them.  Device-side status (a bounded wait that ran out) is not
- * reported by this call.  Async. */
+ * Limit: 256 + B*(4*D + Kp*(2*D + 32)) bytes (each of the three parts
+ * rounded up to 256-byte blocks) must fit in FKM_NOALLOC_SCRATCH_BYTES, Kp = K
+ * rounded up to 256; larger shapes return FKM_ERR_UNSUPPORTED.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress) and
+ * raises the kernel's shared-memory limit; make that first call before any
+ * stream capture.  The address is kept for the life of the process: a device
+ * reset while the library is loaded is not supported.  All calls share the one
+ * array, which keeps the last call's contents (the status word is cleared at
+ * the start of each call, the rest is rewritten): calls that can overlap on the
+ * GPU (other streams, other threads) race with each other, so serialise them.
+ * Device-side status (a bounded wait that ran out) is read with
+ * fkm_assign_noalloc_status.  Async. */
 FKM_API fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, const void* x,
                                       const float* centers, int32_t* ids, void* stream);
+
+/* Status of the fkm_assign_noalloc calls on the current device (no
+ * counterpart in the paper): waits for `stream`, then reads and clears the
+ * status word in the static scratch array.  FKM_OK, or FKM_ERR_TIMEOUT when a
+ * device-side bounded wait ran out (the ids of that call are then not valid).
+ * Allocates nothing; call it on the stream of the fkm_assign_noalloc calls it
+ * reports on. */
+FKM_API fkm_status fkm_assign_noalloc_status(void* stream);
 
 /* Waits for `stream`, then reads and clears the workspace's status word:
  * FKM_OK, FKM_ERR_TIMEOUT, FKM_ERR_BAD_ID or FKM_ERR_INTERNAL. */
