@@ -56,6 +56,7 @@ _SIG = {
     "fkm_baseline_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_baseline_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_assign_noalloc": ([_I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
+    "fkm_assign_noalloc_status": ([_P], _I),
     "fkm_sync_status": ([_P, _Z, _P], _I),
     "fkm_profile": ([_I], _I),
     "fkm_profile_read": ([_P, ctypes.POINTER(ctypes.c_longlong), _I], _I),
@@ -112,6 +113,82 @@ def _ptr(t, dtype=None):
     return t.data_ptr()
 
 
+class _Args:
+    """Argument checks of one call, made before the C call: every tensor must
+    hold exactly the elements its role needs (the C side trusts the sizes it
+    derives from B, N, K, D) and sit on the call's CUDA device (the stream's,
+    else that of the first device tensor given, else the current one); only
+    the host-streamed calls take their points from (pinned) host memory.
+    Contiguity, dtype and size are checked as each argument is marshalled;
+    a device mismatch is raised by done() (ws() calls it), after every
+    argument has passed those."""
+
+    def __init__(self, fn, stream=None, *tensors):
+        self.fn = fn
+        self.pending = None
+        self.device = None
+        if stream is not None and not isinstance(stream, int):
+            self.device = stream.device
+        else:
+            for t in tensors:
+                if torch.is_tensor(t) and t.is_cuda:
+                    self.device = t.device
+                    break
+
+    def _count(self, name, t, shape):
+        want = 1
+        for n in shape:
+            want *= int(n)
+        if t.numel() != want:
+            raise ValueError(f"{self.fn}: {name} has shape {tuple(t.shape)}, expected "
+                             f"{tuple(int(n) for n in shape)}")
+
+    def dev(self, name, t, shape, dtype=None):
+        """Pointer of a device tensor of `shape` (None and raw addresses pass)."""
+        if t is None or isinstance(t, int):
+            return t
+        p = _ptr(t, dtype)
+        self._count(name, t, shape)
+        if not t.is_cuda:
+            self.pending = self.pending or f"{name} must be a CUDA tensor, got one on {t.device}"
+        elif self.device is None:
+            self.device = t.device
+        elif t.device != self.device:
+            self.pending = self.pending or (f"{name} is on {t.device}, the call runs on "
+                                            f"{self.device}")
+        return p
+
+    def done(self):
+        if self.pending:
+            raise ValueError(f"{self.fn}: {self.pending}")
+
+    def ws(self, t):
+        """Pointer and size of a workspace tensor on the call's device."""
+        self.done()
+        if not t.is_cuda:
+            raise ValueError(f"{self.fn}: the workspace must be a CUDA tensor")
+        if self.device is not None and t.device != self.device:
+            raise ValueError(f"{self.fn}: the workspace is on {t.device}, the call runs on "
+                             f"{self.device}")
+        return _ptr(t), t.numel() * t.element_size()
+
+    def host(self, name, t, shape, dtype=None):
+        """Pointer of a host tensor of `shape` (raw addresses pass)."""
+        if isinstance(t, int):
+            return t
+        p = _ptr(t, dtype)
+        self._count(name, t, shape)
+        if t.is_cuda:
+            raise ValueError(f"{self.fn}: {name} must be in (pinned) host memory")
+        return p
+
+
+def _dims(fn, t, n, what):
+    if t.dim() != n:
+        raise ValueError(f"{fn}: {what} must be {n}-D, got shape {tuple(t.shape)}")
+    return tuple(t.shape)
+
+
 def _stream(stream):
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -155,35 +232,53 @@ def workspace(nbytes, device=None) -> torch.Tensor:
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
 
 
+def _ws(ws, nbytes, device):
+    return ws if ws is not None else workspace(nbytes, device)
+
+
 def fkm_assign(x, centers, ids, inertia=None, ws=None, stream=None):
-    B, N, D = x.shape
-    K = centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_assign", lib().fkm_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers, torch.float32), _ptr(ids, torch.int32),
-                                          _ptr(inertia, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
+    f = "fkm_assign"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, centers, 3, "centers")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("ids", ids, (B, N), torch.int32), A.dev("inertia", inertia, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
+    _check(f, lib().fkm_assign(B, N, K, D, _dt(x), *args, wp, wn, _stream(stream)))
 
 
 def fkm_update(x, ids, prev_centers, centers, counts, shift=None, inertia=None, ws=None,
                stream=None):
-    B, N, D = x.shape
-    K = prev_centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_update", lib().fkm_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids, torch.int32),
-                                          _ptr(prev_centers, torch.float32), _ptr(centers, torch.float32), _ptr(counts, torch.int32),
-                                          _ptr(shift, torch.float64), _ptr(inertia, torch.float64), _ptr(ws), ws.numel(),
-                                          _stream(stream)))
+    f = "fkm_update"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, prev_centers, 3, "prev_centers")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("prev_centers", prev_centers, (B, K, D), torch.float32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("shift", shift, (B,), torch.float64),
+            A.dev("inertia", inertia, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
+    _check(f, lib().fkm_update(B, N, K, D, _dt(x), *args, wp, wn, _stream(stream)))
 
 
 def fkm_lloyd(x, init_centers, max_iters, tol, ids, centers, counts, inertia=None, ws=None,
               stream=None) -> int:
-    B, N, D = x.shape
-    K = init_centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    f = "fkm_lloyd"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, init_centers, 3, "init_centers")[1]
+    A = _Args(f, stream, x)
+    px = A.dev("x", x, (B, N, D))
+    pi = A.dev("init_centers", init_centers, (B, K, D), torch.float32)
+    outs = (A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("inertia", inertia, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
     n_iter = ctypes.c_int(0)
-    _check("fkm_lloyd", lib().fkm_lloyd(B, N, K, D, _dt(x), _ptr(x), _ptr(init_centers, torch.float32), max_iters,
-                                        float(tol), _ptr(ids, torch.int32), _ptr(centers, torch.float32), _ptr(counts, torch.int32),
-                                        _ptr(inertia, torch.float64), ctypes.byref(n_iter), _ptr(ws), ws.numel(),
-                                        _stream(stream)))
+    _check(f, lib().fkm_lloyd(B, N, K, D, _dt(x), px, pi, max_iters, float(tol), *outs,
+                              ctypes.byref(n_iter), wp, wn, _stream(stream)))
     return n_iter.value
 
 
@@ -195,130 +290,185 @@ def _metric(metric) -> int:
 
 def fkm_assign_metric(x, centers, ids, metric, ws=None, stream=None):
     """ids = the most similar centroid under metric ('euclid', 'dot', 'cosine')."""
-    B, N, D = x.shape
-    K = centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_assign_metric",
-           lib().fkm_assign_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(centers, torch.float32),
-                                   _ptr(ids, torch.int32), _ptr(ws), ws.numel(), _stream(stream)))
+    f = "fkm_assign_metric"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, centers, 3, "centers")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("ids", ids, (B, N), torch.int32))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
+    _check(f, lib().fkm_assign_metric(B, N, K, D, _dt(x), _metric(metric), *args, wp, wn,
+                                      _stream(stream)))
 
 
 def fkm_update_metric(x, ids, prev_centers, centers, counts, metric, shift=None, objective=None,
                       ws=None, stream=None):
-    B, N, D = x.shape
-    K = prev_centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_update_metric",
-           lib().fkm_update_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x), _ptr(ids, torch.int32),
-                                   _ptr(prev_centers, torch.float32), _ptr(centers, torch.float32), _ptr(counts, torch.int32), _ptr(shift, torch.float64),
-                                   _ptr(objective, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
+    f = "fkm_update_metric"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, prev_centers, 3, "prev_centers")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("prev_centers", prev_centers, (B, K, D), torch.float32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("shift", shift, (B,), torch.float64),
+            A.dev("objective", objective, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
+    _check(f, lib().fkm_update_metric(B, N, K, D, _dt(x), _metric(metric), *args, wp, wn,
+                                      _stream(stream)))
 
 
 def fkm_lloyd_metric(x, init_centers, max_iters, tol, ids, centers, counts, metric,
                      objective=None, ws=None, stream=None) -> int:
-    B, N, D = x.shape
-    K = init_centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
+    f = "fkm_lloyd_metric"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, init_centers, 3, "init_centers")[1]
+    A = _Args(f, stream, x)
+    px = A.dev("x", x, (B, N, D))
+    pi = A.dev("init_centers", init_centers, (B, K, D), torch.float32)
+    outs = (A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("objective", objective, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
     n_iter = ctypes.c_int(0)
-    _check("fkm_lloyd_metric",
-           lib().fkm_lloyd_metric(B, N, K, D, _dt(x), _metric(metric), _ptr(x),
-                                  _ptr(init_centers, torch.float32), max_iters, float(tol), _ptr(ids, torch.int32),
-                                  _ptr(centers, torch.float32), _ptr(counts, torch.int32), _ptr(objective, torch.float64),
-                                  ctypes.byref(n_iter), _ptr(ws), ws.numel(), _stream(stream)))
+    _check(f, lib().fkm_lloyd_metric(B, N, K, D, _dt(x), _metric(metric), px, pi, max_iters,
+                                     float(tol), *outs, ctypes.byref(n_iter), wp, wn,
+                                     _stream(stream)))
     return n_iter.value
 
 
 def fkm_lloyd_host(x_host, init_centers, max_iters, tol, chunk_rows, ids, centers, counts,
                    inertia=None, ws=None, stream=None, dtype=None, shape=None) -> int:
     """x_host: a pinned CPU tensor [B, N, D] (or a raw address with dtype and shape)."""
+    f = "fkm_lloyd_host"
     if isinstance(x_host, int):
         B, N, D = shape
         dt = _dt(dtype)
     else:
-        B, N, D = x_host.shape
+        B, N, D = _dims(f, x_host, 3, "x_host")
         dt = _dt(x_host)
-    K = init_centers.shape[1]
-    if ws is None:
-        ws = workspace(fkm_host_workspace_size(B, N, K, D, dt, chunk_rows), init_centers.device)
+    K = _dims(f, init_centers, 3, "init_centers")[1]
+    A = _Args(f, stream, init_centers)
+    px = A.host("x_host", x_host, (B, N, D))
+    pi = A.dev("init_centers", init_centers, (B, K, D), torch.float32)
+    outs = (A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("inertia", inertia, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_host_workspace_size(B, N, K, D, dt, chunk_rows),
+                      init_centers.device))
     n_iter = ctypes.c_int(0)
-    _check("fkm_lloyd_host",
-           lib().fkm_lloyd_host(B, N, K, D, dt, _ptr(x_host), _ptr(init_centers, torch.float32), max_iters,
-                                float(tol), int(chunk_rows), _ptr(ids, torch.int32), _ptr(centers, torch.float32),
-                                _ptr(counts, torch.int32), _ptr(inertia, torch.float64), ctypes.byref(n_iter), _ptr(ws),
-                                ws.numel(), _stream(stream)))
+    _check(f, lib().fkm_lloyd_host(B, N, K, D, dt, px, pi, max_iters, float(tol),
+                                   int(chunk_rows), *outs, ctypes.byref(n_iter), wp, wn,
+                                   _stream(stream)))
     return n_iter.value
 
 
 def fkm_argsort(keys, n_keys, idx, sorted_keys=None, ws=None, stream=None):
+    f = "fkm_argsort"
     n = keys.numel()
-    ws = ws if ws is not None else workspace(fkm_argsort_workspace_size(n, n_keys), keys.device)
-    _check("fkm_argsort", lib().fkm_argsort(_ptr(keys, torch.int32), n, n_keys, _ptr(idx, torch.int32), _ptr(sorted_keys, torch.int32),
-                                            _ptr(ws), ws.numel(), _stream(stream)))
+    A = _Args(f, stream, keys)
+    args = (A.dev("keys", keys, (n,), torch.int32), n, n_keys,
+            A.dev("idx", idx, (n,), torch.int32),
+            A.dev("sorted_keys", sorted_keys, (n,), torch.int32))
+    wp, wn = A.ws(_ws(ws, fkm_argsort_workspace_size(n, n_keys), keys.device))
+    _check(f, lib().fkm_argsort(*args, wp, wn, _stream(stream)))
 
 
 def fkm_baseline_assign(x, centers, dist, ids, ws=None, stream=None):
-    B, N, D = x.shape
-    K = centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_baseline_assign",
-           lib().fkm_baseline_assign(B, N, K, D, _dt(x), _ptr(x), _ptr(centers, torch.float32), _ptr(dist),
-                                     _ptr(ids, torch.int32), _ptr(ws), ws.numel(), _stream(stream)))
+    f = "fkm_baseline_assign"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, centers, 3, "centers")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("dist", dist, (B, N, K), torch.float32), A.dev("ids", ids, (B, N), torch.int32))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
+    _check(f, lib().fkm_baseline_assign(B, N, K, D, _dt(x), *args, wp, wn, _stream(stream)))
 
 
 def fkm_baseline_update(x, ids, prev_centers, centers, counts, ws=None, stream=None):
-    B, N, D = x.shape
-    K = prev_centers.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_baseline_update",
-           lib().fkm_baseline_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids, torch.int32), _ptr(prev_centers, torch.float32),
-                                     _ptr(centers, torch.float32), _ptr(counts, torch.int32), _ptr(ws), ws.numel(),
-                                     _stream(stream)))
+    f = "fkm_baseline_update"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, prev_centers, 3, "prev_centers")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("prev_centers", prev_centers, (B, K, D), torch.float32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts", counts, (B, K), torch.int32))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
+    _check(f, lib().fkm_baseline_update(B, N, K, D, _dt(x), *args, wp, wn, _stream(stream)))
 
 
 def fkm_assign_noalloc(x, centers, ids, stream=None):
     """fkm_assign without a workspace, for callers that cannot allocate device
     memory: its scratch is a static 16 MiB device array inside the library
     (bf16/fp16 points only; calls that overlap on the GPU race)."""
-    B, N, D = x.shape
-    K = centers.shape[1]
-    _check("fkm_assign_noalloc", lib().fkm_assign_noalloc(B, N, K, D, _dt(x), _ptr(x),
-                                                          _ptr(centers, torch.float32), _ptr(ids, torch.int32),
-                                                          _stream(stream)))
+    f = "fkm_assign_noalloc"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, centers, 3, "centers")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("ids", ids, (B, N), torch.int32))
+    A.done()
+    _check(f, lib().fkm_assign_noalloc(B, N, K, D, _dt(x), *args, _stream(stream)))
+
+
+def fkm_assign_noalloc_status(stream=None):
+    """Wait for the stream, then read and clear the status word of the
+    fkm_assign_noalloc calls on the current device (raises FkmError with
+    FKM_ERR_TIMEOUT if a device-side bounded wait ran out)."""
+    _check("fkm_assign_noalloc_status", lib().fkm_assign_noalloc_status(_stream(stream)))
 
 
 def fkm_partial_update(x, ids, prev, sums, counts, obj=None, ws=None, stream=None):
     """Add one shard's per-cluster sums / counts (and objective) to sums [B, K, D]
     float64, counts [B, K] int32 (and obj [B] float64); see fkm.h."""
-    B, N, D = x.shape
-    K = prev.shape[1]
-    ws = ws if ws is not None else workspace(fkm_workspace_size(B, N, K, D, x.dtype), x.device)
-    _check("fkm_partial_update",
-           lib().fkm_partial_update(B, N, K, D, _dt(x), _ptr(x), _ptr(ids, torch.int32), _ptr(prev, torch.float32), _ptr(sums, torch.float64),
-                                    _ptr(counts, torch.int32), _ptr(obj, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
+    f = "fkm_partial_update"
+    B, N, D = _dims(f, x, 3, "x")
+    K = _dims(f, prev, 3, "prev")[1]
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("prev", prev, (B, K, D), torch.float32),
+            A.dev("sums", sums, (B, K, D), torch.float64),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("obj", obj, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
+    _check(f, lib().fkm_partial_update(B, N, K, D, _dt(x), *args, wp, wn, _stream(stream)))
 
 
 def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=None, ws=None,
                             stream=None):
     """fkm_partial_update for a shard in pinned host memory x_host [B, N, D],
     streamed in chunks of chunk_rows points; also writes the shard's ids."""
-    B, N, D = x_host.shape
-    K = centers.shape[1]
-    if ws is None:
-        ws = workspace(fkm_host_workspace_size(B, N, K, D, _dt(x_host), chunk_rows),
-                       centers.device)
-    _check("fkm_partial_update_host",
-           lib().fkm_partial_update_host(B, N, K, D, _dt(x_host), _ptr(x_host), _ptr(centers, torch.float32),
-                                         int(chunk_rows), _ptr(ids, torch.int32), _ptr(sums, torch.float64), _ptr(counts, torch.int32),
-                                         _ptr(obj, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
+    f = "fkm_partial_update_host"
+    B, N, D = _dims(f, x_host, 3, "x_host")
+    K = _dims(f, centers, 3, "centers")[1]
+    A = _Args(f, stream, centers)
+    px = A.host("x_host", x_host, (B, N, D))
+    args = (A.dev("centers", centers, (B, K, D), torch.float32), int(chunk_rows),
+            A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("sums", sums, (B, K, D), torch.float64),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("obj", obj, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_host_workspace_size(B, N, K, D, _dt(x_host), chunk_rows),
+                      centers.device))
+    _check(f, lib().fkm_partial_update_host(B, N, K, D, _dt(x_host), px, *args, wp, wn,
+                                            _stream(stream)))
 
 
 def fkm_finalize_sums(sums, counts, prev, centers, shift=None, ws=None, stream=None):
     """centers = sums / counts (prev where a cluster is empty); shift [B] optional."""
-    B, K, D = prev.shape
-    ws = ws if ws is not None else workspace(256 + 8 * B * K, prev.device)
-    _check("fkm_finalize_sums",
-           lib().fkm_finalize_sums(B, K, D, _ptr(sums, torch.float64), _ptr(counts, torch.int32), _ptr(prev, torch.float32), _ptr(centers, torch.float32),
-                                   _ptr(shift, torch.float64), _ptr(ws), ws.numel(), _stream(stream)))
+    f = "fkm_finalize_sums"
+    B, K, D = _dims(f, prev, 3, "prev")
+    A = _Args(f, stream, prev)
+    args = (A.dev("sums", sums, (B, K, D), torch.float64),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("prev", prev, (B, K, D), torch.float32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("shift", shift, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, 256 + 8 * B * K, prev.device))
+    _check(f, lib().fkm_finalize_sums(B, K, D, *args, wp, wn, _stream(stream)))
 
 
 def reduce_partials(tensors, group=None):
@@ -412,24 +562,30 @@ def fkm_centre_workspace_size_bytes(B, N, D) -> int:
 def fkm_centre(x, mu=None, out=None, ws=None, stream=None):
     """Per-batch mean of x [B, N, D] and x minus it, rounded to x's dtype (see
     fkm.h).  out may be x itself.  Returns (out, mu float32 [B, D])."""
-    B, N, D = x.shape
+    f = "fkm_centre"
+    B, N, D = _dims(f, x, 3, "x")
     mu = mu if mu is not None else torch.empty(B, D, dtype=torch.float32, device=x.device)
     out = out if out is not None else torch.empty_like(x)
-    if ws is None:
-        ws = workspace(fkm_centre_workspace_size_bytes(B, N, D), x.device)
-    _check("fkm_centre", lib().fkm_centre(B, N, D, _dt(x), _ptr(x), _ptr(mu, torch.float32), _ptr(out), _ptr(ws),
-                                          ws.numel(), _stream(stream)))
+    A = _Args(f, stream, x)
+    args = (A.dev("x", x, (B, N, D)), A.dev("mu", mu, (B, D), torch.float32),
+            A.dev("out", out, (B, N, D), x.dtype))
+    wp, wn = A.ws(_ws(ws, fkm_centre_workspace_size_bytes(B, N, D), x.device))
+    _check(f, lib().fkm_centre(B, N, D, _dt(x), *args, wp, wn, _stream(stream)))
     return out, mu
 
 
 def fkm_selftest_wait_timeout(timeout_ns, ws, stream=None):
     """Launch a kernel whose bounded wait runs out after timeout_ns (see fkm.h)."""
+    A = _Args("fkm_selftest_wait_timeout", stream, ws)
+    wp, wn = A.ws(ws)
     _check("fkm_selftest_wait_timeout",
-           lib().fkm_selftest_wait_timeout(int(timeout_ns), _ptr(ws), ws.numel(), _stream(stream)))
+           lib().fkm_selftest_wait_timeout(int(timeout_ns), wp, wn, _stream(stream)))
 
 
 def fkm_sync_status(ws, stream=None):
-    _check("fkm_sync_status", lib().fkm_sync_status(_ptr(ws), ws.numel(), _stream(stream)))
+    A = _Args("fkm_sync_status", stream, ws)
+    wp, wn = A.ws(ws)
+    _check("fkm_sync_status", lib().fkm_sync_status(wp, wn, _stream(stream)))
 
 
 def fkm_profile(enable: bool) -> None:

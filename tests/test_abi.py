@@ -151,3 +151,63 @@ def test_binding_refuses_strided_views_and_wrong_dtypes(fkm):
     with pytest.raises(TypeError, match="float64"):
         fkm.fkm_partial_update(x, ids, c, torch.zeros(2, 4, 16), torch.zeros(2, 4, dtype=torch.int32),
                                ws=ws)
+
+
+def test_binding_refuses_wrong_sizes_and_host_tensors(fkm):
+    """Every tensor must hold the elements its role needs and sit on the GPU
+    (host memory only for the streamed points): checked before any C call,
+    so a mis-sized or host tensor never reaches a kernel."""
+    import torch
+    x = torch.zeros(2, 64, 16, dtype=torch.bfloat16)
+    c = torch.zeros(2, 4, 16)
+    ids = torch.zeros(2, 64, dtype=torch.int32)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="ids has shape"):
+        fkm.fkm_assign(x, c, ids[:, :32].contiguous(), ws=ws)
+    with pytest.raises(ValueError, match="inertia has shape"):
+        fkm.fkm_assign(x, c, ids, torch.zeros(3, dtype=torch.float64), ws=ws)
+    with pytest.raises(ValueError, match="centers has shape"):
+        fkm.fkm_update(x, ids, c, torch.zeros(2, 5, 16), torch.zeros(2, 4, dtype=torch.int32),
+                       ws=ws)
+    with pytest.raises(ValueError, match="counts has shape"):
+        fkm.fkm_lloyd(x, c, 3, 0.0, ids, torch.zeros(2, 4, 16), torch.zeros(2, 5, dtype=torch.int32),
+                      ws=ws)
+    with pytest.raises(ValueError, match="must be 3-D"):
+        fkm.fkm_assign(x, c[0], ids, ws=ws)
+    # sizes right, but host tensors where device memory is required
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        fkm.fkm_assign(x, c, ids, ws=ws)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        fkm.fkm_assign_noalloc(x, c, ids)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        fkm.fkm_lloyd_host(x, c, 3, 0.0, 16, ids, torch.zeros(2, 4, 16),
+                           torch.zeros(2, 4, dtype=torch.int32), ws=ws)
+    with pytest.raises(ValueError, match="sums has shape"):
+        fkm.fkm_finalize_sums(torch.zeros(2, 4, 8, dtype=torch.float64),
+                              torch.zeros(2, 4, dtype=torch.int32), c, torch.zeros(2, 4, 16), ws=ws)
+    with pytest.raises(ValueError, match="idx has shape"):
+        fkm.fkm_argsort(torch.zeros(10, dtype=torch.int32), 4, torch.zeros(9, dtype=torch.int32),
+                        ws=ws)
+
+
+def test_noalloc_size_limit_matches_the_header(fkm):
+    """The header's limit, 256 + B*(4D + Kp*(2D + 32)) bytes with each part
+    rounded up to 256, against FKM_NOALLOC_SCRATCH_BYTES: the first K past
+    the limit is refused as unsupported before any device work.  (The shape
+    just inside is not called here: it would go on to launch.)"""
+    src = open(HEADER).read()
+    assert "Kp*(2*D + 32)" in src
+    L = fkm.lib()
+    limit = 16 << 20
+    D = 128
+
+    def need(B, K):
+        Kp = -(-K // 256) * 256
+        r = lambda v: -(-v // 256) * 256
+        return 256 + r(B * D * 4) + r(B * Kp * D * 2) + r(B * Kp * 32)
+
+    K_in = 256 * ((limit - 256 - 512) // (256 * (2 * D + 32)))
+    assert need(1, K_in) <= limit < need(1, K_in + 256)
+    a = 1 << 12   # a 16-byte-aligned non-null stand-in; validation runs before any access
+    rc_out = L.fkm_assign_noalloc(1, 128, K_in + 256, D, 2, a, a, a, None)
+    assert rc_out == 2 and b"static scratch" in L.fkm_last_error()
