@@ -18,6 +18,11 @@
 //     acc = x.q(c - m) - n/2 = -(score)/2 + (a per-point constant),
 // and the nearest centroid is the argmax of acc: the epilogue only compares.
 //
+// Two kernels share this design.  16-bit points whose point tile fits in
+// shared memory (D <= 256) run on CTA pairs (assign_pair_kernel below: one
+// MMA of M = 256 spans two SMs).  fp32 points, large D and the comparison
+// mode run on single CTAs (assign_tc_kernel), described first.
+//
 // B200 design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: the point tile [128 x D] once per work item into
 //               one of nA buffers; per centroid tile, 256 x 64 chunks through
@@ -55,6 +60,7 @@
 #include <cfloat>
 #include <cstddef>
 #include <cstdio>
+#include <cstring>
 
 #include "fkm_internal.cuh"
 #include "ptx_sm100.cuh"
@@ -498,6 +504,305 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA pairs
+// The main path (16-bit points, point tile resident in shared memory): a
+// cluster of two CTAs on neighbouring SMs shares every MMA (tcgen05
+// cta_group::2, M = 256).  CTA r of the pair holds rows [256 w + 128 r, +128)
+// of work item w and rows [128 r, +128) of every 256-centroid tile; the even
+// CTA issues the MMAs, and each CTA's TMEM receives its own 128 x 256
+// accumulator, which its own epilogue warps reduce as above.  Per SM this
+// halves the centroid bytes streamed from L2 and the B-operand bytes the
+// tensor cores read from shared memory per MMA: with one CTA per tile those
+// reads plus the TMA refills exceed the SM's shared-memory bandwidth and
+// hold the tensor pipe well below its peak.
+//
+// Synchronisation across the pair: TMA loads of both CTAs complete on the
+// even CTA's "full" barriers (cta_group::2 form, no multicast), whose
+// expected byte count covers both halves; tcgen05.commit with a two-CTA mask
+// arrives on the "empty" and accumulator-full barriers of both CTAs; each
+// epilogue warp of either CTA arrives on the even CTA's accumulator-empty
+// barrier (16 arrivals) once its TMEM reads are done.  Every wait is bounded
+// as in the single-CTA kernel; a cluster barrier precedes the TMEM release.
+constexpr int PAIR_BH = BN / 2;                          // centroid rows per CTA
+constexpr int PAIR_B_CHUNK = PAIR_BH * KC * 2;           // 16 KB
+constexpr int PAIR_AUG_B = PAIR_BH * AUG_COLS * 2;       // 4 KB
+constexpr int PAIR_STAGE = PAIR_B_CHUNK + PAIR_AUG_B;    // 20 KB (1024-byte multiple)
+constexpr int PAIR_ROWS = 2 * BM;                        // points per work item
+
+struct __align__(8) PairCtl {
+  uint64_t a_full[2], a_empty[2];
+  uint64_t b_full[8], b_empty[8];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t merge_full, merge_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  float2 merge[BM];   // (best, index as float bits) of warpgroup 1
+};
+
+// fold_chunk keeping the improving chunk in registers (no shared memory).
+__device__ __forceinline__ void fold_chunk_reg(const uint32_t (&r)[32], int col0, int K,
+                                               float& best, int& bcol, float (&sv)[32]) {
+  float s[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(r[j]);
+  if (col0 + 32 > K) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j >= K) s[j] = -INFINITY;
+  }
+  const float cm = max32(s);
+  if (cm > best) {
+    best = cm;
+    bcol = col0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) sv[j] = s[j];
+  }
+}
+
+__device__ __forceinline__ int find_first_reg(const float (&sv)[32], float best) {
+  uint32_t mask = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) mask |= (uint32_t)(sv[j] == best) << j;
+  return mask ? __ffs(mask) - 1 : 0;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
+    assign_pair_kernel(const __grid_constant__ CUtensorMap tm_x,    // points, box 64 x 128
+                       const __grid_constant__ CUtensorMap tm_c,    // centroid offsets, box 64 x 128
+                       const __grid_constant__ CUtensorMap tm_aug,  // bias slabs, box 16 x 128
+                       const AssignKParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* a_base = smem;
+  uint8_t* aug_a = a_base + (size_t)p.nA * p.a_bytes;
+  uint8_t* b_base = aug_a + AUG_A_BYTES;
+  PairCtl* ctl = reinterpret_cast<PairCtl*>(b_base + (size_t)p.nS * PAIR_STAGE);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const uint32_t cid = ptx::cluster_id_x(), ncl = ptx::n_clusters_x();
+  volatile int* abort_flag = &ctl->abort;
+
+  write_aug_a(aug_a, p.f16);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.nA; ++i) {
+      ptx::mbar_init(&ctl->a_full[i], 1);
+      ptx::mbar_init(&ctl->a_empty[i], 1);
+    }
+    for (int i = 0; i < p.nS; ++i) {
+      ptx::mbar_init(&ctl->b_full[i], 1);
+      ptx::mbar_init(&ctl->b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&ctl->acc_full[i], 1);
+      ptx::mbar_init(&ctl->acc_empty[i], 16);   // 8 epilogue warps in each CTA
+    }
+    ptx::mbar_init(&ctl->merge_full, 128);
+    ptx::mbar_init(&ctl->merge_empty, 128);
+    ptx::mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncwarp();
+  // both CTAs' barriers exist and their TMEM is allocated before any
+  // cross-CTA arrival or MMA
+  ptx::cluster_sync();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_x);
+      ptx::prefetch_tmap(&tm_c);
+      ptx::prefetch_tmap(&tm_aug);
+      uint32_t a_arms = 0, s_arms = 0;
+      bool ok = true;
+      for (int w = (int)cid; w < p.n_work && ok; w += (int)ncl) {
+        const int b = w / p.m_tiles, mt = w % p.m_tiles;
+        const int row0 = mt * PAIR_ROWS + (int)rank * BM;
+        const int ab = a_arms % p.nA;
+        const uint32_t apar = ((a_arms / p.nA) & 1) ^ 1;
+        if (!ptx::mbar_wait_bounded_cl(&ctl->a_empty[ab], apar, abort_flag, p.status, ST_TIMEOUT,
+                                       kWaitTimeoutNs)) { ok = false; break; }
+        if (leader) ptx::mbar_arrive_expect_tx(&ctl->a_full[ab], 2 * p.a_bytes);
+        const uint32_t afull = ptx::mapa_rank(&ctl->a_full[ab], 0);
+        uint8_t* abuf = a_base + (size_t)ab * p.a_bytes;
+        for (int dc = 0; dc < p.nD; ++dc)
+          ptx::tma_load_3d_pair(abuf + dc * A_CHUNK_BYTES, &tm_x, afull, dc * KC, row0, b);
+        ++a_arms;
+        for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
+          const int crow = kt * BN + (int)rank * PAIR_BH;
+          for (int q = 0; q < p.nD; ++q) {
+            const int sb = s_arms % p.nS;
+            const uint32_t spar = ((s_arms / p.nS) & 1) ^ 1;
+            if (!ptx::mbar_wait_bounded_cl(&ctl->b_empty[sb], spar, abort_flag, p.status,
+                                           ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+            if (leader)
+              ptx::mbar_arrive_expect_tx(&ctl->b_full[sb],
+                                         2 * (PAIR_B_CHUNK + (q == 0 ? PAIR_AUG_B : 0)));
+            const uint32_t bfull = ptx::mapa_rank(&ctl->b_full[sb], 0);
+            uint8_t* sbuf = b_base + (size_t)sb * PAIR_STAGE;
+            ptx::tma_load_3d_pair(sbuf, &tm_c, bfull, q * KC, crow, b);
+            if (q == 0) ptx::tma_load_3d_pair(sbuf + PAIR_B_CHUNK, &tm_aug, bfull, 0, crow, b);
+            ++s_arms;
+          }
+        }
+      }
+      // Drain: the last use of every buffer was consumed by the MMAs (which
+      // also means its loads landed) before this CTA may leave.
+      for (uint32_t i = 0; i < (uint32_t)p.nA && i < a_arms; ++i) {
+        const uint32_t last = i + p.nA * ((a_arms - 1 - i) / p.nA);
+        ptx::mbar_wait_bounded_cl(&ctl->a_empty[i], (last / p.nA) & 1, abort_flag, p.status,
+                                  ST_TIMEOUT, kWaitTimeoutNs);
+      }
+      for (uint32_t i = 0; i < (uint32_t)p.nS && i < s_arms; ++i) {
+        const uint32_t last = i + p.nS * ((s_arms - 1 - i) / p.nS);
+        ptx::mbar_wait_bounded_cl(&ctl->b_empty[i], (last / p.nS) & 1, abort_flag, p.status,
+                                  ST_TIMEOUT, kWaitTimeoutNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      const uint32_t aug_a_addr = ptx::smem_u32(aug_a);
+      uint32_t a_uses = 0, s_uses = 0, acc_uses = 0;
+      bool ok = true, issued = false;
+      for (int w = (int)cid; w < p.n_work && ok; w += (int)ncl) {
+        const int ab = a_uses % p.nA;
+        if (!ptx::mbar_wait_bounded_cl(&ctl->a_full[ab], (a_uses / p.nA) & 1, abort_flag,
+                                       p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t a_addr = ptx::smem_u32(a_base + (size_t)ab * p.a_bytes);
+        for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
+          const int acc = acc_uses & 1;
+          if (!ptx::mbar_wait_bounded_cl(&ctl->acc_empty[acc], ((acc_uses >> 1) & 1) ^ 1,
+                                         abort_flag, p.status, ST_TIMEOUT, kWaitTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+          for (int q = 0; q < p.nD; ++q) {
+            const int sb = s_uses % p.nS;
+            if (!ptx::mbar_wait_bounded_cl(&ctl->b_full[sb], (s_uses / p.nS) & 1, abort_flag,
+                                           p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint32_t b_addr = ptx::smem_u32(b_base + (size_t)sb * PAIR_STAGE);
+            if (q == 0)   // the bias product starts the tile's accumulation
+              ptx::mma_f16_ss_pair(d_tmem, ptx::umma_desc_sw32(aug_a_addr),
+                                   ptx::umma_desc_sw32(b_addr + PAIR_B_CHUNK), p.idesc, 0u);
+            const uint32_t xa = a_addr + q * A_CHUNK_BYTES;
+#pragma unroll
+            for (int k = 0; k < KC / 16; ++k)
+              ptx::mma_f16_ss_pair(d_tmem, ptx::umma_desc_sw128(xa + 32 * k),
+                                   ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc, 1u);
+            issued = true;
+            ptx::mma_commit_pair_mc(&ctl->b_empty[sb], 0x3);
+            ++s_uses;
+          }
+          if (!ok) break;
+          ptx::mma_commit_pair_mc(&ctl->acc_full[acc], 0x3);
+          ++acc_uses;
+        }
+        if (!ok) break;
+        ptx::mma_commit_pair_mc(&ctl->a_empty[ab], 0x3);
+        ++a_uses;
+      }
+      // Drain: all MMAs issued must finish before TMEM is freed.
+      if (issued) {
+        ptx::mma_commit_pair_mc(&ctl->drain, 0x1);
+        ptx::mbar_wait_bounded_cl(&ctl->drain, 0, abort_flag, p.status, ST_TIMEOUT,
+                                  kWaitTimeoutNs);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int half = ew >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
+    const uint32_t acc_empty_cl[2] = {ptx::mapa_rank(&ctl->acc_empty[0], 0),
+                                      ptx::mapa_rank(&ctl->acc_empty[1], 0)};
+    uint32_t acc_uses = 0, items = 0;
+    bool ok = true;
+    float sv[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) sv[j] = -INFINITY;
+    for (int w = (int)cid; w < p.n_work && ok; w += (int)ncl, ++items) {
+      const int b = w / p.m_tiles, mt = w % p.m_tiles;
+      const int gi = mt * PAIR_ROWS + (int)rank * BM + row;
+      float best = -INFINITY;
+      int bcol = 0;
+      for (int kt = 0; kt < p.k_tiles; ++kt) {
+        const int acc = acc_uses & 1;
+        const uint32_t par = (acc_uses >> 1) & 1;
+        if (!ptx::mbar_wait_bounded_cl(&ctl->acc_full[acc], par, abort_flag, p.status,
+                                       ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t taddr = lane_addr + (uint32_t)(acc * BN + half * 128);
+        const int colb = kt * BN + half * 128;
+        // two batches of 64 columns keep the live registers within the
+        // 320-thread block's budget (the improving chunk is kept in
+        // registers); the accumulator goes back once the second batch landed
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld32(taddr, r0);
+        ptx::tmem_ld32(taddr + 32, r1);
+        ptx::tmem_wait_ld64(r0, r1);
+        fold_chunk_reg(r0, colb, p.K, best, bcol, sv);
+        fold_chunk_reg(r1, colb + 32, p.K, best, bcol, sv);
+        __syncwarp();   // the folds branch per lane; tcgen05.ld is warp-wide
+        ptx::tmem_ld32(taddr + 64, r0);
+        ptx::tmem_ld32(taddr + 96, r1);
+        ptx::tmem_wait_ld64(r0, r1);
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(acc_empty_cl[acc]);
+        ++acc_uses;
+        fold_chunk_reg(r0, colb + 64, p.K, best, bcol, sv);
+        fold_chunk_reg(r1, colb + 96, p.K, best, bcol, sv);
+      }
+      if (!ok) break;
+      const int idx = best > -INFINITY ? bcol + find_first_reg(sv, best) : 0;
+      const uint32_t mpar = items & 1;
+      if (half == 1) {
+        if (!ptx::mbar_wait_bounded(&ctl->merge_empty, mpar ^ 1, abort_flag, p.status,
+                                    ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+        ctl->merge[row] = make_float2(best, __int_as_float(idx));
+        ptx::mbar_arrive(&ctl->merge_full);
+      } else {
+        if (!ptx::mbar_wait_bounded(&ctl->merge_full, mpar, abort_flag, p.status, ST_TIMEOUT,
+                                    kWaitTimeoutNs)) { ok = false; break; }
+        const float2 o = ctl->merge[row];
+        ptx::mbar_arrive(&ctl->merge_empty);
+        const int oidx = __float_as_int(o.y);
+        const int fidx = (o.x > best || (o.x == best && oidx < idx)) ? oidx : idx;
+        if (gi < p.N) p.ids[(size_t)b * p.N + gi] = fidx;
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncwarp();
+  // both CTAs are done with TMEM and with each other's barriers
+  ptx::cluster_sync();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -580,6 +885,29 @@ bool assign_smem_plan(int D, bool split, int* nA_out, int* nS_out, size_t* smem_
   return true;
 }
 
+// Shared-memory plan of the CTA-pair kernel (16-bit points, D <= 256).
+static bool assign_pair_plan(int D, int* nA_out, int* nS_out, size_t* smem_out) {
+  if (D > 256) return false;
+  const int nD = (int)ceil_div(D, KC);
+  const long a_bytes = (long)nD * A_CHUNK_BYTES;
+  const long ctl = (long)((sizeof(PairCtl) + 127) & ~size_t(127)) + AUG_A_BYTES;
+  int nA = 2;
+  long nS = (kSmemBudget - ctl - 2 * a_bytes) / PAIR_STAGE;
+  if (nS < 3) {
+    nA = 1;
+    nS = (kSmemBudget - ctl - a_bytes) / PAIR_STAGE;
+  }
+  if (nS > 8) nS = 8;
+  if (nS < 2) return false;
+  if (nA_out) *nA_out = nA;
+  if (nS_out) *nS_out = (int)nS;
+  if (smem_out) *smem_out = (size_t)(nA * a_bytes + nS * PAIR_STAGE + ctl + 1024);
+  return true;
+}
+
+// Clusters of two the pair kernel keeps resident at once (per device).
+static int pair_clusters[64] = {0};
+
 // Raises the kernels' dynamic shared-memory limit once per device.  Called
 // before any stream capture (the attribute call is not a stream operation).
 fkm_status assign_prepare() {
@@ -604,11 +932,73 @@ fkm_status assign_prepare() {
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
   FKM_CUDA_TRY(cudaFuncSetAttribute(assign_tc_kernel<true, true, true>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+  FKM_CUDA_TRY(cudaFuncSetAttribute(assign_pair_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+  // resident clusters of the pair kernel at its largest shared-memory plan
+  {
+    size_t smem = 0;
+    assign_pair_plan(64, nullptr, nullptr, &smem);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(2 * (num_sms() / 2)), 1, 1);
+    cfg.blockDim = dim3(ASSIGN_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)lim;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, assign_pair_kernel, &cfg) != cudaSuccess ||
+        n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    if (dev >= 0 && dev < 64) pair_clusters[dev] = n;
+  }
   if (dev >= 0 && dev < 64) done[dev] = true;
   return FKM_OK;
 }
 
+static fkm_status launch_assign_pair(const AssignArgs& a, cudaStream_t st) {
+  int nA = 0, nS = 0;
+  size_t smem = 0;
+  assign_pair_plan(a.D, &nA, &nS, &smem);
+  const int nD = (int)ceil_div(a.D, KC);
+  const bool bf16 = a.dtype == FKM_BF16;
+  CUtensorMap tx, tc, taug;
+  FKM_TRY(make_map(&tx, a.xq, bf16, a.D, a.N, a.B, a.x_row_elems, KC, BM));
+  FKM_TRY(make_map(&tc, a.cq, bf16, a.D, a.Kp, a.B, a.D, KC, PAIR_BH));
+  FKM_TRY(make_map(&taug, a.caug, bf16, AUG_COLS, a.Kp, a.B, AUG_COLS, AUG_COLS, PAIR_BH,
+                   CU_TENSOR_MAP_SWIZZLE_32B));
+  AssignKParams p;
+  memset(&p, 0, sizeof(p));
+  p.B = a.B;
+  p.N = a.N;
+  p.Kp = a.Kp;
+  p.K = a.K;
+  p.nD = nD;
+  p.m_tiles = (int)ceil_div(a.N, PAIR_ROWS);
+  p.k_tiles = a.Kp / BN;
+  p.n_work = a.B * p.m_tiles;
+  p.nA = nA;
+  p.nS = nS;
+  p.a_bytes = (uint32_t)(nD * A_CHUNK_BYTES);
+  p.idesc = ptx::umma_idesc_f16(bf16, 2 * BM, BN);
+  p.f16 = bf16 ? 0 : 1;
+  p.ids = a.ids;
+  p.status = a.status;
+  FKM_TRY(assign_prepare());
+  int dev = 0;
+  FKM_CUDA_TRY(cudaGetDevice(&dev));
+  int clusters = (dev >= 0 && dev < 64 && pair_clusters[dev] > 0) ? pair_clusters[dev]
+                                                                    : num_sms() / 2;
+  if (clusters > p.n_work) clusters = p.n_work;
+  assign_pair_kernel<<<2 * clusters, ASSIGN_THREADS, smem, st>>>(tx, tc, taug, p);
+  note_launch();
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
 fkm_status launch_assign(const AssignArgs& a, cudaStream_t st) {
+  // 16-bit points with the point tile resident in shared memory: CTA pairs
+  if (!a.split && !a.dist && assign_pair_plan(a.D, nullptr, nullptr, nullptr))
+    return launch_assign_pair(a, st);
   int nA = 0, nS = 0;
   size_t smem = 0;
   bool stream = false;

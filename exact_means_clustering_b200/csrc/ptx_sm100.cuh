@@ -52,21 +52,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Polls between checks of the abort flag and the clock in a bounded wait.
+// try_wait itself suspends the thread for a while before it reports "not
+// yet", so the polls alone pace the loop; reading %globaltimer (a
+// long-latency read) on every poll would put that latency between a phase
+// completing and the waiter noticing it, on the critical path of the
+// pipelines that wait here.
+constexpr uint32_t kPollsPerCheck = 64;
+
 // Waits for the phase of `parity` to complete.  Gives up (returns false) when
-// *abort becomes non-zero or after timeout_ns; on a timeout it raises *abort
-// and ORs err_bit into the global status word so every waiter leaves quickly.
+// *abort becomes non-zero or after timeout_ns (both checked every
+// kPollsPerCheck polls); on a timeout it raises *abort and ORs err_bit into
+// the global status word so every waiter leaves quickly.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, int* status,
                                                   int err_bit, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
-  for (;;) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t polls = 1;; ++polls) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > timeout_ns) {
-      *abort = 1;
-      atomicOr(status, err_bit);
-      return false;
+    if (polls % kPollsPerCheck == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        atomicOr(status, err_bit);
+        return false;
+      }
     }
   }
 }
@@ -162,6 +173,22 @@ __device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
                : "memory");
 }
 
+// Pins 32 registers after a wait: code that reads them cannot move above it.
+__device__ __forceinline__ void pin32(uint32_t (&b)[32]) {
+  asm volatile("" : "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]),
+               "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]),
+               "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15]), "+r"(b[16]), "+r"(b[17]),
+               "+r"(b[18]), "+r"(b[19]), "+r"(b[20]), "+r"(b[21]), "+r"(b[22]), "+r"(b[23]),
+               "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]),
+               "+r"(b[30]), "+r"(b[31])::"memory");
+}
+
+// tcgen05.wait::ld naming two 32-register destination arrays.
+__device__ __forceinline__ void tmem_wait_ld64(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  tmem_wait_ld32(a);
+  pin32(b);
+}
+
 // tcgen05.wait::ld naming four 32-register destination arrays.
 __device__ __forceinline__ void tmem_wait_ld128(uint32_t (&a)[32], uint32_t (&b)[32],
                                                 uint32_t (&c)[32], uint32_t (&d)[32]) {
@@ -185,6 +212,106 @@ __device__ __forceinline__ void tmem_wait_ld128(uint32_t (&a)[32], uint32_t (&b)
                "+r"(d[18]), "+r"(d[19]), "+r"(d[20]), "+r"(d[21]), "+r"(d[22]), "+r"(d[23]),
                "+r"(d[24]), "+r"(d[25]), "+r"(d[26]), "+r"(d[27]), "+r"(d[28]), "+r"(d[29]),
                "+r"(d[30]), "+r"(d[31])::"memory");
+}
+
+// ------------------------------------------------ CTA pairs (cta_group::2)
+// A cluster of two CTAs on neighbouring SMs shares one MMA: the even CTA
+// (rank 0) issues tcgen05.mma.cta_group::2, which reads 128 rows of A from
+// each CTA's shared memory (M = 256) and the two halves of B (N/2 rows each),
+// and writes each CTA's 128 accumulator rows into that CTA's TMEM.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t n_clusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+
+// Address, in the cluster's shared window, of the object at the same offset
+// as `p` in the shared memory of CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_rank(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier of either CTA of the pair, given by its cluster
+// address.  The TMEM reads this arrival releases were completed
+// (tcgen05.wait::ld) and ordered before it (tcgen05.fence::before_thread_sync)
+// by the caller.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Bounded wait on a barrier that the other CTA of the pair also arrives on
+// (the same wait: an arrival's release is observed by the try_wait's acquire).
+__device__ __forceinline__ bool mbar_wait_bounded_cl(uint64_t* bar, uint32_t parity,
+                                                     volatile int* abort, int* status,
+                                                     int err_bit, uint64_t timeout_ns) {
+  return mbar_wait_bounded(bar, parity, abort, status, err_bit, timeout_ns);
+}
+
+// 3-D tiled TMA load into this CTA's shared memory whose completion (bytes)
+// is signalled on an mbarrier of either CTA of the pair, given by its
+// cluster address.  No multicast.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const void* tmap,
+                                                 uint32_t bar_cluster_addr, int c0, int c1,
+                                                 int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A (128 rows from each CTA) * B (N/2 rows from each)^T
+__device__ __forceinline__ void mma_f16_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the mbarrier at the offset of `bar` in every CTA of
+// cta_mask when all previously issued MMAs of this thread complete.
+__device__ __forceinline__ void mma_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// Whole-cluster barrier (every thread of both CTAs).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
 }
 
 // 3-input minimum (sm_100a).
