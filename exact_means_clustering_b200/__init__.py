@@ -36,10 +36,11 @@ _SIG = {
     "fkm_selftest_wait_timeout": ([ctypes.c_uint64, _P, _Z, _P], _I),
     "fkm_centre_workspace_size": ([_I, _I, _I, ctypes.POINTER(_Z)], _I),
     "fkm_partial_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
-    "fkm_finalize_sums": ([_I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_finalize_sums": ([_I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_partial_update_host": ([_I, _I, _I, _I, _I, _P, _P, _L, _P, _P, _P, _P, _P, _Z, _P],
                                 _I),
     "fkm_centre": ([_I, _I, _I, _I, _P, _P, _P, _P, _Z, _P], _I),
+    "fkm_shift_centroids": ([_I, _I, _I, _P, _P, _I, _P, _P], _I),
     "fkm_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_lloyd": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _P, _P, ctypes.POINTER(_I), _P, _Z,
@@ -58,6 +59,8 @@ _SIG = {
     "fkm_assign_noalloc": ([_I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
     "fkm_assign_noalloc_status": ([_P], _I),
     "fkm_sync_status": ([_P, _Z, _P], _I),
+    "fkm_segsum_stats": ([_P, _Z, _L, _I, ctypes.POINTER(ctypes.c_ulonglong),
+                          ctypes.POINTER(_I), _P], _I),
     "fkm_profile": ([_I], _I),
     "fkm_profile_read": ([_P, ctypes.POINTER(ctypes.c_longlong), _I], _I),
     "fkm_kernel_launches": ([], ctypes.c_longlong),
@@ -422,8 +425,8 @@ def fkm_assign_noalloc_status(stream=None):
 
 
 def fkm_partial_update(x, ids, prev, sums, counts, obj=None, ws=None, stream=None):
-    """Add one shard's per-cluster sums / counts (and objective) to sums [B, K, D]
-    float64, counts [B, K] int32 (and obj [B] float64); see fkm.h."""
+    """Add one shard's per-cluster sums / counts (and objective) to sums [B, K, D],
+    counts [B, K] (and obj [B]), all float64; see fkm.h."""
     f = "fkm_partial_update"
     B, N, D = _dims(f, x, 3, "x")
     K = _dims(f, prev, 3, "prev")[1]
@@ -431,7 +434,7 @@ def fkm_partial_update(x, ids, prev, sums, counts, obj=None, ws=None, stream=Non
     args = (A.dev("x", x, (B, N, D)), A.dev("ids", ids, (B, N), torch.int32),
             A.dev("prev", prev, (B, K, D), torch.float32),
             A.dev("sums", sums, (B, K, D), torch.float64),
-            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("counts", counts, (B, K), torch.float64),
             A.dev("obj", obj, (B,), torch.float64))
     wp, wn = A.ws(_ws(ws, fkm_workspace_size(B, N, K, D, x.dtype), x.device))
     _check(f, lib().fkm_partial_update(B, N, K, D, _dt(x), *args, wp, wn, _stream(stream)))
@@ -449,7 +452,7 @@ def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=
     args = (A.dev("centers", centers, (B, K, D), torch.float32), int(chunk_rows),
             A.dev("ids", ids, (B, N), torch.int32),
             A.dev("sums", sums, (B, K, D), torch.float64),
-            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("counts", counts, (B, K), torch.float64),
             A.dev("obj", obj, (B,), torch.float64))
     wp, wn = A.ws(_ws(ws, fkm_host_workspace_size(B, N, K, D, _dt(x_host), chunk_rows),
                       centers.device))
@@ -457,24 +460,28 @@ def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=
                                             _stream(stream)))
 
 
-def fkm_finalize_sums(sums, counts, prev, centers, shift=None, ws=None, stream=None):
-    """centers = sums / counts (prev where a cluster is empty); shift [B] optional."""
+def fkm_finalize_sums(sums, counts, prev, centers, shift=None, ws=None, stream=None,
+                      counts_out=None):
+    """centers = sums / counts (prev where a cluster is empty; sums and counts
+    float64); shift [B] and counts_out [B, K] int32 optional."""
     f = "fkm_finalize_sums"
     B, K, D = _dims(f, prev, 3, "prev")
     A = _Args(f, stream, prev)
     args = (A.dev("sums", sums, (B, K, D), torch.float64),
-            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("counts", counts, (B, K), torch.float64),
             A.dev("prev", prev, (B, K, D), torch.float32),
             A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts_out", counts_out, (B, K), torch.int32),
             A.dev("shift", shift, (B,), torch.float64))
     wp, wn = A.ws(_ws(ws, 256 + 8 * B * K, prev.device))
     _check(f, lib().fkm_finalize_sums(B, K, D, *args, wp, wn, _stream(stream)))
 
 
 def reduce_partials(tensors, group=None):
-    """Sum the shards' partial sums / counts / objectives over the ranks of a
-    torch.distributed group (NCCL over NVLink for CUDA tensors): one
-    all-reduce each.  A no-op without an initialised group of 2+ ranks."""
+    """Sum the shards' partials over the ranks of a torch.distributed group
+    (NCCL over NVLink for CUDA tensors): one all-reduce per tensor given --
+    the sharded loop gives one packed buffer.  A no-op without an
+    initialised group of 2+ ranks."""
     import torch.distributed as dist
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) < 2:
         return
@@ -482,16 +489,30 @@ def reduce_partials(tensors, group=None):
         dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
 
 
+def partial_buffers(B, K, D, device):
+    """One float64 buffer holding a shard's partials, and its views (sums
+    [B, K, D], counts [B, K], obj [B]); each view starts 16-byte aligned.
+    Reducing the buffer reduces all three with one collective."""
+    def up2(n):
+        return n + (n & 1)
+    o1 = up2(B * K * D)
+    o2 = o1 + up2(B * K)
+    buf = torch.zeros(o2 + up2(B), dtype=torch.float64, device=device)
+    return (buf, buf[:B * K * D].view(B, K, D), buf[o1:o1 + B * K].view(B, K),
+            buf[o2:o2 + B])
+
+
 def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None, chunk_rows=None):
     """Data-parallel Lloyd k-means over the ranks of a torch.distributed group
     (README "Multi-GPU Support"): every rank passes its own contiguous shard
     x [B, N_r, D] of the same B problems and the same init_centers [B, K, D];
     per iteration each rank assigns its shard, forms its partial sums and
-    counts, the partials are all-reduced, and every rank forms the same
-    centroids.  A shard in pinned host memory (x on the CPU) is streamed to
-    init_centers' device in chunks of chunk_rows points every iteration, as
-    fkm_lloyd_host does.  Returns (ids of this shard [B, N_r], centers
-    [B, K, D], counts [B, K] of all shards, inertia [B] of all shards, n_iter)."""
+    counts, the partials are all-reduced (one packed buffer, one
+    collective), and every rank forms the same centroids.  A shard in pinned
+    host memory (x on the CPU) is streamed to init_centers' device in chunks
+    of chunk_rows points every iteration, as fkm_lloyd_host does.  Returns
+    (ids of this shard [B, N_r], centers [B, K, D], counts [B, K] int32 of
+    all shards, inertia [B] of all shards, n_iter)."""
     B, N, D = x.shape
     K = init_centers.shape[1]
     on_host = not x.is_cuda
@@ -514,43 +535,78 @@ def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None, chun
             fkm_assign(x, c, ids, ws=ws)
             fkm_partial_update(x, ids, c, sums, counts, obj, ws=ws)
 
-    def finalize(sums, counts, c, nxt, shift):
-        fkm_finalize_sums(sums, counts, c, nxt, shift, ws=ws)
+    def finalize(sums, counts, c, nxt, shift, counts_out):
+        fkm_finalize_sums(sums, counts, c, nxt, shift, ws=ws, counts_out=counts_out)
 
     c, counts, obj, n_iter = sharded_loop(partials, finalize, c, max_iters, tol, group)
     fkm_sync_status(ws)
     return ids, c, counts, obj, n_iter
 
 
+def _group_size(group=None):
+    """Ranks of an initialised torch.distributed group (1 without one)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return 1
+    return dist.get_world_size(group)
+
+
+def shard_rows(N, rank, world):
+    """Contiguous rows [r0, r1) of N that rank `rank` of `world` holds: the
+    first N % world ranks take one row more."""
+    q, r = divmod(int(N), int(world))
+    r0 = rank * q + min(rank, r)
+    return r0, r0 + q + (1 if rank < r else 0)
+
+
+def gather_shard_ids(ids, N, group=None):
+    """All ranks' shard labels [B, N_r] put back in row order, [B, N] on every
+    rank (shards from shard_rows; one all_gather of equal-size padded
+    blocks)."""
+    import torch.distributed as dist
+    world = _group_size(group)
+    if world < 2:
+        return ids
+    B = ids.shape[0]
+    width = shard_rows(N, 0, world)[1]
+    pad = torch.full((B, width), -1, dtype=ids.dtype, device=ids.device)
+    pad[:, :ids.shape[1]] = ids
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    out = torch.empty(B, N, dtype=ids.dtype, device=ids.device)
+    for r, part in enumerate(parts):
+        r0, r1 = shard_rows(N, r, world)
+        out[:, r0:r1] = part[:, :r1 - r0]
+    return out
+
+
 def sharded_loop(partials, finalize, c, max_iters, tol=0.0, group=None):
     """The rank-side control of the data-parallel loop, independent of where
     the shard lives: per iteration partials(c, sums, counts, obj) adds this
-    rank's shard into zeroed sums [B, K, D] float64, counts [B, K] int32 and
-    obj [B] float64; reduce_partials sums them over the group; finalize(sums,
-    counts, c, nxt, shift) forms the next centroids and the shift [B].  The
-    stop test (max shift < tol) reads reduced values only, so every rank takes
-    the same number of iterations and the same collectives.  Returns (centers,
-    counts and objective of all shards, n_iter)."""
+    rank's shard into the zeroed float64 views sums [B, K, D], counts [B, K]
+    and obj [B] of one packed buffer; reduce_partials sums that buffer over
+    the group with one all-reduce; finalize(sums, counts, c, nxt, shift,
+    counts_out) forms the next centroids, the shift [B] and the int32 counts.
+    The stop test (max shift < tol) reads reduced values only, so every rank
+    takes the same number of iterations and the same collectives.  Returns
+    (centers, counts [B, K] int32 and objective [B] of all shards, n_iter)."""
     B, K, D = c.shape
     dev = c.device
-    sums = torch.empty(B, K, D, dtype=torch.float64, device=dev)
-    counts = torch.empty(B, K, dtype=torch.int32, device=dev)
-    obj = torch.empty(B, dtype=torch.float64, device=dev)
+    buf, sums, counts, obj = partial_buffers(B, K, D, dev)
+    counts_out = torch.empty(B, K, dtype=torch.int32, device=dev)
     shift = torch.empty(B, dtype=torch.float64, device=dev)
     n_iter = 0
     for t in range(max_iters):
-        sums.zero_()
-        counts.zero_()
-        obj.zero_()
+        buf.zero_()
         partials(c, sums, counts, obj)
-        reduce_partials((sums, counts, obj), group)
+        reduce_partials((buf,), group)
         nxt = torch.empty_like(c)
-        finalize(sums, counts, c, nxt, shift)
+        finalize(sums, counts, c, nxt, shift, counts_out)
         c = nxt
         n_iter = t + 1
         if tol > 0.0 and shift.max().item() < tol:
             break
-    return c, counts, obj, n_iter
+    return c, counts_out, obj, n_iter
 
 
 def fkm_centre_workspace_size_bytes(B, N, D) -> int:
@@ -574,12 +630,40 @@ def fkm_centre(x, mu=None, out=None, ws=None, stream=None):
     return out, mu
 
 
+def fkm_shift_centroids(centers, mu, sign, out=None, stream=None):
+    """out = centers + sign * mu per batch (fp32, sign +1 or -1; out may be
+    centers): the centroid side of centring.  Returns out."""
+    f = "fkm_shift_centroids"
+    B, K, D = _dims(f, centers, 3, "centers")
+    out = out if out is not None else torch.empty_like(centers)
+    A = _Args(f, stream, centers)
+    args = (A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("mu", mu, (B, D), torch.float32), int(sign),
+            A.dev("out", out, (B, K, D), torch.float32))
+    A.done()
+    _check(f, lib().fkm_shift_centroids(B, K, D, *args, _stream(stream)))
+    return out
+
+
 def fkm_selftest_wait_timeout(timeout_ns, ws, stream=None):
     """Launch a kernel whose bounded wait runs out after timeout_ns (see fkm.h)."""
     A = _Args("fkm_selftest_wait_timeout", stream, ws)
     wp, wn = A.ws(ws)
     _check("fkm_selftest_wait_timeout",
            lib().fkm_selftest_wait_timeout(int(timeout_ns), wp, wn, _stream(stream)))
+
+
+def fkm_segsum_stats(ws, n_rows, reset=False, stream=None):
+    """(fp64 element atomics the segment sums made into ws's cluster sums since
+    the last reset, sorted rows per segment-sum range for n_rows points)."""
+    A = _Args("fkm_segsum_stats", stream, ws)
+    wp, wn = A.ws(ws)
+    cnt = ctypes.c_ulonglong(0)
+    rng = ctypes.c_int(0)
+    _check("fkm_segsum_stats", lib().fkm_segsum_stats(wp, wn, int(n_rows), 1 if reset else 0,
+                                                      ctypes.byref(cnt), ctypes.byref(rng),
+                                                      _stream(stream)))
+    return cnt.value, rng.value
 
 
 def fkm_sync_status(ws, stream=None):
@@ -670,16 +754,27 @@ class FlashKMeans:
                copy of x
     chunk_rows rows per streamed chunk when the points are in host memory
 
+    device     the GPU to run on.  None: the current CUDA device, or, when a
+               torch.distributed process group of two or more ranks is
+               initialised (one process per GPU, e.g. under torchrun), every
+               rank clusters its contiguous shard of the points on its own
+               GPU and the ranks combine their partial sums with one
+               all-reduce per iteration (README "Multi-GPU Support");
+               labels_ then holds every point's label on every rank
+    group      the process group for that case (None: the default group)
+
     Points are [N, D] or [B, N, D] (B independent problems).  After fit:
     centroids [B, K, D] float32 (or [K, D]), labels_ int32 [B, N] (or [N]),
     n_iter, inertia [B] (the objective of the last assignment).
     """
 
     def __init__(self, d, k, niter=100, tol=0.0, dtype=None, centre=False, seed=0,
-                 chunk_rows=1 << 23, device=None):
+                 chunk_rows=1 << 23, device=None, group=None):
         self.d, self.k, self.niter, self.tol = int(d), int(k), int(niter), float(tol)
         self.dtype, self.centre, self.seed = dtype, bool(centre), int(seed)
         self.chunk_rows = int(chunk_rows)
+        self.group = group
+        self._sharded = device is None and _group_size(group) > 1
         self.device = torch.device(device) if device is not None else torch.device("cuda")
         self.centroids = None
         self.labels_ = None
@@ -700,6 +795,8 @@ class FlashKMeans:
         B, N, D = x.shape
         if init_centroids is not None:
             return init_centroids.reshape(B, self.k, D).to(self.device, torch.float32).contiguous()
+        if N < self.k:
+            raise ValueError(f"k = {self.k} clusters need at least as many points, got {N}")
         g = torch.Generator(device="cpu").manual_seed(self.seed)
         idx = torch.stack([torch.randperm(N, generator=g)[:self.k] for _ in range(B)])
         rows = torch.gather(x, 1, idx.to(x.device).unsqueeze(-1).expand(B, self.k, D))
@@ -708,6 +805,8 @@ class FlashKMeans:
     def fit(self, x, init_centroids=None):
         self._squeeze = x.dim() == 2
         x = self._shape(x)
+        if self._sharded:
+            return self._fit_sharded(x, init_centroids)
         if not x.is_cuda:
             return self._fit_host(x, init_centroids)
         B, N, D = x.shape
@@ -715,7 +814,8 @@ class FlashKMeans:
         if self.centre:
             x, mu = fkm_centre(x)
             if init_centroids is not None:
-                init_centroids = init_centroids.reshape(B, self.k, D).to(x.device) - mu[:, None, :]
+                c = init_centroids.reshape(B, self.k, D).to(x.device, torch.float32).contiguous()
+                init_centroids = fkm_shift_centroids(c, mu, -1)
         init = self._init(x, init_centroids)
         ids = torch.empty(B, N, dtype=torch.int32, device=x.device)
         centers = torch.empty(B, self.k, D, dtype=torch.float32, device=x.device)
@@ -723,7 +823,7 @@ class FlashKMeans:
         inertia = torch.empty(B, dtype=torch.float64, device=x.device)
         self.n_iter = fkm_lloyd(x, init, self.niter, self.tol, ids, centers, counts, inertia)
         if mu is not None:
-            centers += mu[:, None, :]
+            fkm_shift_centroids(centers, mu, +1, out=centers)
         self._store(ids, centers, inertia)
         return self
 
@@ -740,6 +840,29 @@ class FlashKMeans:
         self.n_iter = fkm_lloyd_host(xh, init, self.niter, self.tol, self.chunk_rows, ids, centers,
                                      counts, inertia)
         self._store(ids, centers, inertia)
+        return self
+
+    def _fit_sharded(self, x, init_centroids):
+        """One shard of the points per rank: rows shard_rows(N, rank, world)
+        of every problem, in pinned host memory (streamed) when x is on the
+        host, else on this rank's GPU."""
+        import torch.distributed as dist
+        if self.centre:
+            raise ValueError("centre=True is not supported with sharded fitting")
+        rank, world = dist.get_rank(self.group), dist.get_world_size(self.group)
+        dev = torch.device("cuda", torch.cuda.current_device())
+        B, N, D = x.shape
+        r0, r1 = shard_rows(N, rank, world)
+        shard = x[:, r0:r1].contiguous()
+        if shard.is_cuda:
+            shard = shard.to(dev)
+        elif not shard.is_pinned():
+            shard = shard.pin_memory()
+        init = self._init(x, init_centroids).to(dev)   # the same seed on every rank
+        ids, centers, _, inertia, self.n_iter = lloyd_sharded(
+            shard, init, self.niter, self.tol, self.group,
+            chunk_rows=None if shard.is_cuda else self.chunk_rows)
+        self._store(gather_shard_ids(ids, N, self.group), centers, inertia)
         return self
 
     def _store(self, ids, centers, inertia):

@@ -196,6 +196,8 @@ struct Ws {
   T* at(size_t off) const { return ws_ptr<T>(base, off); }
   int* status() const { return at<int>(L->status); }
   double* max_shift() const { return at<double>(L->status + 64); }
+  // fp64 atomic additions made by the segment sums (fkm_segsum_stats)
+  unsigned long long* atomics() const { return at<unsigned long long>(L->status + 128); }
 };
 
 static fkm_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
@@ -296,7 +298,7 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   // from the cluster sums in the finalize step
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK,
                         w.at<double>(L.sums64), next, false,
-                        obj_args(w, prev, euclid ? obj : nullptr), st, range));
+                        obj_args(w, prev, euclid ? obj : nullptr), st, range, w.atomics()));
   if (ev) FKM_TRY(record_stage(ev[3], st));
   if (euclid) {
     FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64),
@@ -800,6 +802,26 @@ fkm_status fkm_baseline_update(int B, int N, int K, int D, int dtype, const void
   return launch_baseline_update(x, dtype, ids, B, N, K, D, w.at<float>(L.sums64),
                                 w.at<int32_t>(L.segstart), prev_centers, centers, counts,
                                 w.status(), static_cast<cudaStream_t>(stream));
+}
+
+fkm_status fkm_segsum_stats(void* ws, size_t ws_bytes, int64_t n_rows, int reset,
+                            unsigned long long* atomics, int* range_rows, void* stream) {
+  if (!ws || ws_bytes < 256 || !aligned16(ws) || n_rows < 0) {
+    set_error("workspace null, misaligned or smaller than 256 bytes, or n_rows < 0");
+    return FKM_ERR_INVALID_ARG;
+  }
+  if (range_rows) *range_rows = segsum_range_rows(n_rows > 0 ? n_rows : 1);
+  if (!atomics && !reset) return FKM_OK;
+  Layout L;
+  memset(&L, 0, sizeof(L));
+  Ws w{ws, &L};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned long long host = 0;
+  FKM_CUDA_TRY(cudaMemcpyAsync(&host, w.atomics(), sizeof(host), cudaMemcpyDeviceToHost, st));
+  if (reset) FKM_CUDA_TRY(cudaMemsetAsync(w.atomics(), 0, sizeof(host), st));
+  FKM_CUDA_TRY(cudaStreamSynchronize(st));
+  if (atomics) *atomics = host;
+  return FKM_OK;
 }
 
 fkm_status fkm_sync_status(void* ws, size_t ws_bytes, void* stream) {

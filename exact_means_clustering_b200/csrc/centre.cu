@@ -95,6 +95,18 @@ __global__ void __launch_bounds__(CENTRE_THREADS) centre_subtract_kernel(
 
 int64_t centre_partials(int N) { return ceil_div(N, CENTRE_ROWS); }
 
+// out[b, k, d] = fp32(c[b, k, d] + sign * mu[b, d]): one IEEE fp32 addition
+// (or subtraction) per element; out may be c.
+__global__ void __launch_bounds__(CENTRE_THREADS) shift_centroids_kernel(
+    const float* c, const float* __restrict__ mu, float sign, int K, int D, int64_t n,
+    float* out) {
+  const int64_t e = (int64_t)blockIdx.x * CENTRE_THREADS + threadIdx.x;
+  if (e >= n) return;
+  const int64_t d = e % D, b = e / ((int64_t)K * D);
+  const float m = mu[b * D + d];
+  out[e] = sign > 0.0f ? c[e] + m : c[e] - m;
+}
+
 }  // namespace
 }  // namespace fkm
 
@@ -146,6 +158,25 @@ extern "C" fkm_status fkm_centre(int B, int N, int D, int dtype, const void* x, 
   else
     centre_subtract_kernel<FKM_F32><<<grid, CENTRE_THREADS, 0, st>>>(x, x_out, mu, N, D, nvec);
   note_launch(3);
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+extern "C" fkm_status fkm_shift_centroids(int B, int K, int D, const float* centers,
+                                          const float* mu, int sign, float* out, void* stream) {
+  if (B < 1 || K < 1 || D < 1 || (sign != 1 && sign != -1)) {
+    set_error("B, K, D must be >= 1 and sign +1 or -1");
+    return FKM_ERR_INVALID_ARG;
+  }
+  if (!centers || !mu || !out) {
+    set_error("centers, mu and out must be non-null");
+    return FKM_ERR_INVALID_ARG;
+  }
+  const int64_t n = (int64_t)B * K * D;
+  shift_centroids_kernel<<<(unsigned)ceil_div(n, CENTRE_THREADS), CENTRE_THREADS, 0,
+                           static_cast<cudaStream_t>(stream)>>>(centers, mu, (float)sign, K, D,
+                                                                n, out);
+  note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
 }

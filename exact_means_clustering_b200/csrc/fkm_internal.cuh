@@ -165,9 +165,12 @@ struct ObjArgs {
   int K = 1;
   double* obj = nullptr;
 };
+// atomics (optional): incremented by the number of fp64 element atomics the
+// segment sums add into sums64 (D per flush of a run that crosses a range).
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
-                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range = 0);
+                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range = 0,
+                         unsigned long long* atomics = nullptr);
 // Rows per warp range of the segment sums for n sorted rows: SEG_RANGE for
 // large n, fewer (down to 32) when n is small, so a small problem still
 // spreads over many warps.  finalize must be given the same value.
@@ -179,11 +182,13 @@ fkm_status segsum_prepare();
 fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const int32_t* ids,
                             const ObjArgs& oa, cudaStream_t st);
 // clear_sums: zero sums64 after reading it (the library's own accumulators);
-// false leaves a caller's reduced sums untouched.
+// false leaves a caller's reduced sums untouched.  counts_in64 (fp64 counts,
+// the shard partials reduced across GPUs) takes precedence over counts_in.
 fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
                            const int32_t* counts_in, double* sums64, const float* prev,
                            float* centers, int32_t* counts, double* shiftk, cudaStream_t st,
-                           int range = SEG_RANGE, bool clear_sums = true);
+                           int range = SEG_RANGE, bool clear_sums = true,
+                           const double* counts_in64 = nullptr);
 fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
                                double* max_shift, cudaStream_t st);
 // dot-product / cosine k-means: new centroids, per-cluster shift and

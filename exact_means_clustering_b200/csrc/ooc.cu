@@ -24,11 +24,12 @@ namespace fkm {
 
 namespace {
 
+template <typename T>
 __global__ void accumulate_counts_kernel(const int32_t* __restrict__ segstart,
                                          const int32_t* __restrict__ segend, int K,
-                                         int32_t* __restrict__ acc) {
+                                         T* __restrict__ acc) {
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k < K) acc[k] += segend[k] - segstart[k];
+  if (k < K) acc[k] += (T)(segend[k] - segstart[k]);
 }
 
 struct HostLayout {
@@ -138,7 +139,7 @@ int64_t injected_h2d_fault_chunk() {
 // to the caller's buffers instead of finalizing.
 struct HostPartial {
   double* sums;
-  int32_t* counts;
+  double* counts;
   double* obj;
 };
 
@@ -177,18 +178,21 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
 
 fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype, const void* x_host,
                                    const float* centers, int64_t chunk_rows, int32_t* ids,
-                                   double* sums, int32_t* counts, double* obj, void* ws,
+                                   double* sums, double* counts, double* obj, void* ws,
                                    size_t ws_bytes, void* stream) {
-  if (!sums || (reinterpret_cast<uintptr_t>(sums) & 15) ||
+  if (!sums || !counts || (reinterpret_cast<uintptr_t>(sums) & 15) ||
+      (reinterpret_cast<uintptr_t>(counts) & 15) ||
       (obj && (reinterpret_cast<uintptr_t>(obj) & 15))) {
-    set_error("sums must be non-null; sums and obj 16-byte aligned");
+    set_error("sums and counts must be non-null; sums, counts and obj 16-byte aligned");
     return FKM_ERR_INVALID_ARG;
   }
   HostPartial part{sums, counts, obj};
   int n_iter = 0;
+  // counts is only checked for null and alignment on this path: the partial
+  // pass adds into part.counts (fp64), never into the int32 output
   return lloyd_host_impl(B, N, K, D, dtype, x_host, centers, 1, 0.0f, chunk_rows, ids,
-                         const_cast<float*>(centers), counts, obj, &n_iter, ws, ws_bytes, stream,
-                         &part);
+                         const_cast<float*>(centers), reinterpret_cast<int32_t*>(counts), obj,
+                         &n_iter, ws, ws_bytes, stream, &part);
 }
 
 }  // extern "C"
@@ -234,7 +238,7 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
   float* cA = static_cast<float*>(at(L.cbuf));
   float* cB = cA + (size_t)B * K * D;
   double* sums64 = part ? part->sums : static_cast<double*>(at(L.sums64));
-  int32_t* counts_acc = part ? part->counts : static_cast<int32_t*>(at(L.counts_acc));
+  int32_t* counts_acc = static_cast<int32_t*>(at(L.counts_acc));
 
   StreamSet ss;
   FKM_CUDA_TRY(cudaStreamCreateWithFlags(&ss.copy, cudaStreamNonBlocking));
@@ -333,8 +337,12 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
         }
         FKM_TRY(launch_segsum(xb, dtype, D, so.keys_out, so.vals_out, rows, K,
                               sums64 + (size_t)b * K * D, nullptr, true, oa, st));
-        accumulate_counts_kernel<<<(unsigned)ceil_div(K, 256), 256, 0, st>>>(
-            segstart, segend, K, counts_acc + (size_t)b * K);
+        if (part)
+          accumulate_counts_kernel<double><<<(unsigned)ceil_div(K, 256), 256, 0, st>>>(
+              segstart, segend, K, part->counts + (size_t)b * K);
+        else
+          accumulate_counts_kernel<int32_t><<<(unsigned)ceil_div(K, 256), 256, 0, st>>>(
+              segstart, segend, K, counts_acc + (size_t)b * K);
         note_launch();
         FKM_CUDA_TRY(cudaGetLastError());
         FKM_CUDA_TRY(cudaEventRecord(ss.freed[buf], st));

@@ -5,7 +5,8 @@
 // and counts (a few MB) are reduced across the GPUs; and every GPU forms the
 // same new centroids from the reduced sums.  These two calls are the
 // per-shard halves of that iteration; the reduction between them is the
-// caller's (one all-reduce).
+// caller's: sums, counts and objective are all fp64, so the caller can lay
+// them out in one buffer and reduce it with one all-reduce.
 #include "fkm_internal.cuh"
 
 namespace fkm {
@@ -13,9 +14,9 @@ namespace {
 
 __global__ void add_counts_kernel(const int32_t* __restrict__ segstart,
                                   const int32_t* __restrict__ segend, int64_t keys,
-                                  int32_t* __restrict__ counts) {
+                                  double* __restrict__ counts) {
   const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (k < keys) counts[k] += segend[k] - segstart[k];
+  if (k < keys) counts[k] += (double)(segend[k] - segstart[k]);
 }
 
 fkm_status aligned_or_null(const void* p, const char* name) {
@@ -29,7 +30,7 @@ fkm_status aligned_or_null(const void* p, const char* name) {
 }  // namespace
 
 fkm_status shard_partial_update(const Layout& L, const void* x, const int32_t* ids,
-                                const float* prev, double* sums, int32_t* counts, double* obj,
+                                const float* prev, double* sums, double* counts, double* obj,
                                 void* ws, cudaStream_t st);
 
 }  // namespace fkm
@@ -38,7 +39,7 @@ using namespace fkm;
 
 extern "C" fkm_status fkm_partial_update(int B, int N, int K, int D, int dtype, const void* x,
                                          const int32_t* ids, const float* prev, double* sums,
-                                         int32_t* counts, double* obj, void* ws, size_t ws_bytes,
+                                         double* counts, double* obj, void* ws, size_t ws_bytes,
                                          void* stream) {
   size_t need = 0;
   FKM_TRY(fkm_workspace_size(B, N, K, D, dtype, &need));
@@ -60,8 +61,9 @@ extern "C" fkm_status fkm_partial_update(int B, int N, int K, int D, int dtype, 
 }
 
 extern "C" fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
-                                        const int32_t* counts, const float* prev, float* centers,
-                                        double* shift, void* ws, size_t ws_bytes, void* stream) {
+                                        const double* counts, const float* prev, float* centers,
+                                        int32_t* counts_out, double* shift, void* ws,
+                                        size_t ws_bytes, void* stream) {
   if (B < 1 || K < 1 || D < 1 || (int64_t)B * K >= (int64_t(1) << 31)) {
     set_error("B, K, D must be >= 1 and B*K < 2^31");
     return FKM_ERR_INVALID_ARG;
@@ -75,13 +77,14 @@ extern "C" fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
     set_error("centers must not alias prev");
     return FKM_ERR_INVALID_ARG;
   }
-  const void* ptrs[] = {sums, counts, prev, centers, shift, ws};
-  const char* names[] = {"sums", "counts", "prev", "centers", "shift", "ws"};
-  for (int i = 0; i < 6; ++i) FKM_TRY(aligned_or_null(ptrs[i], names[i]));
+  const void* ptrs[] = {sums, counts, prev, centers, shift, ws, counts_out};
+  const char* names[] = {"sums", "counts", "prev", "centers", "shift", "ws", "counts_out"};
+  for (int i = 0; i < 7; ++i) FKM_TRY(aligned_or_null(ptrs[i], names[i]));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   double* shiftk = reinterpret_cast<double*>(static_cast<char*>(ws) + 256);
-  FKM_TRY(launch_finalize(B, K, D, nullptr, nullptr, counts, const_cast<double*>(sums), prev,
-                          centers, nullptr, shiftk, st, SEG_RANGE, /*clear_sums=*/false));
+  FKM_TRY(launch_finalize(B, K, D, nullptr, nullptr, nullptr, const_cast<double*>(sums), prev,
+                          centers, counts_out, shiftk, st, SEG_RANGE, /*clear_sums=*/false,
+                          counts));
   if (shift) FKM_TRY(launch_batch_reduce(B, K, shiftk, shift, nullptr, st));
   return FKM_OK;
 }
@@ -89,7 +92,7 @@ extern "C" fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
 namespace fkm {
 
 fkm_status shard_partial_update(const Layout& L, const void* x, const int32_t* ids,
-                                const float* prev, double* sums, int32_t* counts, double* obj,
+                                const float* prev, double* sums, double* counts, double* obj,
                                 void* wsp, cudaStream_t st) {
   char* w = static_cast<char*>(wsp);
   auto at = [&](size_t off) { return static_cast<void*>(w + off); };

@@ -71,7 +71,8 @@ template <bool kFirst>
 __device__ __forceinline__ void load_key(const KeySrc& s, int64_t j, int32_t& key, int32_t& val) {
   if (kFirst) {
     const int32_t id = s.ids[j];
-    const int32_t b = (int32_t)(j / s.N);
+    // j < 2^31 (B*N is bounded by validation): a 32-bit division suffices
+    const int32_t b = (int32_t)((uint32_t)j / (uint32_t)s.N);
     if (id < 0 || id >= s.K) {
       atomicOr(s.status, ST_BAD_ID);
       key = s.sentinel;

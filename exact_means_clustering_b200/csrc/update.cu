@@ -60,6 +60,7 @@ struct SegParams {
   float* centers;
   bool accumulate_all;   // out-of-core chunks: every run goes to sums64
   ObjArgs oa;
+  unsigned long long* atomics;   // optional: count of fp64 atomic additions to sums64
 };
 
 // 16-byte vectors of the storage type, widened to float.
@@ -151,6 +152,8 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
 #pragma unroll
       for (int e = 0; e < E; ++e)
         if (col0 + e < p.D) atomicAdd(sd + e, acc[e]);
+      // instrumentation: this flush made p.D element atomics in all
+      if (sub == 0 && p.atomics) atomicAdd(p.atomics, (unsigned long long)p.D);
     }
   }
 #pragma unroll
@@ -478,6 +481,7 @@ struct FinParams {
   int32_t* counts;
   double* shiftk;
   const int32_t* counts_in;  // out-of-core: accumulated counts (segstart/end unused)
+  const double* counts_in64;  // shard partials reduced across GPUs: counts as fp64
   int range;                 // the segment sums' rows per warp range
   bool clear_sums;           // zero sums64 after use (the library's own accumulators)
 };
@@ -491,7 +495,9 @@ __global__ void finalize_kernel(FinParams p) {
   if (key >= (int64_t)p.B * p.K) return;
   int32_t nk;
   bool interior = false;
-  if (p.counts_in) {
+  if (p.counts_in64) {
+    nk = (int32_t)p.counts_in64[key];
+  } else if (p.counts_in) {
     nk = p.counts_in[key];
   } else {
     const int32_t s = p.segstart[key], t = p.segend[key];
@@ -787,7 +793,8 @@ fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* s
 
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
-                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range) {
+                         bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range,
+                         unsigned long long* atomics) {
   if (n == 0) return FKM_OK;
   if (range <= 0) range = segsum_range_rows(n);
   FKM_TRY(segsum_prepare());
@@ -810,6 +817,7 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
     sp.centers = centers ? centers + c0 : nullptr;
     sp.accumulate_all = accumulate_all;
     sp.oa = oa;
+    sp.atomics = atomics;
     if (oa.chat) sp.oa.chat = static_cast<const char*>(oa.chat) + (int64_t)c0 * eb;
     if (oa.m) sp.oa.m = oa.m + c0;
     if (dtype == FKM_BF16) FKM_TRY(run_segsum_dt<FKM_BF16>(sp, st));
@@ -839,8 +847,9 @@ fkm_status launch_objective(const void* x, int dtype, int B, int N, int D, const
 fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const int32_t* segend,
                            const int32_t* counts_in, double* sums64, const float* prev,
                            float* centers, int32_t* counts, double* shiftk, cudaStream_t st,
-                           int range, bool clear_sums) {
+                           int range, bool clear_sums, const double* counts_in64) {
   FinParams fp;
+  fp.counts_in64 = counts_in64;
   fp.range = range;
   fp.clear_sums = clear_sums;
   fp.B = B;

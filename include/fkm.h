@@ -219,30 +219,34 @@ FKM_API fkm_status fkm_argsort(const int32_t* keys, int64_t n, int n_keys, int32
  * contiguous shards, one per GPU.  One iteration on each GPU is
  *   fkm_assign(shard, c)                        -> shard ids
  *   fkm_partial_update(shard, ids, c)           -> += shard sums / counts / objective
- *   all-reduce of sums, counts (and objective) across the GPUs (the caller's)
+ *   all-reduce of sums, counts and objective across the GPUs (the caller's;
+ *   all three are fp64, so one buffer holding them takes one all-reduce)
  *   fkm_finalize_sums(reduced sums, counts, c)  -> the same new centroids everywhere
  *
  * fkm_partial_update: for the shard x [B, N, D] (this GPU's N points of each
  * problem) and its ids [B, N], ADDS the per-cluster fp64 sums of the points
- * to sums [B, K, D] (double), their counts to counts [B, K] (int32), and,
- * when obj is non-null, the shard's objective sum ||x - c_hat||^2 against the
- * centroids prev [B, K, D] the ids were assigned with to obj [B] (double).
- * The caller zeroes sums / counts / obj once per iteration.  ws: a workspace
- * of fkm_workspace_size(B, N, K, D, dtype) bytes.  All device pointers.
- * An id outside [0, K) sets FKM_ERR_BAD_ID in the status word.  Async.
+ * to sums [B, K, D] (double), their counts to counts [B, K] (double: exact
+ * integers up to 2^53), and, when obj is non-null, the shard's objective
+ * sum ||x - c_hat||^2 against the centroids prev [B, K, D] the ids were
+ * assigned with to obj [B] (double).  The caller zeroes sums / counts / obj
+ * once per iteration.  ws: a workspace of fkm_workspace_size(B, N, K, D,
+ * dtype) bytes.  All device pointers, 16-byte aligned.  An id outside
+ * [0, K) sets FKM_ERR_BAD_ID in the status word.  Async.
  *
  * fkm_finalize_sums: centers = sums / counts per cluster (IEEE division in
- * fp64, rounded to fp32), prev for a cluster with no points; shift [B] (may
- * be NULL) = sum_k ||centers - prev||^2.  sums and counts are not modified.
- * ws: device scratch of at least 256 + 8 * B * K bytes.  centers must not
- * alias prev.  Async. */
+ * fp64, rounded to fp32), prev for a cluster with no points; counts_out
+ * [B, K] int32 (may be NULL) receives the counts; shift [B] (may be NULL) =
+ * sum_k ||centers - prev||^2.  sums and counts are not modified.  ws: device
+ * scratch of at least 256 + 8 * B * K bytes.  centers must not alias prev.
+ * Async. */
 FKM_API fkm_status fkm_partial_update(int B, int N, int K, int D, int dtype, const void* x,
                                       const int32_t* ids, const float* prev, double* sums,
-                                      int32_t* counts, double* obj, void* ws, size_t ws_bytes,
+                                      double* counts, double* obj, void* ws, size_t ws_bytes,
                                       void* stream);
 FKM_API fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
-                                     const int32_t* counts, const float* prev, float* centers,
-                                     double* shift, void* ws, size_t ws_bytes, void* stream);
+                                     const double* counts, const float* prev, float* centers,
+                                     int32_t* counts_out, double* shift, void* ws,
+                                     size_t ws_bytes, void* stream);
 
 /* fkm_partial_update_host: the same shard step for a shard that stays in HOST
  * memory (pinned), as fkm_lloyd_host streams it: each chunk of chunk_rows
@@ -256,7 +260,7 @@ FKM_API fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
 FKM_API fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype,
                                            const void* x_host, const float* centers,
                                            int64_t chunk_rows, int32_t* ids, double* sums,
-                                           int32_t* counts, double* obj, void* ws,
+                                           double* counts, double* obj, void* ws,
                                            size_t ws_bytes, void* stream);
 
 /* Centring ("Flash-KMeans" GitHub README, section "Centre your data"):
@@ -272,6 +276,16 @@ FKM_API fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype
 FKM_API fkm_status fkm_centre_workspace_size(int B, int N, int D, size_t* bytes);
 FKM_API fkm_status fkm_centre(int B, int N, int D, int dtype, const void* x, float* mu,
                               void* x_out, void* ws, size_t ws_bytes, void* stream);
+
+/* The centroid side of the same recipe ("Flash-KMeans" GitHub README, section
+ * "Centre your data": cluster the centred points, then shift the centroids
+ * back by the mean): out[b,k,d] = fp32(centers[b,k,d] + sign * mu[b,d]), one
+ * IEEE fp32 addition (sign = +1, back to the original frame) or subtraction
+ * (sign = -1, initial centroids into the centred frame) per element.
+ * centers, out: device float32 [B, K, D] (out may be centers); mu: device
+ * float32 [B, D].  Async on `stream`. */
+FKM_API fkm_status fkm_shift_centroids(int B, int K, int D, const float* centers,
+                                       const float* mu, int sign, float* out, void* stream);
 
 /* Comparison point, NOT the method: the "standard" iteration the pages
  * measure against.  Assign materialises the full fp32 distance matrix
@@ -340,6 +354,22 @@ FKM_API fkm_status fkm_assign_noalloc(int B, int N, int K, int D, int dtype, con
  * Allocates nothing; call it on the stream of the fkm_assign_noalloc calls it
  * reports on. */
 FKM_API fkm_status fkm_assign_noalloc_status(void* stream);
+
+/* Instrumentation of the Sort-Inverse Update's atomics ("Flash-KMeans：快速且
+ * 内存高效精确K-Means聚类" summary, sections 前置知识 / argsort与分段规约 and
+ * 方法步骤详情 step (2): one atomic add per segment boundary, O((K + N/B_N) d)
+ * in all instead of O(N d)).  Reads the number of fp64 element atomics the
+ * segment sums of fkm_update / fkm_lloyd added into the workspace's cluster
+ * sums since the count was last reset (a zeroed workspace, the start of each
+ * fkm_lloyd call, or a call here with reset != 0), after waiting for `stream`.
+ * range_rows (optional) receives B_N, the sorted rows per segment-sum range
+ * that an update of n_rows = B*N points uses on the current device: runs that
+ * lie inside one range make no atomics, a run that crosses a range boundary
+ * makes D per range it touches.  ws: the workspace of those calls (its first
+ * 256 bytes hold the count).  Either output may be NULL. */
+FKM_API fkm_status fkm_segsum_stats(void* ws, size_t ws_bytes, int64_t n_rows, int reset,
+                                    unsigned long long* atomics, int* range_rows,
+                                    void* stream);
 
 /* Waits for `stream`, then reads and clears the workspace's status word:
  * FKM_OK, FKM_ERR_TIMEOUT, FKM_ERR_BAD_ID or FKM_ERR_INTERNAL. */

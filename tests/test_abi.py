@@ -95,9 +95,9 @@ def test_shard_calls_validate_before_any_launch(fkm):
     # fkm_partial_update: x is required
     assert L.fkm_partial_update(1, 16, 4, 64, 2, None, a, a, a, a, None, a, 1 << 19, None) == 1
     # fkm_finalize_sums: centers may not alias prev; the scratch must hold 256 + 8*B*K bytes
-    assert L.fkm_finalize_sums(1, 4, 64, a, a + 4096, a + 8192, a + 8192, None, a + 16384,
+    assert L.fkm_finalize_sums(1, 4, 64, a, a + 4096, a + 8192, a + 8192, None, None, a + 16384,
                                1024, None) == 1
-    assert L.fkm_finalize_sums(1, 4, 64, a, a + 4096, a + 8192, a + 12288, None, a + 16384,
+    assert L.fkm_finalize_sums(1, 4, 64, a, a + 4096, a + 8192, a + 12288, None, None, a + 16384,
                                200, None) == 4
     # fkm_partial_update_host: sums are required and 16-byte aligned; the host workspace
     # is sized by fkm_host_workspace_size
@@ -184,7 +184,8 @@ def test_binding_refuses_wrong_sizes_and_host_tensors(fkm):
                            torch.zeros(2, 4, dtype=torch.int32), ws=ws)
     with pytest.raises(ValueError, match="sums has shape"):
         fkm.fkm_finalize_sums(torch.zeros(2, 4, 8, dtype=torch.float64),
-                              torch.zeros(2, 4, dtype=torch.int32), c, torch.zeros(2, 4, 16), ws=ws)
+                              torch.zeros(2, 4, dtype=torch.float64), c, torch.zeros(2, 4, 16),
+                              ws=ws)
     with pytest.raises(ValueError, match="idx has shape"):
         fkm.fkm_argsort(torch.zeros(10, dtype=torch.int32), 4, torch.zeros(9, dtype=torch.int32),
                         ws=ws)

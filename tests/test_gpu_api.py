@@ -101,3 +101,19 @@ def test_class_train_on_host_data_streams_it():
     fkm.fkm_lloyd_host(xh.pin_memory(), c0t, 3, 0.0, 4096, ids, cen, cnt)
     assert torch.equal(km.labels_, ids)
     assert torch.equal(km.centroids, cen)
+
+
+@pytest.mark.parametrize("sign", [1, -1])
+def test_shift_centroids_is_one_fp32_operation(sign):
+    """fkm_shift_centroids: out = fp32(c + sign * mu) per batch, exactly the
+    single IEEE fp32 operation numpy performs; in place as well."""
+    rng = np.random.default_rng(3 + sign)
+    B, K, D = 3, 1000, 40
+    c = (rng.standard_normal((B, K, D)) * 100).astype(np.float32)
+    mu = (rng.standard_normal((B, D)) * 1e4).astype(np.float32)
+    ref = c + mu[:, None, :] if sign > 0 else c - mu[:, None, :]
+    ct = torch.from_numpy(c).cuda()
+    out = fkm.fkm_shift_centroids(ct, torch.from_numpy(mu).cuda(), sign)
+    assert np.array_equal(out.cpu().numpy(), ref)
+    fkm.fkm_shift_centroids(ct, torch.from_numpy(mu).cuda(), sign, out=ct)
+    assert np.array_equal(ct.cpu().numpy(), ref)

@@ -23,16 +23,17 @@ def test_shard_partials_add_up_to_the_whole_update(dtype, B, N, K, D, cuts):
     c = torch.from_numpy(c0).cuda()
     ids = torch.empty(B, N, dtype=torch.int32, device="cuda")
     fkm.fkm_assign(xt, c, ids)
-    sums = torch.zeros(B, K, D, dtype=torch.float64, device="cuda")
-    counts = torch.zeros(B, K, dtype=torch.int32, device="cuda")
-    obj = torch.zeros(B, dtype=torch.float64, device="cuda")
+    buf, sums, counts, obj = fkm.partial_buffers(B, K, D, "cuda")
     edges = (0,) + tuple(cuts) + (N,)
     for a, b in zip(edges[:-1], edges[1:]):
         fkm.fkm_partial_update(xt[:, a:b].contiguous(), ids[:, a:b].contiguous(), c, sums, counts,
                                obj)
     cen = torch.empty_like(c)
     shift = torch.empty(B, dtype=torch.float64, device="cuda")
-    fkm.fkm_finalize_sums(sums, counts, c, cen, shift)
+    cnt32 = torch.empty(B, K, dtype=torch.int32, device="cuda")
+    fkm.fkm_finalize_sums(sums, counts, c, cen, shift, counts_out=cnt32)
+    assert torch.equal(cnt32.double(), counts)
+    counts = cnt32
     check_update(x, dtype, ids.cpu().numpy(), c0, cen.cpu().numpy(), counts.cpu().numpy())
     whole = torch.empty_like(c)
     n_whole = torch.empty(B, K, dtype=torch.int32, device="cuda")
@@ -81,10 +82,8 @@ def test_host_shard_partials_match_device_partials(dtype, B, N, K, D, cut, chunk
     w = datagen.Workload("host-shards", B, N, D, K, dtype, K, sigma=0.5, iters=1, seed=N + D)
     x, xt, c0 = problem(w)
     c = torch.from_numpy(c0).cuda()
-    ref = [torch.zeros(B, K, D, dtype=torch.float64, device="cuda"),
-           torch.zeros(B, K, dtype=torch.int32, device="cuda"),
-           torch.zeros(B, dtype=torch.float64, device="cuda")]
-    got = [torch.zeros_like(t) for t in ref]
+    ref = list(fkm.partial_buffers(B, K, D, "cuda")[1:])
+    got = list(fkm.partial_buffers(B, K, D, "cuda")[1:])
     ids_ref = torch.empty(B, N, dtype=torch.int32, device="cuda")
     fkm.fkm_assign(xt, c, ids_ref)
     ids = torch.full((B, N), -1, dtype=torch.int32, device="cuda")
@@ -104,7 +103,8 @@ def test_host_shard_partials_match_device_partials(dtype, B, N, K, D, cut, chunk
     assert torch.allclose(got[2], ref[2], rtol=1e-6)
     cen = torch.empty_like(c)
     fkm.fkm_finalize_sums(got[0], got[1], c, cen)
-    check_update(x, dtype, ids.cpu().numpy(), c0, cen.cpu().numpy(), got[1].cpu().numpy())
+    check_update(x, dtype, ids.cpu().numpy(), c0, cen.cpu().numpy(),
+                 got[1].cpu().numpy().astype(np.int64))
 
 
 def test_sharded_loop_from_host_matches_lloyd_host():

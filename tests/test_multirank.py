@@ -34,10 +34,11 @@ def _rank_main(rank, world, port, q):
         digest = float(datagen.widen(x, w.dtype).astype(np.float64).sum())
         # the sharded loop's all-reduce of partial sums / counts / objectives
         import exact_means_clustering_b200 as fkm
-        sums = torch.full((2, 3, 4), float(rank + 1), dtype=torch.float64)
-        counts = torch.full((2, 3), rank + 1, dtype=torch.int32)
-        obj = torch.tensor([0.5 * (rank + 1), 1.0], dtype=torch.float64)
-        fkm.reduce_partials((sums, counts, obj))
+        buf, sums, counts, obj = fkm.partial_buffers(2, 3, 4, "cpu")
+        sums.fill_(float(rank + 1))
+        counts.fill_(float(rank + 1))
+        obj.copy_(torch.tensor([0.5 * (rank + 1), 1.0], dtype=torch.float64))
+        fkm.reduce_partials((buf,))      # one collective for all three
         reduced = (float(sums.sum()), int(counts.sum()), obj.tolist())
         dist.barrier()
         q.put((rank, t, n, w.seed, digest, reduced))
@@ -75,14 +76,15 @@ def _cpu_steps(x):
             d = torch.cdist(x[b], c[b].double()) ** 2
             dmin, ids = d.min(1)
             sums[b].index_add_(0, ids, x[b])
-            counts[b] += torch.bincount(ids, minlength=c.shape[1]).to(torch.int32)
+            counts[b] += torch.bincount(ids, minlength=c.shape[1]).double()
             obj[b] += dmin.sum()
 
-    def finalize(sums, counts, c, nxt, shift):
-        n = counts.unsqueeze(-1).double()
+    def finalize(sums, counts, c, nxt, shift, counts_out):
+        n = counts.unsqueeze(-1)
         new = torch.where(n > 0, sums / n.clamp(min=1), c.double())
         nxt.copy_(new.float())
         shift.copy_(((nxt.double() - c.double()) ** 2).sum((1, 2)))
+        counts_out.copy_(counts.to(torch.int32))
 
     return partials, finalize
 
@@ -140,3 +142,52 @@ def test_sharded_loop_two_gloo_ranks_match_one_rank(tol):
         assert np.allclose(c, c1.numpy(), rtol=1e-6, atol=1e-6)
         assert np.allclose(o, o1.numpy(), rtol=1e-9)
     assert np.array_equal(out[0][1], out[1][1])   # every rank forms the same centroids
+
+
+# ---- the class API's sharded fit: shard layout and label gathering over two
+# ranks (the GPU steps replaced by the CPU stand-ins above)
+def _class_rank(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import exact_means_clustering_b200 as fkm
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        x, c0 = _problem(N=601)            # an odd N: the shards differ by one row
+        N = x.shape[1]
+        r0, r1 = fkm.shard_rows(N, rank, world)
+        c, counts, obj, n_iter = fkm.sharded_loop(*_cpu_steps(x[:, r0:r1]), c0.clone(), 30)
+        # the labels of the final centroids, per shard, gathered in row order
+        ids = torch.cdist(x[:, r0:r1], c.double()).argmin(-1).to(torch.int32)
+        full = fkm.gather_shard_ids(ids, N)
+        q.put((rank, full.numpy(), c.numpy(), counts.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_class_sharding_two_gloo_ranks():
+    """shard_rows covers every row once, the two ranks reach the one-rank
+    centroids and counts, and gather_shard_ids gives every rank the labels
+    of all points in row order."""
+    sys.path.insert(0, ROOT)
+    import exact_means_clustering_b200 as fkm
+    N, world = 601, 2
+    spans = [fkm.shard_rows(N, r, world) for r in range(world)]
+    assert spans == [(0, 301), (301, 601)]
+    assert [fkm.shard_rows(10, r, 4) for r in range(4)] == [(0, 3), (3, 6), (6, 8), (8, 10)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_class_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    x, c0 = _problem(N=N)
+    c1, k1, _, _ = fkm.sharded_loop(*_cpu_steps(x), c0.clone(), 30)
+    want = torch.cdist(x, c1.double()).argmin(-1).to(torch.int32).numpy()
+    for rank, full, c, counts in out:
+        assert np.allclose(c, c1.numpy(), rtol=1e-6, atol=1e-6)
+        assert np.array_equal(counts, k1.numpy())
+        assert np.array_equal(full, want)
