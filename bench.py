@@ -548,6 +548,9 @@ def main():
     ap.add_argument("--sharded", action="store_true",
                     help="one problem split over the ranks' GPUs (strong scaling)")
     ap.add_argument("--oracle-iters", type=int, default=10)
+    ap.add_argument("--points", type=int, default=0,
+                    help="a smaller case of the workload for profiling: N points per batch "
+                         "(same recipe; the line's config names the reduced size)")
     ap.add_argument("--metric", default="euclid", choices=["euclid", "dot", "cosine"],
                     help="similarity of the clustering (dot and cosine k-means: fkm_lloyd_metric)")
     args = ap.parse_args()
@@ -556,6 +559,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = datagen.CONFIGS[args.config]
+    if args.points > 0:
+        w = w.scaled(N=args.points, name=f"{w.name}_reduced_N{args.points}")
     if args.metric != "euclid" and (w.host_resident or args.sharded or args.impl == "reference"):
         print("bench.py: --metric dot/cosine runs on device-resident workloads with --impl fkm "
               "only (the host-streamed and sharded runs are Euclidean)", file=sys.stderr)

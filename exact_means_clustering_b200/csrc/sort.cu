@@ -95,17 +95,23 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_upsweep(KeySrc s, int64_t 
     (&h[0][0])[i] = 0;
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * SORT_TILE;
-#pragma unroll 4
+  // every load of the tile first, so they are in flight together; the
+  // shared-memory atomics after them would otherwise keep each load behind
+  // the previous item's update
+  int digit[SORT_ITEMS];
+#pragma unroll
   for (int it = 0; it < SORT_ITEMS; ++it) {
     const int64_t j = base + (int64_t)it * SORT_THREADS + threadIdx.x;
-    int digit = RADIX_BINS;  // out of range: matches nothing real
+    digit[it] = RADIX_BINS;  // out of range: matches nothing real
     if (j < n) {
       int32_t key, val;
       load_key<kFirst>(s, j, key, val);
-      digit = (key >> shift) & (RADIX_BINS - 1);
+      digit[it] = (key >> shift) & (RADIX_BINS - 1);
     }
-    if (digit < RADIX_BINS) atomicAdd(&h[warp][digit], 1u);
   }
+#pragma unroll
+  for (int it = 0; it < SORT_ITEMS; ++it)
+    if (digit[it] < RADIX_BINS) atomicAdd(&h[warp][digit[it]], 1u);
   __syncthreads();
   for (int d = threadIdx.x; d < RADIX_BINS; d += SORT_THREADS) {
     uint32_t t = 0;
@@ -187,7 +193,7 @@ __global__ void __launch_bounds__(kScanBlock) scan_apply(uint32_t* data, int64_t
 }
 
 template <bool kFirst>
-__global__ void __launch_bounds__(SORT_THREADS) radix_downsweep(KeySrc s, int64_t n, int shift,
+__global__ void __launch_bounds__(SORT_THREADS, 2) radix_downsweep(KeySrc s, int64_t n, int shift,
                                                                 int n_tiles,
                                                                 const uint32_t* __restrict__ hist,
                                                                 int32_t* __restrict__ keys_out,
@@ -208,8 +214,9 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_downsweep(KeySrc s, int64_
   const int64_t base = (int64_t)blockIdx.x * SORT_TILE + (int64_t)warp * PER_WARP;
   const unsigned lt_mask = (1u << lane) - 1u;
   int32_t key[SORT_ITEMS], val[SORT_ITEMS];
-  uint32_t rank[SORT_ITEMS];
-  int dig[SORT_ITEMS];
+  uint32_t dr[SORT_ITEMS];   // digit (9 bits) | rank inside the warp's items << 9
+  // every load first, so they are in flight together (the ranking below
+  // goes through shared memory item by item)
 #pragma unroll
   for (int r = 0; r < SORT_ITEMS; ++r) {
     const int64_t j = base + r * 32 + lane;
@@ -220,10 +227,14 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_downsweep(KeySrc s, int64_
       load_key<kFirst>(s, j, key[r], val[r]);
       d = (key[r] >> shift) & (RADIX_BINS - 1);
     }
-    dig[r] = d;
+    dr[r] = (uint32_t)d;
+  }
+#pragma unroll
+  for (int r = 0; r < SORT_ITEMS; ++r) {
+    const int d = (int)dr[r];
     const unsigned peers = warp_peers((unsigned)d, 9);   // digits 0..RADIX_BINS
     const uint32_t before = cnt[warp][d];
-    rank[r] = before + __popc(peers & lt_mask);
+    dr[r] = (uint32_t)d | ((before + __popc(peers & lt_mask)) << 9);
     __syncwarp();
     if (lane == __ffs(peers) - 1) cnt[warp][d] = before + __popc(peers);
     __syncwarp();
@@ -246,8 +257,9 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_downsweep(KeySrc s, int64_
   __syncthreads();
 #pragma unroll
   for (int r = 0; r < SORT_ITEMS; ++r) {
-    if (dig[r] < RADIX_BINS) {
-      const uint32_t lp = tdo[dig[r]] + cnt[warp][dig[r]] + rank[r];
+    const int d = (int)(dr[r] & 511u);
+    if (d < RADIX_BINS) {
+      const uint32_t lp = tdo[d] + cnt[warp][d] + (dr[r] >> 9);
       sk[lp] = key[r];
       sv[lp] = val[r];
     }

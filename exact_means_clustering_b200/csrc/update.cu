@@ -31,14 +31,31 @@
 namespace fkm {
 namespace {
 
+// Four sorted keys per thread (one 16-byte load; skeys is 16-byte aligned),
+// compared with their neighbours: a key that differs from the one before it
+// starts its run, one that differs from the one after it ends it.
 __global__ void seg_bounds_kernel(const int32_t* __restrict__ skeys, int64_t n, int BK,
                                   int32_t* __restrict__ segstart, int32_t* __restrict__ segend) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const int32_t k = skeys[i];
-  if (k < 0 || k >= BK) return;  // sentinel of a rejected id
-  if (i == 0 || skeys[i - 1] != k) segstart[k] = (int32_t)i;
-  if (i == n - 1 || skeys[i + 1] != k) segend[k] = (int32_t)(i + 1);
+  const int64_t i0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i0 >= n) return;
+  int32_t k[6];   // k[0] the key before i0, k[1..4] keys i0..i0+3, k[5] the one after
+  if (i0 + 4 <= n) {
+    const int4 v = *reinterpret_cast<const int4*>(skeys + i0);
+    k[1] = v.x; k[2] = v.y; k[3] = v.z; k[4] = v.w;
+  } else {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) k[1 + t] = i0 + t < n ? skeys[i0 + t] : -1;
+  }
+  k[0] = i0 > 0 ? skeys[i0 - 1] : -1;
+  k[5] = i0 + 4 < n ? skeys[i0 + 4] : -1;
+#pragma unroll
+  for (int t = 1; t <= 4; ++t) {
+    const int64_t i = i0 + t - 1;
+    const int32_t key = k[t];
+    if (i >= n || key < 0 || key >= BK) continue;  // past the end, or a rejected id
+    if (k[t - 1] != key) segstart[key] = (int32_t)i;
+    if (k[t + 1] != key) segend[key] = (int32_t)(i + 1);
+  }
 }
 
 // Rows longer than 512 bytes are summed in slabs of columns, one launch per
@@ -142,11 +159,13 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
   if (g == 0 && lane_has_vec) {
     const int64_t col0 = (int64_t)sub * E;
     if (interior) {
-      const double n = (double)nk;
+      // one fp64 reciprocal per run (its error, below 2^-52 relative, is
+      // far below the fp32 rounding that follows)
+      const double rn = 1.0 / (double)nk;
       float* c = p.centers + (int64_t)key * p.Dfull + col0;
 #pragma unroll
       for (int e = 0; e < E; ++e)
-        if (col0 + e < p.D) c[e] = (float)(acc[e] / n);
+        if (col0 + e < p.D) c[e] = (float)(acc[e] * rn);
     } else {
       double* sd = p.sums64 + (int64_t)key * p.Dfull + col0;
 #pragma unroll
@@ -350,6 +369,11 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     flush_run<E, LPR>(p, cur, g, sub, lane_has_vec, !p.accumulate_all && !crossing,
                       end - run_start, acc);
   };
+  // this lane's piece of the current batch's mean centroid (16-bit points),
+  // loaded when the batch changes
+  float2 m2[E / 2];
+#pragma unroll
+  for (int e = 0; e < E / 2; ++e) m2[e] = make_float2(0.0f, 0.0f);
   auto start_run = [&](int kg, int i) {
     cur = kg;
     ++run;
@@ -365,18 +389,18 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
       }
       obj = 0.0;
       cur_b = b;
+      if (p.oa.m && lane_has_vec) {
+        const float2* mb =
+            reinterpret_cast<const float2*>(p.oa.m + (int64_t)b * p.Dfull) + sub * (E / 2);
+#pragma unroll
+        for (int e = 0; e < E / 2; ++e) m2[e] = mb[e];
+      }
     }
     if (lane_has_vec) {
       float2 c2[E / 2];
       Vec<DT>::widen2(chat_next, c2);
-      if (p.oa.m) {   // the batch's mean centroid: a few KB, cache-resident
-        const float2* mb =
-            reinterpret_cast<const float2*>(p.oa.m + (int64_t)b * p.Dfull) + sub * (E / 2);
 #pragma unroll
-        for (int e = 0; e < E / 2; ++e) c2[e] = __fadd2_rn(c2[e], mb[e]);
-      }
-#pragma unroll
-      for (int e = 0; e < E / 2; ++e) chat2[e] = c2[e];
+      for (int e = 0; e < E / 2; ++e) chat2[e] = __fadd2_rn(c2[e], m2[e]);
     }
     prefetch_chat(run + 1);
   };
@@ -784,7 +808,8 @@ fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* s
   FKM_CUDA_TRY(cudaMemsetAsync(segstart, 0, sizeof(int32_t) * (size_t)BK, st));
   FKM_CUDA_TRY(cudaMemsetAsync(segend, 0, sizeof(int32_t) * (size_t)BK, st));
   if (n > 0) {
-    seg_bounds_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(skeys, n, BK, segstart, segend);
+    seg_bounds_kernel<<<(unsigned)ceil_div(n, 1024), 256, 0, st>>>(skeys, n, BK, segstart,
+                                                                  segend);
     note_launch();
     FKM_CUDA_TRY(cudaGetLastError());
   }
