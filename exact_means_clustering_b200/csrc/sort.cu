@@ -192,33 +192,44 @@ __global__ void __launch_bounds__(kScanBlock) scan_apply(uint32_t* data, int64_t
   }
 }
 
+// The downsweep runs DS_THREADS threads of DS_ITEMS keys on the same
+// SORT_TILE-key tile as the upsweep: with half the per-thread state of a
+// 256-thread block, twice as many warps stay resident to cover the loads.
+constexpr int DS_THREADS = 2 * SORT_THREADS;
+constexpr int DS_ITEMS = SORT_TILE / DS_THREADS;
+static_assert(DS_THREADS >= RADIX_BINS, "one thread per digit in the digit scan");
+
 template <bool kFirst>
-__global__ void __launch_bounds__(SORT_THREADS, 2) radix_downsweep(KeySrc s, int64_t n, int shift,
-                                                                int n_tiles,
-                                                                const uint32_t* __restrict__ hist,
-                                                                int32_t* __restrict__ keys_out,
-                                                                int32_t* __restrict__ vals_out) {
-  constexpr int NW = SORT_THREADS / 32;
-  constexpr int PER_WARP = SORT_TILE / NW;  // 512 consecutive keys per warp
-  __shared__ uint32_t cnt[NW][RADIX_BINS + 1];
+__global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64_t n, int shift,
+                                                              int n_tiles,
+                                                              const uint32_t* __restrict__ hist,
+                                                              int32_t* __restrict__ keys_out,
+                                                              int32_t* __restrict__ vals_out) {
+  constexpr int NW = DS_THREADS / 32;
+  constexpr int PER_WARP = SORT_TILE / NW;  // 256 consecutive keys per warp
+  static_assert(NW * (RADIX_BINS + 1) <= 2 * SORT_TILE, "the counters fit the staging area");
+  // the per-warp digit counters are only needed until every key knows its
+  // place in the tile, so they share memory with the staged keys and values
+  __shared__ int32_t stage[2 * SORT_TILE];
   __shared__ uint32_t tdo[RADIX_BINS];      // tile-local exclusive digit offsets
   __shared__ uint32_t gofs[RADIX_BINS];     // global base of (digit, this tile)
   __shared__ uint32_t sw[32];
-  __shared__ int32_t sk[SORT_TILE];
-  __shared__ int32_t sv[SORT_TILE];
+  int32_t* sk = stage;
+  int32_t* sv = stage + SORT_TILE;
+  uint32_t (*cnt)[RADIX_BINS + 1] = reinterpret_cast<uint32_t (*)[RADIX_BINS + 1]>(stage);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < NW * (RADIX_BINS + 1); i += SORT_THREADS) (&cnt[0][0])[i] = 0;
+  for (int i = threadIdx.x; i < NW * (RADIX_BINS + 1); i += DS_THREADS) (&cnt[0][0])[i] = 0;
   __syncthreads();
 
   const int64_t base = (int64_t)blockIdx.x * SORT_TILE + (int64_t)warp * PER_WARP;
   const unsigned lt_mask = (1u << lane) - 1u;
-  int32_t key[SORT_ITEMS], val[SORT_ITEMS];
-  uint32_t dr[SORT_ITEMS];   // digit (9 bits) | rank inside the warp's items << 9
+  int32_t key[DS_ITEMS], val[DS_ITEMS];
+  uint32_t dr[DS_ITEMS];   // digit (9 bits) | rank inside the warp's items << 9
   // every load first, so they are in flight together (the ranking below
   // goes through shared memory item by item)
 #pragma unroll
-  for (int r = 0; r < SORT_ITEMS; ++r) {
+  for (int r = 0; r < DS_ITEMS; ++r) {
     const int64_t j = base + r * 32 + lane;
     int d = RADIX_BINS;  // keys past the end use an extra bin and are never written
     key[r] = 0;
@@ -230,7 +241,7 @@ __global__ void __launch_bounds__(SORT_THREADS, 2) radix_downsweep(KeySrc s, int
     dr[r] = (uint32_t)d;
   }
 #pragma unroll
-  for (int r = 0; r < SORT_ITEMS; ++r) {
+  for (int r = 0; r < DS_ITEMS; ++r) {
     const int d = (int)dr[r];
     const unsigned peers = warp_peers((unsigned)d, 9);   // digits 0..RADIX_BINS
     const uint32_t before = cnt[warp][d];
@@ -240,34 +251,45 @@ __global__ void __launch_bounds__(SORT_THREADS, 2) radix_downsweep(KeySrc s, int
     __syncwarp();
   }
   __syncthreads();
-  // per digit: exclusive prefix over warps, tile total, tile-local digit offsets
+  // per digit (threads 0..255): exclusive prefix over warps, tile total,
+  // tile-local digit offsets; the other threads add zeros to the block scan
   {
-    const int d = threadIdx.x;  // SORT_THREADS == RADIX_BINS
+    const int d = threadIdx.x;
     uint32_t run = 0;
+    if (d < RADIX_BINS) {
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      uint32_t c = cnt[w][d];
-      cnt[w][d] = run;
-      run += c;
+      for (int w = 0; w < NW; ++w) {
+        uint32_t c = cnt[w][d];
+        cnt[w][d] = run;
+        run += c;
+      }
     }
     uint32_t ex = block_exclusive_scan(run, sw, nullptr);
-    tdo[d] = ex;
-    gofs[d] = hist[(size_t)d * n_tiles + blockIdx.x];
+    if (d < RADIX_BINS) {
+      tdo[d] = ex;
+      gofs[d] = hist[(size_t)d * n_tiles + blockIdx.x];
+    }
   }
   __syncthreads();
+  // every key's place in the tile (while the counters are still there) ...
 #pragma unroll
-  for (int r = 0; r < SORT_ITEMS; ++r) {
+  for (int r = 0; r < DS_ITEMS; ++r) {
     const int d = (int)(dr[r] & 511u);
-    if (d < RADIX_BINS) {
-      const uint32_t lp = tdo[d] + cnt[warp][d] + (dr[r] >> 9);
-      sk[lp] = key[r];
-      sv[lp] = val[r];
+    dr[r] = d < RADIX_BINS ? tdo[d] + cnt[warp][d] + (dr[r] >> 9) : 0xffffffffu;
+  }
+  __syncthreads();
+  // ... then the keys staged there in sorted order
+#pragma unroll
+  for (int r = 0; r < DS_ITEMS; ++r) {
+    if (dr[r] != 0xffffffffu) {
+      sk[dr[r]] = key[r];
+      sv[dr[r]] = val[r];
     }
   }
   __syncthreads();
   const int64_t tile0 = (int64_t)blockIdx.x * SORT_TILE;
   const int valid = (int)((n - tile0) < SORT_TILE ? (n - tile0) : SORT_TILE);
-  for (int j = threadIdx.x; j < valid; j += SORT_THREADS) {
+  for (int j = threadIdx.x; j < valid; j += DS_THREADS) {
     const int32_t k = sk[j];
     const int d = (k >> shift) & (RADIX_BINS - 1);
     const int64_t g = (int64_t)gofs[d] + (j - (int64_t)tdo[d]);
@@ -630,14 +652,14 @@ fkm_status launch_argsort_ids(SortArgs& a, cudaStream_t st) {
       s.vals = nullptr;
       radix_upsweep<true><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist);
       FKM_TRY(device_scan(a.hist, hlen, a.hist_part, st));
-      radix_downsweep<true><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist,
+      radix_downsweep<true><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist,
                                                               kout[0], vout[0]);
     } else {
       s.keys = kout[(p - 1) & 1];
       s.vals = vout[(p - 1) & 1];
       radix_upsweep<false><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist);
       FKM_TRY(device_scan(a.hist, hlen, a.hist_part, st));
-      radix_downsweep<false><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist,
+      radix_downsweep<false><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist,
                                                                kout[p & 1], vout[p & 1]);
     }
     FKM_CUDA_TRY(cudaGetLastError());
