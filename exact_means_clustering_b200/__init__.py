@@ -62,6 +62,7 @@ _SIG = {
     "fkm_segsum_stats": ([_P, _Z, _L, _I, ctypes.POINTER(ctypes.c_ulonglong),
                           ctypes.POINTER(_I), _P], _I),
     "fkm_profile": ([_I], _I),
+    "fkm_set_verbose": ([_I], _I),
     "fkm_profile_read": ([_P, ctypes.POINTER(ctypes.c_longlong), _I], _I),
     "fkm_kernel_launches": ([], ctypes.c_longlong),
     "fkm_status_string": ([_I], ctypes.c_char_p),
@@ -672,6 +673,11 @@ def fkm_sync_status(ws, stream=None):
     _check("fkm_sync_status", lib().fkm_sync_status(wp, wn, _stream(stream)))
 
 
+def fkm_set_verbose(level) -> None:
+    """Per-iteration progress lines of fkm_lloyd on stderr (level > 0)."""
+    _check("fkm_set_verbose", lib().fkm_set_verbose(int(level)))
+
+
 def fkm_profile(enable: bool) -> None:
     _check("fkm_profile", lib().fkm_profile(1 if enable else 0))
 
@@ -700,12 +706,13 @@ def fkm_version() -> str:
 # ---------------------------------------------------------------- wrapper
 def batch_kmeans(x: torch.Tensor, n_clusters: int, max_iters: int = 100, tol: float = 0.0,
                  init_centroids: torch.Tensor | None = None, seed: int = 0,
-                 metric: str = "euclid"):
+                 metric: str = "euclid", verbose: bool = False):
     """Exact batched Lloyd k-means under metric 'euclid', 'dot' or 'cosine'
     (fkm.h, fkm_metric).  x: [B, N, D] (or [N, D]) CUDA tensor in float32 /
     float16 / bfloat16.  Returns (cluster_ids int32 [B, N], centers float32
     [B, K, D], n_iter).  Default initial centroids: per batch, the points at
-    the first K positions of a seeded random permutation."""
+    the first K positions of a seeded random permutation.  verbose prints one
+    progress line per iteration (fkm_set_verbose)."""
     squeeze = x.dim() == 2
     if squeeze:
         x = x.unsqueeze(0)
@@ -722,20 +729,27 @@ def batch_kmeans(x: torch.Tensor, n_clusters: int, max_iters: int = 100, tol: fl
     ids = torch.empty(B, N, dtype=torch.int32, device=dev)
     centers = torch.empty(B, K, D, dtype=torch.float32, device=dev)
     counts = torch.empty(B, K, dtype=torch.int32, device=dev)
-    if _metric(metric) == METRICS["euclid"]:
-        n_iter = fkm_lloyd(x, init, max_iters, tol, ids, centers, counts)
-    else:
-        n_iter = fkm_lloyd_metric(x, init, max_iters, tol, ids, centers, counts, metric)
+    if verbose:
+        fkm_set_verbose(1)
+    try:
+        if _metric(metric) == METRICS["euclid"]:
+            n_iter = fkm_lloyd(x, init, max_iters, tol, ids, centers, counts)
+        else:
+            n_iter = fkm_lloyd_metric(x, init, max_iters, tol, ids, centers, counts, metric)
+    finally:
+        if verbose:
+            fkm_set_verbose(0)
     if squeeze:
         return ids[0], centers[0], n_iter
     return ids, centers, n_iter
 
 
 def batch_kmeans_Euclid(x: torch.Tensor, n_clusters: int, max_iters: int = 100, tol: float = 0.0,
-                        init_centroids: torch.Tensor | None = None, seed: int = 0):
+                        init_centroids: torch.Tensor | None = None, seed: int = 0,
+                        verbose: bool = False):
     """Exact batched Lloyd k-means (Euclidean), the README's call shape; see
     batch_kmeans."""
-    return batch_kmeans(x, n_clusters, max_iters, tol, init_centroids, seed, "euclid")
+    return batch_kmeans(x, n_clusters, max_iters, tol, init_centroids, seed, "euclid", verbose)
 
 
 # ---------------------------------------------------------------- class API

@@ -42,6 +42,9 @@ int num_sms() {
 }
 
 static std::atomic<long long> g_launches{0};
+// progress output of the Lloyd loops (fkm_set_verbose)
+static std::atomic<int> g_verbose{0};
+int verbose_level() { return g_verbose.load(); }
 void note_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 // ---- stage timing (fkm_profile): CUDA events around each stage of every
@@ -538,7 +541,8 @@ static fkm_status lloyd_impl(int metric, int B, int N, int K, int D, int dtype, 
   }
   cudaEvent_t* ev_base = prof ? g_prof.ev.data() : nullptr;
   int done = 0;
-  if (tol == 0.0f) {
+  // verbose runs take the stepped loop, which reads every iteration's results
+  if (tol == 0.0f && g_verbose.load() == 0) {
     // every iteration runs: replay one captured graph of the whole loop
     int dev = 0;
     cudaGetDevice(&dev);
@@ -595,12 +599,26 @@ static fkm_status lloyd_impl(int metric, int B, int N, int K, int D, int dtype, 
     FKM_CUDA_TRY(cudaGraphLaunch(hit->exec, st));
     done = max_iters;
   } else {
+    // verbose: the objective of every iteration's assignment is reported, in
+    // the caller's buffer or, without one, in spare workspace doubles
+    const bool verbose = g_verbose.load() > 0;
+    double* obj = inertia ? inertia : (verbose ? shift_dev + B : nullptr);
+    std::vector<double> host_obj(verbose ? (size_t)B : 0);
     for (int t = 0; t < max_iters; ++t) {
-      FKM_TRY(lloyd_iterations(w, x, 1, ids, counts, inertia, shift_dev, true, t, st, ev_base));
+      FKM_TRY(lloyd_iterations(w, x, 1, ids, counts, obj, shift_dev, true, t, st, ev_base));
       double mx = 0.0;
       FKM_CUDA_TRY(cudaMemcpyAsync(&mx, w.max_shift(), sizeof(double), cudaMemcpyDeviceToHost, st));
+      if (verbose)
+        FKM_CUDA_TRY(cudaMemcpyAsync(host_obj.data(), obj, sizeof(double) * B,
+                                     cudaMemcpyDeviceToHost, st));
       FKM_CUDA_TRY(cudaStreamSynchronize(st));
       done = t + 1;
+      if (verbose) {
+        double total = 0.0;
+        for (double v : host_obj) total += v;
+        fprintf(stderr, "fkm_lloyd: iteration %d/%d  objective %.9g (sum over %d batches)  "
+                "max shift %.6g\n", t + 1, max_iters, total, B, mx);
+      }
       if (mx < (double)tol) break;
     }
   }
@@ -654,6 +672,11 @@ fkm_status fkm_lloyd_metric(int B, int N, int K, int D, int dtype, int metric, c
                             void* ws, size_t ws_bytes, void* stream) {
   return lloyd_impl(metric, B, N, K, D, dtype, x, init_centers, max_iters, tol, ids, centers,
                     counts, objective, n_iter, ws, ws_bytes, stream);
+}
+
+fkm_status fkm_set_verbose(int level) {
+  g_verbose = level > 0 ? 1 : 0;
+  return FKM_OK;
 }
 
 fkm_status fkm_profile(int enable) {

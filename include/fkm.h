@@ -301,6 +301,15 @@ FKM_API fkm_status fkm_baseline_update(int B, int N, int K, int D, int dtype, co
                                const int32_t* ids, const float* prev_centers, float* centers,
                                int32_t* counts, void* ws, size_t ws_bytes, void* stream);
 
+/* Progress output of the Lloyd loops ("Flash-KMeans" GitHub README, section
+ * "Usage": the verbose argument of batch_kmeans_Euclid).  With level > 0,
+ * fkm_lloyd and fkm_lloyd_metric run their stepped loop (also when tol = 0)
+ * and print one line per iteration to stderr: the objective of that
+ * iteration's assignment summed over the batches, and the largest per-batch
+ * centroid shift.  Results are unchanged; the stepped loop syncs every
+ * iteration.  Process-wide; level 0 (the default) turns it off. */
+FKM_API fkm_status fkm_set_verbose(int level);
+
 /* Stage timing of fkm_lloyd (tracing).  While enabled, fkm_lloyd records CUDA
  * events on its stream (inside its captured graph too) around each stage of
  * every iteration; fkm_profile_read returns the accumulated milliseconds per

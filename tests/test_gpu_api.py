@@ -117,3 +117,33 @@ def test_shift_centroids_is_one_fp32_operation(sign):
     assert np.array_equal(out.cpu().numpy(), ref)
     fkm.fkm_shift_centroids(ct, torch.from_numpy(mu).cuda(), sign, out=ct)
     assert np.array_equal(ct.cpu().numpy(), ref)
+
+
+def test_verbose_progress_lines(capfd):
+    """fkm_set_verbose: one progress line per iteration on stderr (README
+    "Usage", verbose), the same results as a quiet run, and the last line's
+    objective is the loop's reported objective."""
+    w = datagen.CONFIGS[2].scaled(B=2, N=3000, K=100, iters=3)
+    x, xt, c0 = problem(w)
+    c0t = torch.from_numpy(c0).cuda()
+    outs = []
+    for verbose in (0, 1):
+        ids = torch.empty(w.B, w.N, dtype=torch.int32, device="cuda")
+        cen = torch.empty(w.B, w.K, w.D, device="cuda")
+        cnt = torch.empty(w.B, w.K, dtype=torch.int32, device="cuda")
+        obj = torch.empty(w.B, dtype=torch.float64, device="cuda")
+        fkm.fkm_set_verbose(verbose)
+        try:
+            n = fkm.fkm_lloyd(xt, c0t, 3, 0.0, ids, cen, cnt, obj)
+        finally:
+            fkm.fkm_set_verbose(0)
+        outs.append((n, ids, cen, cnt, obj))
+    err = capfd.readouterr().err
+    lines = [l for l in err.splitlines() if l.startswith("fkm_lloyd: iteration")]
+    assert [l.split()[2] for l in lines] == ["1/3", "2/3", "3/3"]
+    (n0, i0, c_0, k0, o0), (n1, i1, c_1, k1, o1) = outs
+    assert n0 == n1 == 3
+    assert torch.equal(i0, i1) and torch.equal(k0, k1)
+    assert torch.allclose(c_0, c_1, rtol=1e-6, atol=1e-7)
+    printed = float(lines[-1].split("objective")[1].split()[0])
+    assert abs(printed - o1.sum().item()) <= 1e-6 * abs(printed)
