@@ -289,9 +289,9 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   int32_t* segend = w.at<int32_t>(L.segend);
   if (L.count_sort) {
     FKM_TRY(launch_count_sort_ids(s, L.B, segstart, segend, st, ids_valid));
-  } else {
+  } else {   // the segment sums write the bounds
     FKM_TRY(launch_argsort_ids(s, st));
-    FKM_TRY(launch_seg_bounds(s.keys_out, L.n_sort, BK, segstart, segend, st));
+    FKM_TRY(clear_seg_bounds(BK, segstart, segend, st));
   }
   if (ev) FKM_TRY(record_stage(ev[2], st));
   const bool euclid = L.metric == FKM_METRIC_EUCLID;
@@ -301,7 +301,8 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   // from the cluster sums in the finalize step
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK,
                         w.at<double>(L.sums64), next, false,
-                        obj_args(w, prev, euclid ? obj : nullptr), st, range, w.atomics()));
+                        obj_args(w, prev, euclid ? obj : nullptr), st, range, w.atomics(),
+                        L.count_sort ? nullptr : segstart, L.count_sort ? nullptr : segend));
   if (ev) FKM_TRY(record_stage(ev[3], st));
   if (euclid) {
     FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64),

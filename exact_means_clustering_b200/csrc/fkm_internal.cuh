@@ -150,8 +150,6 @@ fkm_status launch_count_sort_ids(SortArgs& a, int B, int32_t* segstart, int32_t*
                                  cudaStream_t st, bool ids_valid = false);
 fkm_status count_sort_prepare();
 
-fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
-                             int32_t* segend, cudaStream_t st);
 // Objective of the assignment being summed against c_hat, the centroid the
 // assign step measured against: m + q(c - m) for 16-bit points (chat = the
 // q(c - m) rows [B][Kp][D], m = the per-batch mean centroid), the fp32
@@ -167,10 +165,14 @@ struct ObjArgs {
 };
 // atomics (optional): incremented by the number of fp64 element atomics the
 // segment sums add into sums64 (D per flush of a run that crosses a range).
+// segstart / segend (optional, cleared by clear_seg_bounds first): the
+// segment bounds of the sorted keys are written by the same pass.
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
                          bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range = 0,
-                         unsigned long long* atomics = nullptr);
+                         unsigned long long* atomics = nullptr, int32_t* segstart = nullptr,
+                         int32_t* segend = nullptr);
+fkm_status clear_seg_bounds(int BK, int32_t* segstart, int32_t* segend, cudaStream_t st);
 // Rows per warp range of the segment sums for n sorted rows: SEG_RANGE for
 // large n, fewer (down to 32) when n is small, so a small problem still
 // spreads over many warps.  finalize must be given the same value.

@@ -323,7 +323,7 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
         FKM_TRY(launch_argsort_ids(so, st));
         int32_t* segstart = static_cast<int32_t*>(at(L.segstart));
         int32_t* segend = static_cast<int32_t*>(at(L.segend));
-        FKM_TRY(launch_seg_bounds(so.keys_out, rows, K, segstart, segend, st));
+        FKM_TRY(clear_seg_bounds(K, segstart, segend, st));   // the segment sums write them
         ObjArgs oa;
         oa.K = K;
         oa.obj = inertia ? inertia + b : nullptr;
@@ -336,7 +336,8 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
           oa.m = mvec + (size_t)b * D;
         }
         FKM_TRY(launch_segsum(xb, dtype, D, so.keys_out, so.vals_out, rows, K,
-                              sums64 + (size_t)b * K * D, nullptr, true, oa, st));
+                              sums64 + (size_t)b * K * D, nullptr, true, oa, st, 0, nullptr,
+                              segstart, segend));
         if (part)
           accumulate_counts_kernel<double><<<(unsigned)ceil_div(K, 256), 256, 0, st>>>(
               segstart, segend, K, part->counts + (size_t)b * K);

@@ -118,9 +118,9 @@ fkm_status shard_partial_update(const Layout& L, const void* x, const int32_t* i
   int32_t* segend = static_cast<int32_t*>(at(L.segend));
   if (L.count_sort) {
     FKM_TRY(launch_count_sort_ids(s, L.B, segstart, segend, st));
-  } else {
+  } else {   // the segment sums write the bounds
     FKM_TRY(launch_argsort_ids(s, st));
-    FKM_TRY(launch_seg_bounds(s.keys_out, L.n_sort, BK, segstart, segend, st));
+    FKM_TRY(clear_seg_bounds(BK, segstart, segend, st));
   }
   ObjArgs oa;
   oa.K = L.K;
@@ -134,7 +134,8 @@ fkm_status shard_partial_update(const Layout& L, const void* x, const int32_t* i
     oa.m = static_cast<float*>(at(L.mvec));
   }
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK, sums, nullptr,
-                        true, oa, st));
+                        true, oa, st, 0, nullptr, L.count_sort ? nullptr : segstart,
+                        L.count_sort ? nullptr : segend));
   add_counts_kernel<<<(unsigned)ceil_div(BK, 256), 256, 0, st>>>(segstart, segend, BK, counts);
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());

@@ -2,8 +2,9 @@
 // 聚类" summary, section 方法步骤详情 step (2); "Flash-KMeans: Fast and
 // Memory-Efficient Exact K-Means" summary, section "Method"):
 //
-//   seg_bounds  runs of equal keys in the sorted order: start/end per key, so
-//               counts = end - start are exact integers.
+//   bounds      runs of equal keys in the sorted order: start/end per key, so
+//               counts = end - start are exact integers (from the counting
+//               sort's scan, or written by segsum from its staged keys).
 //   segsum      the sorted order is cut into ranges of SEG_RANGE rows, one warp
 //               per range.  The warp walks its rows in order, gathering each
 //               row of the UNPERMUTED x by the sorted index with 16-byte loads
@@ -31,33 +32,6 @@
 namespace fkm {
 namespace {
 
-// Four sorted keys per thread (one 16-byte load; skeys is 16-byte aligned),
-// compared with their neighbours: a key that differs from the one before it
-// starts its run, one that differs from the one after it ends it.
-__global__ void seg_bounds_kernel(const int32_t* __restrict__ skeys, int64_t n, int BK,
-                                  int32_t* __restrict__ segstart, int32_t* __restrict__ segend) {
-  const int64_t i0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-  if (i0 >= n) return;
-  int32_t k[6];   // k[0] the key before i0, k[1..4] keys i0..i0+3, k[5] the one after
-  if (i0 + 4 <= n) {
-    const int4 v = *reinterpret_cast<const int4*>(skeys + i0);
-    k[1] = v.x; k[2] = v.y; k[3] = v.z; k[4] = v.w;
-  } else {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) k[1 + t] = i0 + t < n ? skeys[i0 + t] : -1;
-  }
-  k[0] = i0 > 0 ? skeys[i0 - 1] : -1;
-  k[5] = i0 + 4 < n ? skeys[i0 + 4] : -1;
-#pragma unroll
-  for (int t = 1; t <= 4; ++t) {
-    const int64_t i = i0 + t - 1;
-    const int32_t key = k[t];
-    if (i >= n || key < 0 || key >= BK) continue;  // past the end, or a rejected id
-    if (k[t - 1] != key) segstart[key] = (int32_t)i;
-    if (k[t + 1] != key) segend[key] = (int32_t)(i + 1);
-  }
-}
-
 // Rows longer than 512 bytes are summed in slabs of columns, one launch per
 // slab: x, centers, sums64, the centroid rows and the mean point at the slab's
 // first column, D its width, Dfull the whole row length.
@@ -78,6 +52,8 @@ struct SegParams {
   bool accumulate_all;   // out-of-core chunks: every run goes to sums64
   ObjArgs oa;
   unsigned long long* atomics;   // optional: count of fp64 atomic additions to sums64
+  int32_t* segstart;   // optional (cleared to zero by the caller): run bounds per key,
+  int32_t* segend;     // written here from the staged keys
 };
 
 // 16-byte vectors of the storage type, widened to float.
@@ -267,6 +243,9 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
   __syncwarp();
   // run starts (ids that are rejected sort after every valid key, so the
   // valid rows are a prefix of the range)
+  // With p.segstart, also the segment bounds: a run that starts (ends) in
+  // this range starts (ends) its key's segment unless the key continues from
+  // the range before (into the range after).
   int nruns = 0, nvalid = 0;
 #pragma unroll
   for (int t = 0; t < SEG_RANGE / 32; ++t) {
@@ -278,6 +257,11 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     if (start) ws.runs[nruns + __popc(bal & ((1u << lane) - 1u))] = (int16_t)i;
     nruns += __popc(bal);
     nvalid += __popc(__ballot_sync(0xffffffffu, k >= 0));
+    if (p.segstart && k >= 0) {
+      if (start && !(i == 0 && key_before == k)) p.segstart[k] = (int32_t)(j0 + i);
+      const int kn = ws.kv[i + 1].x;   // the (-1, 0) entries past the range end it
+      if (kn != k && !(i + 1 == nrows && key_after == k)) p.segend[k] = (int32_t)(j0 + i + 1);
+    }
   }
   if (lane == 0) ws.runs[nruns] = (int16_t)nvalid;
   __syncwarp();
@@ -803,23 +787,16 @@ fkm_status segsum_prepare() {
   return FKM_OK;
 }
 
-fkm_status launch_seg_bounds(const int32_t* skeys, int64_t n, int BK, int32_t* segstart,
-                             int32_t* segend, cudaStream_t st) {
+fkm_status clear_seg_bounds(int BK, int32_t* segstart, int32_t* segend, cudaStream_t st) {
   FKM_CUDA_TRY(cudaMemsetAsync(segstart, 0, sizeof(int32_t) * (size_t)BK, st));
   FKM_CUDA_TRY(cudaMemsetAsync(segend, 0, sizeof(int32_t) * (size_t)BK, st));
-  if (n > 0) {
-    seg_bounds_kernel<<<(unsigned)ceil_div(n, 1024), 256, 0, st>>>(skeys, n, BK, segstart,
-                                                                  segend);
-    note_launch();
-    FKM_CUDA_TRY(cudaGetLastError());
-  }
   return FKM_OK;
 }
 
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
                          bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range,
-                         unsigned long long* atomics) {
+                         unsigned long long* atomics, int32_t* segstart, int32_t* segend) {
   if (n == 0) return FKM_OK;
   if (range <= 0) range = segsum_range_rows(n);
   FKM_TRY(segsum_prepare());
@@ -843,6 +820,8 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
     sp.accumulate_all = accumulate_all;
     sp.oa = oa;
     sp.atomics = atomics;
+    sp.segstart = c0 == 0 ? segstart : nullptr;   // the first column slab writes them
+    sp.segend = c0 == 0 ? segend : nullptr;
     if (oa.chat) sp.oa.chat = static_cast<const char*>(oa.chat) + (int64_t)c0 * eb;
     if (oa.m) sp.oa.m = oa.m + c0;
     if (dtype == FKM_BF16) FKM_TRY(run_segsum_dt<FKM_BF16>(sp, st));
