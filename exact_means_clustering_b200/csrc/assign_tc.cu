@@ -540,23 +540,35 @@ struct __align__(8) PairCtl {
   float2 merge[BM];   // (best, index as float bits) of warpgroup 1
 };
 
-// fold_chunk keeping the improving chunk in registers (no shared memory).
-__device__ __forceinline__ void fold_chunk_reg(const uint32_t (&r)[32], int col0, int K,
-                                               float& best, int& bcol, float (&sv)[32]) {
-  float s[32];
+// Two adjacent chunks (64 columns from col0) folded at once: the chunk
+// holding the larger maximum (the lower one on a tie, so the lowest column
+// still wins) replaces the saved chunk when it beats the running maximum.
+// One decision per 64 columns halves the copies a warp makes, which every
+// lane pays for when any lane improves.
+__device__ __forceinline__ void fold_pair_reg(const uint32_t (&r0)[32], const uint32_t (&r1)[32],
+                                              int col0, int K, float& best, int& bcol,
+                                              float (&sv)[32]) {
+  float s0[32], s1[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(r[j]);
-  if (col0 + 32 > K) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (col0 + j >= K) s[j] = -INFINITY;
+  for (int j = 0; j < 32; ++j) {
+    s0[j] = __uint_as_float(r0[j]);
+    s1[j] = __uint_as_float(r1[j]);
   }
-  const float cm = max32(s);
-  if (cm > best) {
-    best = cm;
-    bcol = col0;
+  if (col0 + 64 > K) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) sv[j] = s[j];
+    for (int j = 0; j < 32; ++j) {
+      if (col0 + j >= K) s0[j] = -INFINITY;
+      if (col0 + 32 + j >= K) s1[j] = -INFINITY;
+    }
+  }
+  const float cm0 = max32(s0), cm1 = max32(s1);
+  const float bm = fmaxf(cm0, cm1);
+  if (bm > best) {
+    best = bm;
+    const bool first = cm0 >= cm1;
+    bcol = first ? col0 : col0 + 32;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) sv[j] = first ? s0[j] : s1[j];
   }
 }
 
@@ -760,8 +772,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
         ptx::tmem_ld32(taddr, r0);
         ptx::tmem_ld32(taddr + 32, r1);
         ptx::tmem_wait_ld64(r0, r1);
-        fold_chunk_reg(r0, colb, p.K, best, bcol, sv);
-        fold_chunk_reg(r1, colb + 32, p.K, best, bcol, sv);
+        fold_pair_reg(r0, r1, colb, p.K, best, bcol, sv);
         __syncwarp();   // the folds branch per lane; tcgen05.ld is warp-wide
         ptx::tmem_ld32(taddr + 64, r0);
         ptx::tmem_ld32(taddr + 96, r1);
@@ -770,8 +781,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive_cluster(acc_empty_cl[acc]);
         ++acc_uses;
-        fold_chunk_reg(r0, colb + 64, p.K, best, bcol, sv);
-        fold_chunk_reg(r1, colb + 96, p.K, best, bcol, sv);
+        fold_pair_reg(r0, r1, colb + 64, p.K, best, bcol, sv);
       }
       if (!ok) break;
       const int idx = best > -INFINITY ? bcol + find_first_reg(sv, best) : 0;
