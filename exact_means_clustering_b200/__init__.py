@@ -20,7 +20,10 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfkm.so")
+# FKM_LIB_VARIANT=checked loads the checked build (kernels verify their
+# gather / scatter indices and report an out-of-range one in the status word)
+LIB_PATH = os.path.join(_HERE, "libfkm_checked.so" if os.environ.get("FKM_LIB_VARIANT") ==
+                        "checked" else "libfkm.so")
 
 FKM_OK = 0
 STATUS_NAMES = {0: "FKM_OK", 1: "FKM_ERR_INVALID_ARG", 2: "FKM_ERR_UNSUPPORTED",
@@ -37,8 +40,8 @@ _SIG = {
     "fkm_centre_workspace_size": ([_I, _I, _I, ctypes.POINTER(_Z)], _I),
     "fkm_partial_update": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_finalize_sums": ([_I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
-    "fkm_partial_update_host": ([_I, _I, _I, _I, _I, _P, _P, _L, _P, _P, _P, _P, _P, _Z, _P],
-                                _I),
+    "fkm_partial_update_host": ([_I, _I, _I, _I, _I, _P, _P, _L, _P, _P, _P, _P, _I, _P, _Z,
+                                 _P], _I),
     "fkm_centre": ([_I, _I, _I, _I, _P, _P, _P, _P, _Z, _P], _I),
     "fkm_shift_centroids": ([_I, _I, _I, _P, _P, _I, _P, _P], _I),
     "fkm_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
@@ -441,10 +444,15 @@ def fkm_partial_update(x, ids, prev, sums, counts, obj=None, ws=None, stream=Non
     _check(f, lib().fkm_partial_update(B, N, K, D, _dt(x), *args, wp, wn, _stream(stream)))
 
 
+FKM_HOST_COPY_AT_ONCE = 1
+
+
 def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=None, ws=None,
-                            stream=None):
+                            stream=None, copy_at_once=False):
     """fkm_partial_update for a shard in pinned host memory x_host [B, N, D],
-    streamed in chunks of chunk_rows points; also writes the shard's ids."""
+    streamed in chunks of chunk_rows points; also writes the shard's ids.
+    copy_at_once: the workspace's chunk buffers are idle (an earlier call on
+    it returned), so the first copy need not wait for the stream (fkm.h)."""
     f = "fkm_partial_update_host"
     B, N, D = _dims(f, x_host, 3, "x_host")
     K = _dims(f, centers, 3, "centers")[1]
@@ -454,7 +462,8 @@ def fkm_partial_update_host(x_host, centers, chunk_rows, ids, sums, counts, obj=
             A.dev("ids", ids, (B, N), torch.int32),
             A.dev("sums", sums, (B, K, D), torch.float64),
             A.dev("counts", counts, (B, K), torch.float64),
-            A.dev("obj", obj, (B,), torch.float64))
+            A.dev("obj", obj, (B,), torch.float64),
+            FKM_HOST_COPY_AT_ONCE if copy_at_once else 0)
     wp, wn = A.ws(_ws(ws, fkm_host_workspace_size(B, N, K, D, _dt(x_host), chunk_rows),
                       centers.device))
     _check(f, lib().fkm_partial_update_host(B, N, K, D, _dt(x_host), px, *args, wp, wn,
@@ -528,10 +537,15 @@ def lloyd_sharded(x, init_centers, max_iters, tol=0.0, group=None, ws=None, chun
         ws = workspace(fkm_workspace_size(B, N, K, D, x.dtype), dev)
     c = init_centers.to(dev, torch.float32).contiguous().clone()
     ids = torch.empty(B, N, dtype=torch.int32, device=dev)
+    calls = [0]
 
     def partials(c, sums, counts, obj):
         if on_host:
-            fkm_partial_update_host(x, c, chunk_rows, ids, sums, counts, obj, ws=ws)
+            # after the first call the chunk buffers are idle, so the next
+            # iteration's first copy overlaps this iteration's all-reduce
+            fkm_partial_update_host(x, c, chunk_rows, ids, sums, counts, obj, ws=ws,
+                                    copy_at_once=calls[0] > 0)
+            calls[0] += 1
         else:
             fkm_assign(x, c, ids, ws=ws)
             fkm_partial_update(x, ids, c, sums, counts, obj, ws=ws)

@@ -141,6 +141,7 @@ struct HostPartial {
   double* sums;
   double* counts;
   double* obj;
+  int flags;   // FKM_HOST_COPY_AT_ONCE
 };
 
 }  // namespace
@@ -178,15 +179,19 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
 
 fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype, const void* x_host,
                                    const float* centers, int64_t chunk_rows, int32_t* ids,
-                                   double* sums, double* counts, double* obj, void* ws,
-                                   size_t ws_bytes, void* stream) {
+                                   double* sums, double* counts, double* obj, int flags,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  if (flags & ~FKM_HOST_COPY_AT_ONCE) {
+    set_error("unknown flags 0x%x", flags);
+    return FKM_ERR_INVALID_ARG;
+  }
   if (!sums || !counts || (reinterpret_cast<uintptr_t>(sums) & 15) ||
       (reinterpret_cast<uintptr_t>(counts) & 15) ||
       (obj && (reinterpret_cast<uintptr_t>(obj) & 15))) {
     set_error("sums and counts must be non-null; sums, counts and obj 16-byte aligned");
     return FKM_ERR_INVALID_ARG;
   }
-  HostPartial part{sums, counts, obj};
+  HostPartial part{sums, counts, obj, flags};
   int n_iter = 0;
   // counts is only checked for null and alignment on this path: the partial
   // pass adds into part.counts (fp64), never into the int32 output
@@ -255,9 +260,15 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
   float* mvec = static_cast<float*>(at(L.mvec));
   FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, mvec, at(L.cq),
                                 at(L.caug), st));
-  // the copy stream may only touch the workspace after the caller's earlier work
-  FKM_CUDA_TRY(cudaEventRecord(ss.start, st));
-  FKM_CUDA_TRY(cudaStreamWaitEvent(ss.copy, ss.start, 0));
+  // The copy stream may only touch the workspace after the caller's earlier
+  // work, unless the caller vouches that the chunk buffers are idle: then
+  // the first chunk's copy starts at once and overlaps whatever is still
+  // queued on the caller's stream (in a data-parallel loop, the previous
+  // iteration's all-reduce and finalize).
+  if (!(part && (part->flags & FKM_HOST_COPY_AT_ONCE))) {
+    FKM_CUDA_TRY(cudaEventRecord(ss.start, st));
+    FKM_CUDA_TRY(cudaStreamWaitEvent(ss.copy, ss.start, 0));
+  }
 
   int done = 0;
   int64_t chunk_no = 0;
@@ -337,7 +348,7 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
         }
         FKM_TRY(launch_segsum(xb, dtype, D, so.keys_out, so.vals_out, rows, K,
                               sums64 + (size_t)b * K * D, nullptr, true, oa, st, 0, nullptr,
-                              segstart, segend));
+                              segstart, segend, status));
         if (part)
           accumulate_counts_kernel<double><<<(unsigned)ceil_div(K, 256), 256, 0, st>>>(
               segstart, segend, K, part->counts + (size_t)b * K);
@@ -378,6 +389,10 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
   if (host_status & ST_TIMEOUT) {
     set_error("a device-side bounded wait ran out");
     return FKM_ERR_TIMEOUT;
+  }
+  if (host_status & ST_OOB) {
+    set_error("checked build: a kernel met an out-of-range gather or scatter index");
+    return FKM_ERR_INTERNAL;
   }
   if (host_status) {
     set_error("device status 0x%x", host_status);

@@ -256,11 +256,19 @@ FKM_API fkm_status fkm_finalize_sums(int B, int K, int D, const double* sums,
  * workspace of fkm_host_workspace_size(B, N, K, D, dtype, chunk_rows) bytes.
  * sums, counts, obj as in fkm_partial_update (the caller zeroes them once per
  * iteration; obj may be NULL).  Synchronous, like fkm_lloyd_host, and
- * FKM_FAULT_INJECT applies to its chunk copies in the same way. */
+ * FKM_FAULT_INJECT applies to its chunk copies in the same way.
+ * flags: 0, or FKM_HOST_COPY_AT_ONCE when no work still queued on `stream`
+ * touches this workspace (true after an earlier host-streamed call on it,
+ * which synchronises before returning): the first chunk's copy then starts
+ * at once instead of after that queued work, so in a data-parallel loop it
+ * overlaps the previous iteration's all-reduce and finalize (README
+ * "Multi-GPU Support": the first block of the next iteration is prefetched
+ * during the all-reduce).  Without the flag the copies wait for the stream. */
+#define FKM_HOST_COPY_AT_ONCE 1
 FKM_API fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype,
                                            const void* x_host, const float* centers,
                                            int64_t chunk_rows, int32_t* ids, double* sums,
-                                           double* counts, double* obj, void* ws,
+                                           double* counts, double* obj, int flags, void* ws,
                                            size_t ws_bytes, void* stream);
 
 /* Centring ("Flash-KMeans" GitHub README, section "Centre your data"):

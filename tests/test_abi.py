@@ -101,11 +101,15 @@ def test_shard_calls_validate_before_any_launch(fkm):
                                200, None) == 4
     # fkm_partial_update_host: sums are required and 16-byte aligned; the host workspace
     # is sized by fkm_host_workspace_size
-    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, None, a, None, a, 1 << 19,
+    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, None, a, None, 0, a, 1 << 19,
                                      None) == 1
-    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a + 8, a, None, a, 1 << 19,
+    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a + 8, a, None, 0, a, 1 << 19,
                                      None) == 1
-    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a, a, None, a, 64, None) == 4
+    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a, a, None, 0, a, 64,
+                                     None) == 4
+    # unknown flags
+    assert L.fkm_partial_update_host(1, 16, 4, 64, 2, a, a, 16, a, a, a, None, 6, a, 1 << 19,
+                                     None) == 1
 
 
 def test_metric_calls_reject_unknown_metric(fkm):

@@ -124,3 +124,27 @@ def test_sharded_loop_from_host_matches_lloyd_host():
     assert (cnt - n2).abs().sum().item() <= 2 * (ids != i2).sum().item()
     assert torch.allclose(cen, c2, rtol=1e-6, atol=1e-6)
     assert torch.allclose(inertia, in2, rtol=1e-6)
+
+
+def test_host_shard_copy_at_once_gives_the_same_partials():
+    """With FKM_HOST_COPY_AT_ONCE (the chunk buffers idle after an earlier call
+    on the workspace) the first copy starts without waiting for the stream;
+    the partials and ids are those of a call without the flag."""
+    w = datagen.Workload("host-flags", 2, 7000, 128, 200, "bf16", 200, sigma=0.5, iters=1, seed=3)
+    x, xt, c0 = problem(w)
+    c = torch.from_numpy(c0).cuda()
+    xh = xt.cpu().pin_memory()
+    ws = fkm.workspace(fkm.fkm_host_workspace_size(w.B, w.N, w.K, w.D, xt.dtype, 2048))
+    outs = []
+    for at_once in (False, True, True):
+        buf, sums, counts, obj = fkm.partial_buffers(w.B, w.K, w.D, "cuda")
+        ids = torch.empty(w.B, w.N, dtype=torch.int32, device="cuda")
+        # queued work on the stream that the flagged copy does not wait for
+        torch.cuda._sleep(1_000_000)
+        fkm.fkm_partial_update_host(xh, c, 2048, ids, sums, counts, obj, ws=ws,
+                                    copy_at_once=at_once)
+        outs.append((ids, counts.clone(), sums.clone(), obj.clone()))
+    for ids, counts, sums, obj in outs[1:]:
+        assert torch.equal(ids, outs[0][0]) and torch.equal(counts, outs[0][1])
+        assert torch.allclose(sums, outs[0][2], rtol=1e-12, atol=1e-9)
+        assert torch.allclose(obj, outs[0][3], rtol=1e-12)
