@@ -1,6 +1,11 @@
 """Builds libfkm.so in-tree with nvcc for sm_100a.
 
-    python -m exact_means_clustering_b200.build [--force] [--verbose]
+    python -m exact_means_clustering_b200.build [--force] [--verbose] [--checked]
+
+--checked builds libfkm_checked.so instead: the same sources with
+FKM_CHECKED defined, so the kernels verify the indices they gather and
+scatter with and record an out-of-range one in the status word (instead of
+touching memory); the binding loads it when FKM_LIB_VARIANT=checked.
 
 Sources: csrc/*.cu; public header: include/fkm.h.  The CUDA runtime is linked
 statically and the driver's tensor-map encoder is looked up at run time, so
@@ -19,7 +24,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libfkm.so")
+LIB_CHECKED = os.path.join(HERE, "libfkm_checked.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
+BUILD_DIR_CHECKED = os.path.join(ROOT, "_build_checked")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -40,23 +47,25 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib=LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "fkm.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    bdir = BUILD_DIR_CHECKED if checked else BUILD_DIR
+    if not force and not _stale(lib):
+        return lib
+    os.makedirs(bdir, exist_ok=True)
     objs = []
     procs = []
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        cmd = [_nvcc(), *NVCC_FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [_nvcc(), *NVCC_FLAGS, *(["-DFKM_CHECKED"] if checked else []), "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
@@ -71,14 +80,14 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     link = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
             "-Xcompiler", "-fvisibility=hidden"]
     subprocess.run(link, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                checked="--checked" in sys.argv))

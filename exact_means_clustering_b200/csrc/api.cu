@@ -302,7 +302,8 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK,
                         w.at<double>(L.sums64), next, false,
                         obj_args(w, prev, euclid ? obj : nullptr), st, range, w.atomics(),
-                        L.count_sort ? nullptr : segstart, L.count_sort ? nullptr : segend));
+                        L.count_sort ? nullptr : segstart, L.count_sort ? nullptr : segend,
+                        w.status()));
   if (ev) FKM_TRY(record_stage(ev[3], st));
   if (euclid) {
     FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64),
@@ -334,6 +335,11 @@ static fkm_status read_status(const Ws& w, cudaStream_t st) {
   if (host & ST_BAD_ID) {
     set_error("an id outside [0, K) was passed to the update (status 0x%x)", host);
     return FKM_ERR_BAD_ID;
+  }
+  if (host & ST_OOB) {
+    set_error("checked build: a kernel met an out-of-range gather or scatter index (status "
+              "0x%x)", host);
+    return FKM_ERR_INTERNAL;
   }
   set_error("device status 0x%x", host);
   return FKM_ERR_INTERNAL;
@@ -400,7 +406,9 @@ static fkm_status lloyd_iterations(const Ws& w, const void* x, int iters, int32_
 
 extern "C" {
 
-const char* fkm_version(void) { return "fkm 0.1.0 (sm_100a)"; }
+const char* fkm_version(void) {
+  return kChecked ? "fkm 0.2.0 (sm_100a, checked build)" : "fkm 0.2.0 (sm_100a)";
+}
 
 const char* fkm_last_error(void) { return g_err; }
 

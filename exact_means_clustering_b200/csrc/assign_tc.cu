@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
         ptx::mbar_arrive(&ctl->merge_empty);
         const int oidx = __float_as_int(o.y);
         const int fidx = (o.x > best || (o.x == best && oidx < idx)) ? oidx : idx;
-        if (gi < p.N) p.ids[(size_t)b * p.N + gi] = fidx;
+        if (gi < p.N && fkm_in_range(fidx, p.K, p.status)) p.ids[(size_t)b * p.N + gi] = fidx;
       }
     }
   }
@@ -798,7 +798,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
         ptx::mbar_arrive(&ctl->merge_empty);
         const int oidx = __float_as_int(o.y);
         const int fidx = (o.x > best || (o.x == best && oidx < idx)) ? oidx : idx;
-        if (gi < p.N) p.ids[(size_t)b * p.N + gi] = fidx;
+        if (gi < p.N && fkm_in_range(fidx, p.K, p.status)) p.ids[(size_t)b * p.N + gi] = fidx;
       }
     }
   }

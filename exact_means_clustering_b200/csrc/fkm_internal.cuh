@@ -13,7 +13,23 @@ enum : int {
   ST_TIMEOUT = 1,     // a bounded wait on an mbarrier ran out
   ST_BAD_ID = 2,      // fkm_update got an id outside [0, K)
   ST_INTERNAL = 4,    // an internal consistency check failed
+  ST_OOB = 8,         // checked build: a gather / scatter index was out of range
 };
+
+// The checked build (FKM_CHECKED): kernels verify the indices they gather and
+// scatter with before using them; an out-of-range one sets ST_OOB and the
+// access is skipped.  fkm_in_range is always true in the normal build.
+#ifdef FKM_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+__device__ __forceinline__ bool fkm_in_range(int64_t i, int64_t n, int* status) {
+  if (!kChecked) return true;
+  if (i >= 0 && i < n) return true;
+  if (status) atomicOr(status, ST_OOB);
+  return false;
+}
 
 // Assign tiling: 128 points (TMEM lanes) x 256 centroids (TMEM columns) per
 // accumulator; K-chunks of 64 16-bit values (one 128-byte swizzled row).
@@ -171,7 +187,7 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
                          bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range = 0,
                          unsigned long long* atomics = nullptr, int32_t* segstart = nullptr,
-                         int32_t* segend = nullptr);
+                         int32_t* segend = nullptr, int* status = nullptr);
 fkm_status clear_seg_bounds(int BK, int32_t* segstart, int32_t* segend, cudaStream_t st);
 // Rows per warp range of the segment sums for n sorted rows: SEG_RANGE for
 // large n, fewer (down to 32) when n is small, so a small problem still

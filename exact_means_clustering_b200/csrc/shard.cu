@@ -135,7 +135,7 @@ fkm_status shard_partial_update(const Layout& L, const void* x, const int32_t* i
   }
   FKM_TRY(launch_segsum(x, L.dtype, L.D, s.keys_out, s.vals_out, L.n_sort, BK, sums, nullptr,
                         true, oa, st, 0, nullptr, L.count_sort ? nullptr : segstart,
-                        L.count_sort ? nullptr : segend));
+                        L.count_sort ? nullptr : segend, static_cast<int*>(at(L.status))));
   add_counts_kernel<<<(unsigned)ceil_div(BK, 256), 256, 0, st>>>(segstart, segend, BK, counts);
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());

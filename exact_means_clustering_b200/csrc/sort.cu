@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
     const int32_t k = sk[j];
     const int d = (k >> shift) & (RADIX_BINS - 1);
     const int64_t g = (int64_t)gofs[d] + (j - (int64_t)tdo[d]);
+    if (!fkm_in_range(g, n, s.status)) continue;
     keys_out[g] = k;
     vals_out[g] = sv[j];
   }
@@ -455,6 +456,7 @@ __global__ void __launch_bounds__(SORT_THREADS, 4) cs_scatter_kernel(CsArgs a) {
   for (int j = threadIdx.x; j < nrows; j += SORT_THREADS) {
     const int k = sk[j];
     const int64_t g = (int64_t)j + shift[k];
+    if (!fkm_in_range(g, (int64_t)a.B * a.N, a.status)) continue;
     a.keys_out[g] = k < a.K ? b * a.K + k : a.B * a.K;
     a.vals_out[g] = sv[j];
   }
@@ -541,6 +543,7 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_single_tile_kernel(CsArgs a) 
   for (int r = 0; r < SORT_ITEMS; ++r) {
     if (bin[r] < a.K) {
       const uint32_t pos = start[bin[r]] + wc[bin[r]] + rank[r];
+      if (!fkm_in_range(pos, (int64_t)a.B * a.N, a.status)) continue;
       a.keys_out[pos] = b * a.K + bin[r];
       a.vals_out[pos] = (int32_t)(row0 + warp * PER_WARP + r * 32 + lane);
     }

@@ -54,6 +54,7 @@ struct SegParams {
   unsigned long long* atomics;   // optional: count of fp64 atomic additions to sums64
   int32_t* segstart;   // optional (cleared to zero by the caller): run bounds per key,
   int32_t* segend;     // written here from the staged keys
+  int* status;         // checked build: out-of-range row indices are reported here
 };
 
 // 16-byte vectors of the storage type, widened to float.
@@ -139,9 +140,18 @@ __device__ __forceinline__ void flush_run(const SegParams& p, int key, int g, in
       // far below the fp32 rounding that follows)
       const double rn = 1.0 / (double)nk;
       float* c = p.centers + (int64_t)key * p.Dfull + col0;
+      if (col0 + E <= p.D && (E & 3) == 0) {
+        // whole 16-byte pieces (row starts and col0 are 16-byte aligned)
 #pragma unroll
-      for (int e = 0; e < E; ++e)
-        if (col0 + e < p.D) c[e] = (float)(acc[e] * rn);
+        for (int e = 0; e < E; e += 4)
+          *reinterpret_cast<float4*>(c + e) =
+              make_float4((float)(acc[e] * rn), (float)(acc[e + 1] * rn),
+                          (float)(acc[e + 2] * rn), (float)(acc[e + 3] * rn));
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          if (col0 + e < p.D) c[e] = (float)(acc[e] * rn);
+      }
     } else {
       double* sd = p.sums64 + (int64_t)key * p.Dfull + col0;
 #pragma unroll
@@ -227,6 +237,7 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     if (i < nrows) {
       e_[t].x = p.skeys[j0 + i];
       e_[t].y = p.svals[j0 + i];
+      if (!fkm_in_range(e_[t].y, p.n, p.status)) e_[t].x = -1;   // the row is skipped
     }
   }
   int kedge = -1;   // lane 0: the key before the range; lane 1: the key after it
@@ -286,10 +297,17 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
 
   // centroid rows for the objective: raw 16-byte piece of the next run's row
   uint4 chat_next = make_uint4(0, 0, 0, 0);
+  // (batch, cluster) of a sorted key b*K + id: keys only grow along the
+  // range, so the batch is found by division only when it changes
+  int pf_b = -1, pf_base = 0;
   auto prefetch_chat = [&](int run) {
     if (!want_obj || run >= nruns || !lane_has_vec) return;
     const int kg = ws.kv[ws.runs[run]].x;
-    const int b = kg / p.oa.K, k = kg % p.oa.K;
+    if (pf_b < 0 || kg - pf_base >= p.oa.K) {
+      pf_b = kg / p.oa.K;
+      pf_base = pf_b * p.oa.K;
+    }
+    const int b = pf_b, k = kg - pf_base;
     const char* row = static_cast<const char*>(p.oa.chat) +
                       ((int64_t)b * p.oa.chat_bstride + (int64_t)k * p.Dfull) * elem_bytes_;
     chat_next = ldg_nc_v4(row + (int64_t)sub * 16);
@@ -358,6 +376,7 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
   float2 m2[E / 2];
 #pragma unroll
   for (int e = 0; e < E / 2; ++e) m2[e] = make_float2(0.0f, 0.0f);
+  int cur_base = 0;   // cur_b * K
   auto start_run = [&](int kg, int i) {
     cur = kg;
     ++run;
@@ -365,14 +384,15 @@ __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     run_end = ws.runs[run + 1];
     if (!want_obj) return;
     fold_obj();
-    const int b = kg / p.oa.K;
-    if (b != cur_b) {
+    if (cur_b < 0 || kg - cur_base >= p.oa.K) {   // a new batch (keys only grow)
+      const int b = kg / p.oa.K;
       if (cur_b >= 0) {
         const double t = warp_sum(obj);
         if (lane == 0) atomicAdd(p.oa.obj + cur_b, t);
       }
       obj = 0.0;
       cur_b = b;
+      cur_base = b * p.oa.K;
       if (p.oa.m && lane_has_vec) {
         const float2* mb =
             reinterpret_cast<const float2*>(p.oa.m + (int64_t)b * p.Dfull) + sub * (E / 2);
@@ -796,7 +816,8 @@ fkm_status clear_seg_bounds(int BK, int32_t* segstart, int32_t* segend, cudaStre
 fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
                          const int32_t* svals, int64_t n, int BK, double* sums64, float* centers,
                          bool accumulate_all, const ObjArgs& oa, cudaStream_t st, int range,
-                         unsigned long long* atomics, int32_t* segstart, int32_t* segend) {
+                         unsigned long long* atomics, int32_t* segstart, int32_t* segend,
+                         int* status) {
   if (n == 0) return FKM_OK;
   if (range <= 0) range = segsum_range_rows(n);
   FKM_TRY(segsum_prepare());
@@ -822,6 +843,7 @@ fkm_status launch_segsum(const void* x, int dtype, int D, const int32_t* skeys,
     sp.atomics = atomics;
     sp.segstart = c0 == 0 ? segstart : nullptr;   // the first column slab writes them
     sp.segend = c0 == 0 ? segend : nullptr;
+    sp.status = status;
     if (oa.chat) sp.oa.chat = static_cast<const char*>(oa.chat) + (int64_t)c0 * eb;
     if (oa.m) sp.oa.m = oa.m + c0;
     if (dtype == FKM_BF16) FKM_TRY(run_segsum_dt<FKM_BF16>(sp, st));
