@@ -639,26 +639,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
       ptx::prefetch_tmap(&tm_c);
       ptx::prefetch_tmap(&tm_aug);
       uint32_t a_arms = 0, s_arms = 0;
+      uint32_t ab = 0, a_ph = 0, sb = 0, s_ph = 0;   // ring positions, as in the issuer
       bool ok = true;
       for (int w = (int)cid; w < p.n_work && ok; w += (int)ncl) {
         const int b = w / p.m_tiles, mt = w % p.m_tiles;
         const int row0 = mt * PAIR_ROWS + (int)rank * BM;
-        const int ab = a_arms % p.nA;
-        const uint32_t apar = ((a_arms / p.nA) & 1) ^ 1;
-        if (!ptx::mbar_wait_bounded_cl(&ctl->a_empty[ab], apar, abort_flag, p.status, ST_TIMEOUT,
-                                       kWaitTimeoutNs)) { ok = false; break; }
+        if (!ptx::mbar_wait_bounded_cl(&ctl->a_empty[ab], a_ph ^ 1, abort_flag, p.status,
+                                       ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
         if (leader) ptx::mbar_arrive_expect_tx(&ctl->a_full[ab], 2 * p.a_bytes);
         const uint32_t afull = ptx::mapa_rank(&ctl->a_full[ab], 0);
         uint8_t* abuf = a_base + (size_t)ab * p.a_bytes;
         for (int dc = 0; dc < p.nD; ++dc)
           ptx::tma_load_3d_pair(abuf + dc * A_CHUNK_BYTES, &tm_x, afull, dc * KC, row0, b);
         ++a_arms;
+        if (++ab == (uint32_t)p.nA) { ab = 0; a_ph ^= 1; }
         for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
           const int crow = kt * BN + (int)rank * PAIR_BH;
           for (int q = 0; q < p.nD; ++q) {
-            const int sb = s_arms % p.nS;
-            const uint32_t spar = ((s_arms / p.nS) & 1) ^ 1;
-            if (!ptx::mbar_wait_bounded_cl(&ctl->b_empty[sb], spar, abort_flag, p.status,
+            if (!ptx::mbar_wait_bounded_cl(&ctl->b_empty[sb], s_ph ^ 1, abort_flag, p.status,
                                            ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
             if (leader)
               ptx::mbar_arrive_expect_tx(&ctl->b_full[sb],
@@ -668,6 +666,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
             ptx::tma_load_3d_pair(sbuf, &tm_c, bfull, q * KC, crow, b);
             if (q == 0) ptx::tma_load_3d_pair(sbuf + PAIR_B_CHUNK, &tm_aug, bfull, 0, crow, b);
             ++s_arms;
+            if (++sb == (uint32_t)p.nS) { sb = 0; s_ph ^= 1; }
           }
         }
       }
@@ -686,50 +685,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
+    // One thread feeds the tensor pipe, and an M = 256, N = 256, K = 16 MMA
+    // occupies it for only ~128 cycles, so this loop keeps its own work per
+    // MMA to a few instructions: ring indices and phases advance without
+    // divisions, and every operand descriptor is a base descriptor plus the
+    // operand's byte offset >> 4 (the start-address field, bits 0-13, cannot
+    // carry below 256 KB).  A division or a rebuilt descriptor per MMA was
+    // enough to leave the pipe idle half of the time.
     if (leader && lane == 0) {
-      const uint32_t aug_a_addr = ptx::smem_u32(aug_a);
-      uint32_t a_uses = 0, s_uses = 0, acc_uses = 0;
+      const uint64_t d_aug_a = ptx::umma_desc_sw32(ptx::smem_u32(aug_a));
+      const uint64_t d_a0 = ptx::umma_desc_sw128(ptx::smem_u32(a_base));
+      const uint64_t d_b0 = ptx::umma_desc_sw128(ptx::smem_u32(b_base));
+      const uint64_t d_aug_b0 = ptx::umma_desc_sw32(ptx::smem_u32(b_base + PAIR_B_CHUNK));
+      constexpr uint32_t kStageStep = PAIR_STAGE >> 4, kChunkStep = A_CHUNK_BYTES >> 4;
+      const uint32_t a_step = p.a_bytes >> 4;
+      uint32_t ab = 0, a_ph = 0, sb = 0, s_ph = 0, acc = 0, acc_ph = 0;
       bool ok = true, issued = false;
       for (int w = (int)cid; w < p.n_work && ok; w += (int)ncl) {
-        const int ab = a_uses % p.nA;
-        if (!ptx::mbar_wait_bounded_cl(&ctl->a_full[ab], (a_uses / p.nA) & 1, abort_flag,
-                                       p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+        if (!ptx::mbar_wait_bounded_cl(&ctl->a_full[ab], a_ph, abort_flag, p.status, ST_TIMEOUT,
+                                       kWaitTimeoutNs)) { ok = false; break; }
         ptx::tc_fence_after();
-        const uint32_t a_addr = ptx::smem_u32(a_base + (size_t)ab * p.a_bytes);
+        const uint64_t d_a = d_a0 + ab * a_step;
         for (int kt = 0; kt < p.k_tiles && ok; ++kt) {
-          const int acc = acc_uses & 1;
-          if (!ptx::mbar_wait_bounded_cl(&ctl->acc_empty[acc], ((acc_uses >> 1) & 1) ^ 1,
-                                         abort_flag, p.status, ST_TIMEOUT, kWaitTimeoutNs)) {
-            ok = false;
-            break;
-          }
+          if (!ptx::mbar_wait_bounded_cl(&ctl->acc_empty[acc], acc_ph ^ 1, abort_flag, p.status,
+                                         ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+          const uint32_t d_tmem = tmem_base + acc * BN;
           for (int q = 0; q < p.nD; ++q) {
-            const int sb = s_uses % p.nS;
-            if (!ptx::mbar_wait_bounded_cl(&ctl->b_full[sb], (s_uses / p.nS) & 1, abort_flag,
-                                           p.status, ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
+            if (!ptx::mbar_wait_bounded_cl(&ctl->b_full[sb], s_ph, abort_flag, p.status,
+                                           ST_TIMEOUT, kWaitTimeoutNs)) { ok = false; break; }
             ptx::tc_fence_after();
-            const uint32_t b_addr = ptx::smem_u32(b_base + (size_t)sb * PAIR_STAGE);
+            const uint64_t d_b = d_b0 + sb * kStageStep;
             if (q == 0)   // the bias product starts the tile's accumulation
-              ptx::mma_f16_ss_pair(d_tmem, ptx::umma_desc_sw32(aug_a_addr),
-                                   ptx::umma_desc_sw32(b_addr + PAIR_B_CHUNK), p.idesc, 0u);
-            const uint32_t xa = a_addr + q * A_CHUNK_BYTES;
+              ptx::mma_f16_ss_pair(d_tmem, d_aug_a, d_aug_b0 + sb * kStageStep, p.idesc, 0u);
+            const uint64_t d_aq = d_a + q * kChunkStep;
 #pragma unroll
-            for (int k = 0; k < KC / 16; ++k)
-              ptx::mma_f16_ss_pair(d_tmem, ptx::umma_desc_sw128(xa + 32 * k),
-                                   ptx::umma_desc_sw128(b_addr + 32 * k), p.idesc, 1u);
+            for (int k = 0; k < KC / 16; ++k)   // K = 16 steps are 32 bytes apart
+              ptx::mma_f16_ss_pair(d_tmem, d_aq + 2 * k, d_b + 2 * k, p.idesc, 1u);
             issued = true;
             ptx::mma_commit_pair_mc(&ctl->b_empty[sb], 0x3);
-            ++s_uses;
+            if (++sb == (uint32_t)p.nS) { sb = 0; s_ph ^= 1; }
           }
           if (!ok) break;
           ptx::mma_commit_pair_mc(&ctl->acc_full[acc], 0x3);
-          ++acc_uses;
+          if (++acc == 2) { acc = 0; acc_ph ^= 1; }
         }
         if (!ok) break;
         ptx::mma_commit_pair_mc(&ctl->a_empty[ab], 0x3);
-        ++a_uses;
+        if (++ab == (uint32_t)p.nA) { ab = 0; a_ph ^= 1; }
       }
       // Drain: all MMAs issued must finish before TMEM is freed.
       if (issued) {
