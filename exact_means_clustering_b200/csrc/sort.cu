@@ -6,8 +6,8 @@
 // argsort与分段规约 and 方法步骤详情 step (2)).  Keys are key = b*K + id (so
 // batches stay apart); values are the row indices b*N + i.
 //
-// LSD radix sort, 8-bit digits, as many passes as the key width needs
-// (1 for B*K < 256, 2 up to 65536).  Per pass:
+// LSD radix sort: as many passes as digits of at most 8 bits need (1 for
+// B*K < 256, 2 up to 65536), the key bits split evenly over them.  Per pass:
 //   upsweep    tile histograms (4096 keys per 256-thread tile), digit-major
 //   scan       exclusive scan of the histogram matrix: global base per
 //              (digit, tile)
@@ -88,7 +88,9 @@ __device__ __forceinline__ void load_key(const KeySrc& s, int64_t j, int32_t& ke
 
 template <bool kFirst>
 __global__ void __launch_bounds__(SORT_THREADS) radix_upsweep(KeySrc s, int64_t n, int shift,
-                                                              int n_tiles, uint32_t* hist) {
+                                                              int bits, int n_tiles,
+                                                              uint32_t* hist) {
+  const int nbins = 1 << bits;
   __shared__ uint32_t h[SORT_THREADS / 32][RADIX_BINS];
   const int warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < (SORT_THREADS / 32) * RADIX_BINS; i += SORT_THREADS)
@@ -102,18 +104,18 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_upsweep(KeySrc s, int64_t 
 #pragma unroll
   for (int it = 0; it < SORT_ITEMS; ++it) {
     const int64_t j = base + (int64_t)it * SORT_THREADS + threadIdx.x;
-    digit[it] = RADIX_BINS;  // out of range: matches nothing real
+    digit[it] = nbins;  // out of range: matches nothing real
     if (j < n) {
       int32_t key, val;
       load_key<kFirst>(s, j, key, val);
-      digit[it] = (key >> shift) & (RADIX_BINS - 1);
+      digit[it] = (key >> shift) & (nbins - 1);
     }
   }
 #pragma unroll
   for (int it = 0; it < SORT_ITEMS; ++it)
-    if (digit[it] < RADIX_BINS) atomicAdd(&h[warp][digit[it]], 1u);
+    if (digit[it] < nbins) atomicAdd(&h[warp][digit[it]], 1u);
   __syncthreads();
-  for (int d = threadIdx.x; d < RADIX_BINS; d += SORT_THREADS) {
+  for (int d = threadIdx.x; d < nbins; d += SORT_THREADS) {
     uint32_t t = 0;
 #pragma unroll
     for (int w = 0; w < SORT_THREADS / 32; ++w) t += h[w][d];
@@ -201,7 +203,7 @@ static_assert(DS_THREADS >= RADIX_BINS, "one thread per digit in the digit scan"
 
 template <bool kFirst>
 __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64_t n, int shift,
-                                                              int n_tiles,
+                                                              int bits, int n_tiles,
                                                               const uint32_t* __restrict__ hist,
                                                               int32_t* __restrict__ keys_out,
                                                               int32_t* __restrict__ vals_out) {
@@ -219,7 +221,12 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
   uint32_t (*cnt)[RADIX_BINS + 1] = reinterpret_cast<uint32_t (*)[RADIX_BINS + 1]>(stage);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nbins = 1 << bits;
   for (int i = threadIdx.x; i < NW * (RADIX_BINS + 1); i += DS_THREADS) (&cnt[0][0])[i] = 0;
+  // this tile's global base of every digit (the scanned histogram), loaded
+  // now so its latency overlaps the key loads and the ranking
+  const uint32_t gbase =
+      (int)threadIdx.x < nbins ? hist[(size_t)threadIdx.x * n_tiles + blockIdx.x] : 0u;
   __syncthreads();
 
   const int64_t base = (int64_t)blockIdx.x * SORT_TILE + (int64_t)warp * PER_WARP;
@@ -231,19 +238,19 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
 #pragma unroll
   for (int r = 0; r < DS_ITEMS; ++r) {
     const int64_t j = base + r * 32 + lane;
-    int d = RADIX_BINS;  // keys past the end use an extra bin and are never written
+    int d = nbins;  // keys past the end use an extra bin and are never written
     key[r] = 0;
     val[r] = 0;
     if (j < n) {
       load_key<kFirst>(s, j, key[r], val[r]);
-      d = (key[r] >> shift) & (RADIX_BINS - 1);
+      d = (key[r] >> shift) & (nbins - 1);
     }
     dr[r] = (uint32_t)d;
   }
 #pragma unroll
   for (int r = 0; r < DS_ITEMS; ++r) {
     const int d = (int)dr[r];
-    const unsigned peers = warp_peers((unsigned)d, 9);   // digits 0..RADIX_BINS
+    const unsigned peers = warp_peers((unsigned)d, bits + 1);   // digits 0..nbins
     const uint32_t before = cnt[warp][d];
     dr[r] = (uint32_t)d | ((before + __popc(peers & lt_mask)) << 9);
     __syncwarp();
@@ -256,7 +263,7 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
   {
     const int d = threadIdx.x;
     uint32_t run = 0;
-    if (d < RADIX_BINS) {
+    if (d < nbins) {
 #pragma unroll
       for (int w = 0; w < NW; ++w) {
         uint32_t c = cnt[w][d];
@@ -265,9 +272,9 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
       }
     }
     uint32_t ex = block_exclusive_scan(run, sw, nullptr);
-    if (d < RADIX_BINS) {
+    if (d < nbins) {
       tdo[d] = ex;
-      gofs[d] = hist[(size_t)d * n_tiles + blockIdx.x];
+      gofs[d] = gbase;
     }
   }
   __syncthreads();
@@ -275,7 +282,7 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
 #pragma unroll
   for (int r = 0; r < DS_ITEMS; ++r) {
     const int d = (int)(dr[r] & 511u);
-    dr[r] = d < RADIX_BINS ? tdo[d] + cnt[warp][d] + (dr[r] >> 9) : 0xffffffffu;
+    dr[r] = d < nbins ? tdo[d] + cnt[warp][d] + (dr[r] >> 9) : 0xffffffffu;
   }
   __syncthreads();
   // ... then the keys staged there in sorted order
@@ -291,7 +298,7 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
   const int valid = (int)((n - tile0) < SORT_TILE ? (n - tile0) : SORT_TILE);
   for (int j = threadIdx.x; j < valid; j += DS_THREADS) {
     const int32_t k = sk[j];
-    const int d = (k >> shift) & (RADIX_BINS - 1);
+    const int d = (k >> shift) & (nbins - 1);
     const int64_t g = (int64_t)gofs[d] + (j - (int64_t)tdo[d]);
     if (!fkm_in_range(g, n, s.status)) continue;
     keys_out[g] = k;
@@ -391,6 +398,26 @@ __global__ void __launch_bounds__(SORT_THREADS, 4) cs_scatter_kernel(CsArgs a) {
       bin[r] = (id < 0 || id >= a.K) ? a.K : id;
     }
   }
+  // thread t owns bins [t*kpt, (t+1)*kpt) in the bin scan below; their global
+  // bases (the scanned histogram) are loaded together with the ids and parked
+  // in `shift`, so the latency of these scattered words is paid once
+  const int kpt = (KB + SORT_THREADS - 1) / SORT_THREADS;
+  const int k0 = threadIdx.x * kpt;
+  {
+    constexpr int KPT_MAX = (CS_MAX_K + 1 + SORT_THREADS - 1) / SORT_THREADS;
+    uint32_t gv[KPT_MAX];   // every load issued before the first store waits
+#pragma unroll
+    for (int i = 0; i < KPT_MAX; ++i) {
+      const int k = k0 + i;
+      gv[i] = 0;
+      if (i < kpt && k < KB)
+        gv[i] = k < a.K ? a.hist[((int64_t)b * a.K + k) * a.tpb + t]
+                        : a.hist[(int64_t)a.B * a.K * a.tpb + tg];
+    }
+#pragma unroll
+    for (int i = 0; i < KPT_MAX; ++i)
+      if (i < kpt && k0 + i < KB) shift[k0 + i] = (int32_t)gv[i];
+  }
   __syncthreads();
   const unsigned lt_mask = (1u << lane) - 1u;
   const int nbits = value_bits((unsigned)a.K + 1);   // bins 0..K+1
@@ -411,8 +438,6 @@ __global__ void __launch_bounds__(SORT_THREADS, 4) cs_scatter_kernel(CsArgs a) {
   __syncthreads();
   // per bin: earlier warps' counts become offsets inside the bin; thread t
   // owns bins [t*kpt, (t+1)*kpt) and scans their totals across the block
-  const int kpt = (KB + SORT_THREADS - 1) / SORT_THREADS;
-  const int k0 = threadIdx.x * kpt;
   uint32_t local = 0;
   for (int k = k0; k < k0 + kpt && k < KB; ++k) {
     uint32_t run = 0;
@@ -428,10 +453,8 @@ __global__ void __launch_bounds__(SORT_THREADS, 4) cs_scatter_kernel(CsArgs a) {
   uint32_t pos = block_exclusive_scan(local, sw, nullptr);
   for (int k = k0; k < k0 + kpt && k < KB; ++k) {
     const uint32_t n = start[k];
-    const uint32_t g = k < a.K ? a.hist[((int64_t)b * a.K + k) * a.tpb + t]
-                               : a.hist[(int64_t)a.B * a.K * a.tpb + tg];
     start[k] = pos;
-    shift[k] = (int32_t)(g - pos);
+    shift[k] -= (int32_t)pos;   // global base - tile position
     pos += n;
   }
   __syncthreads();
@@ -639,7 +662,11 @@ fkm_status launch_argsort_ids(SortArgs& a, cudaStream_t st) {
   }
   const int n_tiles = (int)ceil_div(a.n, SORT_TILE);
   const int passes = (a.key_bits + RADIX_BITS - 1) / RADIX_BITS;
-  const int64_t hlen = (int64_t)n_tiles * RADIX_BINS;
+  // the key bits split evenly over the passes (12-bit keys: two 6-bit
+  // digits), so no pass ranks more bins than it needs, and the scatter's runs
+  // per digit stay long in every pass
+  const int bits = passes > 0 ? (a.key_bits + passes - 1) / passes : 1;
+  const int64_t hlen = (int64_t)n_tiles << bits;
   KeySrc s;
   s.ids = a.ids;
   s.N = a.N;
@@ -649,21 +676,23 @@ fkm_status launch_argsort_ids(SortArgs& a, cudaStream_t st) {
   int32_t* kout[2] = {a.keys0, a.keys1};
   int32_t* vout[2] = {a.vals0, a.vals1};
   for (int p = 0; p < (passes > 0 ? passes : 1); ++p) {
-    const int shift = p * RADIX_BITS;
+    const int shift = p * bits;
     if (p == 0) {
       s.keys = nullptr;
       s.vals = nullptr;
-      radix_upsweep<true><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist);
+      radix_upsweep<true><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
+                                                            a.hist);
       FKM_TRY(device_scan(a.hist, hlen, a.hist_part, st));
-      radix_downsweep<true><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist,
-                                                              kout[0], vout[0]);
+      radix_downsweep<true><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
+                                                              a.hist, kout[0], vout[0]);
     } else {
       s.keys = kout[(p - 1) & 1];
       s.vals = vout[(p - 1) & 1];
-      radix_upsweep<false><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist);
+      radix_upsweep<false><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
+                                                             a.hist);
       FKM_TRY(device_scan(a.hist, hlen, a.hist_part, st));
-      radix_downsweep<false><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, n_tiles, a.hist,
-                                                               kout[p & 1], vout[p & 1]);
+      radix_downsweep<false><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
+                                                               a.hist, kout[p & 1], vout[p & 1]);
     }
     FKM_CUDA_TRY(cudaGetLastError());
     note_launch(2);

@@ -157,7 +157,11 @@ def test_assign_teacher_forced(wid, scale):
 @pytest.mark.parametrize("dtype,B,N,K,D", [("bf16", 2, 9000, 300, 128), ("f16", 3, 4097, 50, 64),
                                            ("f32", 1, 20000, 40, 64), ("f32", 2, 3000, 100, 128),
                                            ("bf16", 1, 70000, 9, 256), ("bf16", 2, 1, 3, 8),
-                                           ("bf16", 2, 30000, 3000, 64), ("f16", 1, 9000, 2049, 32)])
+                                           ("bf16", 2, 30000, 3000, 64), ("f16", 1, 9000, 2049, 32),
+                                           # rows of 12, 25 and 10 16-byte vectors: lanes whose
+                                           # second vector lies past the row
+                                           ("bf16", 2, 5000, 200, 96), ("bf16", 1, 6000, 100, 200),
+                                           ("f32", 1, 4000, 64, 40)])
 def test_update_teacher_forced(dtype, B, N, K, D):
     rng = np.random.default_rng(N + K)
     w = datagen.Workload("t", B, N, D, K, dtype, 0, sigma=2.0, seed=N)
