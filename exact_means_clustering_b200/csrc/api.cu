@@ -266,10 +266,19 @@ static ObjArgs obj_args(const Ws& w, const float* prev, double* obj) {
 // argsort + bounds + segment sums (+ objective) + finalize; prev -> next.
 // obj (device [B], zeroed here) receives the objective of ids against prev.
 // ids_valid: the ids were written by the assign kernel (all in [0, K)).
+// shifts (Lloyd loop): where given, the Euclidean finalize, the next assign's
+// operands (requant) and the batch shifts go into one launch, which writes
+// shift_out / max_shift and sets *shifts->done; otherwise the caller reduces
+// the per-cluster shifts itself.
+struct LoopShifts {
+  double* shift_out;
+  double* max_shift;
+  bool done;
+};
 static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, const float* prev,
                               float* next, int32_t* counts, bool requant, double* obj,
                               cudaStream_t st, cudaEvent_t* ev = nullptr,
-                              bool ids_valid = false) {
+                              bool ids_valid = false, LoopShifts* shifts = nullptr) {
   const Layout& L = *w.L;
   SortArgs s;
   s.ids = ids;
@@ -305,6 +314,14 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
                         L.count_sort ? nullptr : segstart, L.count_sort ? nullptr : segend,
                         w.status()));
   if (ev) FKM_TRY(record_stage(ev[3], st));
+  if (euclid && requant && shifts && finalize_prep_fits(L.B, L.Kp, L.D)) {
+    FKM_TRY(launch_finalize_prep(L.B, L.K, L.Kp, L.D, L.dtype, range, segstart, segend,
+                                 w.at<double>(L.sums64), prev, next, counts, w.at<float>(L.mvec),
+                                 w.at<void>(L.cq), w.at<void>(L.caug), shifts->shift_out,
+                                 shifts->max_shift, st));
+    shifts->done = true;
+    return FKM_OK;
+  }
   if (euclid) {
     FKM_TRY(launch_finalize(L.B, L.K, L.D, segstart, segend, nullptr, w.at<double>(L.sums64),
                             prev, next, counts, w.at<double>(L.shiftk), st, range));
@@ -395,10 +412,12 @@ static fkm_status lloyd_iterations(const Ws& w, const void* x, int iters, int32_
     if (ev) FKM_TRY(record_stage(ev[0], st));
     FKM_TRY(step_assign(w, x, ids, st));
     if (ev) FKM_TRY(record_stage(ev[1], st));
-    FKM_TRY(step_update(w, x, ids, cur, nxt, counts, true, inertia, st, ev, true));
     if (track_max) FKM_CUDA_TRY(cudaMemsetAsync(w.max_shift(), 0, sizeof(double), st));
-    FKM_TRY(launch_batch_reduce(L.B, L.K, w.at<double>(L.shiftk), shift_dev,
-                                track_max ? w.max_shift() : nullptr, st));
+    LoopShifts sh{shift_dev, track_max ? w.max_shift() : nullptr, false};
+    FKM_TRY(step_update(w, x, ids, cur, nxt, counts, true, inertia, st, ev, true, &sh));
+    if (!sh.done)
+      FKM_TRY(launch_batch_reduce(L.B, L.K, w.at<double>(L.shiftk), shift_dev,
+                                  track_max ? w.max_shift() : nullptr, st));
     if (ev) FKM_TRY(record_stage(ev[4], st));
   }
   return FKM_OK;

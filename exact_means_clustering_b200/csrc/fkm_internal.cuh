@@ -46,6 +46,14 @@ constexpr int TMEM_COLS = 512;               // two 256-column fp32 accumulators
 // finished by that warp; one that spans ranges is summed with fp64 atomics.
 constexpr int SEG_RANGE = 256;
 
+// The mean centroid's fixed summation order (center_kernel and the fused
+// end-of-iteration kernel): MEAN_CHUNKS contiguous chunks of Kp / MEAN_CHUNKS
+// padded rows, MEAN_WAYS strided partials per chunk.  Kp is a multiple of BN,
+// so every chunk holds whole rounds of the partials.
+constexpr int MEAN_CHUNKS = 8;
+constexpr int MEAN_WAYS = 16;
+static_assert(BN % (MEAN_CHUNKS * MEAN_WAYS) == 0, "whole rounds of partials per chunk");
+
 // Radix argsort: 8-bit digits, 256 threads x 16 keys per tile.
 constexpr int RADIX_BITS = 8;
 constexpr int RADIX_BINS = 1 << RADIX_BITS;
@@ -131,6 +139,18 @@ constexpr int AUG_SLAB = 16;
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
                                  float* m, void* cq, void* caug, cudaStream_t st,
                                  int metric = FKM_METRIC_EUCLID, double* cnorm = nullptr);
+// The end of a Euclidean Lloyd iteration in one launch: finalize (counts,
+// new centroids from the segment sums, sums64 cleared), the mean centroid m
+// (bit for bit launch_prep_centroids'), the next assign's operands and bias
+// slabs, and the batch shifts (shift_out [B], optional; max_shift optional,
+// zeroed by the caller).  For D <= 256, Kp <= 1024 and B <= 65535
+// (finalize_prep_fits).
+bool finalize_prep_fits(int B, int Kp, int D);
+fkm_status launch_finalize_prep(int B, int K, int Kp, int D, int dtype, int range,
+                                const int32_t* segstart, const int32_t* segend, double* sums64,
+                                const float* prev, float* centers, int32_t* counts, float* m,
+                                void* cq, void* caug, double* shift_out, double* max_shift,
+                                cudaStream_t st);
 // fp32 points: split rows into xs; xn (optional) = ||x - m[row / N]||^2
 // (||x||^2 when m is null).
 fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,

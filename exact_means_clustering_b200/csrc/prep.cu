@@ -1,7 +1,7 @@
 // Operand preparation for the assign kernel.
 //
-//  center: per batch the mean centroid m (fp64 sum over k in a fixed order --
-//    32 strided partial sums, then their sum -- divided by K, rounded to fp32).  The assignment works on offsets from m:
+//  center: per batch the mean centroid m (fp64 sum over k in a fixed order,
+//    divided by K, rounded to fp32).  The assignment works on offsets from m:
 //    k-means is translation invariant ("Flash-KMeans" README, section "Centre
 //    your data"), and with the offsets small the tensor-core products and
 //    their fp32 accumulation keep their precision even for data far from the
@@ -31,6 +31,7 @@
 #include <cuda_fp16.h>
 
 #include "fkm_internal.cuh"
+#include "ptx_sm100.cuh"
 
 namespace fkm {
 namespace {
@@ -64,40 +65,67 @@ __global__ void row_norms_kernel(const float* __restrict__ c, int64_t rows, int 
   if (lane == 0) cn[row] = sqrt(s);
 }
 
-// m[b][d] = fp32(S / K) with S summed in fp64 in a fixed order that does not
-// depend on the launch: 32 partial sums P_w = sum over k = w, w+32, w+64, ...
-// (each in ascending k), then S = P_0 + P_1 + ... + P_31 in that order.
-// Block (b, 32-dimension group) of 32 warps: warp w forms P_w for the 32
-// dimensions of its lanes (coalesced rows), warp 0 adds the partials.
-__global__ void __launch_bounds__(1024) center_kernel(const float* __restrict__ c, int B, int K,
-                                                      int D, float* __restrict__ m,
-                                                      const double* __restrict__ cn) {
-  __shared__ double part[32][33];
+// m[b][d] = fp32(S / K), S summed in fp64 in one fixed order that does not
+// depend on the launch (the fused end-of-iteration kernel below follows the
+// same order, so both give m bit for bit): the padded rows [0, Kp) are cut
+// into MEAN_CHUNKS contiguous chunks of R = Kp / MEAN_CHUNKS rows; partial
+// (r, w) of chunk r sums the rows r*R + w, r*R + w + MEAN_WAYS, ... below K in
+// ascending order; a chunk adds its partials in order w = 0, 1, ..., and S
+// adds the chunks in order r = 0, 1, ....  Grid (B, 32-dimension groups,
+// MEAN_CHUNKS), one cluster of MEAN_CHUNKS CTAs per (batch, group): CTA r
+// forms chunk r, warp w partial (r, w) for the 32 dimensions of its lanes
+// (coalesced rows, eight rows' loads in flight), and CTA 0 adds the chunks
+// from distributed shared memory.
+__global__ void __cluster_dims__(1, 1, MEAN_CHUNKS) __launch_bounds__(MEAN_WAYS * 32)
+    center_kernel(const float* __restrict__ c, int B, int K, int Kp, int D,
+                  float* __restrict__ m, const double* __restrict__ cn) {
+  __shared__ double part[MEAN_WAYS][33];
+  __shared__ double chunk[32];
   const int b = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int r = (int)ptx::cluster_ctarank();   // == blockIdx.z
   const int d = blockIdx.y * 32 + lane;
+  const int R = Kp / MEAN_CHUNKS;
   double s = 0.0;
   if (d < D) {
     const float* p = c + (int64_t)b * K * D + d;
     const int64_t row0 = (int64_t)b * K;
-    int k = w;
-    // sixteen rows' loads in flight at once, added in the same ascending order
-    for (; k + 15 * 32 < K; k += 16 * 32) {
-      float v[16];
+    const int k0 = r * R + w;
+    int i = 0;
+    for (; i + 7 * MEAN_WAYS < R; i += 8 * MEAN_WAYS) {
+      float v[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = p[(int64_t)(k + 32 * j) * D];
+      for (int j = 0; j < 8; ++j) {
+        const int k = k0 + i + j * MEAN_WAYS;
+        v[j] = k < K ? p[(int64_t)k * D] : 0.0f;
+      }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) s += (double)metric_elem(v[j], cn, row0 + k + 32 * j);
+      for (int j = 0; j < 8; ++j) {
+        const int k = k0 + i + j * MEAN_WAYS;
+        if (k < K) s += (double)metric_elem(v[j], cn, row0 + k);
+      }
     }
-    for (; k < K; k += 32) s += (double)metric_elem(p[(int64_t)k * D], cn, row0 + k);
+    for (; i < R; i += MEAN_WAYS) {
+      const int k = k0 + i;
+      if (k < K) s += (double)metric_elem(p[(int64_t)k * D], cn, row0 + k);
+    }
   }
   part[w][lane] = s;
   __syncthreads();
-  if (w == 0 && d < D) {
+  if (w == 0) {
     double t = 0.0;
 #pragma unroll 1
-    for (int j = 0; j < 32; ++j) t += part[j][lane];
+    for (int q = 0; q < MEAN_WAYS; ++q) t += part[q][lane];
+    chunk[lane] = t;
+  }
+  ptx::cluster_sync();   // every chunk's sums visible across the cluster
+  if (r == 0 && w == 0 && d < D) {
+    double t = 0.0;
+#pragma unroll 1
+    for (int q = 0; q < MEAN_CHUNKS; ++q)
+      t += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&chunk[lane], q));
     m[(int64_t)b * D + d] = (float)(t / (double)K);
   }
+  ptx::cluster_sync();   // no CTA leaves while CTA 0 still reads its shared memory
 }
 
 // v split into three 16-bit parts whose weighted sum is v to about 24 bits:
@@ -142,21 +170,17 @@ __device__ __forceinline__ uint16_t q16(float v, bool bf, float* back) {
   return __half_as_ushort(q);
 }
 
-// Four padded centroid rows per warp, eight lanes per row; each lane takes
-// four consecutive elements at a time (D is a multiple of 4 for every dtype:
-// the rows of x are 16-byte multiples).
-__global__ void prep_centroids_kernel(const float* __restrict__ c, const float* __restrict__ m,
-                                      int B, int K, int Kp, int D, int dtype,
-                                      void* __restrict__ cq, uint16_t* __restrict__ caug,
-                                      const double* __restrict__ cn, bool bias) {
-  const int lane = threadIdx.x & 31, l8 = lane & 7;
-  const int64_t row =
-      ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
-  const bool valid = row < (int64_t)B * Kp;
-  const int b = valid ? (int)(row / Kp) : 0, k = valid ? (int)(row % Kp) : 0;
-  const bool real = valid && k < K;
-  const float* src = c + ((int64_t)b * K + k) * D;
-  const float* mb = m + (int64_t)b * D;
+// One padded centroid row, eight lanes per row (l8 = lane & 7); each lane
+// takes four consecutive elements at a time (D is a multiple of 4 for every
+// dtype: the rows of x are 16-byte multiples).  src: the fp32 centroid row
+// (read only when real), mb: the batch's mean centroid, crow: the row's index
+// b*K + k (cosine norms), row: its index b*Kp + k in the operands.  Every lane
+// of the warp calls this (the row's lanes exchange partial sums).
+__device__ __forceinline__ void prep_row(const float* __restrict__ src,
+                                         const float* __restrict__ mb, bool valid, bool real,
+                                         int64_t crow, int64_t row, int D, int dtype,
+                                         void* __restrict__ cq, uint16_t* __restrict__ caug,
+                                         const double* __restrict__ cn, bool bias, int l8) {
   double acc = 0.0;
   if (dtype == FKM_F32) {
     const int Dp = (D + 7) & ~7;
@@ -164,11 +188,9 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
     for (int d = 4 * l8; valid && d < D; d += 32) {
       const float4 mm = *reinterpret_cast<const float4*>(mb + d);
       float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
-      if (real && cn) {
-        const int64_t r = (int64_t)b * K + k;
-        cv = make_float4(metric_elem(cv.x, cn, r), metric_elem(cv.y, cn, r),
-                         metric_elem(cv.z, cn, r), metric_elem(cv.w, cn, r));
-      }
+      if (real && cn)
+        cv = make_float4(metric_elem(cv.x, cn, crow), metric_elem(cv.y, cn, crow),
+                         metric_elem(cv.z, cn, crow), metric_elem(cv.w, cn, crow));
       const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
       const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
       uint16_t hb[4], lb[4];
@@ -190,11 +212,9 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
     for (int d = 4 * l8; valid && d < D; d += 32) {
       const float4 mm = *reinterpret_cast<const float4*>(mb + d);
       float4 cv = real ? *reinterpret_cast<const float4*>(src + d) : mm;
-      if (real && cn) {
-        const int64_t r = (int64_t)b * K + k;
-        cv = make_float4(metric_elem(cv.x, cn, r), metric_elem(cv.y, cn, r),
-                         metric_elem(cv.z, cn, r), metric_elem(cv.w, cn, r));
-      }
+      if (real && cn)
+        cv = make_float4(metric_elem(cv.x, cn, crow), metric_elem(cv.y, cn, crow),
+                         metric_elem(cv.z, cn, crow), metric_elem(cv.w, cn, crow));
       const float v[4] = {cv.x - mm.x, cv.y - mm.y, cv.z - mm.z, cv.w - mm.w};
       const float mv[4] = {mm.x, mm.y, mm.z, mm.w};
       uint16_t qb[4];
@@ -221,6 +241,162 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
     const uint32_t lo = e == 0 ? parts[0] : e == 2 ? parts[2] : 0u;
     const uint32_t hi = e == 0 ? parts[1] : 0u;
     *reinterpret_cast<uint32_t*>(caug + row * AUG_SLAB + e) = lo | (hi << 16);
+  }
+}
+
+// Four padded centroid rows per warp.
+__global__ void prep_centroids_kernel(const float* __restrict__ c, const float* __restrict__ m,
+                                      int B, int K, int Kp, int D, int dtype,
+                                      void* __restrict__ cq, uint16_t* __restrict__ caug,
+                                      const double* __restrict__ cn, bool bias) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row =
+      ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
+  const bool valid = row < (int64_t)B * Kp;
+  const int b = valid ? (int)(row / Kp) : 0, k = valid ? (int)(row % Kp) : 0;
+  const bool real = valid && k < K;
+  prep_row(c + ((int64_t)b * K + k) * D, m + (int64_t)b * D, valid, real, (int64_t)b * K + k,
+           row, D, dtype, cq, caug, cn, bias, lane & 7);
+}
+
+// The end of a Euclidean Lloyd iteration in one launch: one thread-block
+// cluster of MEAN_CHUNKS CTAs per batch (grid MEAN_CHUNKS x B), CTA r owning
+// the padded rows [r R, (r+1) R), R = Kp / MEAN_CHUNKS.
+//   1. finalize (as finalize_kernel): warp w takes the rows r R + w,
+//      r R + w + MEAN_WAYS, ...: count, new centroid (s/n of a crossing run,
+//      the value the segment sums wrote for an interior one, the previous
+//      centroid for an empty cluster), its shift, and the running fp64 sums
+//      of the new centroid's columns -- partial (r, w) of the mean's order;
+//   2. the CTA adds its partials (w = 0, 1, ...), the cluster barrier makes
+//      every CTA's sums visible, and every CTA adds the chunks (r = 0, 1, ...)
+//      from distributed shared memory: m, bit for bit center_kernel's; CTA 0
+//      also writes m and the batch's shift (same chunked order);
+//   3. the CTA prepares the operands of its rows (prep_row) against m.
+// Columns are held four per lane, so D <= FP_MAX_D.
+constexpr int FP_WARPS = MEAN_WAYS;
+constexpr int FP_MAX_D = 256;
+
+struct FinPrepParams {
+  int B, K, Kp, D, dtype, range;
+  const int32_t* segstart;
+  const int32_t* segend;
+  double* sums64;      // crossing runs' fp64 sums, zeroed after use
+  const float* prev;
+  float* centers;
+  int32_t* counts;
+  float* m;
+  void* cq;
+  uint16_t* caug;
+  double* shift_out;   // optional [B]
+  double* max_shift;   // optional (zeroed by the caller): max over batches
+};
+
+__global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS * 32)
+    finalize_prep_kernel(FinPrepParams p) {
+  __shared__ double colsum[FP_WARPS][FP_MAX_D];
+  __shared__ double cta_sum[FP_MAX_D];
+  __shared__ double wshift[FP_WARPS];
+  __shared__ double cta_shift;
+  __shared__ __align__(16) float msh[FP_MAX_D];
+  const int r = (int)ptx::cluster_ctarank();
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int R = p.Kp / MEAN_CHUNKS;
+  const int D = p.D;
+  const int64_t kb = (int64_t)b * p.K;
+
+  // ---- 1. finalize this CTA's rows
+  constexpr int J = FP_MAX_D / 128;   // four-column pieces per lane
+  double cs[J][4];
+#pragma unroll
+  for (int j = 0; j < J; ++j) cs[j][0] = cs[j][1] = cs[j][2] = cs[j][3] = 0.0;
+  double shw = 0.0;
+  for (int k = r * R + warp; k < r * R + R && k < p.K; k += FP_WARPS) {
+    const int64_t key = kb + k;
+    const int32_t s0 = p.segstart[key], s1 = p.segend[key];
+    const int32_t nk = s1 - s0;
+    const bool interior = nk > 0 && (s0 / p.range) == ((s1 - 1) / p.range);
+    if (lane == 0 && p.counts) p.counts[key] = nk;
+    double sh = 0.0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int d = 4 * lane + 128 * j;
+      if (d >= D) break;
+      const int64_t e = key * D + d;
+      const float4 pv = *reinterpret_cast<const float4*>(p.prev + e);
+      float4 v;
+      if (nk == 0) {
+        v = pv;
+      } else if (interior) {
+        v = *reinterpret_cast<const float4*>(p.centers + e);
+      } else {
+        double2* s2 = reinterpret_cast<double2*>(p.sums64 + e);
+        const double2 a = s2[0], c = s2[1];
+        const double n = (double)nk;
+        v = make_float4((float)(a.x / n), (float)(a.y / n), (float)(c.x / n), (float)(c.y / n));
+        s2[0] = make_double2(0.0, 0.0);
+        s2[1] = make_double2(0.0, 0.0);
+      }
+      *reinterpret_cast<float4*>(p.centers + e) = v;
+      const double d0 = (double)v.x - (double)pv.x, d1 = (double)v.y - (double)pv.y;
+      const double d2 = (double)v.z - (double)pv.z, d3 = (double)v.w - (double)pv.w;
+      sh += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
+      cs[j][0] += (double)v.x;
+      cs[j][1] += (double)v.y;
+      cs[j][2] += (double)v.z;
+      cs[j][3] += (double)v.w;
+    }
+    shw += warp_sum(sh);   // the same value in every lane
+  }
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int d = 4 * lane + 128 * j;
+    if (d < D) {
+      colsum[warp][d] = cs[j][0];
+      colsum[warp][d + 1] = cs[j][1];
+      colsum[warp][d + 2] = cs[j][2];
+      colsum[warp][d + 3] = cs[j][3];
+    }
+  }
+  if (lane == 0) wshift[warp] = shw;
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    double t = 0.0;
+#pragma unroll 1
+    for (int w = 0; w < FP_WARPS; ++w) t += colsum[w][d];
+    cta_sum[d] = t;
+  }
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+#pragma unroll 1
+    for (int w = 0; w < FP_WARPS; ++w) t += wshift[w];
+    cta_shift = t;
+  }
+  // ---- 2. the batch's mean and shift across the cluster
+  ptx::cluster_sync();   // release / acquire: every CTA's sums (and centroids) visible
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    double t = 0.0;
+#pragma unroll 1
+    for (int q = 0; q < MEAN_CHUNKS; ++q) t += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&cta_sum[d], q));
+    msh[d] = (float)(t / (double)p.K);
+    if (r == 0) p.m[(int64_t)b * D + d] = msh[d];
+  }
+  if (r == 0 && threadIdx.x == 0) {
+    double t = 0.0;
+#pragma unroll 1
+    for (int q = 0; q < MEAN_CHUNKS; ++q) t += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&cta_shift, q));
+    if (p.shift_out) p.shift_out[b] = t;
+    if (p.max_shift)   // shift >= 0: the bit pattern orders like the value
+      atomicMax(reinterpret_cast<unsigned long long*>(p.max_shift),
+                (unsigned long long)__double_as_longlong(t));
+  }
+  ptx::cluster_sync();   // no CTA leaves while another still reads its shared memory
+  // ---- 3. the next assign's operands for this CTA's rows
+  for (int i = warp * 4 + (lane >> 3); i < R; i += FP_WARPS * 4) {
+    const int k = r * R + i;
+    const bool real = k < p.K;
+    prep_row(p.centers + (kb + k) * D, msh, true, real, kb + k, (int64_t)b * p.Kp + k, D,
+             p.dtype, p.cq, p.caug, nullptr, true, lane & 7);
   }
 }
 
@@ -289,14 +465,54 @@ fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int
     note_launch();
     cn = cnorm;
   }
-  center_kernel<<<dim3((unsigned)B, (unsigned)ceil_div(D, 32)), 1024, 0, st>>>(centers, B, K, D,
-                                                                              m, cn);
+  center_kernel<<<dim3((unsigned)B, (unsigned)ceil_div(D, 32), MEAN_CHUNKS), MEAN_WAYS * 32, 0,
+                  st>>>(centers, B, K, Kp, D, m, cn);
   const int64_t rows = (int64_t)B * Kp;
   const int wpb = 8;   // 4 rows per warp
   prep_centroids_kernel<<<(unsigned)ceil_div(rows, 4 * wpb), wpb * 32, 0, st>>>(
       centers, m, B, K, Kp, D, dtype, cq, static_cast<uint16_t*>(caug), cn,
       metric == FKM_METRIC_EUCLID);
   note_launch(2);
+  FKM_CUDA_TRY(cudaGetLastError());
+  return FKM_OK;
+}
+
+// A CTA finalizes and prepares Kp / MEAN_CHUNKS rows, one after another per
+// warp; beyond 128 rows (Kp > 1024) the separate kernels, with every row
+// in its own warp, finish sooner.
+bool finalize_prep_fits(int B, int Kp, int D) {
+  return D <= FP_MAX_D && B <= 65535 && Kp <= 1024;
+}
+
+fkm_status launch_finalize_prep(int B, int K, int Kp, int D, int dtype, int range,
+                                const int32_t* segstart, const int32_t* segend, double* sums64,
+                                const float* prev, float* centers, int32_t* counts, float* m,
+                                void* cq, void* caug, double* shift_out, double* max_shift,
+                                cudaStream_t st) {
+  if (!finalize_prep_fits(B, Kp, D) || Kp % BN != 0) {
+    set_error("finalize_prep: D = %d or Kp = %d out of range", D, Kp);
+    return FKM_ERR_INTERNAL;
+  }
+  FinPrepParams p;
+  p.B = B;
+  p.K = K;
+  p.Kp = Kp;
+  p.D = D;
+  p.dtype = dtype;
+  p.range = range;
+  p.segstart = segstart;
+  p.segend = segend;
+  p.sums64 = sums64;
+  p.prev = prev;
+  p.centers = centers;
+  p.counts = counts;
+  p.m = m;
+  p.cq = cq;
+  p.caug = static_cast<uint16_t*>(caug);
+  p.shift_out = shift_out;
+  p.max_shift = max_shift;
+  finalize_prep_kernel<<<dim3(MEAN_CHUNKS, (unsigned)B), FP_WARPS * 32, 0, st>>>(p);
+  note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
 }

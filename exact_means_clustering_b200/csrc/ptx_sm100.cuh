@@ -1,6 +1,7 @@
-// Thin inline-PTX wrappers for the sm_100a features the assign kernel uses:
+// Thin inline-PTX wrappers for the sm_100a features the kernels use:
 // mbarriers (with bounded waits), TMA tile loads (no multicast), tcgen05
-// tensor-memory allocation, MMA, commit, loads and fences.
+// tensor-memory allocation, MMA, commit, loads and fences, and the cluster
+// barrier and distributed-shared-memory loads.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -308,10 +309,19 @@ __device__ __forceinline__ void mma_commit_pair_mc(uint64_t* bar, uint16_t cta_m
       : "memory");
 }
 
-// Whole-cluster barrier (every thread of both CTAs).
+// Whole-cluster barrier (every thread of every CTA of the cluster), with
+// release / acquire ordering of the memory operations around it.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
+}
+
+// fp64 load from the shared memory of a CTA of this cluster, at a cluster
+// address from mapa_rank.
+__device__ __forceinline__ double ld_shared_cluster_f64(uint32_t addr) {
+  double v;
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // 3-input minimum (sm_100a).

@@ -24,6 +24,9 @@
 //               centroid for empty clusters (a reading: the pages give only
 //               c = s/n), and the shift ||c_new - c_old||^2.
 //   batch_reduce  per batch, in fixed order: shift = sum_k shift_k.
+// Inside the Lloyd loop, for D <= 256 and Kp <= 1024, finalize and the batch
+// shifts run fused with the next assign's operand preparation
+// (finalize_prep_kernel, prep.cu).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
