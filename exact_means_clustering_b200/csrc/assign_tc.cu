@@ -277,6 +277,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   const int nQ = p.nD * (kSplit ? 2 : 1);   // stages per centroid tile
+  // the set-up above touched only this CTA's shared memory and TMEM; global
+  // memory waits for the previous kernel of the stream
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -631,6 +635,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ASSIGN_THREADS, 1)
   ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+  // the set-up above touched only the pair's shared memory and TMEM; global
+  // memory waits for the previous kernel of the stream
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producers (both CTAs)
@@ -1002,7 +1010,8 @@ static fkm_status launch_assign_pair(const AssignArgs& a, cudaStream_t st) {
   int clusters = (dev >= 0 && dev < 64 && pair_clusters[dev] > 0) ? pair_clusters[dev]
                                                                     : num_sms() / 2;
   if (clusters > p.n_work) clusters = p.n_work;
-  assign_pair_kernel<<<2 * clusters, ASSIGN_THREADS, smem, st>>>(tx, tc, taug, p);
+  FKM_CUDA_TRY(launch_pdl(assign_pair_kernel, dim3(2 * clusters), dim3(ASSIGN_THREADS), smem, st,
+                          tx, tc, taug, p));
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;

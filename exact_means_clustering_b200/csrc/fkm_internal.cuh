@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "fkm.h"
@@ -29,6 +30,33 @@ __device__ __forceinline__ bool fkm_in_range(int64_t i, int64_t n, int* status) 
   if (i >= 0 && i < n) return true;
   if (status) atomicOr(status, ST_OOB);
   return false;
+}
+
+// Programmatic dependent launch.  The kernels of one Lloyd iteration follow
+// each other on one stream; launched with launch_pdl, a kernel's CTAs may be
+// scheduled while the kernel before it drains.  Every such kernel calls
+// pdl_wait() before it reads or writes global memory: it returns once the
+// previous grid has completed and its writes are visible (at once for a
+// kernel launched the ordinary way).  pdl_trigger() lets the next kernel be
+// scheduled once every CTA of this grid has called it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Assign tiling: 128 points (TMEM lanes) x 256 centroids (TMEM columns) per

@@ -53,6 +53,8 @@ __device__ __forceinline__ float metric_elem(float c, const double* cn, int64_t 
 // ||c|| of every centroid row (fp64 sum of squares); one warp per row.
 __global__ void row_norms_kernel(const float* __restrict__ c, int64_t rows, int D,
                                  double* __restrict__ cn) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -79,6 +81,8 @@ __global__ void row_norms_kernel(const float* __restrict__ c, int64_t rows, int 
 __global__ void __cluster_dims__(1, 1, MEAN_CHUNKS) __launch_bounds__(MEAN_WAYS * 32)
     center_kernel(const float* __restrict__ c, int B, int K, int Kp, int D,
                   float* __restrict__ m, const double* __restrict__ cn) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   __shared__ double part[MEAN_WAYS][33];
   __shared__ double chunk[32];
   const int b = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -249,6 +253,8 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
                                       int B, int K, int Kp, int D, int dtype,
                                       void* __restrict__ cq, uint16_t* __restrict__ caug,
                                       const double* __restrict__ cn, bool bias) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t row =
       ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
@@ -293,6 +299,8 @@ struct FinPrepParams {
 
 __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS * 32)
     finalize_prep_kernel(FinPrepParams p) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   __shared__ double colsum[FP_WARPS][FP_MAX_D];
   __shared__ double cta_sum[FP_MAX_D];
   __shared__ double wshift[FP_WARPS];
@@ -377,14 +385,16 @@ __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS *
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     double t = 0.0;
 #pragma unroll 1
-    for (int q = 0; q < MEAN_CHUNKS; ++q) t += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&cta_sum[d], q));
+    for (int q = 0; q < MEAN_CHUNKS; ++q)
+      t += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&cta_sum[d], q));
     msh[d] = (float)(t / (double)p.K);
     if (r == 0) p.m[(int64_t)b * D + d] = msh[d];
   }
   if (r == 0 && threadIdx.x == 0) {
     double t = 0.0;
 #pragma unroll 1
-    for (int q = 0; q < MEAN_CHUNKS; ++q) t += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&cta_shift, q));
+    for (int q = 0; q < MEAN_CHUNKS; ++q)
+      t += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&cta_shift, q));
     if (p.shift_out) p.shift_out[b] = t;
     if (p.max_shift)   // shift >= 0: the bit pattern orders like the value
       atomicMax(reinterpret_cast<unsigned long long*>(p.max_shift),
@@ -461,17 +471,18 @@ fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int
   const double* cn = nullptr;
   if (metric == FKM_METRIC_COSINE) {
     const int64_t rows = (int64_t)B * K;
-    row_norms_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(centers, rows, D, cnorm);
+    FKM_CUDA_TRY(launch_pdl(row_norms_kernel, dim3((unsigned)ceil_div(rows, 8)), dim3(256), 0, st,
+                            centers, rows, D, cnorm));
     note_launch();
     cn = cnorm;
   }
-  center_kernel<<<dim3((unsigned)B, (unsigned)ceil_div(D, 32), MEAN_CHUNKS), MEAN_WAYS * 32, 0,
-                  st>>>(centers, B, K, Kp, D, m, cn);
+  FKM_CUDA_TRY(launch_pdl(center_kernel, dim3((unsigned)B, (unsigned)ceil_div(D, 32), MEAN_CHUNKS),
+                          dim3(MEAN_WAYS * 32), 0, st, centers, B, K, Kp, D, m, cn));
   const int64_t rows = (int64_t)B * Kp;
   const int wpb = 8;   // 4 rows per warp
-  prep_centroids_kernel<<<(unsigned)ceil_div(rows, 4 * wpb), wpb * 32, 0, st>>>(
-      centers, m, B, K, Kp, D, dtype, cq, static_cast<uint16_t*>(caug), cn,
-      metric == FKM_METRIC_EUCLID);
+  FKM_CUDA_TRY(launch_pdl(prep_centroids_kernel, dim3((unsigned)ceil_div(rows, 4 * wpb)),
+                          dim3(wpb * 32), 0, st, centers, m, B, K, Kp, D, dtype, cq,
+                          static_cast<uint16_t*>(caug), cn, metric == FKM_METRIC_EUCLID));
   note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
@@ -511,7 +522,8 @@ fkm_status launch_finalize_prep(int B, int K, int Kp, int D, int dtype, int rang
   p.caug = static_cast<uint16_t*>(caug);
   p.shift_out = shift_out;
   p.max_shift = max_shift;
-  finalize_prep_kernel<<<dim3(MEAN_CHUNKS, (unsigned)B), FP_WARPS * 32, 0, st>>>(p);
+  FKM_CUDA_TRY(launch_pdl(finalize_prep_kernel, dim3(MEAN_CHUNKS, (unsigned)B), dim3(FP_WARPS * 32),
+                          0, st, p));
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;

@@ -90,6 +90,8 @@ template <bool kFirst>
 __global__ void __launch_bounds__(SORT_THREADS) radix_upsweep(KeySrc s, int64_t n, int shift,
                                                               int bits, int n_tiles,
                                                               uint32_t* hist) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   const int nbins = 1 << bits;
   __shared__ uint32_t h[SORT_THREADS / 32][RADIX_BINS];
   const int warp = threadIdx.x >> 5;
@@ -153,6 +155,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 
 __global__ void __launch_bounds__(kScanBlock) scan_reduce(const uint32_t* in, int64_t len,
                                                           uint32_t* part) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   __shared__ uint32_t sw[32];
   uint32_t t = 0;
   const int64_t base = (int64_t)blockIdx.x * kScanChunk;
@@ -170,6 +174,8 @@ __global__ void __launch_bounds__(kScanBlock) scan_reduce(const uint32_t* in, in
 // a few thousand words in L2), so no separate pass scans the chunk totals.
 __global__ void __launch_bounds__(kScanBlock) scan_apply(uint32_t* data, int64_t len,
                                                          const uint32_t* part) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   __shared__ uint32_t sw[32];
   uint32_t earlier = 0;
   for (int64_t j = threadIdx.x; j < (int64_t)blockIdx.x; j += kScanBlock) earlier += part[j];
@@ -207,6 +213,8 @@ __global__ void __launch_bounds__(DS_THREADS, 2) radix_downsweep(KeySrc s, int64
                                                               const uint32_t* __restrict__ hist,
                                                               int32_t* __restrict__ keys_out,
                                                               int32_t* __restrict__ vals_out) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   constexpr int NW = DS_THREADS / 32;
   constexpr int PER_WARP = SORT_TILE / NW;  // 256 consecutive keys per warp
   static_assert(NW * (RADIX_BINS + 1) <= 2 * SORT_TILE, "the counters fit the staging area");
@@ -321,6 +329,8 @@ struct CsArgs {
 
 // Tile histogram: bins 0..K-1 are the ids, bin K the rejected ids.
 __global__ void __launch_bounds__(SORT_THREADS) cs_hist_kernel(CsArgs a) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   extern __shared__ uint32_t h[];   // K + 1
   const int tg = blockIdx.x, b = tg / a.tpb, t = tg % a.tpb;
   for (int i = threadIdx.x; i <= a.K; i += SORT_THREADS) h[i] = 0;
@@ -375,6 +385,8 @@ __host__ __device__ __forceinline__ size_t cs_scatter_smem_bytes(int K) {
 // Tile 0 of each batch also writes that batch's segment bounds.  Four blocks
 // per SM keep a 32-batch grid of 16 tiles each (512 blocks) in one wave.
 __global__ void __launch_bounds__(SORT_THREADS, 4) cs_scatter_kernel(CsArgs a) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   constexpr int NW = SORT_THREADS / 32;
   constexpr int PER_WARP = SORT_TILE / NW;
   extern __shared__ uint32_t smem[];
@@ -498,6 +510,8 @@ __global__ void __launch_bounds__(SORT_THREADS, 4) cs_scatter_kernel(CsArgs a) {
 // and writes the batch's segment bounds.  Batch b's keys occupy positions
 // [b*N, (b+1)*N).  One launch instead of five.
 __global__ void __launch_bounds__(SORT_THREADS) cs_single_tile_kernel(CsArgs a) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   constexpr int NW = SORT_THREADS / 32;
   constexpr int PER_WARP = SORT_TILE / NW;
   extern __shared__ uint32_t cnt[];   // NW * (K + 1) per-warp counters, then K + 1 bin starts
@@ -575,8 +589,10 @@ __global__ void __launch_bounds__(SORT_THREADS) cs_single_tile_kernel(CsArgs a) 
 
 fkm_status device_scan(uint32_t* data, int64_t len, uint32_t* part, cudaStream_t st) {
   const int64_t nparts = ceil_div(len, kScanChunk);
-  scan_reduce<<<(unsigned)nparts, kScanBlock, 0, st>>>(data, len, part);
-  scan_apply<<<(unsigned)nparts, kScanBlock, 0, st>>>(data, len, part);
+  FKM_CUDA_TRY(launch_pdl(scan_reduce, dim3((unsigned)nparts), dim3(kScanBlock), 0, st,
+                          data, len, part));
+  FKM_CUDA_TRY(launch_pdl(scan_apply, dim3((unsigned)nparts), dim3(kScanBlock), 0, st,
+                          data, len, part));
   note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
@@ -639,14 +655,16 @@ fkm_status launch_count_sort_ids(SortArgs& s, int B, int32_t* segstart, int32_t*
   const unsigned tiles = (unsigned)((int64_t)B * a.tpb);
   if (ids_valid && a.tpb == 1) {
     const size_t smem = (size_t)(SORT_THREADS / 32 + 1) * (a.K + 1) * 4;
-    cs_single_tile_kernel<<<(unsigned)B, SORT_THREADS, smem, st>>>(a);
+    FKM_CUDA_TRY(launch_pdl(cs_single_tile_kernel, dim3((unsigned)B), dim3(SORT_THREADS), smem,
+                            st, a));
     note_launch();
     FKM_CUDA_TRY(cudaGetLastError());
     return FKM_OK;
   }
-  cs_hist_kernel<<<tiles, SORT_THREADS, (a.K + 1) * 4, st>>>(a);
+  FKM_CUDA_TRY(launch_pdl(cs_hist_kernel, dim3(tiles), dim3(SORT_THREADS), (a.K + 1) * 4, st, a));
   FKM_TRY(device_scan(a.hist, cs_hist_words(B, s.N, s.K), s.hist_part, st));
-  cs_scatter_kernel<<<tiles, SORT_THREADS, cs_scatter_smem_bytes(a.K), st>>>(a);
+  FKM_CUDA_TRY(launch_pdl(cs_scatter_kernel, dim3(tiles), dim3(SORT_THREADS),
+                          cs_scatter_smem_bytes(a.K), st, a));
   note_launch(2);
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
@@ -680,19 +698,19 @@ fkm_status launch_argsort_ids(SortArgs& a, cudaStream_t st) {
     if (p == 0) {
       s.keys = nullptr;
       s.vals = nullptr;
-      radix_upsweep<true><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
-                                                            a.hist);
+      FKM_CUDA_TRY(launch_pdl((radix_upsweep<true>), dim3(n_tiles), dim3(SORT_THREADS), 0, st,
+                              s, a.n, shift, bits, n_tiles, a.hist));
       FKM_TRY(device_scan(a.hist, hlen, a.hist_part, st));
-      radix_downsweep<true><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
-                                                              a.hist, kout[0], vout[0]);
+      FKM_CUDA_TRY(launch_pdl((radix_downsweep<true>), dim3(n_tiles), dim3(DS_THREADS), 0, st,
+                              s, a.n, shift, bits, n_tiles, a.hist, kout[0], vout[0]));
     } else {
       s.keys = kout[(p - 1) & 1];
       s.vals = vout[(p - 1) & 1];
-      radix_upsweep<false><<<n_tiles, SORT_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
-                                                             a.hist);
+      FKM_CUDA_TRY(launch_pdl((radix_upsweep<false>), dim3(n_tiles), dim3(SORT_THREADS), 0, st,
+                              s, a.n, shift, bits, n_tiles, a.hist));
       FKM_TRY(device_scan(a.hist, hlen, a.hist_part, st));
-      radix_downsweep<false><<<n_tiles, DS_THREADS, 0, st>>>(s, a.n, shift, bits, n_tiles,
-                                                               a.hist, kout[p & 1], vout[p & 1]);
+      FKM_CUDA_TRY(launch_pdl((radix_downsweep<false>), dim3(n_tiles), dim3(DS_THREADS), 0, st,
+                              s, a.n, shift, bits, n_tiles, a.hist, kout[p & 1], vout[p & 1]));
     }
     FKM_CUDA_TRY(cudaGetLastError());
     note_launch(2);

@@ -216,6 +216,8 @@ __device__ __forceinline__ void cp_async_wait_stages() {
 template <int DT, int RPS>
 __global__ void __launch_bounds__(SEG_WARPS * 32, FKM_SEG_MIN_BLOCKS)
     segsum_kernel(SegParams p) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   constexpr int E = Vec<DT>::E;
   constexpr int LPR = 32 / RPS;
   extern __shared__ __align__(16) uint8_t seg_smem[];
@@ -521,6 +523,8 @@ struct FinParams {
 // consecutive elements per step (16-byte loads and stores), so a cluster of
 // D <= 128 takes one step.
 __global__ void finalize_kernel(FinParams p) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   const int64_t key = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (key >= (int64_t)p.B * p.K) return;
@@ -606,6 +610,8 @@ struct FinSimParams {
 };
 
 __global__ void finalize_sim_kernel(FinSimParams p) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   const int64_t key = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (key >= (int64_t)p.B * p.K) return;
@@ -733,6 +739,8 @@ __global__ void finalize_sim_kernel(FinSimParams p) {
 // one block per batch; fixed-order tree sum
 __global__ void __launch_bounds__(256) batch_reduce_kernel(int K, const double* __restrict__ shiftk,
                                                            double* shift_out, double* max_shift) {
+  pdl_wait();   // the previous kernel of the stream has completed
+  pdl_trigger();
   __shared__ double s1[256];
   const int b = blockIdx.x;
   double a = 0.0;
@@ -755,7 +763,8 @@ template <int DT, int RPS>
 fkm_status run_segsum(const SegParams& sp, cudaStream_t st) {
   const int64_t nranges = ceil_div(sp.n, sp.range);
   const int64_t blocks = ceil_div(nranges, SEG_WARPS);
-  segsum_kernel<DT, RPS><<<(unsigned)blocks, SEG_WARPS * 32, SEG_SMEM_BYTES, st>>>(sp);
+  FKM_CUDA_TRY(launch_pdl((segsum_kernel<DT, RPS>), dim3((unsigned)blocks), dim3(SEG_WARPS * 32),
+                          SEG_SMEM_BYTES, st, sp));
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
@@ -894,7 +903,8 @@ fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const i
   fp.counts_in = counts_in;
   const int64_t keys = (int64_t)B * K;
   const int wpb = 8;
-  finalize_kernel<<<(unsigned)ceil_div(keys, wpb), wpb * 32, 0, st>>>(fp);
+  FKM_CUDA_TRY(launch_pdl(finalize_kernel, dim3((unsigned)ceil_div(keys, wpb)), dim3(wpb * 32), 0,
+                          st, fp));
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
@@ -920,7 +930,8 @@ fkm_status launch_finalize_sim(int B, int K, int D, int metric, const int32_t* s
   fp.objk = objk;
   fp.clear_sums = true;
   const int64_t keys = (int64_t)B * K;
-  finalize_sim_kernel<<<(unsigned)ceil_div(keys, 8), 256, 0, st>>>(fp);
+  FKM_CUDA_TRY(launch_pdl(finalize_sim_kernel, dim3((unsigned)ceil_div(keys, 8)), dim3(256), 0, st,
+                          fp));
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
@@ -928,7 +939,8 @@ fkm_status launch_finalize_sim(int B, int K, int D, int metric, const int32_t* s
 
 fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift_out,
                                double* max_shift, cudaStream_t st) {
-  batch_reduce_kernel<<<B, 256, 0, st>>>(K, shiftk, shift_out, max_shift);
+  FKM_CUDA_TRY(launch_pdl(batch_reduce_kernel, dim3(B), dim3(256), 0, st,
+                          K, shiftk, shift_out, max_shift));
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
