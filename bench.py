@@ -659,7 +659,9 @@ def main():
     else:
         bound_note = "bf16/fp16 operands, fp32 accumulate"
     traffic = assign_traffic(wr.name)
-    roofline = {"bound": "tensor", "kernel": "assign_tc_kernel", "achieved": tflops,
+    # 16-bit points with rows of at most 256 elements run on CTA pairs
+    kname = "assign_pair_kernel" if wr.dtype != "f32" and wr.D <= 256 else "assign_tc_kernel"
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": tflops,
                 "peak": peak_t, "unit": "TFLOP/s",
                 "frac": (tflops / peak_t) if tflops else None, "traffic": traffic,
                 "peak_source": f"{peak_src} (bf16 burst, MEASURED_PEAKS.json)",

@@ -55,6 +55,8 @@ _SIG = {
     "fkm_host_workspace_size": ([_I, _I, _I, _I, _I, _L, ctypes.POINTER(_Z)], _I),
     "fkm_lloyd_host": ([_I, _I, _I, _I, _I, _P, _P, _I, _F, _L, _P, _P, _P, _P,
                         ctypes.POINTER(_I), _P, _Z, _P], _I),
+    "fkm_lloyd_host_metric": ([_I, _I, _I, _I, _I, _I, _P, _P, _I, _F, _L, _P, _P, _P, _P,
+                               ctypes.POINTER(_I), _P, _Z, _P], _I),
     "fkm_argsort_workspace_size": ([_L, _I, ctypes.POINTER(_Z)], _I),
     "fkm_argsort": ([_P, _L, _I, _P, _P, _P, _Z, _P], _I),
     "fkm_baseline_assign": ([_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P], _I),
@@ -369,6 +371,30 @@ def fkm_lloyd_host(x_host, init_centers, max_iters, tol, chunk_rows, ids, center
     _check(f, lib().fkm_lloyd_host(B, N, K, D, dt, px, pi, max_iters, float(tol),
                                    int(chunk_rows), *outs, ctypes.byref(n_iter), wp, wn,
                                    _stream(stream)))
+    return n_iter.value
+
+
+def fkm_lloyd_host_metric(x_host, init_centers, max_iters, tol, chunk_rows, ids, centers,
+                          counts, metric, objective=None, ws=None, stream=None) -> int:
+    """fkm_lloyd_host under metric ('euclid', 'dot', 'cosine'); x_host: a pinned
+    CPU tensor [B, N, D]."""
+    f = "fkm_lloyd_host_metric"
+    B, N, D = _dims(f, x_host, 3, "x_host")
+    dt = _dt(x_host)
+    K = _dims(f, init_centers, 3, "init_centers")[1]
+    A = _Args(f, stream, init_centers)
+    px = A.host("x_host", x_host, (B, N, D))
+    pi = A.dev("init_centers", init_centers, (B, K, D), torch.float32)
+    outs = (A.dev("ids", ids, (B, N), torch.int32),
+            A.dev("centers", centers, (B, K, D), torch.float32),
+            A.dev("counts", counts, (B, K), torch.int32),
+            A.dev("objective", objective, (B,), torch.float64))
+    wp, wn = A.ws(_ws(ws, fkm_host_workspace_size(B, N, K, D, dt, chunk_rows),
+                      init_centers.device))
+    n_iter = ctypes.c_int(0)
+    _check(f, lib().fkm_lloyd_host_metric(B, N, K, D, dt, _metric(metric), px, pi, max_iters,
+                                          float(tol), int(chunk_rows), *outs,
+                                          ctypes.byref(n_iter), wp, wn, _stream(stream)))
     return n_iter.value
 
 

@@ -259,10 +259,12 @@ fkm_status launch_batch_reduce(int B, int K, const double* shiftk, double* shift
                                double* max_shift, cudaStream_t st);
 // dot-product / cosine k-means: new centroids, per-cluster shift and
 // objective share (objk [B*K]) from the segment sums; sums64 left zeroed.
+// counts_in (out-of-core): accumulated counts, every cluster's sum in sums64
+// (segstart / segend unused).
 fkm_status launch_finalize_sim(int B, int K, int D, int metric, const int32_t* segstart,
                                const int32_t* segend, double* sums64, const float* prev,
                                float* centers, int32_t* counts, double* shiftk, double* objk,
-                               cudaStream_t st, int range);
+                               cudaStream_t st, int range, const int32_t* counts_in = nullptr);
 
 fkm_status launch_baseline_argmin(const float* dist, int64_t rows, int K, int32_t* ids,
                                   cudaStream_t st);

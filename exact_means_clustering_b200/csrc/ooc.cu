@@ -40,7 +40,7 @@ struct HostLayout {
   int tiles_per_chunk;
   int key_bits;
   size_t status, xbuf[2], mvec, cq, caug, xs, xn, keys0, vals0, keys1, vals1, hist, hist_part,
-      segstart, segend, sums64, counts_acc, shiftk, cbuf, total;
+      segstart, segend, sums64, counts_acc, shiftk, cnorm, objk, cbuf, total;
 };
 
 int bits_for_value(int64_t v) {
@@ -104,6 +104,8 @@ fkm_status make_host_layout(int B, int N, int K, int D, int dtype, int64_t chunk
   l.sums64 = take(BK * D * 8);
   l.counts_acc = take(BK * 4);
   l.shiftk = take(BK * 8);
+  l.cnorm = take(BK * 8);   // cosine: centroid row norms
+  l.objk = take(BK * 8);    // dot / cosine: each cluster's share of the objective
   l.cbuf = take(2 * BK * D * 4);
   l.total = off;
   *out = l;
@@ -149,9 +151,9 @@ struct HostPartial {
 
 using namespace fkm;
 
-static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const void* x_host,
-                                  const float* init_centers, int max_iters, float tol,
-                                  int64_t chunk_rows, int32_t* ids, float* centers,
+static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, int metric,
+                                  const void* x_host, const float* init_centers, int max_iters,
+                                  float tol, int64_t chunk_rows, int32_t* ids, float* centers,
                                   int32_t* counts, double* inertia, int* n_iter, void* ws,
                                   size_t ws_bytes, void* stream, const HostPartial* part);
 
@@ -173,8 +175,23 @@ fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const void* x_h
                           const float* init_centers, int max_iters, float tol,
                           int64_t chunk_rows, int32_t* ids, float* centers, int32_t* counts,
                           double* inertia, int* n_iter, void* ws, size_t ws_bytes, void* stream) {
-  return lloyd_host_impl(B, N, K, D, dtype, x_host, init_centers, max_iters, tol, chunk_rows, ids,
-                         centers, counts, inertia, n_iter, ws, ws_bytes, stream, nullptr);
+  return lloyd_host_impl(B, N, K, D, dtype, FKM_METRIC_EUCLID, x_host, init_centers, max_iters,
+                         tol, chunk_rows, ids, centers, counts, inertia, n_iter, ws, ws_bytes,
+                         stream, nullptr);
+}
+
+fkm_status fkm_lloyd_host_metric(int B, int N, int K, int D, int dtype, int metric,
+                                 const void* x_host, const float* init_centers, int max_iters,
+                                 float tol, int64_t chunk_rows, int32_t* ids, float* centers,
+                                 int32_t* counts, double* objective, int* n_iter, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  if (metric != FKM_METRIC_EUCLID && metric != FKM_METRIC_DOT && metric != FKM_METRIC_COSINE) {
+    set_error("unknown metric %d", metric);
+    return FKM_ERR_INVALID_ARG;
+  }
+  return lloyd_host_impl(B, N, K, D, dtype, metric, x_host, init_centers, max_iters, tol,
+                         chunk_rows, ids, centers, counts, objective, n_iter, ws, ws_bytes,
+                         stream, nullptr);
 }
 
 fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype, const void* x_host,
@@ -195,16 +212,20 @@ fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype, const 
   int n_iter = 0;
   // counts is only checked for null and alignment on this path: the partial
   // pass adds into part.counts (fp64), never into the int32 output
-  return lloyd_host_impl(B, N, K, D, dtype, x_host, centers, 1, 0.0f, chunk_rows, ids,
-                         const_cast<float*>(centers), reinterpret_cast<int32_t*>(counts), obj,
-                         &n_iter, ws, ws_bytes, stream, &part);
+  return lloyd_host_impl(B, N, K, D, dtype, FKM_METRIC_EUCLID, x_host, centers, 1, 0.0f,
+                         chunk_rows, ids, const_cast<float*>(centers),
+                         reinterpret_cast<int32_t*>(counts), obj, &n_iter, ws, ws_bytes, stream,
+                         &part);
 }
 
 }  // extern "C"
 
-static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const void* x_host,
-                                  const float* init_centers, int max_iters, float tol,
-                                  int64_t chunk_rows, int32_t* ids, float* centers,
+// metric: FKM_METRIC_EUCLID, or dot / cosine k-means (fkm_lloyd_metric's
+// arithmetic: operands of the scaled rows, no bias, every cluster's objective
+// share from its sums in the finalize; inertia then receives that objective).
+static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, int metric,
+                                  const void* x_host, const float* init_centers, int max_iters,
+                                  float tol, int64_t chunk_rows, int32_t* ids, float* centers,
                                   int32_t* counts, double* inertia, int* n_iter, void* ws,
                                   size_t ws_bytes, void* stream, const HostPartial* part) {
   HostLayout L;
@@ -258,8 +279,11 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
   if (!part) FKM_CUDA_TRY(cudaMemsetAsync(sums64, 0, (size_t)B * K * D * 8, st));
   FKM_CUDA_TRY(cudaMemcpyAsync(cA, init_centers, cbytes, cudaMemcpyDeviceToDevice, st));
   float* mvec = static_cast<float*>(at(L.mvec));
+  const bool euclid = metric == FKM_METRIC_EUCLID;
+  double* cnorm = static_cast<double*>(at(L.cnorm));
+  double* objk = static_cast<double*>(at(L.objk));
   FKM_TRY(launch_prep_centroids(cA, B, K, L.Kp, D, dtype, mvec, at(L.cq),
-                                at(L.caug), st));
+                                at(L.caug), st, metric, cnorm));
   // The copy stream may only touch the workspace after the caller's earlier
   // work, unless the caller vouches that the chunk buffers are idle: then
   // the first chunk's copy starts at once and overlaps whatever is still
@@ -337,7 +361,8 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
         FKM_TRY(clear_seg_bounds(K, segstart, segend, st));   // the segment sums write them
         ObjArgs oa;
         oa.K = K;
-        oa.obj = inertia ? inertia + b : nullptr;
+        // the similarity objectives come from the cluster sums in the finalize
+        oa.obj = (inertia && euclid) ? inertia + b : nullptr;
         if (L.split) {
           oa.chat = cur + (size_t)b * K * D;
           oa.chat_bstride = 0;
@@ -364,10 +389,17 @@ static fkm_status lloyd_host_impl(int B, int N, int K, int D, int dtype, const v
       done = 1;
       break;
     }
-    FKM_TRY(launch_finalize(B, K, D, nullptr, nullptr, counts_acc, sums64, cur, nxt, counts,
-                            static_cast<double*>(at(L.shiftk)), st));
+    if (euclid) {
+      FKM_TRY(launch_finalize(B, K, D, nullptr, nullptr, counts_acc, sums64, cur, nxt, counts,
+                              static_cast<double*>(at(L.shiftk)), st));
+    } else {
+      FKM_TRY(launch_finalize_sim(B, K, D, metric, nullptr, nullptr, sums64, cur, nxt, counts,
+                                  static_cast<double*>(at(L.shiftk)), objk, st, SEG_RANGE,
+                                  counts_acc));
+      if (inertia) FKM_TRY(launch_batch_reduce(B, K, objk, inertia, nullptr, st));
+    }
     FKM_TRY(launch_prep_centroids(nxt, B, K, L.Kp, D, dtype, mvec, at(L.cq),
-                                  at(L.caug), st));
+                                  at(L.caug), st, metric, cnorm));
     if (tol > 0.0f) FKM_CUDA_TRY(cudaMemsetAsync(max_shift, 0, sizeof(double), st));
     FKM_TRY(launch_batch_reduce(B, K, static_cast<double*>(at(L.shiftk)), nullptr,
                                 tol > 0.0f ? max_shift : nullptr, st));

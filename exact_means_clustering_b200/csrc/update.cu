@@ -600,6 +600,7 @@ struct FinSimParams {
   int B, K, D, metric, range;
   const int32_t* segstart;
   const int32_t* segend;
+  const int32_t* counts_in;  // out-of-core: accumulated counts, every sum in sums64
   double* sums64;
   const float* prev;
   float* centers;
@@ -615,9 +616,15 @@ __global__ void finalize_sim_kernel(FinSimParams p) {
   const int64_t key = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (key >= (int64_t)p.B * p.K) return;
-  const int32_t s0 = p.segstart[key], t0 = p.segend[key];
-  const int32_t nk = t0 - s0;
-  const bool interior = nk > 0 && (s0 / p.range) == ((t0 - 1) / p.range);
+  int32_t nk;
+  bool interior = false;
+  if (p.counts_in) {
+    nk = p.counts_in[key];
+  } else {
+    const int32_t s0 = p.segstart[key], t0 = p.segend[key];
+    nk = t0 - s0;
+    interior = nk > 0 && (s0 / p.range) == ((t0 - 1) / p.range);
+  }
   const bool cosine = p.metric == FKM_METRIC_COSINE;
   const double n = (double)nk;
   if (p.D <= 128 && (p.D & 3) == 0) {
@@ -913,8 +920,9 @@ fkm_status launch_finalize(int B, int K, int D, const int32_t* segstart, const i
 fkm_status launch_finalize_sim(int B, int K, int D, int metric, const int32_t* segstart,
                                const int32_t* segend, double* sums64, const float* prev,
                                float* centers, int32_t* counts, double* shiftk, double* objk,
-                               cudaStream_t st, int range) {
+                               cudaStream_t st, int range, const int32_t* counts_in) {
   FinSimParams fp;
+  fp.counts_in = counts_in;
   fp.B = B;
   fp.K = K;
   fp.D = D;

@@ -201,6 +201,23 @@ FKM_API fkm_status fkm_lloyd_host(int B, int N, int K, int D, int dtype, const v
                           int64_t chunk_rows, int32_t* ids, float* centers, int32_t* counts,
                           double* inertia, int* n_iter, void* ws, size_t ws_bytes, void* stream);
 
+/* fkm_lloyd_host under a metric (fkm_metric): dot-product or cosine k-means
+ * with the host-streamed points, the same arithmetic as fkm_lloyd_metric
+ * (the README lists the metrics beside the Euclidean one; the pages stream
+ * host data for any run, "Large tensor Benchmark").  Every chunk's segment
+ * sums go to fp64 accumulators, and one finalize per iteration forms the new
+ * centroids, the shift and the objective [B] (may be NULL: the objective of
+ * the last assignment, against the centroids it used) from them.  Same
+ * workspace (fkm_host_workspace_size), validation and synchronisation as
+ * fkm_lloyd_host; FKM_METRIC_EUCLID gives exactly fkm_lloyd_host.  An
+ * unknown metric returns FKM_ERR_INVALID_ARG before any launch. */
+FKM_API fkm_status fkm_lloyd_host_metric(int B, int N, int K, int D, int dtype, int metric,
+                                         const void* x_host, const float* init_centers,
+                                         int max_iters, float tol, int64_t chunk_rows,
+                                         int32_t* ids, float* centers, int32_t* counts,
+                                         double* objective, int* n_iter, void* ws,
+                                         size_t ws_bytes, void* stream);
+
 /* Stable argsort of n int32 keys in [0, n_keys) on the device (the sort inside
  * fkm_update, exposed for tests): idx[r] = index of the r-th smallest key,
  * equal keys in index order ("Flash-KMeans：快速且内存高效精确K-Means聚类" summary,

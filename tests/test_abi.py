@@ -121,6 +121,12 @@ def test_metric_calls_reject_unknown_metric(fkm):
     assert b"metric" in L.fkm_last_error()
     # a known metric still validates its pointers first
     assert L.fkm_assign_metric(1, 16, 4, 64, 2, 2, None, a, a, a, 1 << 19, None) == 1
+    n = ctypes.c_int(0)
+    assert L.fkm_lloyd_host_metric(1, 16, 4, 64, 2, 3, a, a, 1, 0.0, 16, a, a, a, None,
+                                   ctypes.byref(n), a, 1 << 19, None) == 1
+    assert b"metric" in L.fkm_last_error()
+    assert L.fkm_lloyd_host_metric(1, 16, 4, 64, 2, 1, None, a, 1, 0.0, 16, a, a, a, None,
+                                   ctypes.byref(n), a, 1 << 19, None) == 1
 
 
 def test_status_strings_and_version(fkm):

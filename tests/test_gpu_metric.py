@@ -156,3 +156,72 @@ def test_batch_kmeans_metric_call(metric):
     n2 = torch.empty(w.B, w.K, dtype=torch.int32, device="cuda")
     assert n == fkm.fkm_lloyd_metric(xt, torch.from_numpy(c0).cuda(), 3, 0.0, i2, c2, n2, metric)
     assert torch.equal(ids, i2) and torch.equal(centers, c2)
+
+
+@pytest.mark.parametrize("metric", ["dot", "cosine"])
+@pytest.mark.parametrize("cfg,B,N,K,chunk", [(1, None, None, None, 1000),
+                                             (2, 2, 8192, 256, 3000)])
+def test_host_streamed_loop_against_oracle(metric, cfg, B, N, K, chunk):
+    """fkm_lloyd_host_metric streams pinned points in chunks (ragged last
+    chunk, several chunks per batch): (i) its objective is the oracle's
+    objective of its own last assignment; (ii) walked iteration by iteration
+    against the oracle (check_free_running) it ends within 1e-4 of the
+    oracle's objective; (iii) its ids match the device-resident loop's up to
+    near-tie flips (the two add the cluster sums in different orders)."""
+    it = 4
+    w = datagen.CONFIGS[cfg].scaled(B=B, N=N, K=K, iters=it) if B else \
+        datagen.CONFIGS[cfg].scaled(iters=it)
+    x, xt, c0 = problem(w)
+    xh = xt.cpu().pin_memory()
+    c = torch.from_numpy(c0).cuda()
+
+    def run(n_it):
+        ids = torch.empty(w.B, w.N, dtype=torch.int32, device="cuda")
+        cen = torch.empty_like(c)
+        cnt = torch.empty(w.B, w.K, dtype=torch.int32, device="cuda")
+        obj = torch.empty(w.B, dtype=torch.float64, device="cuda")
+        assert fkm.fkm_lloyd_host_metric(xh, c, n_it, 0.0, chunk, ids, cen, cnt, metric,
+                                         obj) == n_it
+        return ids, cen, cnt, obj
+
+    ids, cen, cnt, obj = run(it)
+    assert np.all(cnt.cpu().numpy().sum(1) == w.N)
+    _, c_prev, _, _ = run(it - 1)
+    g_ids, g_obj = ids.cpu().numpy(), obj.cpu().numpy()
+    check_assign_sim(x, w.dtype, c_prev.cpu().numpy(), g_ids, metric)
+    check_objective(x, w.dtype, g_ids, c_prev.cpu().numpy(), g_obj, metric)
+
+    def prefix(t):
+        i, ce, n, _ = run(t)
+        return i.cpu().numpy(), ce.cpu().numpy(), n.cpu().numpy()
+
+    check_free_running(x, w.dtype, c0, it, 0.0, prefix, lambda: (g_ids, g_obj, it),
+                       f"host-streamed {metric} workload {cfg}", metric=metric)
+    i2 = torch.empty_like(ids)
+    c2 = torch.empty_like(c)
+    n2 = torch.empty_like(cnt)
+    assert fkm.fkm_lloyd_metric(xt, c, it, 0.0, i2, c2, n2, metric) == it
+    assert (ids != i2).float().mean().item() <= 1e-3
+
+
+def test_host_streamed_euclid_metric_is_the_plain_host_loop():
+    w = datagen.CONFIGS[2].scaled(B=2, N=5000, K=200, iters=3)
+    x, xt, c0 = problem(w)
+    xh = xt.cpu().pin_memory()
+    c = torch.from_numpy(c0).cuda()
+    outs = []
+    for use_metric in (False, True):
+        ids = torch.empty(w.B, w.N, dtype=torch.int32, device="cuda")
+        cen = torch.empty_like(c)
+        cnt = torch.empty(w.B, w.K, dtype=torch.int32, device="cuda")
+        obj = torch.empty(w.B, dtype=torch.float64, device="cuda")
+        if use_metric:
+            n = fkm.fkm_lloyd_host_metric(xh, c, 3, 0.0, 1500, ids, cen, cnt, "euclid", obj)
+        else:
+            n = fkm.fkm_lloyd_host(xh, c, 3, 0.0, 1500, ids, cen, cnt, obj)
+        outs.append((n, ids, cen, cnt, obj))
+    (n0, i0, c_0, k0, o0), (n1, i1, c_1, k1, o1) = outs
+    assert n0 == n1 == 3
+    assert torch.equal(i0, i1) and torch.equal(k0, k1)
+    assert torch.allclose(c_0, c_1, rtol=1e-6, atol=1e-6)   # fp64 atomics: order may differ
+    assert torch.allclose(o0, o1, rtol=1e-9)
