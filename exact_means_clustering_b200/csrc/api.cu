@@ -314,11 +314,12 @@ static fkm_status step_update(const Ws& w, const void* x, const int32_t* ids, co
                         L.count_sort ? nullptr : segstart, L.count_sort ? nullptr : segend,
                         w.status()));
   if (ev) FKM_TRY(record_stage(ev[3], st));
-  if (euclid && requant && shifts && finalize_prep_fits(L.B, L.Kp, L.D)) {
+  if (requant && shifts && finalize_prep_fits(L.B, L.Kp, L.D, L.metric)) {
     FKM_TRY(launch_finalize_prep(L.B, L.K, L.Kp, L.D, L.dtype, range, segstart, segend,
                                  w.at<double>(L.sums64), prev, next, counts, w.at<float>(L.mvec),
                                  w.at<void>(L.cq), w.at<void>(L.caug), shifts->shift_out,
-                                 shifts->max_shift, st));
+                                 shifts->max_shift, st, L.metric, w.at<double>(L.cnorm),
+                                 euclid ? nullptr : obj));
     shifts->done = true;
     return FKM_OK;
   }

@@ -167,18 +167,21 @@ constexpr int AUG_SLAB = 16;
 fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int D, int dtype,
                                  float* m, void* cq, void* caug, cudaStream_t st,
                                  int metric = FKM_METRIC_EUCLID, double* cnorm = nullptr);
-// The end of a Euclidean Lloyd iteration in one launch: finalize (counts,
-// new centroids from the segment sums, sums64 cleared), the mean centroid m
+// The end of a Lloyd iteration in one launch: finalize (counts, new
+// centroids from the segment sums, sums64 cleared), the mean centroid m
 // (bit for bit launch_prep_centroids'), the next assign's operands and bias
 // slabs, and the batch shifts (shift_out [B], optional; max_shift optional,
-// zeroed by the caller).  For D <= 256, Kp <= 1024 and B <= 65535
-// (finalize_prep_fits).
-bool finalize_prep_fits(int B, int Kp, int D);
+// zeroed by the caller).  metric: Euclidean, or dot / cosine (the similarity
+// finalize; cnorm [B*K] receives the cosine row norms; obj_out [B], optional,
+// the objective of the assignment).  For Kp <= 1024, B <= 65535 and D <= 256
+// (Euclidean) or D <= 128 (finalize_prep_fits).
+bool finalize_prep_fits(int B, int Kp, int D, int metric);
 fkm_status launch_finalize_prep(int B, int K, int Kp, int D, int dtype, int range,
                                 const int32_t* segstart, const int32_t* segend, double* sums64,
                                 const float* prev, float* centers, int32_t* counts, float* m,
                                 void* cq, void* caug, double* shift_out, double* max_shift,
-                                cudaStream_t st);
+                                cudaStream_t st, int metric = FKM_METRIC_EUCLID,
+                                double* cnorm = nullptr, double* obj_out = nullptr);
 // fp32 points: split rows into xs; xn (optional) = ||x - m[row / N]||^2
 // (||x||^2 when m is null).
 fkm_status launch_points_prep(const void* x, int64_t rows, int D, int dtype, void* xs, float* xn,

@@ -295,16 +295,113 @@ struct FinPrepParams {
   uint16_t* caug;
   double* shift_out;   // optional [B]
   double* max_shift;   // optional (zeroed by the caller): max over batches
+  int metric;          // FKM_METRIC_*; dot and cosine need D <= 128
+  double* cnorm;       // cosine: the new centroids' row norms [B*K]
+  double* obj_out;     // dot / cosine, optional [B]: the objective of the assignment
 };
 
-__global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS * 32)
+// One cluster of the dot / cosine finalize (finalize_sim_kernel's arithmetic
+// for D <= 128, one 16-byte piece per lane): writes the new centroid (the
+// mean, its unit direction for cosine, or prev for an empty or zero-sum
+// cluster) and the count; returns the shift in every lane and adds the
+// cluster's objective share to *obj; cs receives the column values the mean
+// centroid adds (the row scaled by its norm for cosine, whose norm, summed
+// in row_norms_kernel's order, goes to cnorm).
+__device__ __forceinline__ double finalize_sim_row(const FinPrepParams& p, int64_t key,
+                                                   int32_t nk, bool interior, int lane,
+                                                   double* obj, double (&cs)[4]) {
+  const bool cosine = p.metric == FKM_METRIC_COSINE;
+  const int d = 4 * lane;
+  const bool on = d < p.D;
+  const int64_t e = key * p.D + d;
+  const double n = (double)nk;
+  float4 pv = make_float4(0.f, 0.f, 0.f, 0.f), v = pv;
+  double sd[4] = {0.0, 0.0, 0.0, 0.0};
+  if (on) {
+    pv = *reinterpret_cast<const float4*>(p.prev + e);
+    if (nk > 0 && interior) {
+      v = *reinterpret_cast<const float4*>(p.centers + e);
+      sd[0] = (double)v.x * n;
+      sd[1] = (double)v.y * n;
+      sd[2] = (double)v.z * n;
+      sd[3] = (double)v.w * n;
+    } else if (nk > 0) {
+      double2* s2 = reinterpret_cast<double2*>(p.sums64 + e);
+      const double2 a = s2[0], c = s2[1];
+      sd[0] = a.x;
+      sd[1] = a.y;
+      sd[2] = c.x;
+      sd[3] = c.y;
+      v = make_float4((float)(a.x / n), (float)(a.y / n), (float)(c.x / n), (float)(c.y / n));
+      s2[0] = make_double2(0.0, 0.0);
+      s2[1] = make_double2(0.0, 0.0);
+    }
+  }
+  const float vv4[4] = {v.x, v.y, v.z, v.w}, pv4[4] = {pv.x, pv.y, pv.z, pv.w};
+  double vv = 0.0, pp = 0.0, sp = 0.0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    vv += (double)vv4[j] * (double)vv4[j];
+    pp += (double)pv4[j] * (double)pv4[j];
+    sp += sd[j] * (double)pv4[j];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    vv += __shfl_xor_sync(0xffffffffu, vv, o);
+    pp += __shfl_xor_sync(0xffffffffu, pp, o);
+    sp += __shfl_xor_sync(0xffffffffu, sp, o);
+  }
+  const double pn = sqrt(pp), vn = sqrt(vv);
+  const bool keep = nk == 0 || (cosine && !(vv > 0.0));
+  float o4[4];
+  double sh = 0.0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    o4[j] = keep ? pv4[j] : cosine ? (float)((double)vv4[j] / vn) : vv4[j];
+    const double df = (double)o4[j] - (double)pv4[j];
+    sh += df * df;
+  }
+  if (on) *reinterpret_cast<float4*>(p.centers + e) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sh += __shfl_xor_sync(0xffffffffu, sh, o);
+  *obj += cosine ? (pn > 0.0 ? sp / pn : 0.0) : sp;
+  if (lane == 0 && p.counts) p.counts[key] = nk;
+  if (!cosine) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) cs[j] += on ? (double)o4[j] : 0.0;
+    return sh;
+  }
+  // ||o|| in row_norms_kernel's order: lane l sums elements l, l + 32, ...,
+  // which lanes (l + 32 q) / 4 hold as their component l % 4
+  double s = 0.0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int src = (lane >> 2) + 8 * q;
+    float t[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) t[j] = __shfl_sync(0xffffffffu, o4[j], src);
+    const float ov = t[lane & 3];
+    if (lane + 32 * q < p.D) s += (double)ov * (double)ov;
+  }
+  s = warp_sum(s);
+  const double cn = sqrt(s);
+  if (lane == 0) p.cnorm[key] = cn;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    cs[j] += on ? (double)(cn > 0.0 ? (float)((double)o4[j] / cn) : 0.0f) : 0.0;
+  return sh;
+}
+
+__global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS * 32, 2)
     finalize_prep_kernel(FinPrepParams p) {
   pdl_wait();   // the previous kernel of the stream has completed
   pdl_trigger();
   __shared__ double colsum[FP_WARPS][FP_MAX_D];
   __shared__ double cta_sum[FP_MAX_D];
   __shared__ double wshift[FP_WARPS];
+  __shared__ double wobj[FP_WARPS];
   __shared__ double cta_shift;
+  __shared__ double cta_obj;
   __shared__ __align__(16) float msh[FP_MAX_D];
   const int r = (int)ptx::cluster_ctarank();
   const int b = blockIdx.y;
@@ -318,12 +415,17 @@ __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS *
   double cs[J][4];
 #pragma unroll
   for (int j = 0; j < J; ++j) cs[j][0] = cs[j][1] = cs[j][2] = cs[j][3] = 0.0;
-  double shw = 0.0;
+  double shw = 0.0, objw = 0.0;
+  const bool euclid = p.metric == FKM_METRIC_EUCLID;
   for (int k = r * R + warp; k < r * R + R && k < p.K; k += FP_WARPS) {
     const int64_t key = kb + k;
     const int32_t s0 = p.segstart[key], s1 = p.segend[key];
     const int32_t nk = s1 - s0;
     const bool interior = nk > 0 && (s0 / p.range) == ((s1 - 1) / p.range);
+    if (!euclid) {
+      shw += finalize_sim_row(p, key, nk, interior, lane, &objw, cs[0]);
+      continue;
+    }
     if (lane == 0 && p.counts) p.counts[key] = nk;
     double sh = 0.0;
 #pragma unroll
@@ -366,7 +468,10 @@ __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS *
       colsum[warp][d + 3] = cs[j][3];
     }
   }
-  if (lane == 0) wshift[warp] = shw;
+  if (lane == 0) {
+    wshift[warp] = shw;
+    wobj[warp] = objw;
+  }
   __syncthreads();
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     double t = 0.0;
@@ -375,10 +480,14 @@ __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS *
     cta_sum[d] = t;
   }
   if (threadIdx.x == 0) {
-    double t = 0.0;
+    double t = 0.0, o = 0.0;
 #pragma unroll 1
-    for (int w = 0; w < FP_WARPS; ++w) t += wshift[w];
+    for (int w = 0; w < FP_WARPS; ++w) {
+      t += wshift[w];
+      o += wobj[w];
+    }
     cta_shift = t;
+    cta_obj = o;
   }
   // ---- 2. the batch's mean and shift across the cluster
   ptx::cluster_sync();   // release / acquire: every CTA's sums (and centroids) visible
@@ -399,6 +508,13 @@ __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS *
     if (p.max_shift)   // shift >= 0: the bit pattern orders like the value
       atomicMax(reinterpret_cast<unsigned long long*>(p.max_shift),
                 (unsigned long long)__double_as_longlong(t));
+    if (!euclid && p.obj_out) {
+      double o = 0.0;
+#pragma unroll 1
+      for (int q = 0; q < MEAN_CHUNKS; ++q)
+        o += ptx::ld_shared_cluster_f64(ptx::mapa_rank(&cta_obj, q));
+      p.obj_out[b] = o;
+    }
   }
   ptx::cluster_sync();   // no CTA leaves while another still reads its shared memory
   // ---- 3. the next assign's operands for this CTA's rows
@@ -406,7 +522,8 @@ __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS *
     const int k = r * R + i;
     const bool real = k < p.K;
     prep_row(p.centers + (kb + k) * D, msh, true, real, kb + k, (int64_t)b * p.Kp + k, D,
-             p.dtype, p.cq, p.caug, nullptr, true, lane & 7);
+             p.dtype, p.cq, p.caug, p.metric == FKM_METRIC_COSINE ? p.cnorm : nullptr, euclid,
+             lane & 7);
   }
 }
 
@@ -491,16 +608,17 @@ fkm_status launch_prep_centroids(const float* centers, int B, int K, int Kp, int
 // A CTA finalizes and prepares Kp / MEAN_CHUNKS rows, one after another per
 // warp; beyond 128 rows (Kp > 1024) the separate kernels, with every row
 // in its own warp, finish sooner.
-bool finalize_prep_fits(int B, int Kp, int D) {
-  return D <= FP_MAX_D && B <= 65535 && Kp <= 1024;
+bool finalize_prep_fits(int B, int Kp, int D, int metric) {
+  return D <= (metric == FKM_METRIC_EUCLID ? FP_MAX_D : 128) && B <= 65535 && Kp <= 1024;
 }
 
 fkm_status launch_finalize_prep(int B, int K, int Kp, int D, int dtype, int range,
                                 const int32_t* segstart, const int32_t* segend, double* sums64,
                                 const float* prev, float* centers, int32_t* counts, float* m,
                                 void* cq, void* caug, double* shift_out, double* max_shift,
-                                cudaStream_t st) {
-  if (!finalize_prep_fits(B, Kp, D) || Kp % BN != 0) {
+                                cudaStream_t st, int metric, double* cnorm, double* obj_out) {
+  if (!finalize_prep_fits(B, Kp, D, metric) || Kp % BN != 0 ||
+      (metric == FKM_METRIC_COSINE && !cnorm)) {
     set_error("finalize_prep: D = %d or Kp = %d out of range", D, Kp);
     return FKM_ERR_INTERNAL;
   }
@@ -522,6 +640,9 @@ fkm_status launch_finalize_prep(int B, int K, int Kp, int D, int dtype, int rang
   p.caug = static_cast<uint16_t*>(caug);
   p.shift_out = shift_out;
   p.max_shift = max_shift;
+  p.metric = metric;
+  p.cnorm = cnorm;
+  p.obj_out = obj_out;
   FKM_CUDA_TRY(launch_pdl(finalize_prep_kernel, dim3(MEAN_CHUNKS, (unsigned)B), dim3(FP_WARPS * 32),
                           0, st, p));
   note_launch();
