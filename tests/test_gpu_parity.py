@@ -534,3 +534,31 @@ def test_large_d_host_streaming():
     fkm.fkm_lloyd(xt, torch.from_numpy(c0).cuda(), 2, 0.0, i2, c2, n2)
     assert (ids != i2).float().mean().item() <= 1e-3
     assert torch.allclose(centers, c2, rtol=1e-4, atol=1e-4)
+
+
+def test_inputs_written_by_a_kernel_just_before_the_call():
+    """The loop's kernels are launched as programmatic dependents of the work
+    before them on the stream; an input written by a torch kernel right
+    before the call must be seen in full (every kernel waits for its
+    predecessor before touching memory)."""
+    w = datagen.CONFIGS[2].scaled(B=2, N=6000, K=300, iters=3)
+    x, xt, c0 = problem(w)
+    ref = _empty(w.B, w.N, w.K, w.D)
+    fkm.fkm_lloyd(xt, torch.from_numpy(c0).cuda(), 3, 0.0, *ref)
+    ids_a = torch.empty(w.B, w.N, dtype=torch.int32, device="cuda")
+    fkm.fkm_assign(xt, torch.from_numpy(c0).cuda(), ids_a)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        xs = torch.zeros_like(xt)
+        cs = torch.zeros(w.B, w.K, w.D, device="cuda")
+        got = _empty(w.B, w.N, w.K, w.D)
+        xs.add_(xt)                          # elementwise kernels on the same stream,
+        cs.add_(torch.from_numpy(c0).cuda())  # launched just before the library's
+        fkm.fkm_lloyd(xs, cs, 3, 0.0, *got)
+        assert torch.equal(got[0], ref[0]) and torch.equal(got[2], ref[2])
+        assert torch.allclose(got[1], ref[1], rtol=1e-6, atol=1e-6)
+        xs2 = torch.zeros_like(xt)
+        ids = torch.full((w.B, w.N), -1, dtype=torch.int32, device="cuda")
+        xs2.add_(xt)
+        fkm.fkm_assign(xs2, cs, ids)
+        assert torch.equal(ids, ids_a)
