@@ -21,7 +21,13 @@
  *              depends on N*K (the B x N x K distance matrix is never formed).
  *   Streams    `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *              stream).  Work is stream-ordered; functions marked "async" return
- *              before the GPU finishes.
+ *              before the GPU finishes.  The library's kernels are launched as
+ *              programmatic dependents (each waits for the stream's previous
+ *              work to complete before it touches memory) and let the next
+ *              kernel be scheduled early: a caller kernel launched after a call
+ *              with programmatic stream serialization of its own must wait
+ *              (griddepcontrol.wait) before it reads the call's outputs; an
+ *              ordinary launch is ordered as usual.
  *   Limits     B, N, K, D >= 1; D * sizeof(dtype) a multiple of 16 bytes
  *              (D % 8 == 0 for bf16/fp16, D % 4 == 0 for fp32);
  *              D <= 4096; B*N < 2^31; B*K < 2^31.  Above D = 256 (fp32:
