@@ -392,6 +392,7 @@ __device__ __forceinline__ double finalize_sim_row(const FinPrepParams& p, int64
   return sh;
 }
 
+template <bool kEuclid>
 __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS * 32, 2)
     finalize_prep_kernel(FinPrepParams p) {
   pdl_wait();   // the previous kernel of the stream has completed
@@ -416,13 +417,25 @@ __global__ void __cluster_dims__(MEAN_CHUNKS, 1, 1) __launch_bounds__(FP_WARPS *
 #pragma unroll
   for (int j = 0; j < J; ++j) cs[j][0] = cs[j][1] = cs[j][2] = cs[j][3] = 0.0;
   double shw = 0.0, objw = 0.0;
-  const bool euclid = p.metric == FKM_METRIC_EUCLID;
-  for (int k = r * R + warp; k < r * R + R && k < p.K; k += FP_WARPS) {
+  constexpr bool euclid = kEuclid;   // else dot / cosine (p.metric)
+  // the next row's segment bounds are loaded while the current row is
+  // finalized, so each row waits for one round trip to memory, not two
+  const int kend = min(r * R + R, p.K);
+  int32_t nb0 = 0, nb1 = 0;
+  if (r * R + warp < kend) {
+    nb0 = p.segstart[kb + r * R + warp];
+    nb1 = p.segend[kb + r * R + warp];
+  }
+  for (int k = r * R + warp; k < kend; k += FP_WARPS) {
     const int64_t key = kb + k;
-    const int32_t s0 = p.segstart[key], s1 = p.segend[key];
+    const int32_t s0 = nb0, s1 = nb1;
+    if (k + FP_WARPS < kend) {
+      nb0 = p.segstart[key + FP_WARPS];
+      nb1 = p.segend[key + FP_WARPS];
+    }
     const int32_t nk = s1 - s0;
     const bool interior = nk > 0 && (s0 / p.range) == ((s1 - 1) / p.range);
-    if (!euclid) {
+    if constexpr (!euclid) {
       shw += finalize_sim_row(p, key, nk, interior, lane, &objw, cs[0]);
       continue;
     }
@@ -643,8 +656,12 @@ fkm_status launch_finalize_prep(int B, int K, int Kp, int D, int dtype, int rang
   p.metric = metric;
   p.cnorm = cnorm;
   p.obj_out = obj_out;
-  FKM_CUDA_TRY(launch_pdl(finalize_prep_kernel, dim3(MEAN_CHUNKS, (unsigned)B), dim3(FP_WARPS * 32),
-                          0, st, p));
+  if (metric == FKM_METRIC_EUCLID)
+    FKM_CUDA_TRY(launch_pdl(finalize_prep_kernel<true>, dim3(MEAN_CHUNKS, (unsigned)B),
+                            dim3(FP_WARPS * 32), 0, st, p));
+  else
+    FKM_CUDA_TRY(launch_pdl(finalize_prep_kernel<false>, dim3(MEAN_CHUNKS, (unsigned)B),
+                            dim3(FP_WARPS * 32), 0, st, p));
   note_launch();
   FKM_CUDA_TRY(cudaGetLastError());
   return FKM_OK;
