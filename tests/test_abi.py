@@ -192,6 +192,13 @@ def test_binding_refuses_wrong_sizes_and_host_tensors(fkm):
     with pytest.raises(ValueError, match="must be a CUDA tensor"):
         fkm.fkm_lloyd_host(x, c, 3, 0.0, 16, ids, torch.zeros(2, 4, 16),
                            torch.zeros(2, 4, dtype=torch.int32), ws=ws)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        fkm.fkm_lloyd_host_metric(x, c, 3, 0.0, 16, ids, torch.zeros(2, 4, 16),
+                                  torch.zeros(2, 4, dtype=torch.int32), "cosine", ws=ws)
+    with pytest.raises(ValueError, match="objective has shape"):
+        fkm.fkm_lloyd_host_metric(x, c, 3, 0.0, 16, ids, torch.zeros(2, 4, 16),
+                                  torch.zeros(2, 4, dtype=torch.int32), "dot",
+                                  torch.zeros(3, dtype=torch.float64), ws=ws)
     with pytest.raises(ValueError, match="sums has shape"):
         fkm.fkm_finalize_sums(torch.zeros(2, 4, 8, dtype=torch.float64),
                               torch.zeros(2, 4, dtype=torch.float64), c, torch.zeros(2, 4, 16),
