@@ -265,20 +265,23 @@ __global__ void prep_centroids_kernel(const float* __restrict__ c, const float* 
            row, D, dtype, cq, caug, cn, bias, lane & 7);
 }
 
-// The end of a Euclidean Lloyd iteration in one launch: one thread-block
-// cluster of MEAN_CHUNKS CTAs per batch (grid MEAN_CHUNKS x B), CTA r owning
-// the padded rows [r R, (r+1) R), R = Kp / MEAN_CHUNKS.
-//   1. finalize (as finalize_kernel): warp w takes the rows r R + w,
-//      r R + w + MEAN_WAYS, ...: count, new centroid (s/n of a crossing run,
-//      the value the segment sums wrote for an interior one, the previous
-//      centroid for an empty cluster), its shift, and the running fp64 sums
-//      of the new centroid's columns -- partial (r, w) of the mean's order;
+// The end of a Lloyd iteration in one launch: one thread-block cluster of
+// MEAN_CHUNKS CTAs per batch (grid MEAN_CHUNKS x B), CTA r owning the padded
+// rows [r R, (r+1) R), R = Kp / MEAN_CHUNKS.
+//   1. finalize (as finalize_kernel, or finalize_sim_kernel for dot and
+//      cosine k-means): warp w takes the rows r R + w, r R + w + MEAN_WAYS,
+//      ...: count, new centroid (s/n of a crossing run, the value the segment
+//      sums wrote for an interior one, the previous centroid for an empty
+//      cluster), its shift, and the running fp64 sums of the new centroid's
+//      columns (as the assignment sees them) -- partial (r, w) of the mean's
+//      order;
 //   2. the CTA adds its partials (w = 0, 1, ...), the cluster barrier makes
 //      every CTA's sums visible, and every CTA adds the chunks (r = 0, 1, ...)
 //      from distributed shared memory: m, bit for bit center_kernel's; CTA 0
-//      also writes m and the batch's shift (same chunked order);
+//      also writes m, the batch's shift and, for dot and cosine, its
+//      objective (same chunked order);
 //   3. the CTA prepares the operands of its rows (prep_row) against m.
-// Columns are held four per lane, so D <= FP_MAX_D.
+// Columns are held four per lane, so D <= FP_MAX_D (128 for dot and cosine).
 constexpr int FP_WARPS = MEAN_WAYS;
 constexpr int FP_MAX_D = 256;
 
