@@ -477,6 +477,11 @@ static fkm_status assign_impl(int metric, int B, int N, int K, int D, int dtype,
   FKM_TRY(check_ptr(centers, "centers"));
   FKM_TRY(check_ptr(ids, "ids"));
   if (inertia) FKM_TRY(check_ptr(inertia, "inertia"));
+  if (inertia && B > 65535) {   // the objective kernel runs one grid row per batch
+    set_error("fkm_assign's objective needs B <= 65535 (B = %d); pass inertia = NULL or "
+              "split the batches", B);
+    return FKM_ERR_UNSUPPORTED;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Ws w{ws, &L};
   FKM_TRY(launch_prep_centroids(centers, B, K, L.Kp, D, dtype, w.at<float>(L.mvec),

@@ -129,8 +129,9 @@ extern "C" fkm_status fkm_centre(int B, int N, int D, int dtype, const void* x, 
     set_error("unknown dtype %d", dtype);
     return FKM_ERR_INVALID_ARG;
   }
-  if (((int64_t)D * elem_bytes(dtype)) % 16 != 0 || (int64_t)B * N >= (int64_t(1) << 31)) {
-    set_error("D * element size must be a multiple of 16 bytes and B * N < 2^31");
+  if (((int64_t)D * elem_bytes(dtype)) % 16 != 0 || (int64_t)B * N >= (int64_t(1) << 31) ||
+      B > 65535) {   // the partial sums run one grid row per batch
+    set_error("D * element size must be a multiple of 16 bytes, B * N < 2^31 and B <= 65535");
     return FKM_ERR_UNSUPPORTED;
   }
   const void* ptrs[] = {x, mu, x_out, ws};

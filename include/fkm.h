@@ -109,7 +109,8 @@ FKM_API fkm_status fkm_workspace_size(int B, int N, int K, int D, int dtype, siz
  *   x        device [B,N,D] dtype        centers  device [B,K,D] float32
  *   ids      device [B,N] int32 (out)
  *   inertia  device [B] float64 (out) = sum_i ||x_i - c_hat[b, ids_i]||^2 (direct
- *            difference, fp32 terms summed in fp64), or NULL
+ *            difference, fp32 terms summed in fp64), or NULL; with inertia,
+ *            B <= 65535 (FKM_ERR_UNSUPPORTED above)
  *   ws       device workspace of ws_bytes >= fkm_workspace_size(...)
  * Async. */
 FKM_API fkm_status fkm_assign(int B, int N, int K, int D, int dtype, const void* x, const float* centers,
@@ -303,7 +304,8 @@ FKM_API fkm_status fkm_partial_update_host(int B, int N, int K, int D, int dtype
  *                   to `dtype` (x_out may be x: centring in place)
  * x, x_out: device [B, N, D] in dtype; mu: device float32 [B, D]; ws: device
  * scratch of fkm_centre_workspace_size bytes.  Limits as for fkm_assign
- * (D * element size a multiple of 16, B * N < 2^31).  Async. */
+ * (D * element size a multiple of 16, B * N < 2^31), and B <= 65535
+ * (FKM_ERR_UNSUPPORTED above).  Async. */
 FKM_API fkm_status fkm_centre_workspace_size(int B, int N, int D, size_t* bytes);
 FKM_API fkm_status fkm_centre(int B, int N, int D, int dtype, const void* x, float* mu,
                               void* x_out, void* ws, size_t ws_bytes, void* stream);

@@ -229,3 +229,17 @@ def test_noalloc_size_limit_matches_the_header(fkm):
     a = 1 << 12   # a 16-byte-aligned non-null stand-in; validation runs before any access
     rc_out = L.fkm_assign_noalloc(1, 128, K_in + 256, D, 2, a, a, a, None)
     assert rc_out == 2 and b"static scratch" in L.fkm_last_error()
+
+
+def test_batch_per_grid_row_paths_reject_more_than_65535_batches(fkm):
+    """fkm_assign's objective and fkm_centre run one grid row per batch: more
+    than 65535 batches are refused before any launch (no CUDA call here)."""
+    L = fkm.lib()
+    buf = ctypes.create_string_buffer(1 << 12)
+    a = (ctypes.addressof(buf) + 15) & ~15
+    huge = 1 << 40   # a size check only: nothing is read or written
+    B = 70000
+    assert L.fkm_assign(B, 1, 1, 8, 2, a, a, a, a, a, huge, None) == 2
+    assert b"65535" in L.fkm_last_error()
+    assert L.fkm_centre(B, 1, 8, 2, a, a, a, a, huge, None) == 2
+    assert b"65535" in L.fkm_last_error()
