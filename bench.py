@@ -106,7 +106,7 @@ def assign_traffic(config_name):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
 
     def __init__(self, index):
         self.index = index
